@@ -1,0 +1,18 @@
+"""fp64 CPU oracle of the Sparse-to-Dense hot path.
+
+TEST INFRASTRUCTURE: imported only by the test-suite, ``__graft_entry__.smoke()``
+and the CPU-baseline legs of ``bench.py``; never by the library.
+"""
+from .std_oracle import (  # noqa: F401
+    accept_prefix,
+    attend,
+    decode_round,
+    dense_verify_attn,
+    kv_append,
+    kv_commit,
+    select_topk,
+    selection_scores,
+    softmax,
+    sparse_decode_attn,
+    topk_indices,
+)

@@ -1,0 +1,266 @@
+"""Checks that pin the fp64 oracle to facts outside itself.
+
+Each ``check_*`` takes the oracle module (or a stand-in with the same
+functions) and raises AssertionError on a mismatch, so the same checks can be
+run against deliberately broken copies of the oracle to show that they catch
+plausible mistakes (dropped scale, wrong GQA grouping, off-by-one mask,
+wrong tie rule, non-prefix acceptance, wrong commit window).
+
+Sources of truth used here, none of them the oracle's own formulas:
+  * hand-derived closed forms stored under tests/golden/ (logits ln 1, ln 2, ...
+    make the softmax weights small integers over their sum);
+  * brute-force enumeration on tiny inputs;
+  * library routines: heapq.nlargest, torch's scaled_dot_product_attention in
+    float64, the logistic function written via tanh;
+  * mathematical invariants (a mean of distributions sums to 1, uniform
+    attention when all logits are equal).
+"""
+from __future__ import annotations
+
+import heapq
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def load_golden(name: str) -> dict:
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------------------- attention
+
+def check_golden_attention(orc) -> None:
+    g = load_golden("attention_3key.json")
+    o = orc.attend(np.array(g["q"]), np.array(g["k"]), np.array(g["v"]))
+    np.testing.assert_allclose(o, g["expected"], atol=g["atol"], rtol=0)
+
+
+def check_golden_verify(orc) -> None:
+    g = load_golden("verify_causal_2row.json")
+    k = np.array(g["k"])[None, None, None]          # [L=1][B=1][Hkv=1][n][d]
+    v = np.array(g["v"])[None, None, None]
+    q = np.array(g["q"])[None, None, None]          # [1][1][Hq=1][2][d]
+    o = orc.dense_verify_attn(q, k, v, np.array([g["n_ctx"]]))
+    np.testing.assert_allclose(o[0, 0, 0], g["expected"], atol=g["atol"], rtol=0)
+
+
+def check_attention_vs_sdpa(orc, seed: int = 3) -> None:
+    """Decode and verify attention against torch SDPA (float64) with an explicit mask."""
+    import torch
+    rng = np.random.default_rng(seed)
+    L, B, Hq, Hkv, d, gamma = 2, 2, 6, 2, 16, 3
+    G = Hq // Hkv
+    n_ctx = np.array([11, 5])
+    cap = 20
+    k = rng.standard_normal((L, B, Hkv, cap, d)) * 2
+    v = rng.standard_normal((L, B, Hkv, cap, d))
+    q = rng.standard_normal((L, B, Hq, gamma + 1, d)) * 2
+    o = orc.dense_verify_attn(q, k, v, n_ctx)
+    o_sp = orc.sparse_decode_attn(q[:, :, :, :1], k, v, n_ctx + 1)
+    for l in range(L):
+        for b in range(B):
+            n = int(n_ctx[b]) + gamma + 1
+            kk = torch.from_numpy(np.repeat(k[l, b, :, :n], G, axis=0))    # [Hq][n][d]
+            vv = torch.from_numpy(np.repeat(v[l, b, :, :n], G, axis=0))
+            qq = torch.from_numpy(q[l, b])                                  # [Hq][rows][d]
+            i = torch.arange(gamma + 1)[:, None]
+            j = torch.arange(n)[None, :]
+            mask = j < (int(n_ctx[b]) + i + 1)
+            ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, attn_mask=mask)
+            np.testing.assert_allclose(o[l, b], ref.numpy(), atol=1e-12, rtol=1e-12)
+            np.testing.assert_allclose(o_sp[l, b], ref.numpy()[:, :1], atol=1e-12, rtol=1e-12)
+
+
+def check_attention_closed_forms(orc, seed: int = 4) -> None:
+    rng = np.random.default_rng(seed)
+    d = 8
+    q = rng.standard_normal(d)
+    # one key: the output is that value row
+    v1 = rng.standard_normal((1, d))
+    np.testing.assert_allclose(orc.attend(q, rng.standard_normal((1, d)), v1), v1[0], atol=1e-14)
+    # identical keys: uniform weights, the mean of the values
+    kk = np.repeat(rng.standard_normal((1, d)), 5, axis=0)
+    vv = rng.standard_normal((5, d))
+    np.testing.assert_allclose(orc.attend(q, kk, vv), vv.mean(axis=0), atol=1e-14)
+    # two keys: logistic weighting sigma(x) = (1 + tanh(x/2)) / 2 of the logit gap
+    k2 = rng.standard_normal((2, d))
+    v2 = rng.standard_normal((2, d))
+    x = (q @ k2[0] - q @ k2[1]) / math.sqrt(d)
+    w = 0.5 * (1.0 + math.tanh(0.5 * x))
+    np.testing.assert_allclose(orc.attend(q, k2, v2), w * v2[0] + (1 - w) * v2[1], atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- selection
+
+def check_golden_selection(orc) -> None:
+    g = load_golden("selection_gqa.json")
+    q_text = np.array(g["q_text"])[None, None]                     # [1][1][Hq][T][d]
+    kv = np.array(g["k_vis"])
+    Hkv, nv, d = 2, kv.shape[0], kv.shape[1]
+    T = q_text.shape[3]
+    k_full = np.zeros((1, 1, Hkv, nv + T, d))
+    k_full[0, 0, :, :nv] = kv
+    v_full = np.zeros_like(k_full)
+    for K, key in ((1, "expected_top1"), (2, "expected_top2")):
+        idx, scores, _, _, _ = orc.select_topk(q_text, k_full, v_full, np.array([nv]), T, K, nv + T)
+        np.testing.assert_allclose(scores[0, 0], g["expected_scores"], atol=g["atol"], rtol=0)
+        assert idx[0, 0].tolist() == g[key], (idx[0, 0].tolist(), g[key])
+
+
+def check_selection_invariants(orc, seed: int = 5) -> None:
+    rng = np.random.default_rng(seed)
+    G, T, d, nv = 3, 7, 16, 50
+    q = rng.standard_normal((G, T, d)) * 3
+    k = rng.standard_normal((nv, d))
+    s = orc.selection_scores(q, k)
+    assert s.shape == (nv,)
+    assert abs(s.sum() - 1.0) < 1e-12                       # a mean of distributions
+    assert (s > 0).all()
+    np.testing.assert_allclose(orc.selection_scores(np.zeros_like(q), k), np.full(nv, 1 / nv),
+                               atol=1e-15)                   # zero queries: uniform
+    np.testing.assert_allclose(orc.selection_scores(q, np.repeat(k[:1], nv, axis=0)),
+                               np.full(nv, 1 / nv), atol=1e-15)  # identical keys: uniform
+    # a key that dominates every row's softmax collects almost all mass
+    k2 = k.copy()
+    k2[17] = 40.0 * q.reshape(-1, d).mean(axis=0) / np.linalg.norm(q.reshape(-1, d).mean(axis=0))
+    s2 = orc.selection_scores(q, k2)
+    assert int(np.argmax(s2)) == 17
+
+
+def _brute_topk(s, K):
+    """The unique K-subset whose members all beat all non-members under (score desc, pos asc)."""
+    n = len(s)
+    found = []
+    for sub in itertools.combinations(range(n), K):
+        ins = set(sub)
+        if all((s[a] > s[b]) or (s[a] == s[b] and a < b) for a in ins for b in range(n) if b not in ins):
+            found.append(list(sub))
+    assert len(found) == 1
+    return found[0]
+
+
+def check_topk_bruteforce(orc, seed: int = 6) -> None:
+    rng = np.random.default_rng(seed)
+    for trial in range(40):
+        n = int(rng.integers(1, 8))
+        s = rng.integers(0, 4, size=n).astype(np.float64) / 4   # many ties
+        for K in range(n + 1):
+            got = orc.topk_indices(s, K).tolist()
+            assert got == _brute_topk(s, K), (s, K, got)
+            want = sorted(heapq.nlargest(K, range(n), key=lambda i: (s[i], -i)))
+            assert got == want
+
+
+def check_topk_special(orc, seed: int = 7) -> None:
+    rng = np.random.default_rng(seed)
+    s = rng.random(300)
+    s[[10, 200]] = 2.0                                        # tie at the maximum
+    assert orc.topk_indices(s, 1).tolist() == [int(np.argmax(s))] == [10]
+    assert orc.topk_indices(s, 300).tolist() == list(range(300))
+    assert orc.topk_indices(s, 0).tolist() == []
+
+
+def check_full_k_sparse_equals_dense(orc, seed: int = 8) -> None:
+    """K = Nv keeps every visual row in order, so sparse attention equals dense attention."""
+    rng = np.random.default_rng(seed)
+    L, B, Hq, Hkv, d, nv, T = 1, 1, 4, 2, 8, 30, 5
+    cap = nv + T + 4
+    k = np.zeros((L, B, Hkv, cap, d))
+    v = np.zeros((L, B, Hkv, cap, d))
+    k[..., :nv + T, :] = rng.standard_normal((L, B, Hkv, nv + T, d))
+    v[..., :nv + T, :] = rng.standard_normal((L, B, Hkv, nv + T, d))
+    qt = rng.standard_normal((L, B, Hq, T, d))
+    idx, _, ksp, vsp, lsp = orc.select_topk(qt, k, v, np.array([nv]), T, nv, cap)
+    assert idx[0, 0, 0].tolist() == list(range(nv))
+    np.testing.assert_array_equal(ksp[..., :nv + T, :], k[..., :nv + T, :])
+    q = rng.standard_normal((L, B, Hq, 1, d))
+    a = orc.sparse_decode_attn(q, ksp, vsp, lsp)
+    bb = orc.dense_verify_attn(q, k, v, np.array([nv + T - 1]))
+    np.testing.assert_allclose(a, bb, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- acceptance
+
+def check_golden_accept(orc) -> None:
+    g = load_golden("accept_cases.json")
+    for c in g["cases"]:
+        gm = len(c["draft"])
+        n1, acc = orc.accept_prefix(np.array(c["draft"], dtype=np.int64).reshape(1, gm),
+                                    np.array(c["dense"]).reshape(1, gm + 1))
+        assert int(n1[0]) == c["n_plus_1"], c
+        assert acc[0].tolist() == c["accepted"], c
+
+
+def check_accept_bruteforce(orc) -> None:
+    """Every match pattern for gamma <= 10: n + 1 = (index of the lowest 0 bit) + 1."""
+    for gamma in range(0, 11):
+        pats = np.arange(2 ** gamma)
+        dense = np.tile(np.arange(100, 100 + gamma + 1), (len(pats), 1))
+        bits = (pats[:, None] >> np.arange(gamma)[None, :]) & 1
+        draft = np.where(bits == 1, dense[:, :gamma], dense[:, :gamma] + 7)
+        n1, acc = orc.accept_prefix(draft, dense)
+        for p in range(len(pats)):
+            expect = (~int(p) & (int(p) + 1)).bit_length()
+            assert int(n1[p]) == expect, (gamma, p)
+            assert 1 <= expect <= gamma + 1
+            assert acc[p, :expect].tolist() == dense[p, :expect].tolist()
+            assert (acc[p, expect:] == -1).all()
+
+
+# ----------------------------------------------------------------------------- round bookkeeping
+
+def check_commit(orc, seed: int = 9) -> None:
+    rng = np.random.default_rng(seed)
+    L, B, Hkv, d = 2, 3, 2, 4
+    kf = rng.standard_normal((L, B, Hkv, 20, d))
+    vf = rng.standard_normal((L, B, Hkv, 20, d))
+    ks = np.zeros((L, B, Hkv, 12, d))
+    vs = np.zeros((L, B, Hkv, 12, d))
+    lf = np.array([10, 4, 7])
+    ls = np.array([3, 2, 5])
+    n1 = np.array([1, 4, 2])
+    orc.kv_commit(kf, vf, ks, vs, lf, ls, n1)
+    assert lf.tolist() == [11, 8, 9] and ls.tolist() == [4, 6, 7]
+    for b, (a, s, n) in enumerate(((10, 3, 1), (4, 2, 4), (7, 5, 2))):
+        np.testing.assert_array_equal(ks[:, b, :, s:s + n], kf[:, b, :, a:a + n])
+        np.testing.assert_array_equal(vs[:, b, :, s:s + n], vf[:, b, :, a:a + n])
+        assert (ks[:, b, :, s + n:] == 0).all()
+
+
+def check_round_lossless_extremes(orc, seed: int = 10) -> None:
+    """All drafts right: gamma + 1 tokens per round; all wrong: only the bonus token."""
+    rng = np.random.default_rng(seed)
+    L, B, Hq, Hkv, d, gamma = 1, 2, 2, 1, 4, 3
+    for agree in (True, False):
+        st = {"k_full": np.zeros((L, B, Hkv, 40, d)), "v_full": np.zeros((L, B, Hkv, 40, d)),
+              "k_sp": np.zeros((L, B, Hkv, 30, d)), "v_sp": np.zeros((L, B, Hkv, 30, d)),
+              "len_full": np.array([6, 9]), "len_sp": np.array([3, 4])}
+        st["k_full"][..., :9, :] = rng.standard_normal((L, B, Hkv, 9, d))
+        dense = rng.integers(0, 50, size=(B, gamma + 1))
+        draft = dense[:, :gamma] if agree else dense[:, :gamma] + 1
+        kvv = rng.standard_normal((L, B, Hkv, gamma + 1, d))
+        out = orc.decode_round(st, rng.standard_normal((gamma, L, B, Hq, 1, d)),
+                               rng.standard_normal((gamma, L, B, Hkv, 1, d)),
+                               rng.standard_normal((gamma, L, B, Hkv, 1, d)),
+                               rng.standard_normal((L, B, Hq, gamma + 1, d)), kvv, kvv.copy(),
+                               draft, dense)
+        n = gamma + 1 if agree else 1
+        assert out["n_plus_1"].tolist() == [n, n]
+        assert out["accepted"][:, :n].tolist() == dense[:, :n].tolist()
+        assert st["len_full"].tolist() == [6 + n, 9 + n] and st["len_sp"].tolist() == [3 + n, 4 + n]
+        np.testing.assert_array_equal(st["k_sp"][:, 0, :, 3:3 + n], kvv[:, 0, :, :n])
+        np.testing.assert_array_equal(st["k_full"][:, 1, :, 9:9 + gamma + 1], kvv[:, 1])
+
+
+ALL_CHECKS = [
+    check_golden_attention, check_golden_verify, check_attention_vs_sdpa,
+    check_attention_closed_forms, check_golden_selection, check_selection_invariants,
+    check_topk_bruteforce, check_topk_special, check_full_k_sparse_equals_dense,
+    check_golden_accept, check_accept_bruteforce, check_commit, check_round_lossless_extremes,
+]

@@ -1,0 +1,272 @@
+/*
+ * std_b200.h -- C ABI of the Sparse-to-Dense (StD) decoding hot path on B200 (sm_100a).
+ *
+ * Sparse-to-Dense accelerates Video-LLM decoding without changing its output:
+ * a sparse mode of the model (attention over a top-K subset of the visual KV)
+ * drafts gamma tokens, and the dense mode (attention over the whole cache)
+ * verifies them in one pass; the longest agreeing prefix plus one bonus token
+ * is kept.  Sources: "Sparse-to-Dense: A Free Lunch for Lossless Acceleration
+ * of Video Understanding in LLMs" -- the gist.science technical summary
+ * (sections "Methodik" 2-4) and the paper abstract.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All tensor arguments are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or keeps them.  Scratch space is a caller-provided
+ *    device workspace whose size a *_workspace_size() query returns.
+ *  - Layouts are dense, row-major, head dimension innermost:
+ *        caches   [L][B][Hkv][cap][d]       (cap = dims->cap_full or cap_sparse)
+ *        queries  [L][B][Hq][rows][d]
+ *        outputs  [L][B][Hq][rows][d]  float32
+ *    Query head hq reads KV head hq / G with G = Hq / Hkv (standard grouped-
+ *    query attention; consecutive query heads share a KV head).
+ *  - Element type of Q/K/V is dims->dtype: STD_F32 (float) or STD_BF16
+ *    (bfloat16 bits).  Arithmetic is float32 in every kernel; bf16 operands go
+ *    through the tensor cores with float32 accumulation.
+ *  - Lengths (len_full, len_sparse, nvis) are int32 arrays on the DEVICE, one
+ *    entry per sequence, so whole rounds run without host synchronisation and
+ *    can be captured in a CUDA graph.
+ *  - Every call is asynchronous on `stream` (NULL = the legacy default stream).
+ *  - Return value: STD_OK (0) or a negative STD_ERR_* code.  Arguments that
+ *    the host can check are checked before anything is launched; nothing is
+ *    launched on error.  std_last_error() gives a message (thread-local).
+ *    Conditions that depend on device-resident lengths are checked by the
+ *    kernels: the offending (sequence, head) is skipped and a bit is OR-ed
+ *    into a per-device error word, read with std_get_device_error().
+ *  - No kernel waits on another kernel, CTA or device; nothing spins.
+ */
+#ifndef STD_B200_H
+#define STD_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (the runtime's CUstream_st*); NULL is the legacy default stream. */
+typedef struct CUstream_st* std_stream_t;
+
+enum std_status {
+  STD_OK = 0,
+  STD_ERR_INVALID_ARG = -1, /* null pointer, bad size or shape */
+  STD_ERR_UNSUPPORTED = -2, /* dtype / head dim / group shape this build has no kernel for */
+  STD_ERR_CAPACITY = -3,    /* a host-checkable size exceeds a cache capacity */
+  STD_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed */
+  STD_ERR_DEVICE = -5,      /* std_get_device_error found flags set */
+  STD_ERR_TIMEOUT = -6,     /* reserved: a bounded wait gave up (no current kernel waits) */
+  STD_ERR_WORKSPACE = -7    /* workspace missing or smaller than the size query returned */
+};
+
+enum std_dtype { STD_F32 = 0, STD_BF16 = 1 };
+
+/* Bits of the per-device error word (std_get_device_error). */
+enum std_device_error {
+  STD_DEVERR_CAPACITY = 1,  /* an append / commit / verify would pass the cache capacity */
+  STD_DEVERR_LENGTH = 2,    /* a device length was <= 0 or beyond the capacity in attention */
+  STD_DEVERR_K_RANGE = 4,   /* select: K > nvis[b], or nvis[b] + T > cap_full */
+  STD_DEVERR_NVIS_MAX = 8   /* select: nvis[b] > the host-side nvis_max bound */
+};
+
+/* Shape of the model slice a call works on.  cap_full / cap_sparse are the row
+ * capacities of the full and the sparse (compacted) caches. */
+typedef struct std_dims {
+  int32_t L, B, Hq, Hkv, d, dtype;
+  int64_t cap_full, cap_sparse;
+} std_dims;
+
+/* ---------------------------------------------------------------- library */
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int std_version(void);
+
+/* Message describing the last error returned on this host thread ("" if none). */
+const char* std_last_error(void);
+
+/* Read the current device's error word into *flags (may be NULL), optionally
+ * clearing it.  Orders after all work already queued on `stream` and blocks
+ * the host until that work is done.  Returns STD_ERR_DEVICE if any bit was
+ * set, else STD_OK (or STD_ERR_CUDA). */
+int std_get_device_error(int32_t* flags, int clear, std_stream_t stream);
+
+/* ---------------------------------------------------------------- prefill selection
+ *
+ * "Methodik" item 4 of the summary: the top-K visual KV entries are chosen
+ * once, at prefill, from the attention scores from text tokens to visual
+ * tokens, averaged; the choice differs per layer and head.  Item 2: the
+ * sparse model attends only to those entries.
+ *
+ * For every (layer l, sequence b, KV head h):
+ *   score[n] = 1/(G*T) * sum over the G query heads g of the group and the
+ *              T text rows t of softmax_{n < nvis[b]}( q_text[g,t] . k_n / sqrt(d) )
+ *   idx      = the K highest scores, ties to the lower position, ascending
+ *   sparse cache rows [0, K)     = full rows idx[0..K)   (K and V)
+ *   sparse cache rows [K, K + T) = full rows [nvis[b], nvis[b] + T) (the text)
+ *   len_sparse[b] = K + T
+ * The softmax runs over the visual keys only.
+ */
+
+/* Device workspace bytes std_select_topk needs for these shapes. */
+size_t std_select_workspace_size(const std_dims* dims, int T, int nvis_max);
+
+/*
+ * q_text      [L][B][Hq][T][d]          text-token queries (post-RoPE)
+ * k_full/v_full [L][B][Hkv][cap_full][d] prompt cache: visual rows [0, nvis[b]),
+ *                                        text rows [nvis[b], nvis[b] + T)
+ * nvis        device int32 [B]           visual tokens per sequence
+ * nvis_max    host bound >= every nvis[b]; sizes the launch and the workspace
+ * K           1 <= K <= nvis[b] (checked on the device), K <= nvis_max and
+ *             K + T <= cap_sparse (checked on the host)
+ * idx_out     device int32 [L][B][Hkv][K]  selected visual positions, ascending
+ * k_sparse/v_sparse [L][B][Hkv][cap_sparse][d]  rows [0, K + T) written
+ * len_sparse  device int32 [B]           set to K + T
+ * scores_out  device float [L][B][Hkv][nvis_max] or NULL; entries n >= nvis[b]
+ *             are not written
+ * ws          device workspace of at least std_select_workspace_size() bytes
+ */
+int std_select_topk(const std_dims* dims, const void* q_text, int T, const void* k_full,
+                    const void* v_full, const int32_t* nvis, int nvis_max, int K,
+                    int32_t* idx_out, void* k_sparse, void* v_sparse, int32_t* len_sparse,
+                    float* scores_out, void* ws, size_t ws_bytes, std_stream_t stream);
+
+/* The selection's top-K step alone, on caller-supplied float32 scores:
+ * `rows` independent rows of `n` scores each (row stride n), K <= n.
+ * idx_out [rows][K] receives the K highest positions of each row, ties to the
+ * lower position, ascending.  -0.0 ranks equal to +0.0; NaN is not allowed. */
+int std_topk_from_scores(const float* scores, int rows, int n, int K, int32_t* idx_out,
+                         std_stream_t stream);
+
+/* ---------------------------------------------------------------- decode attention
+ *
+ * Split-K flash decoding: the key range of each (layer, sequence, KV head) is
+ * cut into `splits` pieces processed by separate CTAs; the G query heads of a
+ * KV head (times the query rows) share one tile so each K/V byte is read once.
+ * splits = 0 picks a split count from the device's SM count.  Partial results
+ * go to the workspace and are merged by a second kernel.
+ */
+
+/* Device workspace bytes for a decode-attention call with `q_rows` query rows
+ * per query head (1 for the sparse draft, gamma + 1 for the verify) over a
+ * cache of `cap` rows (dims->cap_sparse for the draft, dims->cap_full for the
+ * verify), and `splits` (0 = the automatic choice, which depends on the number
+ * of (layer, sequence, KV head) problems, `cap` and the current device's SM
+ * count).  Returns 0 when no workspace is needed or the arguments are invalid. */
+size_t std_attn_workspace_size(const std_dims* dims, int q_rows, int64_t cap, int splits);
+
+/* The split count a decode-attention call over a cache of `cap` rows will use
+ * for `splits` (0 = automatic; resolved on the current device), or a negative
+ * STD_ERR_* code.  With more than one split the call launches a second
+ * (merge) kernel. */
+int std_attn_splits(const std_dims* dims, int64_t cap, int splits);
+
+/*
+ * Sparse draft attention ("Methodik" item 2: the draft model M_s uses top-K
+ * attention over the selected KV).  For every query head:
+ *     o = softmax_j(q . k_j / sqrt(d)) v_j   over sparse rows j < len_sparse[b] + len_offset
+ * q          [L][B][Hq][1][d]
+ * k_sparse/v_sparse [L][B][Hkv][cap_sparse][d]
+ * len_sparse device int32 [B]: committed sparse rows; len_offset (>= 0) counts
+ *            rows appended since (std_kv_append with the same offset base)
+ * o          float [L][B][Hq][1][d]
+ */
+int std_sparse_decode_attn(const std_dims* dims, const void* q, const void* k_sparse,
+                           const void* v_sparse, const int32_t* len_sparse, int len_offset,
+                           float* o, int splits, void* ws, size_t ws_bytes, std_stream_t stream);
+
+/*
+ * Dense verify attention ("Methodik" item 3: the dense model verifies the gamma
+ * drafted tokens in parallel with one pass over the full KV cache).  Query row
+ * i = 0..gamma of each query head attends causally:
+ *     o_i = softmax_j(q_i . k_j / sqrt(d)) v_j   over full rows j < len_full[b] + i + 1
+ * q         [L][B][Hq][gamma + 1][d]
+ * k_full/v_full [L][B][Hkv][cap_full][d]; the gamma + 1 new rows must already sit at
+ *           [len_full[b], len_full[b] + gamma + 1) (std_kv_append)
+ * len_full  device int32 [B]: committed context length, before the new rows
+ * o         float [L][B][Hq][gamma + 1][d]
+ * Requires 0 <= gamma <= 31 and G * (gamma + 1) <= 128.
+ */
+int std_dense_verify_attn(const std_dims* dims, const void* q, int gamma, const void* k_full,
+                          const void* v_full, const int32_t* len_full, float* o, int splits,
+                          void* ws, size_t ws_bytes, std_stream_t stream);
+
+/* ---------------------------------------------------------------- acceptance
+ *
+ * "Methodik" item 3: keep the longest prefix of draft tokens that matches the
+ * dense model's predictions (n tokens) plus one bonus token.
+ * draft        device int32 [B][gamma]      drafted tokens d_0..d_{gamma-1}
+ * dense_argmax device int32 [B][gamma + 1]  dense prediction after each input
+ * n_plus_1     device int32 [B]             n + 1, in [1, gamma + 1]
+ * accepted     device int32 [B][gamma + 1]  dense_argmax[b][0..n], then -1
+ * The bonus token is dense_argmax[b][n].  Requires 0 <= gamma <= 31.
+ */
+int std_accept_prefix(int B, int gamma, const int32_t* draft, const int32_t* dense_argmax,
+                      int32_t* n_plus_1, int32_t* accepted, std_stream_t stream);
+
+/* ---------------------------------------------------------------- cache bookkeeping */
+
+/* Write `n_new` rows per (layer, sequence, KV head) into a cache at positions
+ * len[b] + pos_offset + r, r < n_new.  k_new/v_new [L][B][Hkv][n_new][d];
+ * cache [L][B][Hkv][cap][d].  Lengths are not changed.  A sequence whose rows
+ * would pass `cap` is skipped and flags STD_DEVERR_CAPACITY. */
+int std_kv_append(const std_dims* dims, void* k_cache, void* v_cache, int64_t cap,
+                  const int32_t* len, int pos_offset, const void* k_new, const void* v_new,
+                  int n_new, std_stream_t stream);
+
+/* "Methodik" item 3, last step: append the accepted inputs to the context.
+ * For every sequence, the n_plus_1[b] verified rows at full positions
+ * [len_full[b], len_full[b] + n_plus_1[b]) are copied (K and V) to sparse
+ * positions [len_sparse[b], ...), then both lengths grow by n_plus_1[b].
+ * max_n bounds every n_plus_1[b] (gamma + 1) and sizes the launch. */
+int std_kv_commit(const std_dims* dims, void* k_full, void* v_full, void* k_sparse,
+                  void* v_sparse, int32_t* len_full, int32_t* len_sparse,
+                  const int32_t* n_plus_1, int max_n, std_stream_t stream);
+
+/* ---------------------------------------------------------------- one decode round */
+
+typedef struct std_cache {
+  void* k_full;         /* [L][B][Hkv][cap_full][d] */
+  void* v_full;
+  void* k_sparse;       /* [L][B][Hkv][cap_sparse][d] */
+  void* v_sparse;
+  int32_t* len_full;    /* device [B], committed context length */
+  int32_t* len_sparse;  /* device [B], committed sparse length */
+} std_cache;
+
+typedef struct std_round_io {
+  const void* q_draft;          /* [gamma][L][B][Hq][1][d]   query of draft step j */
+  const void* k_draft;          /* [gamma][L][B][Hkv][1][d]  K/V row of draft step j's input */
+  const void* v_draft;
+  const void* q_verify;         /* [L][B][Hq][gamma + 1][d] */
+  const void* k_verify;         /* [L][B][Hkv][gamma + 1][d] K/V rows of the gamma + 1 inputs */
+  const void* v_verify;
+  const int32_t* draft_tokens;  /* [B][gamma] */
+  const int32_t* dense_tokens;  /* [B][gamma + 1] */
+  float* o_draft;               /* [gamma][L][B][Hq][1][d] */
+  float* o_verify;              /* [L][B][Hq][gamma + 1][d] */
+  int32_t* n_plus_1;            /* [B] */
+  int32_t* accepted;            /* [B][gamma + 1] */
+} std_round_io;
+
+/* Workspace bytes for std_decode_round (the larger of its attention calls). */
+size_t std_round_workspace_size(const std_dims* dims, int gamma, int splits_draft,
+                                int splits_verify);
+
+/*
+ * One draft + verify round ("Methodik" item 3), all on `stream`:
+ *   for j < gamma: append draft row j to the sparse cache at len_sparse + j,
+ *                  sparse attention over len_sparse + j + 1 rows;
+ *   append the gamma + 1 verify rows to the full cache at len_full;
+ *   dense verify attention; acceptance; commit (lengths advance by n + 1).
+ * The token ids of the LM head are inputs here (the language-model layers
+ * around attention are not part of this library).
+ */
+int std_decode_round(const std_dims* dims, int gamma, const std_cache* cache,
+                     const std_round_io* io, int splits_draft, int splits_verify, void* ws,
+                     size_t ws_bytes, std_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STD_B200_H */

@@ -1,0 +1,230 @@
+"""ctypes binding of ``libstd_b200.so`` -- the C ABI declared in include/std_b200.h.
+
+Argument marshalling only: every function here has the name of a C entry
+point, turns torch tensors into device pointers and the current torch stream
+into a ``cudaStream_t``, calls the library and raises ``StdError`` on a
+non-zero status.  No step of the method runs in Python, and nothing falls
+back to another implementation: if the library is missing, the first call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libstd_b200.so")
+
+STD_OK = 0
+STD_ERR_INVALID_ARG = -1
+STD_ERR_UNSUPPORTED = -2
+STD_ERR_CAPACITY = -3
+STD_ERR_CUDA = -4
+STD_ERR_DEVICE = -5
+STD_ERR_TIMEOUT = -6
+STD_ERR_WORKSPACE = -7
+
+STD_F32 = 0
+STD_BF16 = 1
+
+STD_DEVERR_CAPACITY = 1
+STD_DEVERR_LENGTH = 2
+STD_DEVERR_K_RANGE = 4
+STD_DEVERR_NVIS_MAX = 8
+
+# every function the header declares, with (restype, argtypes)
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+
+
+class StdDims(ctypes.Structure):
+    _fields_ = [("L", ctypes.c_int32), ("B", ctypes.c_int32), ("Hq", ctypes.c_int32),
+                ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("cap_full", ctypes.c_int64), ("cap_sparse", ctypes.c_int64)]
+
+
+class StdCache(ctypes.Structure):
+    _fields_ = [("k_full", _P), ("v_full", _P), ("k_sparse", _P), ("v_sparse", _P),
+                ("len_full", _P), ("len_sparse", _P)]
+
+
+class StdRoundIO(ctypes.Structure):
+    _fields_ = [("q_draft", _P), ("k_draft", _P), ("v_draft", _P), ("q_verify", _P),
+                ("k_verify", _P), ("v_verify", _P), ("draft_tokens", _P), ("dense_tokens", _P),
+                ("o_draft", _P), ("o_verify", _P), ("n_plus_1", _P), ("accepted", _P)]
+
+
+_DP = ctypes.POINTER(StdDims)
+SIGNATURES = {
+    "std_version": (_I, []),
+    "std_last_error": (ctypes.c_char_p, []),
+    "std_get_device_error": (_I, [ctypes.POINTER(ctypes.c_int32), _I, _P]),
+    "std_select_workspace_size": (_SZ, [_DP, _I, _I]),
+    "std_select_topk": (_I, [_DP, _P, _I, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "std_topk_from_scores": (_I, [_P, _I, _I, _I, _P, _P]),
+    "std_attn_workspace_size": (_SZ, [_DP, _I, _I64, _I]),
+    "std_attn_splits": (_I, [_DP, _I64, _I]),
+    "std_sparse_decode_attn": (_I, [_DP, _P, _P, _P, _P, _I, _P, _I, _P, _SZ, _P]),
+    "std_dense_verify_attn": (_I, [_DP, _P, _I, _P, _P, _P, _P, _I, _P, _SZ, _P]),
+    "std_accept_prefix": (_I, [_I, _I, _P, _P, _P, _P, _P]),
+    "std_kv_append": (_I, [_DP, _P, _P, _I64, _P, _I, _P, _P, _I, _P]),
+    "std_kv_commit": (_I, [_DP, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
+    "std_round_workspace_size": (_SZ, [_DP, _I, _I, _I]),
+    "std_decode_round": (_I, [_DP, _I, ctypes.POINTER(StdCache), ctypes.POINTER(StdRoundIO), _I, _I,
+                              _P, _SZ, _P]),
+}
+
+
+class StdError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"std_b200 error {code}: {msg}")
+        self.code = code
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                       "`python -m sparse_top_kv_std_b200.build`")
+                h = ctypes.CDLL(LIB_PATH)
+                for name, (res, args) in SIGNATURES.items():
+                    f = getattr(h, name)
+                    f.restype = res
+                    f.argtypes = args
+                _lib = h
+    return _lib
+
+
+# ----------------------------------------------------------------------------- marshalling
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if not x.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not x.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return x.data_ptr()
+
+
+def _nbytes(x) -> int:
+    return 0 if x is None else x.numel() * x.element_size()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int) -> None:
+    if rc != STD_OK:
+        raise StdError(rc, lib().std_last_error().decode())
+
+
+def dims(L, B, Hq, Hkv, d, dtype, cap_full, cap_sparse) -> StdDims:
+    return StdDims(int(L), int(B), int(Hq), int(Hkv), int(d), int(dtype), int(cap_full), int(cap_sparse))
+
+
+# ----------------------------------------------------------------------------- entry points
+
+def std_version() -> int:
+    return lib().std_version()
+
+
+def std_last_error() -> str:
+    return lib().std_last_error().decode()
+
+
+def std_get_device_error(clear: bool = True, stream=None) -> int:
+    flags = ctypes.c_int32(0)
+    rc = lib().std_get_device_error(ctypes.byref(flags), int(clear), _stream(stream))
+    if rc not in (STD_OK, STD_ERR_DEVICE):
+        _check(rc)
+    return flags.value
+
+
+def std_select_workspace_size(d: StdDims, T: int, nvis_max: int) -> int:
+    return lib().std_select_workspace_size(ctypes.byref(d), T, nvis_max)
+
+
+def std_select_topk(d: StdDims, q_text, T, k_full, v_full, nvis, nvis_max, K, idx_out, k_sparse,
+                    v_sparse, len_sparse, scores_out, ws, stream=None) -> None:
+    _check(lib().std_select_topk(ctypes.byref(d), _ptr(q_text), T, _ptr(k_full), _ptr(v_full), _ptr(nvis),
+                                 nvis_max, K, _ptr(idx_out), _ptr(k_sparse), _ptr(v_sparse), _ptr(len_sparse),
+                                 _ptr(scores_out), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def std_topk_from_scores(scores, rows, n, K, idx_out, stream=None) -> None:
+    _check(lib().std_topk_from_scores(_ptr(scores), rows, n, K, _ptr(idx_out), _stream(stream)))
+
+
+def std_attn_workspace_size(d: StdDims, q_rows: int, cap: int, splits: int) -> int:
+    return lib().std_attn_workspace_size(ctypes.byref(d), q_rows, cap, splits)
+
+
+def std_attn_splits(d: StdDims, cap: int, splits: int = 0) -> int:
+    rc = lib().std_attn_splits(ctypes.byref(d), cap, splits)
+    if rc < 0:
+        _check(rc)
+    return rc
+
+
+def std_sparse_decode_attn(d: StdDims, q, k_sparse, v_sparse, len_sparse, len_offset, o, splits=0,
+                           ws=None, stream=None) -> None:
+    _check(lib().std_sparse_decode_attn(ctypes.byref(d), _ptr(q), _ptr(k_sparse), _ptr(v_sparse),
+                                        _ptr(len_sparse), len_offset, _ptr(o), splits, _ptr(ws), _nbytes(ws),
+                                        _stream(stream)))
+
+
+def std_dense_verify_attn(d: StdDims, q, gamma, k_full, v_full, len_full, o, splits=0, ws=None,
+                          stream=None) -> None:
+    _check(lib().std_dense_verify_attn(ctypes.byref(d), _ptr(q), gamma, _ptr(k_full), _ptr(v_full),
+                                       _ptr(len_full), _ptr(o), splits, _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def std_accept_prefix(B, gamma, draft, dense_argmax, n_plus_1, accepted, stream=None) -> None:
+    _check(lib().std_accept_prefix(B, gamma, _ptr(draft), _ptr(dense_argmax), _ptr(n_plus_1), _ptr(accepted),
+                                   _stream(stream)))
+
+
+def std_kv_append(d: StdDims, k_cache, v_cache, cap, length, pos_offset, k_new, v_new, n_new,
+                  stream=None) -> None:
+    _check(lib().std_kv_append(ctypes.byref(d), _ptr(k_cache), _ptr(v_cache), cap, _ptr(length), pos_offset,
+                               _ptr(k_new), _ptr(v_new), n_new, _stream(stream)))
+
+
+def std_kv_commit(d: StdDims, k_full, v_full, k_sparse, v_sparse, len_full, len_sparse, n_plus_1, max_n,
+                  stream=None) -> None:
+    _check(lib().std_kv_commit(ctypes.byref(d), _ptr(k_full), _ptr(v_full), _ptr(k_sparse), _ptr(v_sparse),
+                               _ptr(len_full), _ptr(len_sparse), _ptr(n_plus_1), max_n, _stream(stream)))
+
+
+def std_round_workspace_size(d: StdDims, gamma: int, splits_draft: int = 0, splits_verify: int = 0) -> int:
+    return lib().std_round_workspace_size(ctypes.byref(d), gamma, splits_draft, splits_verify)
+
+
+def std_decode_round(d: StdDims, gamma, cache: dict, io: dict, splits_draft=0, splits_verify=0, ws=None,
+                     stream=None) -> None:
+    """cache / io: dicts of tensors keyed by the std_cache / std_round_io field names."""
+    c = StdCache(*[_ptr(cache[f]) for f, _ in StdCache._fields_])
+    r = StdRoundIO(*[_ptr(io[f]) for f, _ in StdRoundIO._fields_])
+    _check(lib().std_decode_round(ctypes.byref(d), gamma, ctypes.byref(c), ctypes.byref(r), splits_draft,
+                                  splits_verify, _ptr(ws), _nbytes(ws), _stream(stream)))

@@ -1,0 +1,384 @@
+// C ABI of the Sparse-to-Dense decoding library: argument checks, workspace
+// sizing, launch configuration.  Declarations and the contract of every entry
+// point are in include/std_b200.h.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "../../include/std_b200.h"
+#include "internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int ok() {
+  g_last_error.clear();
+  return STD_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(STD_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------- per-device state
+__device__ int g_device_error;  // OR of STD_DEVERR_* bits, one word per device
+
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mu;
+int* g_err_ptr[kMaxDevices] = {};
+int g_sm_count[kMaxDevices] = {};
+
+int current_device(int* dev) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (*dev < 0 || *dev >= kMaxDevices) return fail(STD_ERR_UNSUPPORTED, "device ordinal %d", *dev);
+  return STD_OK;
+}
+
+int device_state(int** err_ptr, int* sm_count) {
+  int dev;
+  int rc = current_device(&dev);
+  if (rc) return rc;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_device_error);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(device error word)");
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+    g_err_ptr[dev] = static_cast<int*>(p);
+    g_sm_count[dev] = sms;
+  }
+  if (err_ptr) *err_ptr = g_err_ptr[dev];
+  if (sm_count) *sm_count = g_sm_count[dev];
+  return STD_OK;
+}
+
+// ---------------------------------------------------------------- checks
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int elem_bytes(int dtype) { return dtype == STD_F32 ? 4 : 2; }
+
+int check_dims(const std_dims* d) {
+  if (!d) return fail(STD_ERR_INVALID_ARG, "dims is NULL");
+  if (d->L < 1 || d->B < 1 || d->Hq < 1 || d->Hkv < 1)
+    return fail(STD_ERR_INVALID_ARG, "L, B, Hq, Hkv must be >= 1 (got %d, %d, %d, %d)", d->L, d->B, d->Hq, d->Hkv);
+  if (d->Hq % d->Hkv) return fail(STD_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", d->Hq, d->Hkv);
+  if (d->dtype == STD_BF16) {
+    if (d->d != 64 && d->d != 128) return fail(STD_ERR_UNSUPPORTED, "bf16 head dim %d (supported: 64, 128)", d->d);
+  } else if (d->dtype == STD_F32) {
+    if (d->d != 32 && d->d != 64 && d->d != 96 && d->d != 128)
+      return fail(STD_ERR_UNSUPPORTED, "fp32 head dim %d (supported: 32, 64, 96, 128)", d->d);
+  } else {
+    return fail(STD_ERR_UNSUPPORTED, "dtype %d", d->dtype);
+  }
+  if (d->cap_full < 1 || d->cap_sparse < 1) return fail(STD_ERR_INVALID_ARG, "capacities must be >= 1");
+  if (d->cap_full > INT32_MAX || d->cap_sparse > INT32_MAX) return fail(STD_ERR_INVALID_ARG, "capacity above 2^31-1");
+  return STD_OK;
+}
+
+int check_ptr(const void* p, size_t align, const char* name) {
+  if (!p) return fail(STD_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned(p, align)) return fail(STD_ERR_INVALID_ARG, "%s is not %zu-byte aligned", name, align);
+  return STD_OK;
+}
+
+#define STD_TRY(x)            \
+  do {                        \
+    int rc_ = (x);            \
+    if (rc_ != STD_OK) return rc_; \
+  } while (0)
+
+int probs_of(const std_dims* d) { return d->L * d->B * d->Hkv; }
+
+int auto_splits(int probs, int64_t cap, int sm_count) {
+  // about 8 CTAs per SM over the whole grid, at least 256 keys per split
+  int s = (sm_count * 8 + probs - 1) / probs;
+  const int64_t by_len = cap / 256;
+  if (s > by_len) s = (int)by_len;
+  if (s < 1) s = 1;
+  if (s > 256) s = 256;
+  return s;
+}
+
+int resolve_splits(int splits, int probs, int64_t cap, int* out) {
+  if (splits < 0 || splits > 1024) return fail(STD_ERR_INVALID_ARG, "splits %d out of range [0, 1024]", splits);
+  if (splits > 0) {
+    *out = splits;
+    return STD_OK;
+  }
+  int sms;
+  STD_TRY(device_state(nullptr, &sms));
+  *out = auto_splits(probs, cap, sms);
+  return STD_OK;
+}
+
+size_t attn_ws_bytes(const std_dims* d, int q_rows, int splits) {
+  return stdb::attn_ws_floats(probs_of(d), splits, (d->Hq / d->Hkv) * q_rows, d->d, d->dtype) * sizeof(float);
+}
+
+int run_attn(const std_dims* dims, const void* q, const void* k, const void* v, int64_t cap,
+             const int32_t* len, int len_off, int nq, float* o, int splits, void* ws, size_t ws_bytes,
+             cudaStream_t stream) {
+  const int G = dims->Hq / dims->Hkv;
+  const int rows = G * nq;
+  if (dims->dtype == STD_BF16 && rows > 128)
+    return fail(STD_ERR_UNSUPPORTED, "G * query rows = %d exceeds 128", rows);
+  int sp;
+  STD_TRY(resolve_splits(splits, probs_of(dims), cap, &sp));
+  const size_t need = attn_ws_bytes(dims, nq, sp);
+  if (need > 0 && (!ws || ws_bytes < need))
+    return fail(STD_ERR_WORKSPACE, "attention workspace: need %zu bytes, got %zu", need, ws ? ws_bytes : 0);
+  if (need > 0) STD_TRY(check_ptr(ws, 16, "ws"));
+  int* err;
+  STD_TRY(device_state(&err, nullptr));
+  stdb::AttnArgs a{};
+  a.q = q; a.k = k; a.v = v; a.o = o; a.len = len; a.len_off = len_off;
+  a.L = dims->L; a.B = dims->B; a.Hq = dims->Hq; a.Hkv = dims->Hkv; a.G = G; a.nq = nq; a.rows = rows;
+  a.d = dims->d; a.dtype = dims->dtype; a.cap = cap; a.splits = sp;
+  a.ws = static_cast<float*>(ws); a.err = err;
+  cudaError_t e = stdb::launch_decode_attn(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+int std_version(void) { return 10000; }
+
+const char* std_last_error(void) { return g_last_error.c_str(); }
+
+int std_get_device_error(int32_t* flags, int clear, std_stream_t stream) {
+  int* err;
+  STD_TRY(device_state(&err, nullptr));
+  int32_t host = 0;
+  cudaError_t e = cudaMemcpyAsync(&host, err, sizeof(int32_t), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess && clear) e = cudaMemsetAsync(err, 0, sizeof(int32_t), stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (flags) *flags = host;
+  if (host) return fail(STD_ERR_DEVICE, "device error flags 0x%x", host);
+  return ok();
+}
+
+size_t std_select_workspace_size(const std_dims* dims, int T, int nvis_max) {
+  if (check_dims(dims) || T < 1 || nvis_max < 1) return 0;
+  const size_t probs = probs_of(dims);
+  const size_t M = (size_t)(dims->Hq / dims->Hkv) * T;
+  return (probs * M * 2 + probs * (size_t)nvis_max) * sizeof(float) + 256;
+}
+
+int std_select_topk(const std_dims* dims, const void* q_text, int T, const void* k_full,
+                    const void* v_full, const int32_t* nvis, int nvis_max, int K, int32_t* idx_out,
+                    void* k_sparse, void* v_sparse, int32_t* len_sparse, float* scores_out, void* ws,
+                    size_t ws_bytes, std_stream_t stream) {
+  STD_TRY(check_dims(dims));
+  STD_TRY(check_ptr(q_text, 16, "q_text"));
+  STD_TRY(check_ptr(k_full, 16, "k_full"));
+  STD_TRY(check_ptr(v_full, 16, "v_full"));
+  STD_TRY(check_ptr(nvis, 4, "nvis"));
+  STD_TRY(check_ptr(idx_out, 4, "idx_out"));
+  STD_TRY(check_ptr(k_sparse, 16, "k_sparse"));
+  STD_TRY(check_ptr(v_sparse, 16, "v_sparse"));
+  STD_TRY(check_ptr(len_sparse, 4, "len_sparse"));
+  if (scores_out) STD_TRY(check_ptr(scores_out, 4, "scores_out"));
+  if (T < 1) return fail(STD_ERR_INVALID_ARG, "T = %d must be >= 1", T);
+  if (nvis_max < 1) return fail(STD_ERR_INVALID_ARG, "nvis_max = %d must be >= 1", nvis_max);
+  if (K < 1 || K > nvis_max) return fail(STD_ERR_INVALID_ARG, "K = %d must be in [1, nvis_max = %d]", K, nvis_max);
+  if ((int64_t)K + T > dims->cap_sparse)
+    return fail(STD_ERR_CAPACITY, "K + T = %d exceeds cap_sparse = %lld", K + T, (long long)dims->cap_sparse);
+  if ((int64_t)nvis_max + T > dims->cap_full)
+    return fail(STD_ERR_CAPACITY, "nvis_max + T = %d exceeds cap_full = %lld", nvis_max + T, (long long)dims->cap_full);
+  const size_t need = std_select_workspace_size(dims, T, nvis_max);
+  if (!ws || ws_bytes < need) return fail(STD_ERR_WORKSPACE, "select workspace: need %zu bytes, got %zu", need, ws ? ws_bytes : 0);
+  STD_TRY(check_ptr(ws, 16, "ws"));
+  int* err;
+  STD_TRY(device_state(&err, nullptr));
+
+  const int probs = probs_of(dims);
+  const int G = dims->Hq / dims->Hkv;
+  const size_t M = (size_t)G * T;
+  float* row_m = static_cast<float*>(ws);
+  float* row_l = row_m + probs * M;
+  float* scores = scores_out ? scores_out : row_l + probs * M;
+
+  stdb::ScoreArgs s{};
+  s.q_text = q_text; s.k_full = k_full; s.nvis = nvis; s.nvis_max = nvis_max;
+  s.L = dims->L; s.B = dims->B; s.Hq = dims->Hq; s.Hkv = dims->Hkv; s.G = G; s.T = T; s.d = dims->d;
+  s.dtype = dims->dtype; s.cap = dims->cap_full; s.row_m = row_m; s.row_l = row_l; s.scores = scores; s.err = err;
+  cudaError_t e = stdb::launch_select_scores(s, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "selection score launch");
+  e = stdb::launch_topk(scores, nvis_max, probs, nvis, 0, dims->Hkv, dims->B, K, idx_out, err, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "top-K launch");
+  stdb::GatherArgs g{};
+  g.k_full = k_full; g.v_full = v_full; g.k_sp = k_sparse; g.v_sp = v_sparse; g.idx = idx_out; g.nvis = nvis;
+  g.len_sparse = len_sparse; g.L = dims->L; g.B = dims->B; g.Hkv = dims->Hkv; g.T = T; g.K = K;
+  g.row_bytes = dims->d * elem_bytes(dims->dtype); g.cap_full = dims->cap_full; g.cap_sparse = dims->cap_sparse;
+  g.err = err;
+  e = stdb::launch_gather(g, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+  return ok();
+}
+
+int std_topk_from_scores(const float* scores, int rows, int n, int K, int32_t* idx_out, std_stream_t stream) {
+  STD_TRY(check_ptr(scores, 4, "scores"));
+  STD_TRY(check_ptr(idx_out, 4, "idx_out"));
+  if (rows < 0 || n < 1) return fail(STD_ERR_INVALID_ARG, "rows = %d, n = %d", rows, n);
+  if (K < 1 || K > n) return fail(STD_ERR_INVALID_ARG, "K = %d must be in [1, n = %d]", K, n);
+  int* err;
+  STD_TRY(device_state(&err, nullptr));
+  cudaError_t e = stdb::launch_topk(scores, n, rows, nullptr, n, 1, 1, K, idx_out, err, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "top-K launch");
+  return ok();
+}
+
+size_t std_attn_workspace_size(const std_dims* dims, int q_rows, int64_t cap, int splits) {
+  if (check_dims(dims) || q_rows < 1 || cap < 1) return 0;
+  int sp;
+  if (resolve_splits(splits, probs_of(dims), cap, &sp)) return 0;
+  return attn_ws_bytes(dims, q_rows, sp);
+}
+
+int std_attn_splits(const std_dims* dims, int64_t cap, int splits) {
+  STD_TRY(check_dims(dims));
+  if (cap < 1) return fail(STD_ERR_INVALID_ARG, "cap = %lld", (long long)cap);
+  int sp;
+  STD_TRY(resolve_splits(splits, probs_of(dims), cap, &sp));
+  ok();
+  return sp;
+}
+
+int std_sparse_decode_attn(const std_dims* dims, const void* q, const void* k_sparse, const void* v_sparse,
+                           const int32_t* len_sparse, int len_offset, float* o, int splits, void* ws,
+                           size_t ws_bytes, std_stream_t stream) {
+  STD_TRY(check_dims(dims));
+  STD_TRY(check_ptr(q, 16, "q"));
+  STD_TRY(check_ptr(k_sparse, 16, "k_sparse"));
+  STD_TRY(check_ptr(v_sparse, 16, "v_sparse"));
+  STD_TRY(check_ptr(len_sparse, 4, "len_sparse"));
+  STD_TRY(check_ptr(o, 16, "o"));
+  if (len_offset < 0) return fail(STD_ERR_INVALID_ARG, "len_offset = %d must be >= 0", len_offset);
+  return run_attn(dims, q, k_sparse, v_sparse, dims->cap_sparse, len_sparse, len_offset, 1, o, splits, ws,
+                  ws_bytes, stream);
+}
+
+int std_dense_verify_attn(const std_dims* dims, const void* q, int gamma, const void* k_full, const void* v_full,
+                          const int32_t* len_full, float* o, int splits, void* ws, size_t ws_bytes,
+                          std_stream_t stream) {
+  STD_TRY(check_dims(dims));
+  STD_TRY(check_ptr(q, 16, "q"));
+  STD_TRY(check_ptr(k_full, 16, "k_full"));
+  STD_TRY(check_ptr(v_full, 16, "v_full"));
+  STD_TRY(check_ptr(len_full, 4, "len_full"));
+  STD_TRY(check_ptr(o, 16, "o"));
+  if (gamma < 0 || gamma > 31) return fail(STD_ERR_INVALID_ARG, "gamma = %d must be in [0, 31]", gamma);
+  // row i sees keys j < len_full + 1 + i
+  return run_attn(dims, q, k_full, v_full, dims->cap_full, len_full, 1, gamma + 1, o, splits, ws, ws_bytes,
+                  stream);
+}
+
+int std_accept_prefix(int B, int gamma, const int32_t* draft, const int32_t* dense_argmax, int32_t* n_plus_1,
+                      int32_t* accepted, std_stream_t stream) {
+  if (B < 1) return fail(STD_ERR_INVALID_ARG, "B = %d must be >= 1", B);
+  if (gamma < 0 || gamma > 31) return fail(STD_ERR_INVALID_ARG, "gamma = %d must be in [0, 31]", gamma);
+  if (gamma > 0) STD_TRY(check_ptr(draft, 4, "draft"));
+  STD_TRY(check_ptr(dense_argmax, 4, "dense_argmax"));
+  STD_TRY(check_ptr(n_plus_1, 4, "n_plus_1"));
+  STD_TRY(check_ptr(accepted, 4, "accepted"));
+  cudaError_t e = stdb::launch_accept(B, gamma, draft, dense_argmax, n_plus_1, accepted, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "accept launch");
+  return ok();
+}
+
+int std_kv_append(const std_dims* dims, void* k_cache, void* v_cache, int64_t cap, const int32_t* len,
+                  int pos_offset, const void* k_new, const void* v_new, int n_new, std_stream_t stream) {
+  STD_TRY(check_dims(dims));
+  STD_TRY(check_ptr(k_cache, 16, "k_cache"));
+  STD_TRY(check_ptr(v_cache, 16, "v_cache"));
+  STD_TRY(check_ptr(len, 4, "len"));
+  STD_TRY(check_ptr(k_new, 16, "k_new"));
+  STD_TRY(check_ptr(v_new, 16, "v_new"));
+  if (cap < 1 || cap > INT32_MAX) return fail(STD_ERR_INVALID_ARG, "cap = %lld", (long long)cap);
+  if (n_new < 0 || pos_offset < 0) return fail(STD_ERR_INVALID_ARG, "n_new = %d, pos_offset = %d", n_new, pos_offset);
+  if ((int64_t)n_new + pos_offset > cap) return fail(STD_ERR_CAPACITY, "offset + rows exceed cap");
+  int* err;
+  STD_TRY(device_state(&err, nullptr));
+  cudaError_t e = stdb::launch_append(k_cache, v_cache, cap, len, pos_offset, k_new, v_new, n_new, dims->L,
+                                      dims->B, dims->Hkv, dims->d * elem_bytes(dims->dtype), err, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  return ok();
+}
+
+int std_kv_commit(const std_dims* dims, void* k_full, void* v_full, void* k_sparse, void* v_sparse,
+                  int32_t* len_full, int32_t* len_sparse, const int32_t* n_plus_1, int max_n,
+                  std_stream_t stream) {
+  STD_TRY(check_dims(dims));
+  STD_TRY(check_ptr(k_full, 16, "k_full"));
+  STD_TRY(check_ptr(v_full, 16, "v_full"));
+  STD_TRY(check_ptr(k_sparse, 16, "k_sparse"));
+  STD_TRY(check_ptr(v_sparse, 16, "v_sparse"));
+  STD_TRY(check_ptr(len_full, 4, "len_full"));
+  STD_TRY(check_ptr(len_sparse, 4, "len_sparse"));
+  STD_TRY(check_ptr(n_plus_1, 4, "n_plus_1"));
+  if (max_n < 1 || max_n > 32) return fail(STD_ERR_INVALID_ARG, "max_n = %d must be in [1, 32]", max_n);
+  int* err;
+  STD_TRY(device_state(&err, nullptr));
+  cudaError_t e = stdb::launch_commit(k_full, v_full, k_sparse, v_sparse, len_full, len_sparse, n_plus_1, max_n,
+                                      dims->L, dims->B, dims->Hkv, dims->d * elem_bytes(dims->dtype),
+                                      dims->cap_full, dims->cap_sparse, err, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "commit launch");
+  return ok();
+}
+
+size_t std_round_workspace_size(const std_dims* dims, int gamma, int splits_draft, int splits_verify) {
+  if (check_dims(dims) || gamma < 0 || gamma > 31) return 0;
+  const size_t a = gamma > 0 ? std_attn_workspace_size(dims, 1, dims->cap_sparse, splits_draft) : 0;
+  const size_t b = std_attn_workspace_size(dims, gamma + 1, dims->cap_full, splits_verify);
+  return a > b ? a : b;
+}
+
+int std_decode_round(const std_dims* dims, int gamma, const std_cache* c, const std_round_io* io,
+                     int splits_draft, int splits_verify, void* ws, size_t ws_bytes, std_stream_t stream) {
+  STD_TRY(check_dims(dims));
+  if (!c || !io) return fail(STD_ERR_INVALID_ARG, "cache or io is NULL");
+  if (gamma < 0 || gamma > 31) return fail(STD_ERR_INVALID_ARG, "gamma = %d must be in [0, 31]", gamma);
+  const size_t eb = elem_bytes(dims->dtype);
+  const size_t q_step = (size_t)dims->L * dims->B * dims->Hq * dims->d;   // elements per draft query step
+  const size_t kv_step = (size_t)dims->L * dims->B * dims->Hkv * dims->d;  // elements per draft K/V step
+  for (int j = 0; j < gamma; ++j) {
+    STD_TRY(std_kv_append(dims, c->k_sparse, c->v_sparse, dims->cap_sparse, c->len_sparse, j,
+                          static_cast<const uint8_t*>(io->k_draft) + j * kv_step * eb,
+                          static_cast<const uint8_t*>(io->v_draft) + j * kv_step * eb, 1, stream));
+    STD_TRY(std_sparse_decode_attn(dims, static_cast<const uint8_t*>(io->q_draft) + j * q_step * eb, c->k_sparse,
+                                   c->v_sparse, c->len_sparse, j + 1, io->o_draft + j * q_step, splits_draft, ws,
+                                   ws_bytes, stream));
+  }
+  STD_TRY(std_kv_append(dims, c->k_full, c->v_full, dims->cap_full, c->len_full, 0, io->k_verify, io->v_verify,
+                        gamma + 1, stream));
+  STD_TRY(std_dense_verify_attn(dims, io->q_verify, gamma, c->k_full, c->v_full, c->len_full, io->o_verify,
+                                splits_verify, ws, ws_bytes, stream));
+  STD_TRY(std_accept_prefix(dims->B, gamma, io->draft_tokens, io->dense_tokens, io->n_plus_1, io->accepted,
+                            stream));
+  STD_TRY(std_kv_commit(dims, c->k_full, c->v_full, c->k_sparse, c->v_sparse, c->len_full, c->len_sparse,
+                        io->n_plus_1, gamma + 1, stream));
+  return ok();
+}
+
+}  // extern "C"

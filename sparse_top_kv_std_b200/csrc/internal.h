@@ -1,0 +1,77 @@
+// Host-side launchers shared between the C ABI layer and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace stdb {
+
+// One decode-attention launch: query row r of a KV head (r = g * nq + i, g the
+// query head in the group, i the query position) attends to keys
+// j < len[b] + len_off + i.
+struct AttnArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  float* o;
+  const int32_t* len;
+  int len_off;
+  int L, B, Hq, Hkv, G, nq, rows, d, dtype;
+  int64_t cap;
+  int splits;
+  float* ws;  // partials: [prob][split][rows_pad][d] then [prob][split][rows_pad][2]
+  int* err;
+};
+
+// rows padded to the kernel's row tile, and the workspace floats for `splits`.
+int attn_rows_pad(int rows, int dtype);
+size_t attn_ws_floats(int probs, int splits, int rows, int d, int dtype);
+cudaError_t launch_decode_attn(const AttnArgs& a, cudaStream_t s);
+
+struct ScoreArgs {
+  const void* q_text;   // [L][B][Hq][T][d]
+  const void* k_full;   // [L][B][Hkv][cap][d]
+  const int32_t* nvis;  // device [B]
+  int nvis_max;
+  int L, B, Hq, Hkv, G, T, d, dtype;
+  int64_t cap;
+  float* row_m;   // [prob][G*T]  max of the scaled log2 logits
+  float* row_l;   // [prob][G*T]  sum of 2^(x - m)
+  float* scores;  // [prob][nvis_max]
+  int* err;
+};
+cudaError_t launch_select_scores(const ScoreArgs& a, cudaStream_t s);
+
+// Top-K of `rows` rows of scores at scores + p * stride.  Row p has
+// n_dev[(p / n_div) % n_mod] valid entries (n_const if n_dev is NULL).  idx [rows][K].
+cudaError_t launch_topk(const float* scores, int64_t stride, int rows, const int32_t* n_dev,
+                        int n_const, int n_div, int n_mod, int K, int32_t* idx, int* err,
+                        cudaStream_t s);
+
+struct GatherArgs {
+  const void* k_full;
+  const void* v_full;
+  void* k_sp;
+  void* v_sp;
+  const int32_t* idx;  // [prob][K]
+  const int32_t* nvis;
+  int32_t* len_sparse;
+  int L, B, Hkv, T, K, row_bytes;
+  int64_t cap_full, cap_sparse;
+  int* err;
+};
+cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s);
+
+cudaError_t launch_append(void* k_cache, void* v_cache, int64_t cap, const int32_t* len, int off,
+                          const void* k_new, const void* v_new, int n_new, int L, int B, int Hkv,
+                          int row_bytes, int* err, cudaStream_t s);
+
+cudaError_t launch_commit(void* k_full, void* v_full, void* k_sp, void* v_sp, int32_t* len_full,
+                          int32_t* len_sp, const int32_t* n_plus_1, int max_n, int L, int B,
+                          int Hkv, int row_bytes, int64_t cap_full, int64_t cap_sparse, int* err,
+                          cudaStream_t s);
+
+cudaError_t launch_accept(int B, int gamma, const int32_t* draft, const int32_t* dense,
+                          int32_t* n_plus_1, int32_t* accepted, cudaStream_t s);
+
+}  // namespace stdb

@@ -1,0 +1,97 @@
+"""The C-ABI library loads, exports every entry point the header declares, and
+rejects bad arguments on the host before touching the GPU (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_top_kv_std_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "std_b200.h")
+
+
+def header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(std_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(B.LIB_PATH):
+        from sparse_top_kv_std_b200 import build
+        build.build()
+    return B.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = header_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(B.SIGNATURES), "binding and header disagree"
+
+
+def test_version_and_error_string(lib):
+    assert B.std_version() == 10000
+    assert isinstance(B.std_last_error(), str)
+
+
+def _dims(**kw):
+    base = dict(L=2, B=1, Hq=28, Hkv=4, d=128, dtype=B.STD_BF16, cap_full=1000, cap_sparse=300)
+    base.update(kw)
+    return B.dims(**base)
+
+
+def test_workspace_queries_host_only(lib):
+    d = _dims()
+    ws = B.std_select_workspace_size(d, 64, 512)
+    assert ws >= (2 * 4 * 7 * 64 * 2 + 2 * 4 * 512) * 4
+    # explicit splits: no device query
+    a = B.std_attn_workspace_size(d, 9, 1000, 4)
+    assert a == 2 * 4 * 4 * 64 * (128 + 2) * 4      # rows 63 padded to 64
+    assert B.std_attn_workspace_size(d, 9, 1000, 1) == 0
+    assert B.std_select_workspace_size(_dims(dtype=7), 64, 512) == 0
+    assert B.std_attn_workspace_size(_dims(Hq=5), 1, 1000, 4) == 0
+
+
+FAKE = 1 << 40  # a 16-byte aligned non-null "pointer": never dereferenced, checks fail first
+
+
+@pytest.mark.parametrize("call,code", [
+    (lambda: lib_().std_select_topk(None, FAKE, 64, FAKE, FAKE, FAKE, 512, 16, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_select_topk(ctypes.byref(_dims(dtype=5)), FAKE, 64, FAKE, FAKE, FAKE, 512, 16, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_UNSUPPORTED),
+    (lambda: lib_().std_select_topk(ctypes.byref(_dims(d=80)), FAKE, 64, FAKE, FAKE, FAKE, 512, 16, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_UNSUPPORTED),
+    (lambda: lib_().std_select_topk(ctypes.byref(_dims()), None, 64, FAKE, FAKE, FAKE, 512, 16, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_select_topk(ctypes.byref(_dims()), FAKE + 2, 64, FAKE, FAKE, FAKE, 512, 16, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_select_topk(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, FAKE, 512, 513, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_select_topk(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, FAKE, 512, 0, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_select_topk(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, FAKE, 512, 256, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_CAPACITY),
+    (lambda: lib_().std_select_topk(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, FAKE, 990, 16, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_CAPACITY),
+    (lambda: lib_().std_select_topk(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, FAKE, 512, 16, FAKE, FAKE, FAKE, FAKE, None, FAKE, 16, None), B.STD_ERR_WORKSPACE),
+    (lambda: lib_().std_topk_from_scores(FAKE, 4, 100, 101, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_topk_from_scores(None, 4, 100, 10, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_dense_verify_attn(ctypes.byref(_dims()), FAKE, 32, FAKE, FAKE, FAKE, FAKE, 1, None, 0, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_dense_verify_attn(ctypes.byref(_dims()), FAKE, -1, FAKE, FAKE, FAKE, FAKE, 1, None, 0, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_dense_verify_attn(ctypes.byref(_dims()), FAKE, 18, FAKE, FAKE, FAKE, FAKE, 1, None, 0, None), B.STD_ERR_UNSUPPORTED),
+    (lambda: lib_().std_dense_verify_attn(ctypes.byref(_dims()), FAKE, 4, FAKE, FAKE, FAKE, FAKE, 8, None, 0, None), B.STD_ERR_WORKSPACE),
+    (lambda: lib_().std_dense_verify_attn(ctypes.byref(_dims()), FAKE, 4, FAKE, FAKE, FAKE, FAKE, 2000, None, 0, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_sparse_decode_attn(ctypes.byref(_dims()), FAKE, FAKE, FAKE, FAKE, -1, FAKE, 1, None, 0, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_sparse_decode_attn(ctypes.byref(_dims()), FAKE, FAKE, FAKE, None, 0, FAKE, 1, None, 0, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_accept_prefix(0, 4, FAKE, FAKE, FAKE, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_accept_prefix(2, 32, FAKE, FAKE, FAKE, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_accept_prefix(2, 4, FAKE, FAKE, None, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_kv_append(ctypes.byref(_dims()), FAKE, FAKE, 100, FAKE, 90, FAKE, FAKE, 20, None), B.STD_ERR_CAPACITY),
+    (lambda: lib_().std_kv_append(ctypes.byref(_dims()), FAKE, FAKE, 100, FAKE, -1, FAKE, FAKE, 2, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_kv_commit(ctypes.byref(_dims()), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 33, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_decode_round(ctypes.byref(_dims()), 4, None, None, 0, 0, None, 0, None), B.STD_ERR_INVALID_ARG),
+])
+def test_host_side_rejections(lib, call, code):
+    assert call() == code
+    assert B.std_last_error() != ""
+
+
+def lib_():
+    return B.lib()

@@ -1,0 +1,568 @@
+#!/usr/bin/env python
+"""Benchmark of the Sparse-to-Dense (StD) decoding hot path on B200.
+
+One step = one whole StD decode of a synthetic long-video prompt: the prefill
+top-K selection (selection scores, top-K, gather) followed by R draft+verify
+rounds (gamma sparse draft attentions, one dense verify attention over the
+full cache, acceptance, commit).  All inputs are resident in HBM before the
+timed region; the full KV cache (8.2 GB at the default workload) is larger
+than L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload video_140k]
+    python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
+
+Multi-GPU (torchrun, one rank per GPU): every rank decodes its own prompt
+(independent sequences, no data-path collective), "scaling": "weak"; time is
+the max over ranks.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn HBM GB/s (sparse draft, dense verify) vs 8 TB/s; µs per draft+verify round"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["std", "reference"], default="std")
+    ap.add_argument("--workload", default="video_140k")
+    ap.add_argument("--rounds", type=int, default=None, help="draft+verify rounds per step (default: workload's)")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--threads", type=int, default=0, help="host threads for input generation")
+    return ap.parse_args(argv)
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS if k in d}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- byte / flop model
+
+def attention_bytes(wl, rounds, accepted):
+    """Algorithmic K/V bytes of the draft and verify attention over `rounds` rounds.
+
+    accepted[r][b] = n + 1 of round r.  A step reads, per (layer, KV head), every
+    K and V row each attention call attends to: the verify of round r reads
+    len_full_r + gamma + 1 rows, draft step j reads len_sparse_r + j + 1 rows.
+    Returns (draft_bytes, verify_bytes, per-round verify bytes list).
+    """
+    row = 2 * wl.d * wl.elem_bytes * wl.L * wl.Hkv          # K + V of one position, all layers/heads
+    lf = [n + wl.T for n in wl.nvis]
+    ls = [wl.K + wl.T] * wl.B
+    draft = verify = 0
+    per_round_verify = []
+    for r in range(rounds):
+        v = sum(lf[b] + wl.gamma + 1 for b in range(wl.B)) * row
+        verify += v
+        per_round_verify.append(v)
+        for j in range(wl.gamma):
+            draft += sum(ls[b] + j + 1 for b in range(wl.B)) * row
+        for b in range(wl.B):
+            lf[b] += int(accepted[r][b])
+            ls[b] += int(accepted[r][b])
+    return draft, verify, per_round_verify
+
+
+def select_flops(wl):
+    """Executed MMA flops of the selection (2 passes over the M x Nv logits)."""
+    M = wl.G * wl.T
+    return 2 * sum(2 * M * n * wl.d for n in wl.nvis) * wl.L * wl.Hkv
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            cmd = ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
+                   "-lms", "200"]
+            if self.gpu_id is not None:
+                cmd += ["-i", str(self.gpu_id)]
+            self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == len(self.FIELDS):
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        load = [s for s, p in zip(sm, pw) if pw and p >= 0.5 * max(pw)] or sm
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": num(rows[0][2]), "power_w_max": max(pw) if pw else None,
+                "samples": len(rows), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) sample
+
+def oracle_sample(wl, seed, rounds_sample, heads=((0, 0, 0),)):
+    """Time the fp64 oracle on a bounded sample: for each listed (layer, batch, KV head)
+    slice, its prefill selection and `rounds_sample` draft+verify rounds.
+    Returns (select seconds per head, round seconds per head and round)."""
+    import numpy as np
+
+    import oracle
+    import synth
+    f = lambda a: synth.storage_to_f64(synth.storage(a, wl.dtype), wl.dtype)  # noqa: E731
+    t_sel = t_round = 0.0
+    for (l, b, h) in heads:
+        nv = wl.nvis[b]
+        k, v = synth.kv_head(wl, seed, l, b, h)
+        cap_f = nv + wl.T + rounds_sample * (wl.gamma + 1)
+        cap_s = wl.K + wl.T + rounds_sample * (wl.gamma + 1)
+        kf = np.zeros((1, 1, 1, cap_f, wl.d))
+        vf = np.zeros_like(kf)
+        kf[0, 0, 0, :nv + wl.T] = f(k)
+        vf[0, 0, 0, :nv + wl.T] = f(v)
+        qt = f(synth.q_text_head(wl, seed, l, b, h))[None, None]
+        t0 = time.perf_counter()
+        _, _, ksp, vsp, lsp = oracle.select_topk(qt, kf, vf, np.array([nv]), wl.T, wl.K, cap_s)
+        t_sel += time.perf_counter() - t0
+        qd, qv = synth.decode_queries(wl, seed, l, b, h)
+        kd, vd, kv, vv = synth.decode_kv(wl, seed, l, b, h)
+        dense, draft = synth.tokens(wl, seed, b)
+        st = {"k_full": kf, "v_full": vf, "k_sp": ksp, "v_sp": vsp,
+              "len_full": np.array([nv + wl.T]), "len_sp": lsp.astype(np.int64)}
+        t0 = time.perf_counter()
+        for r in range(rounds_sample):
+            oracle.decode_round(st, f(qd[r])[:, None, None, :, None, :], f(kd[r])[:, None, None, None, None, :],
+                                f(vd[r])[:, None, None, None, None, :], f(qv[r])[None, None],
+                                f(kv[r])[None, None, None], f(vv[r])[None, None, None],
+                                draft[r][None], dense[r][None])
+        t_round += time.perf_counter() - t0
+    n = len(heads)
+    return t_sel / n, t_round / (n * rounds_sample)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_estimate(wl, seed, rounds, step_attn_bytes, rounds_sample, heads):
+    """Oracle GB/s on the sample, scaled to a whole step (all heads, all rounds)."""
+    t_sel, t_round = oracle_sample(wl, seed, rounds_sample, heads)
+    probs = wl.L * wl.B * wl.Hkv
+    est = probs * (t_sel + rounds * t_round)
+    return step_attn_bytes / est / 1e9, t_sel, t_round, est
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import numpy as np
+
+    import oracle
+    import synth
+    wl = synth.workload(args.workload)
+    R = args.rounds or wl.rounds
+    if R > wl.rounds:
+        wl = wl.replace(rounds=R)
+    # acceptance counts of the byte model: the oracle's greedy prefix rule on the token streams
+    streams = [synth.tokens(wl, args.seed, b) for b in range(wl.B)]
+    acc = [oracle.accept_prefix(np.array([s[1][r] for s in streams]), np.array([s[0][r] for s in streams]))[0]
+           for r in range(R)]
+    draft_b, verify_b, _ = attention_bytes(wl, R, acc)
+    step_bytes = draft_b + verify_b
+    heads = [(l, b, h) for l in range(wl.L) for b in range(wl.B) for h in range(wl.Hkv)]
+    vals = []
+    times = []
+    for i in range(args.warmup + args.steps):
+        lbh = heads[i % len(heads)]
+        t0 = time.perf_counter()
+        v, t_sel, t_round, est = cpu_estimate(wl, args.seed, R, step_bytes, 1, [lbh])
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            vals.append(v)
+            times.append(dt)
+    value = statistics.median(vals)
+    cores = blas_threads()
+    sample = (f"each step: the fp64 oracle on one (layer, KV head) slice of {wl.name} -- its prefill "
+              f"selection and 1 draft+verify round -- scaled to all {wl.L * wl.B * wl.Hkv} slices and {R} rounds")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.median(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl, R),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl, R):
+    return {"workload": wl.name, "L": wl.L, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
+            "nvis": list(wl.nvis) if wl.B > 1 else wl.nvis[0], "T": wl.T, "K": wl.K, "gamma": wl.gamma,
+            "rounds_per_step": R, "p_match": wl.p_match, "storage": wl.dtype,
+            "step": f"prefill top-K selection + {R} draft/verify rounds (one StD decode)",
+            "l2": "inputs larger than L2 (no flush)" if kv_bytes(wl) > 126e6 else "L2-resident inputs"}
+
+
+def kv_bytes(wl):
+    return 2 * wl.L * wl.B * wl.Hkv * wl.cap_full * wl.d * wl.elem_bytes
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_std(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import synth
+    from sparse_top_kv_std_b200 import binding as B
+    from sparse_top_kv_std_b200.session import DecodeSession
+
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+        pg = dist
+    B.lib()
+
+    wl = synth.workload(args.workload)
+    R = args.rounds or wl.rounds
+    if R > wl.rounds:
+        wl = wl.replace(rounds=R)
+    seed = args.seed + rank
+    dt = B.STD_F32 if wl.dtype == "f32" else B.STD_BF16
+    sess = DecodeSession(wl.L, wl.B, wl.Hq, wl.Hkv, wl.d, dt, wl.cap_full, wl.cap_sparse, wl.T, wl.K, wl.gamma,
+                         wl.nvis_max, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # ---- inputs: generated on the host (pinned), copied once to HBM
+    host_t = torch.int16 if dt == B.STD_BF16 else torch.float32
+    np_t = np.uint16 if dt == B.STD_BF16 else np.float32
+    pin_k = torch.zeros(tuple(sess.k_full.shape), dtype=host_t, pin_memory=True)
+    pin_v = torch.zeros(tuple(sess.v_full.shape), dtype=host_t, pin_memory=True)
+    nk, nvw = pin_k.numpy().view(np_t), pin_v.numpy().view(np_t)
+
+    def sink(l, b, h, ks, vs):
+        nk[l, b, h, :ks.shape[0]] = ks
+        nvw[l, b, h, :vs.shape[0]] = vs
+
+    t_gen = time.perf_counter()
+    threads = args.threads or min(16, os.cpu_count() or 8)
+    x = synth.host_inputs(wl, seed=seed, threads=threads, kv_sink=sink)
+    t_gen = time.perf_counter() - t_gen
+    names = ["q_text", "q_draft", "k_draft", "v_draft", "q_verify", "k_verify", "v_verify"]
+    pin = {}
+    for n in names:
+        a = np.ascontiguousarray(x[n])
+        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+        pin[n] = t.pin_memory()
+    pin["draft_tokens"] = torch.from_numpy(x["draft_tokens"]).pin_memory()
+    pin["dense_tokens"] = torch.from_numpy(x["dense_tokens"]).pin_memory()
+    sd = torch.bfloat16 if dt == B.STD_BF16 else torch.float32
+
+    def to_dev(t):
+        d = torch.empty(t.shape, dtype=t.dtype, device=dev)
+        return d
+
+    dv = {n: to_dev(pin[n]) for n in pin}
+
+    def h2d_inputs():
+        sess.k_full.view(host_t).copy_(pin_k, non_blocking=True)
+        sess.v_full.view(host_t).copy_(pin_v, non_blocking=True)
+        for n in pin:
+            dv[n].copy_(pin[n], non_blocking=True)
+
+    h2d_inputs()
+    torch.cuda.synchronize()
+
+    def view(n, r=None):
+        t = dv[n] if r is None else dv[n][r]
+        return t.view(sd) if t.dtype == torch.int16 else t
+
+    len0 = torch.tensor([n + wl.T for n in wl.nvis], dtype=torch.int32, device=dev)
+    nvis_dev = torch.tensor(list(wl.nvis), dtype=torch.int32, device=dev)
+    sess.nvis.copy_(nvis_dev)
+    outs = [sess.round_outputs() for _ in range(R)]
+    sp_d = B.std_attn_splits(sess.dims, wl.cap_sparse, 0) if wl.gamma > 0 else 1
+    sp_v = B.std_attn_splits(sess.dims, wl.cap_full, 0)
+    ws = sess.ws_round
+    q_text = view("q_text")
+    launches_per_step = 4 + R * (wl.gamma * (2 + (sp_d > 1)) + 2 + (sp_v > 1) + 1 + 2)
+
+    def step(ev=None):
+        """One StD decode: reset lengths, select, R rounds.  ev: dict of event lists to record."""
+        sess.len_full.copy_(len0, non_blocking=True)
+        if ev is not None:
+            ev["sel0"].record(stream)
+        sess.select(q_text, keep_scores=False)
+        if ev is not None:
+            ev["sel1"].record(stream)
+        for r in range(R):
+            o = outs[r]
+            for j in range(wl.gamma):
+                B.std_kv_append(sess.dims, sess.k_sparse, sess.v_sparse, wl.cap_sparse, sess.len_sparse, j,
+                                view("k_draft", r)[j], view("v_draft", r)[j], 1)
+                if ev is not None:
+                    ev["d0"][r * wl.gamma + j].record(stream)
+                B.std_sparse_decode_attn(sess.dims, view("q_draft", r)[j], sess.k_sparse, sess.v_sparse,
+                                         sess.len_sparse, j + 1, o["o_draft"][j], sp_d, ws)
+                if ev is not None:
+                    ev["d1"][r * wl.gamma + j].record(stream)
+            B.std_kv_append(sess.dims, sess.k_full, sess.v_full, wl.cap_full, sess.len_full, 0,
+                            view("k_verify", r), view("v_verify", r), wl.gamma + 1)
+            if ev is not None:
+                ev["v0"][r].record(stream)
+            B.std_dense_verify_attn(sess.dims, view("q_verify", r), wl.gamma, sess.k_full, sess.v_full,
+                                    sess.len_full, o["o_verify"], sp_v, ws)
+            if ev is not None:
+                ev["v1"][r].record(stream)
+            B.std_accept_prefix(wl.B, wl.gamma, dv["draft_tokens"][r], dv["dense_tokens"][r], o["n_plus_1"],
+                                o["accepted"])
+            B.std_kv_commit(sess.dims, sess.k_full, sess.v_full, sess.k_sparse, sess.v_sparse, sess.len_full,
+                            sess.len_sparse, o["n_plus_1"], wl.gamma + 1)
+        if ev is not None:
+            ev["end"].record(stream)
+
+    def new_events():
+        E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+        return {"sel0": E(), "sel1": E(), "end": E(), "d0": [E() for _ in range(R * wl.gamma)],
+                "d1": [E() for _ in range(R * wl.gamma)], "v0": [E() for _ in range(R)],
+                "v1": [E() for _ in range(R)]}
+
+    # ---- warm-up (also yields the acceptance counts of the byte model)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    flags = B.std_get_device_error(clear=True)
+    if flags:
+        raise RuntimeError(f"device error flags {flags:#x} after warm-up")
+    accepted = [o["n_plus_1"].cpu().tolist() for o in outs]
+    draft_b, verify_b, verify_round_b = attention_bytes(wl, R, accepted)
+    step_attn = draft_b + verify_b
+
+    # ---- timed region
+    evs = [new_events() for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    clk = ClockSampler(gpu_uuid(dev))
+    clk.start()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    if pg:
+        pg.barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    flags = B.std_get_device_error(clear=True)
+    if flags:
+        raise RuntimeError(f"device error flags {flags:#x} in the timed region")
+
+    sel_ms = [e["sel0"].elapsed_time(e["sel1"]) for e in evs]
+    v_ms = [e["v0"][r].elapsed_time(e["v1"][r]) for e in evs for r in range(R)]
+    d_ms = [e["d0"][k].elapsed_time(e["d1"][k]) for e in evs for k in range(R * wl.gamma)]
+    rounds_ms = [e["sel1"].elapsed_time(e["end"]) for e in evs]
+    mx = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(mx, op=pg.ReduceOp.MAX)
+    elapsed_ms = float(mx.item())
+
+    # ---- e2e through the public API with host buffers (H2D of inputs, D2H of the accepted tokens)
+    e2e = None
+    if not args.no_e2e and args.e2e_steps > 0:
+        acc_host = torch.zeros((R, wl.B, wl.gamma + 1), dtype=torch.int32, pin_memory=True)
+        acc_dev = torch.zeros((R, wl.B, wl.gamma + 1), dtype=torch.int32, device=dev)
+
+        def e2e_step():
+            h2d_inputs()
+            step()
+            for r in range(R):
+                acc_dev[r].copy_(outs[r]["accepted"], non_blocking=True)
+            acc_host.copy_(acc_dev, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
+        a0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = torch.tensor([a0.elapsed_time(a1)], dtype=torch.float64, device=dev)
+        if pg:
+            pg.all_reduce(e_ms, op=pg.ReduceOp.MAX)
+        e_ms = float(e_ms.item())
+        h2d = pin_k.numel() * pin_k.element_size() * 2 + sum(t.numel() * t.element_size() for t in pin.values())
+        d2h = acc_host.numel() * 4
+        e2e = {"value": step_attn * args.e2e_steps * world / (e_ms / 1e3) / 1e9, "unit": "GB/s",
+               "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    if rank != 0:
+        if pg:
+            pg.destroy_process_group()
+        return 0
+
+    peaks, peak_src = load_peaks()
+    value = step_attn * args.steps * world / (elapsed_ms / 1e3) / 1e9
+    v_avg_ms = statistics.mean(v_ms)
+    v_bytes_avg = verify_b / R
+    achieved = v_bytes_avg / (v_avg_ms / 1e3) / 1e9
+    d_avg_ms = statistics.mean(d_ms)
+    d_bytes_avg = draft_b / max(1, R * wl.gamma)
+    sel_avg = statistics.mean(sel_ms)
+    traffic = load_traffic("dense_verify_attn", wl.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == B.STD_BF16 else "f32",
+        "data": "synthetic", "config": workload_config(wl, R),
+        "us_per_round": 1e3 * statistics.mean(rounds_ms) / R,
+        "select_ms": sel_avg,
+        "kernels": {
+            "dense_verify_attn": {"ms_per_launch": v_avg_ms, "bytes_per_launch": v_bytes_avg,
+                                  "GBps": achieved, "frac_of_8TBps": achieved / 8000.0, "splits": sp_v},
+            "sparse_decode_attn": {"us_per_launch": 1e3 * d_avg_ms, "bytes_per_launch": d_bytes_avg,
+                                   "GBps": d_bytes_avg / (d_avg_ms / 1e3) / 1e9,
+                                   "frac_of_8TBps": d_bytes_avg / (d_avg_ms / 1e3) / 8e12, "splits": sp_d},
+            "select_topk": {"ms_per_launch": sel_avg, "mma_TFLOPs": select_flops(wl) / (sel_avg / 1e3) / 1e12,
+                            "one_pass_TFLOPs": 0.5 * select_flops(wl) / (sel_avg / 1e3) / 1e12},
+        },
+        "roofline": {"kernel": "dense_verify_attn (verify attention + split merge)", "bound": "hbm",
+                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "peak_source": f"{peak_src} HBM copy bandwidth"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "input_gen_s": t_gen,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        v, t_sel, t_round, est = cpu_estimate(wl, seed, R, step_attn, 2, [(0, 0, 0)])
+        line["cpu_baseline"] = {
+            "value": v, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"fp64 oracle on one (layer, KV head) slice of {wl.name}: its prefill selection "
+                       f"({t_sel:.1f} s) and 2 draft+verify rounds ({2 * t_round:.1f} s), scaled to all "
+                       f"{wl.L * wl.B * wl.Hkv} slices and {R} rounds (est. {est:.0f} s per step)")}
+    print(json.dumps(line), flush=True)
+    if pg:
+        pg.destroy_process_group()
+    return 0
+
+
+def gpu_uuid(dev):
+    try:
+        import torch
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
+
+
+def load_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged since."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel, {})
+    if e.get("workload") != workload:
+        return None
+    src = os.path.join(ROOT, e.get("source", ""))
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    return e.get("dram_bytes_per_launch") if sha == e.get("source_sha256") else None
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local_rank = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_std(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

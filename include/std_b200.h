@@ -190,6 +190,35 @@ int std_dense_verify_attn(const std_dims* dims, const void* q, int gamma, const 
                           const void* v_full, const int32_t* len_full, float* o, int splits,
                           void* ws, size_t ws_bytes, std_stream_t stream);
 
+/* ---------------------------------------------------------------- verify attention, no workspace
+ *
+ * No counterpart in the paper: this entry point exists for callers, not for the method.
+ *
+ * std_dense_verify_attn without the workspace argument, for code that cannot
+ * hand the library device memory while it decodes: a plugin inside another
+ * engine that owns every device allocation, or a latency-bound service that
+ * bans cudaMalloc/cudaFree after start-up because they can synchronise the
+ * device and stall unrelated streams.  The split-K partials go to a scratch
+ * array compiled into the library: STD_NOALLOC_SCRATCH_BYTES on every GPU on
+ * which the library is loaded, held until the process exits.  Arguments,
+ * layouts, requirements and results are those of std_dense_verify_attn.
+ *  - A call whose partials need more than STD_NOALLOC_SCRATCH_BYTES (see
+ *    std_attn_workspace_size; splits = 1 needs none) is rejected with
+ *    STD_ERR_WORKSPACE before anything is launched.  It never allocates.
+ *  - The first call on a device looks up the array's device address with that
+ *    device current; make that first call before capturing any stream.
+ *  - All calls on a device share the one array and it keeps what the last call
+ *    wrote.  Nothing in it has to start at zero (each call writes every partial
+ *    it reads), but two calls whose kernels may overlap on the GPU -- different
+ *    streams with no ordering between them -- race on it and corrupt each
+ *    other's results.
+ */
+#define STD_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+int std_dense_verify_attn_noalloc(const std_dims* dims, const void* q, int gamma, const void* k_full,
+                                  const void* v_full, const int32_t* len_full, float* o, int splits,
+                                  std_stream_t stream);
+
 /* ---------------------------------------------------------------- acceptance
  *
  * "Methodik" item 3: keep the longest prefix of draft tokens that matches the

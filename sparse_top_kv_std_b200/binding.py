@@ -70,6 +70,7 @@ SIGNATURES = {
     "std_attn_splits": (_I, [_DP, _I64, _I]),
     "std_sparse_decode_attn": (_I, [_DP, _P, _P, _P, _P, _I, _P, _I, _P, _SZ, _P]),
     "std_dense_verify_attn": (_I, [_DP, _P, _I, _P, _P, _P, _P, _I, _P, _SZ, _P]),
+    "std_dense_verify_attn_noalloc": (_I, [_DP, _P, _I, _P, _P, _P, _P, _I, _P]),
     "std_accept_prefix": (_I, [_I, _I, _P, _P, _P, _P, _P]),
     "std_kv_append": (_I, [_DP, _P, _P, _I64, _P, _I, _P, _P, _I, _P]),
     "std_kv_commit": (_I, [_DP, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
@@ -198,6 +199,15 @@ def std_dense_verify_attn(d: StdDims, q, gamma, k_full, v_full, len_full, o, spl
                           stream=None) -> None:
     _check(lib().std_dense_verify_attn(ctypes.byref(d), _ptr(q), gamma, _ptr(k_full), _ptr(v_full),
                                        _ptr(len_full), _ptr(o), splits, _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+STD_NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def std_dense_verify_attn_noalloc(d: StdDims, q, gamma, k_full, v_full, len_full, o, splits=0,
+                                  stream=None) -> None:
+    _check(lib().std_dense_verify_attn_noalloc(ctypes.byref(d), _ptr(q), gamma, _ptr(k_full), _ptr(v_full),
+                                               _ptr(len_full), _ptr(o), splits, _stream(stream)))
 
 
 def std_accept_prefix(B, gamma, draft, dense_argmax, n_plus_1, accepted, stream=None) -> None:

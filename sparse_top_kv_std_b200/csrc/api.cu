@@ -382,3 +382,54 @@ int std_decode_round(const std_dims* dims, int gamma, const std_cache* c, const 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- verify attention without a workspace
+// Scratch for std_dense_verify_attn_noalloc: split-K partials live here instead
+// of in a caller-provided workspace.  One copy per device, for the process lifetime.
+static __device__ __align__(256) float g_noalloc_scratch[STD_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name only stands in for the symbol, so the address is looked up
+// once per device (with that device current) and cached.
+int noalloc_scratch(float** out) {
+  int dev;
+  STD_TRY(current_device(&dev));
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return STD_OK;
+}
+
+}  // namespace
+
+extern "C" int std_dense_verify_attn_noalloc(const std_dims* dims, const void* q, int gamma, const void* k_full,
+                                             const void* v_full, const int32_t* len_full, float* o, int splits,
+                                             std_stream_t stream) {
+  STD_TRY(check_dims(dims));
+  STD_TRY(check_ptr(q, 16, "q"));
+  STD_TRY(check_ptr(k_full, 16, "k_full"));
+  STD_TRY(check_ptr(v_full, 16, "v_full"));
+  STD_TRY(check_ptr(len_full, 4, "len_full"));
+  STD_TRY(check_ptr(o, 16, "o"));
+  if (gamma < 0 || gamma > 31) return fail(STD_ERR_INVALID_ARG, "gamma = %d must be in [0, 31]", gamma);
+  int sp;
+  STD_TRY(resolve_splits(splits, probs_of(dims), dims->cap_full, &sp));
+  const size_t need = attn_ws_bytes(dims, gamma + 1, sp);
+  if (need > STD_NOALLOC_SCRATCH_BYTES)
+    return fail(STD_ERR_WORKSPACE, "verify partials need %zu bytes of scratch; the built-in array holds %u "
+                "(use fewer splits or std_dense_verify_attn with a workspace)", need, STD_NOALLOC_SCRATCH_BYTES);
+  float* scratch = nullptr;
+  if (need > 0) STD_TRY(noalloc_scratch(&scratch));
+  return run_attn(dims, q, k_full, v_full, dims->cap_full, len_full, 1, gamma + 1, o, sp, scratch,
+                  need > 0 ? STD_NOALLOC_SCRATCH_BYTES : 0, stream);
+}

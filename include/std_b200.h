@@ -66,7 +66,8 @@ enum std_device_error {
   STD_DEVERR_CAPACITY = 1,  /* an append / commit / verify would pass the cache capacity */
   STD_DEVERR_LENGTH = 2,    /* a device length was <= 0 or beyond the capacity in attention */
   STD_DEVERR_K_RANGE = 4,   /* select: K > nvis[b], or nvis[b] + T > cap_full */
-  STD_DEVERR_NVIS_MAX = 8   /* select: nvis[b] > the host-side nvis_max bound */
+  STD_DEVERR_NVIS_MAX = 8,  /* select: nvis[b] > the host-side nvis_max bound */
+  STD_DEVERR_TIMEOUT = 16   /* a bounded wait inside a kernel gave up; that CTA's output is missing */
 };
 
 /* Shape of the model slice a call works on.  cap_full / cap_sparse are the row

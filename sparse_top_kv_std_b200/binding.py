@@ -33,6 +33,7 @@ STD_DEVERR_CAPACITY = 1
 STD_DEVERR_LENGTH = 2
 STD_DEVERR_K_RANGE = 4
 STD_DEVERR_NVIS_MAX = 8
+STD_DEVERR_TIMEOUT = 16
 
 # every function the header declares, with (restype, argtypes)
 _P = ctypes.c_void_p

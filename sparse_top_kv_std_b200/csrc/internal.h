@@ -41,6 +41,8 @@ struct ScoreArgs {
   int* err;
 };
 cudaError_t launch_select_scores(const ScoreArgs& a, cudaStream_t s);
+// tcgen05 version for bf16 operands; cudaErrorNotSupported for shapes it does not cover.
+cudaError_t launch_select_scores_tc(const ScoreArgs& a, cudaStream_t s);
 
 // Top-K of `rows` rows of scores at scores + p * stride.  Row p has
 // n_dev[(p / n_div) % n_mod] valid entries (n_const if n_dev is NULL).  idx [rows][K].

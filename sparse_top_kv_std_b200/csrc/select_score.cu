@@ -1,3 +1,7 @@
+// Prefill selection scores of Sparse-to-Dense decoding -- mma.sync / FFMA
+// kernels: the fp32 path, and the bf16 fallback for shapes the tcgen05 kernels
+// of select_tc.cu do not cover (more than 2048 text query rows per KV head).
+//
 // Prefill selection scores of Sparse-to-Dense decoding ("Methodik" item 4 of
 // the gist.science summary: top-K visual KV chosen once at prefill from the
 // attention from text tokens to visual tokens, averaged; per layer and head).
@@ -307,6 +311,8 @@ cudaError_t launch_f32_scores(const ScoreArgs& a, cudaStream_t s) {
 
 cudaError_t launch_select_scores(const ScoreArgs& a, cudaStream_t s) {
   if (a.dtype == STD_BF16) {
+    const cudaError_t e = launch_select_scores_tc(a, s);  // tensor-core path
+    if (e != cudaErrorNotSupported) return e;
     if (a.d == 128) return launch_bf16_scores<128>(a, s);
     if (a.d == 64) return launch_bf16_scores<64>(a, s);
   } else {

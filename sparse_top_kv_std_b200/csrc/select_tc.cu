@@ -1,0 +1,486 @@
+// Selection scores on the 5th-generation tensor cores (tcgen05), fed by TMA.
+//
+// Same quantities as select_score.cu ("Methodik" item 4 of the gist.science
+// summary: average text-to-visual attention per (layer, KV head)):
+//   pass 1  m_r = max_n x_rn,  l_r = sum_n 2^(x_rn - m_r)        x = log2(e) q_r . k_n / sqrt(d)
+//   pass 2  score_n = 1/M sum_r 2^(x_rn - m_r) / l_r
+//
+// Pass 1: CTA = 128 text rows (the MMA M axis) of one (layer, seq, KV head);
+//   keys stream through a 3-stage TMA ring in 256-key tiles; S = Q K^T lands
+//   in a double-buffered TMEM accumulator (2 x 256 fp32 columns); each of the
+//   128 epilogue threads owns one row and keeps its running max / sum, so no
+//   cross-thread reduction is needed.
+// Pass 2: transposed.  CTA = 256 keys (two 128-key MMA tiles, M axis) kept in
+//   shared memory; the text rows stream through as 256-row chunks (N axis);
+//   each epilogue thread owns one key and sums its column in registers.
+// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
+// issuer (one elected lane), warps 2-5 epilogue (TMEM lane quarter = warp % 4).
+// Every wait is bounded; on a timeout the CTA raises its abort flag, records
+// the error, lets in-flight copies and MMAs finish (bounded), frees TMEM and
+// returns.  No multicast loads are used.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc100.cuh"
+
+namespace stdb {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int BM = 128;      // MMA M
+constexpr int BN = 256;      // MMA N (keys in pass 1, text rows in pass 2)
+constexpr int kMaxRows = 2048;  // G * T supported by pass 2 (row statistics kept in shared memory)
+constexpr int kTmemCols = 512;
+
+struct Ctl {
+  uint64_t full[8], empty[8];
+  uint64_t qfull, kfull, done;
+  uint64_t accfull[2], accempty[2];
+  uint32_t tmem;
+  int abort_flag;
+  int consumed;
+};
+
+__device__ __forceinline__ bool visual_ok(const ScoreArgs& a, int b, int* nv_out) {
+  const int nv = a.nvis[b];
+  *nv_out = nv;
+  return nv >= 1 && nv <= a.nvis_max && (int64_t)nv + a.T <= a.cap;
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Wait that ignores the abort flag (used while unwinding), bounded in time.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = tc::globaltimer();
+  while (!tc::mbar_try_wait(a, parity)) {
+    if (tc::globaltimer() - t0 > tc::kWaitTimeoutNs) return;
+  }
+}
+
+template <int D>
+struct P1 {
+  static constexpr int KB = D / 64;                  // 128-byte K-blocks per row
+  static constexpr int STAGES = D == 128 ? 3 : 6;
+  static constexpr uint32_t Q_BYTES = KB * BM * 128;
+  static constexpr uint32_t KT_BYTES = KB * BN * 128;
+  static constexpr uint32_t SMEM = 1024 + Q_BYTES + STAGES * KT_BYTES + sizeof(Ctl);
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+rowstats_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const ScoreArgs a) {
+  using C = P1<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sQ = smem_u32(smem);
+  const uint32_t sK = sQ + C::Q_BYTES;
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::Q_BYTES + C::STAGES * C::KT_BYTES);
+
+  const int h = blockIdx.y, lb = blockIdx.z, b = lb % a.B;
+  const int prob = lb * a.Hkv + h;
+  const int M = a.G * a.T;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int nv;
+  if (!visual_ok(a, b, &nv)) {
+    if (blockIdx.x == 0 && threadIdx.x == 0)
+      flag_error(a.err, nv > a.nvis_max ? STD_DEVERR_NVIS_MAX : STD_DEVERR_K_RANGE);
+    return;
+  }
+  const int ntiles = (nv + BN - 1) / BN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      tc::mbar_init(&ctl->full[s], 1);
+      tc::mbar_init(&ctl->empty[s], 1);
+    }
+    tc::mbar_init(&ctl->qfull, 1);
+    tc::mbar_init(&ctl->done, 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&ctl->accfull[i], 1);
+      tc::mbar_init(&ctl->accempty[i], 128);
+    }
+    ctl->abort_flag = 0;
+    ctl->consumed = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tc::tmem_alloc(&ctl->tmem, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = ctl->tmem;
+  volatile int* abort_flag = &ctl->abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::prefetch_tmap(&tm_q);
+      tc::prefetch_tmap(&tm_k);
+      const int qrow = (lb * a.Hq + h * a.G) * a.T + blockIdx.x * BM;
+      tc::mbar_expect_tx(&ctl->qfull, C::Q_BYTES);
+#pragma unroll
+      for (int kb = 0; kb < C::KB; ++kb) tc::tma_load_2d(sQ + kb * BM * 128, &tm_q, kb * 64, qrow, &ctl->qfull);
+      const int krow = prob * (int)a.cap;
+      int issued = 0;
+      for (int t = 0; t < ntiles; ++t) {
+        const int s = t % C::STAGES;
+        const uint32_t ph = (t / C::STAGES) & 1;
+        if (!tc::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag, a.err)) break;
+        tc::mbar_expect_tx(&ctl->full[s], C::KT_BYTES);
+#pragma unroll
+        for (int kb = 0; kb < C::KB; ++kb)
+          tc::tma_load_2d(sK + s * C::KT_BYTES + kb * BN * 128, &tm_k, kb * 64, krow + t * BN, &ctl->full[s]);
+        issued = t + 1;
+      }
+      if (*abort_flag) {  // let the copies still in flight land before the CTA goes away
+        drain_wait(&ctl->qfull, 0);
+        for (int t = *(volatile int*)&ctl->consumed; t < issued; ++t)
+          drain_wait(&ctl->full[t % C::STAGES], (t / C::STAGES) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_bf16(BM, BN);
+      bool ok = tc::mbar_wait(&ctl->qfull, 0, abort_flag, a.err);
+      int t = 0;
+      for (; ok && t < ntiles; ++t) {
+        const int s = t % C::STAGES;
+        const uint32_t ph = (t / C::STAGES) & 1;
+        const int buf = t & 1;
+        const uint32_t aph = (t >> 1) & 1;
+        if (!tc::mbar_wait(&ctl->full[s], ph, abort_flag, a.err)) break;
+        *(volatile int*)&ctl->consumed = t + 1;
+        if (!tc::mbar_wait(&ctl->accempty[buf], aph ^ 1, abort_flag, a.err)) break;
+        tc::fence_after_sync();
+        const uint32_t d = tmem + buf * BN;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k & 3) * 32;  // 16-element K step inside the 128-byte row
+          const uint32_t qa = sQ + (k >> 2) * BM * 128 + off;
+          const uint32_t ka = sK + s * C::KT_BYTES + (k >> 2) * BN * 128 + off;
+          tc::umma_bf16(d, tc::sdesc_sw128(qa), tc::sdesc_sw128(ka), idesc, k > 0 ? 1u : 0u);
+        }
+        tc::umma_commit(&ctl->empty[s]);
+        tc::umma_commit(&ctl->accfull[buf]);
+      }
+      if (*abort_flag && t > 0) {  // MMAs may still read shared memory / write TMEM
+        tc::umma_commit(&ctl->done);
+        drain_wait(&ctl->done, 0);
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const float sc = kLog2e * rsqrtf((float)D);
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int t = 0; t < ntiles; ++t) {
+      const int buf = t & 1;
+      const uint32_t aph = (t >> 1) & 1;
+      if (!tc::mbar_wait_warp(&ctl->accfull[buf], aph, abort_flag, a.err)) {
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+      const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + buf * BN;
+      const int key0 = t * BN;
+      const bool tail = key0 + BN > nv;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        __syncwarp();
+        tc::tmem_ld_x32(base + c * 32, r);
+        tc::tmem_ld_wait(r);
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        if (tail) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (key0 + c * 32 + j >= nv) v[j] = -INFINITY;
+        }
+        float cm = v[0];
+#pragma unroll
+        for (int j = 1; j < 32; ++j) cm = fmaxf(cm, v[j]);
+        if (cm > m) {
+          l *= ex2((m - cm) * sc);
+          m = cm;
+        }
+        const float msc = m * sc;
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          s0 += ex2(fmaf(v[j], sc, -msc));
+          s1 += ex2(fmaf(v[j + 1], sc, -msc));
+        }
+        l += s0 + s1;
+      }
+      tc::fence_before_sync();
+      tc::mbar_arrive(&ctl->accempty[buf]);
+    }
+    const int r_glob = blockIdx.x * BM + row;
+    if (ok && !*abort_flag && r_glob < M) {
+      a.row_m[(size_t)prob * M + r_glob] = m * sc;
+      a.row_l[(size_t)prob * M + r_glob] = l;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D>
+struct P2 {
+  static constexpr int KB = D / 64;
+  static constexpr int QSTAGES = 2;
+  static constexpr uint32_t K_BYTES = KB * 256 * 128;   // 256 keys = two 128-key MMA tiles
+  static constexpr uint32_t QC_BYTES = KB * BN * 128;   // one chunk of 256 text rows
+  static constexpr uint32_t MW_BYTES = kMaxRows * 8;
+  static constexpr uint32_t SMEM = 1024 + K_BYTES + QSTAGES * QC_BYTES + MW_BYTES + sizeof(Ctl);
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const ScoreArgs a) {
+  using C = P2<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sK = smem_u32(smem);
+  const uint32_t sQ = sK + C::K_BYTES;
+  float2* mw = reinterpret_cast<float2*>(smem + C::K_BYTES + C::QSTAGES * C::QC_BYTES);
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::K_BYTES + C::QSTAGES * C::QC_BYTES + C::MW_BYTES);
+
+  const int h = blockIdx.y, lb = blockIdx.z, b = lb % a.B;
+  const int prob = lb * a.Hkv + h;
+  const int M = a.G * a.T;
+  const int nch = (M + BN - 1) / BN;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int nv;
+  if (!visual_ok(a, b, &nv)) return;  // pass 1 flagged it
+  const int key0 = blockIdx.x * 256;
+  if (key0 >= nv) return;
+
+  // row statistics of this head: (m_r, 1 / l_r); padding rows contribute 2^-inf * 0 = 0
+  for (int r = threadIdx.x; r < nch * BN; r += kThreads) {
+    const bool in = r < M;
+    mw[r] = in ? make_float2(a.row_m[(size_t)prob * M + r], 1.f / a.row_l[(size_t)prob * M + r])
+               : make_float2(INFINITY, 0.f);
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::QSTAGES; ++s) {
+      tc::mbar_init(&ctl->full[s], 1);
+      tc::mbar_init(&ctl->empty[s], 1);
+    }
+    tc::mbar_init(&ctl->kfull, 1);
+    tc::mbar_init(&ctl->done, 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&ctl->accfull[i], 1);
+      tc::mbar_init(&ctl->accempty[i], 128);
+    }
+    ctl->abort_flag = 0;
+    ctl->consumed = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tc::tmem_alloc(&ctl->tmem, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = ctl->tmem;
+  volatile int* abort_flag = &ctl->abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::prefetch_tmap(&tm_q);
+      tc::prefetch_tmap(&tm_k);
+      tc::mbar_expect_tx(&ctl->kfull, C::K_BYTES);
+#pragma unroll
+      for (int kb = 0; kb < C::KB; ++kb)
+        tc::tma_load_2d(sK + kb * 256 * 128, &tm_k, kb * 64, prob * (int)a.cap + key0, &ctl->kfull);
+      const int qrow = (lb * a.Hq + h * a.G) * a.T;
+      int issued = 0;
+      for (int c = 0; c < nch; ++c) {
+        const int s = c % C::QSTAGES;
+        const uint32_t ph = (c / C::QSTAGES) & 1;
+        if (!tc::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag, a.err)) break;
+        tc::mbar_expect_tx(&ctl->full[s], C::QC_BYTES);
+#pragma unroll
+        for (int kb = 0; kb < C::KB; ++kb)
+          tc::tma_load_2d(sQ + s * C::QC_BYTES + kb * BN * 128, &tm_q, kb * 64, qrow + c * BN, &ctl->full[s]);
+        issued = c + 1;
+      }
+      if (*abort_flag) {
+        drain_wait(&ctl->kfull, 0);
+        for (int c = *(volatile int*)&ctl->consumed; c < issued; ++c)
+          drain_wait(&ctl->full[c % C::QSTAGES], (c / C::QSTAGES) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_bf16(BM, BN);
+      bool ok = tc::mbar_wait(&ctl->kfull, 0, abort_flag, a.err);
+      bool issued_any = false;
+      for (int c = 0; ok && c < nch; ++c) {
+        const int s = c % C::QSTAGES;
+        const uint32_t ph = (c / C::QSTAGES) & 1;
+        if (!tc::mbar_wait(&ctl->full[s], ph, abort_flag, a.err)) break;
+        *(volatile int*)&ctl->consumed = c + 1;
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
+          if (!tc::mbar_wait(&ctl->accempty[blk], (c & 1) ^ 1, abort_flag, a.err)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t d = tmem + blk * BN;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = (k & 3) * 32;
+            const uint32_t ka = sK + (k >> 2) * 256 * 128 + blk * BM * 128 + off;
+            const uint32_t qa = sQ + s * C::QC_BYTES + (k >> 2) * BN * 128 + off;
+            tc::umma_bf16(d, tc::sdesc_sw128(ka), tc::sdesc_sw128(qa), idesc, k > 0 ? 1u : 0u);
+          }
+          issued_any = true;
+          tc::umma_commit(&ctl->accfull[blk]);
+        }
+        if (!ok) break;
+        tc::umma_commit(&ctl->empty[s]);
+      }
+      if (*abort_flag && issued_any) {
+        tc::umma_commit(&ctl->done);
+        drain_wait(&ctl->done, 0);
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int kl = q * 32 + lane;
+    const float sc = kLog2e * rsqrtf((float)D);
+    float acc[2] = {0.f, 0.f};
+    bool ok = true;
+    for (int c = 0; ok && c < nch; ++c) {
+#pragma unroll
+      for (int blk = 0; blk < 2; ++blk) {
+        if (!tc::mbar_wait_warp(&ctl->accfull[blk], c & 1, abort_flag, a.err)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + blk * BN;
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          uint32_t r[32];
+          __syncwarp();
+          tc::tmem_ld_x32(base + cc * 32, r);
+          tc::tmem_ld_wait(r);
+          const float2* mwc = mw + c * BN + cc * 32;
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float4 p = *reinterpret_cast<const float4*>(mwc + j);  // (m, w) of rows j, j+1
+            s0 += ex2(fmaf(__uint_as_float(r[j]), sc, -p.x)) * p.y;
+            s1 += ex2(fmaf(__uint_as_float(r[j + 1]), sc, -p.z)) * p.w;
+          }
+        }
+        acc[blk] += s0 + s1;
+        tc::fence_before_sync();
+        tc::mbar_arrive(&ctl->accempty[blk]);
+      }
+    }
+    if (ok && !*abort_flag) {
+      const float invM = 1.f / (float)M;
+#pragma unroll
+      for (int blk = 0; blk < 2; ++blk) {
+        const int n = key0 + blk * BM + kl;
+        if (n < nv) a.scores[(size_t)prob * a.nvis_max + n] = acc[blk] * invM;
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+// 2D bf16 tensor map: `rows` rows of `inner` elements, box of 64 x box_rows,
+// 128-byte swizzle (the layout the K-major shared-memory descriptors expect).
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D>
+static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s) {
+  const uint64_t krows = (uint64_t)a.L * a.B * a.Hkv * a.cap;
+  const uint64_t qrows = (uint64_t)a.L * a.B * a.Hq * a.T;
+  CUtensorMap tk, tq128, tq256;
+  if (!make_tmap_bf16_2d(&tk, a.k_full, D, krows, BN) || !make_tmap_bf16_2d(&tq128, a.q_text, D, qrows, BM) ||
+      !make_tmap_bf16_2d(&tq256, a.q_text, D, qrows, BN))
+    return cudaErrorNotSupported;
+  cudaError_t e = cudaFuncSetAttribute(rowstats_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, P1<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(colsum_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, P2<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  const int M = a.G * a.T;
+  rowstats_tc_kernel<D><<<dim3((M + BM - 1) / BM, a.Hkv, a.L * a.B), kThreads, P1<D>::SMEM, s>>>(tq128, tk, a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  colsum_tc_kernel<D><<<dim3((a.nvis_max + 255) / 256, a.Hkv, a.L * a.B), kThreads, P2<D>::SMEM, s>>>(tq256, tk, a);
+  return cudaGetLastError();
+}
+
+// tcgen05 path for bf16 operands; cudaErrorNotSupported for shapes it does not cover.
+cudaError_t launch_select_scores_tc(const ScoreArgs& a, cudaStream_t s) {
+  if (a.dtype != STD_BF16 || (a.d != 64 && a.d != 128)) return cudaErrorNotSupported;
+  if (a.G * a.T > kMaxRows) return cudaErrorNotSupported;
+  if ((uint64_t)a.L * a.B * a.Hkv * a.cap + 256 >= (1ull << 31)) return cudaErrorNotSupported;
+  if ((uint64_t)a.L * a.B * a.Hq * a.T + 256 >= (1ull << 31)) return cudaErrorNotSupported;
+  return a.d == 128 ? launch_tc<128>(a, s) : launch_tc<64>(a, s);
+}
+
+}  // namespace stdb

@@ -38,6 +38,10 @@ SELECT_CASES = {
     "ragged_bf16": small_wl("ragged_bf16", L=2, Bsz=3, nvis=(777, 1500, 64), T=33, K=64, wl_id=91),
     "d64_bf16_G1": small_wl("d64_bf16_G1", Hq=4, Hkv=4, d=64, nvis=(300,), T=7, K=300, wl_id=92),
     "f32_G4_K1": small_wl("f32_G4_K1", dtype="f32", Hq=8, Hkv=2, d=32, nvis=(513,), T=5, K=1, wl_id=93),
+    # more than 2048 text rows per KV head: the mma.sync fallback of the score passes
+    "rows2100_fallback": small_wl("rows2100_fallback", nvis=(700,), T=300, K=64, wl_id=102),
+    # ragged rows: G*T = 7*37 = 259 (two 128-row blocks, two 256-row chunks), ragged keys
+    "tc_ragged_rows": small_wl("tc_ragged_rows", L=2, Bsz=2, nvis=(1025, 300), T=37, K=100, wl_id=103),
 }
 
 

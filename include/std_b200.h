@@ -295,6 +295,15 @@ int std_decode_round(const std_dims* dims, int gamma, const std_cache* cache,
                      const std_round_io* io, int splits_draft, int splits_verify, void* ws,
                      size_t ws_bytes, std_stream_t stream);
 
+/* ---------------------------------------------------------------- test hook
+ *
+ * The selection kernels evaluate part of their exponentials with a polynomial
+ * on the FP32 pipe instead of the special-function unit.  This hook runs both
+ * on n device floats x (x <= 0): y_fma[i] = the polynomial 2^x[i], y_sfu[i] =
+ * the special-function unit's 2^x[i], so tests can bound the polynomial's
+ * error.  Not a step of the method. */
+int std_probe_exp2(const float* x, float* y_fma, float* y_sfu, int n, std_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -76,6 +76,7 @@ SIGNATURES = {
     "std_kv_append": (_I, [_DP, _P, _P, _I64, _P, _I, _P, _P, _I, _P]),
     "std_kv_commit": (_I, [_DP, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
     "std_round_workspace_size": (_SZ, [_DP, _I, _I, _I]),
+    "std_probe_exp2": (_I, [_P, _P, _P, _I, _P]),
     "std_decode_round": (_I, [_DP, _I, ctypes.POINTER(StdCache), ctypes.POINTER(StdRoundIO), _I, _I,
                               _P, _SZ, _P]),
 }
@@ -239,3 +240,7 @@ def std_decode_round(d: StdDims, gamma, cache: dict, io: dict, splits_draft=0, s
     r = StdRoundIO(*[_ptr(io[f]) for f, _ in StdRoundIO._fields_])
     _check(lib().std_decode_round(ctypes.byref(d), gamma, ctypes.byref(c), ctypes.byref(r), splits_draft,
                                   splits_verify, _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def std_probe_exp2(x, y_fma, y_sfu, stream=None) -> None:
+    _check(lib().std_probe_exp2(_ptr(x), _ptr(y_fma), _ptr(y_sfu), x.numel(), _stream(stream)))

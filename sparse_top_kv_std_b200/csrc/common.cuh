@@ -64,6 +64,28 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, for x <= 0 (used beside ex2() to split the exponential
+// work between the special-function unit and the FP32 pipe).  Method: round
+// x to the nearest integer j with the 1.5 * 2^23 shifter (Cody-Waite style
+// reduction, f = x - j in [-1/2, 1/2]), evaluate 2^f = e^(f ln 2) with its
+// Taylor series to degree 6 (truncation error below 1.2e-7 relative), then add
+// j to the exponent field.  Inputs below -125 are clamped (result ~2e-38, far
+// below anything that matters next to the row maximum's 2^0).
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;
+  const float j = t - 12582912.f;
+  const float f = x - j;
+  float p = 1.5403530393381606e-4f;
+  p = fmaf(p, f, 1.3333558146428441e-3f);
+  p = fmaf(p, f, 9.618129107628477e-3f);
+  p = fmaf(p, f, 5.5504108664821576e-2f);
+  p = fmaf(p, f, 2.402265069591007e-1f);
+  p = fmaf(p, f, 6.931471805599453e-1f);
+  p = fmaf(p, f, 1.f);
+  return __int_as_float(__float_as_int(p) + (int)((uint32_t)(__float_as_int(t) - 0x4B400000) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

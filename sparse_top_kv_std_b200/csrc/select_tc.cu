@@ -13,8 +13,12 @@
 // Pass 2: transposed.  CTA = 256 keys (two 128-key MMA tiles, M axis) kept in
 //   shared memory; the text rows stream through as 256-row chunks (N axis);
 //   each epilogue thread owns one key and sums its column in registers.
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
-// issuer (one elected lane), warps 2-5 epilogue (TMEM lane quarter = warp % 4).
+// Warp roles (320 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
+// issuer (one elected lane), warps 2-9 epilogue in two warpgroups that split
+// each accumulator's columns (TMEM lane quarter = warp % 4), so every SM
+// sub-partition has two epilogue warps to hide the TMEM-load latency, which
+// is pipelined one 32-column chunk ahead.  A quarter of the exponentials run
+// as a polynomial on the FMA pipe (exp2_fma) beside the special-function unit.
 // Every wait is bounded; on a timeout the CTA raises its abort flag, records
 // the error, lets in-flight copies and MMAs finish (bounded), frees TMEM and
 // returns.  No multicast loads are used.
@@ -31,11 +35,15 @@
 namespace stdb {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int BM = 128;      // MMA M
 constexpr int BN = 256;      // MMA N (keys in pass 1, text rows in pass 2)
 constexpr int kMaxRows = 2048;  // G * T supported by pass 2 (row statistics kept in shared memory)
 constexpr int kTmemCols = 512;
+constexpr int kHalf = BN / 2;   // accumulator columns per epilogue warpgroup
+constexpr int kPolyLanes = 8;   // of every 32 exponentials, this many on the FMA pipe
 
 struct Ctl {
   uint64_t full[8], empty[8];
@@ -63,6 +71,78 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   while (!tc::mbar_try_wait(a, parity)) {
     if (tc::globaltimer() - t0 > tc::kWaitTimeoutNs) return;
   }
+}
+
+// Pass-1 epilogue on 32 logits of one row: online max / sum of 2^(x - m).
+template <bool TAIL>
+__device__ __forceinline__ void p1_chunk(const uint32_t (&r)[32], int key, int nv, float sc, float& m, float& l) {
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    v[j] = __uint_as_float(r[j]);
+    if (TAIL && key + j >= nv) v[j] = -INFINITY;
+  }
+  float cm = v[0];
+#pragma unroll
+  for (int j = 1; j < 32; ++j) cm = fmaxf(cm, v[j]);
+  if (cm == -INFINITY) return;  // every key of the chunk is past the visual tokens
+  if (cm > m) {
+    l *= ex2((m - cm) * sc);
+    m = cm;
+  }
+  const float msc = m * sc;
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+  for (int j = 0; j < kPolyLanes; j += 2) {
+    s0 += exp2_fma(fmaf(v[j], sc, -msc));
+    s1 += exp2_fma(fmaf(v[j + 1], sc, -msc));
+  }
+#pragma unroll
+  for (int j = kPolyLanes; j < 32; j += 2) {
+    s2 += ex2(fmaf(v[j], sc, -msc));
+    s3 += ex2(fmaf(v[j + 1], sc, -msc));
+  }
+  l += (s0 + s1) + (s2 + s3);
+}
+
+// Pass-2 epilogue on 32 logits of one key: sum_r 2^(x_r - m_r) w_r, (m, w) from shared memory.
+__device__ __forceinline__ float p2_chunk(const uint32_t (&r)[32], const float2* mw, float sc) {
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+  for (int j = 0; j < kPolyLanes; j += 2) {
+    const float4 p = *reinterpret_cast<const float4*>(mw + j);
+    s0 += exp2_fma(fmaf(__uint_as_float(r[j]), sc, -p.x)) * p.y;
+    s1 += exp2_fma(fmaf(__uint_as_float(r[j + 1]), sc, -p.z)) * p.w;
+  }
+#pragma unroll
+  for (int j = kPolyLanes; j < 32; j += 2) {
+    const float4 p = *reinterpret_cast<const float4*>(mw + j);
+    s2 += ex2(fmaf(__uint_as_float(r[j]), sc, -p.x)) * p.y;
+    s3 += ex2(fmaf(__uint_as_float(r[j + 1]), sc, -p.z)) * p.w;
+  }
+  return (s0 + s1) + (s2 + s3);
+}
+
+// Four 32-column TMEM chunks at `base`, each load issued one chunk ahead of its use.
+template <typename F>
+__device__ __forceinline__ void tmem_sweep4(uint32_t base, F&& use) {
+  uint32_t ra[32], rb[32];
+  __syncwarp();
+  tc::tmem_ld_x32(base, ra);
+  tc::tmem_ld_wait(ra);
+  __syncwarp();
+  tc::tmem_ld_x32(base + 32, rb);
+  use(ra, 0);
+  tc::tmem_ld_wait(rb);
+  __syncwarp();
+  tc::tmem_ld_x32(base + 64, ra);
+  use(rb, 1);
+  tc::tmem_ld_wait(ra);
+  __syncwarp();
+  tc::tmem_ld_x32(base + 96, rb);
+  use(ra, 2);
+  tc::tmem_ld_wait(rb);
+  use(rb, 3);
 }
 
 template <int D>
@@ -106,7 +186,7 @@ rowstats_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tc::mbar_init(&ctl->done, 1);
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&ctl->accfull[i], 1);
-      tc::mbar_init(&ctl->accempty[i], 128);
+      tc::mbar_init(&ctl->accempty[i], kEpiThreads);
     }
     ctl->abort_flag = 0;
     ctl->consumed = 0;
@@ -180,60 +260,29 @@ rowstats_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       }
     }
   } else {
-    const int q = warp & 3;
+    const int g = (warp - 2) >> 2;  // warpgroup: which half of the 256 columns
+    const int q = warp & 3;         // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;
     const float sc = kLog2e * rsqrtf((float)D);
     float m = -INFINITY, l = 0.f;
-    bool ok = true;
     for (int t = 0; t < ntiles; ++t) {
       const int buf = t & 1;
       const uint32_t aph = (t >> 1) & 1;
-      if (!tc::mbar_wait_warp(&ctl->accfull[buf], aph, abort_flag, a.err)) {
-        ok = false;
-        break;
-      }
+      if (!tc::mbar_wait_warp(&ctl->accfull[buf], aph, abort_flag, a.err)) break;
       tc::fence_after_sync();
-      const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + buf * BN;
-      const int key0 = t * BN;
-      const bool tail = key0 + BN > nv;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        __syncwarp();
-        tc::tmem_ld_x32(base + c * 32, r);
-        tc::tmem_ld_wait(r);
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-        if (tail) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (key0 + c * 32 + j >= nv) v[j] = -INFINITY;
-        }
-        float cm = v[0];
-#pragma unroll
-        for (int j = 1; j < 32; ++j) cm = fmaxf(cm, v[j]);
-        if (cm > m) {
-          l *= ex2((m - cm) * sc);
-          m = cm;
-        }
-        const float msc = m * sc;
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          s0 += ex2(fmaf(v[j], sc, -msc));
-          s1 += ex2(fmaf(v[j + 1], sc, -msc));
-        }
-        l += s0 + s1;
+      const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + buf * BN + g * kHalf;
+      const int key0 = t * BN + g * kHalf;
+      if (t * BN + BN > nv) {
+        tmem_sweep4(base, [&](const uint32_t(&r)[32], int c) { p1_chunk<true>(r, key0 + c * 32, nv, sc, m, l); });
+      } else {
+        tmem_sweep4(base, [&](const uint32_t(&r)[32], int c) { p1_chunk<false>(r, key0 + c * 32, nv, sc, m, l); });
       }
       tc::fence_before_sync();
       tc::mbar_arrive(&ctl->accempty[buf]);
     }
-    const int r_glob = blockIdx.x * BM + row;
-    if (ok && !*abort_flag && r_glob < M) {
-      a.row_m[(size_t)prob * M + r_glob] = m * sc;
-      a.row_l[(size_t)prob * M + r_glob] = l;
-    }
+    // every MMA has completed once the last accumulator was read: the Q tile is free
+    float2* part = reinterpret_cast<float2*>(smem);
+    part[g * BM + row] = make_float2(m * sc, l);
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -241,6 +290,18 @@ rowstats_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     __syncwarp();
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
+  } else if (warp >= 2 && warp < 6 && !*abort_flag) {
+    // merge the two column halves of each row: (m, l) in the exp2 domain
+    const int row = (warp & 3) * 32 + lane;
+    const int r_glob = blockIdx.x * BM + row;
+    const float2* part = reinterpret_cast<const float2*>(smem);
+    const float2 p0 = part[row], p1 = part[BM + row];
+    const float mm = fmaxf(p0.x, p1.x);
+    const float ll = (p0.y > 0.f ? p0.y * ex2(p0.x - mm) : 0.f) + (p1.y > 0.f ? p1.y * ex2(p1.x - mm) : 0.f);
+    if (r_glob < M) {
+      a.row_m[(size_t)prob * M + r_glob] = mm;
+      a.row_l[(size_t)prob * M + r_glob] = ll;
+    }
   }
 }
 
@@ -291,7 +352,7 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     tc::mbar_init(&ctl->done, 1);
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&ctl->accfull[i], 1);
-      tc::mbar_init(&ctl->accempty[i], 128);
+      tc::mbar_init(&ctl->accempty[i], kEpiThreads);
     }
     ctl->abort_flag = 0;
     ctl->consumed = 0;
@@ -371,6 +432,7 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
     }
   } else {
+    const int g = (warp - 2) >> 2;
     const int q = warp & 3;
     const int kl = q * 32 + lane;
     const float sc = kLog2e * rsqrtf((float)D);
@@ -384,35 +446,19 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           break;
         }
         tc::fence_after_sync();
-        const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + blk * BN;
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll 1
-        for (int cc = 0; cc < BN / 32; ++cc) {
-          uint32_t r[32];
-          __syncwarp();
-          tc::tmem_ld_x32(base + cc * 32, r);
-          tc::tmem_ld_wait(r);
-          const float2* mwc = mw + c * BN + cc * 32;
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float4 p = *reinterpret_cast<const float4*>(mwc + j);  // (m, w) of rows j, j+1
-            s0 += ex2(fmaf(__uint_as_float(r[j]), sc, -p.x)) * p.y;
-            s1 += ex2(fmaf(__uint_as_float(r[j + 1]), sc, -p.z)) * p.w;
-          }
-        }
-        acc[blk] += s0 + s1;
+        const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + blk * BN + g * kHalf;
+        const float2* mwc = mw + c * BN + g * kHalf;
+        float s = 0.f;
+        tmem_sweep4(base, [&](const uint32_t(&r)[32], int cc) { s += p2_chunk(r, mwc + cc * 32, sc); });
+        acc[blk] += s;
         tc::fence_before_sync();
         tc::mbar_arrive(&ctl->accempty[blk]);
       }
     }
-    if (ok && !*abort_flag) {
-      const float invM = 1.f / (float)M;
-#pragma unroll
-      for (int blk = 0; blk < 2; ++blk) {
-        const int n = key0 + blk * BM + kl;
-        if (n < nv) a.scores[(size_t)prob * a.nvis_max + n] = acc[blk] * invM;
-      }
-    }
+    // every MMA has completed once the last accumulator was read: the Q stages are free
+    float* part = reinterpret_cast<float*>(smem + C::K_BYTES);
+    part[(g * 2 + 0) * BM + kl] = acc[0];
+    part[(g * 2 + 1) * BM + kl] = acc[1];
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -420,6 +466,15 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncwarp();
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
+  } else if (warp >= 2 && warp < 6 && !*abort_flag) {
+    const int kl = (warp & 3) * 32 + lane;
+    const float* part = reinterpret_cast<const float*>(smem + C::K_BYTES);
+    const float invM = 1.f / (float)M;
+#pragma unroll
+    for (int blk = 0; blk < 2; ++blk) {
+      const int n = key0 + blk * BM + kl;
+      if (n < nv) a.scores[(size_t)prob * a.nvis_max + n] = (part[blk * BM + kl] + part[(2 + blk) * BM + kl]) * invM;
+    }
   }
 }
 

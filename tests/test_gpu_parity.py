@@ -348,3 +348,24 @@ def test_decode_rounds_match_oracle(name):
     np.testing.assert_array_equal(ksp_g[same], state["k_sp"][same])
     np.testing.assert_array_equal(ksp_g[..., wl.K:, :], state["k_sp"][..., wl.K:, :])
     np.testing.assert_array_equal(H.f64(H.to_host_bits(s.v_full), wl), state["v_full"])
+
+
+# ----------------------------------------------------------------------------- FMA-pipe exponential
+
+def test_exp2_polynomial_error_bound():
+    """The polynomial 2^x used beside the special-function unit: relative error
+    against float64 exp2 within 4e-7 on x in [-125, 0], and no worse than the
+    SFU's own ex2.approx by more than that."""
+    x = np.concatenate([-np.linspace(0.0, 125.0, 1 << 20), -np.random.default_rng(0).random(1 << 16) * 30,
+                        np.array([0.0, -0.5, -1e-8, -0.49999997, -124.99])]).astype(np.float32)
+    xd = torch.from_numpy(x).cuda()
+    yf = torch.empty_like(xd)
+    ys = torch.empty_like(xd)
+    B.std_probe_exp2(xd, yf, ys)
+    torch.cuda.synchronize()
+    ref = np.exp2(x.astype(np.float64))
+    rel_f = np.abs(yf.cpu().numpy() - ref) / ref
+    rel_s = np.abs(ys.cpu().numpy() - ref) / ref
+    assert rel_f.max() < 4e-7, rel_f.max()
+    assert rel_f.mean() < 1e-7
+    assert rel_s.max() < 4e-7     # the SFU reference the polynomial stands beside

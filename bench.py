@@ -356,11 +356,14 @@ def run_std(args, rank, world, local_rank):
     nvis_dev = torch.tensor(list(wl.nvis), dtype=torch.int32, device=dev)
     sess.nvis.copy_(nvis_dev)
     outs = [sess.round_outputs() for _ in range(R)]
-    sp_d = B.std_attn_splits(sess.dims, wl.cap_sparse, 0) if wl.gamma > 0 else 1
-    sp_v = B.std_attn_splits(sess.dims, wl.cap_full, 0)
+    sp_d = B.std_attn_splits(sess.dims, 1, wl.cap_sparse, 0) if wl.gamma > 0 else 1
+    sp_v = B.std_attn_splits(sess.dims, wl.gamma + 1, wl.cap_full, 0)
     ws = sess.ws_round
     q_text = view("q_text")
-    launches_per_step = 4 + R * (wl.gamma * (2 + (sp_d > 1)) + 2 + (sp_v > 1) + 1 + 2)
+    # per attention call: the attention kernel plus its merge kernel (none for a single fp32 split)
+    merge_d = 1 if (dt == B.STD_BF16 or sp_d > 1) else 0
+    merge_v = 1 if (dt == B.STD_BF16 or sp_v > 1) else 0
+    launches_per_step = 4 + R * (wl.gamma * (2 + merge_d) + 2 + merge_v + 1 + 2)
 
     def step(ev=None):
         """One StD decode: reset lengths, select, R rounds.  ev: dict of event lists to record."""
@@ -378,7 +381,7 @@ def run_std(args, rank, world, local_rank):
                 if ev is not None:
                     ev["d0"][r * wl.gamma + j].record(stream)
                 B.std_sparse_decode_attn(sess.dims, view("q_draft", r)[j], sess.k_sparse, sess.v_sparse,
-                                         sess.len_sparse, j + 1, o["o_draft"][j], sp_d, ws)
+                                         sess.len_sparse, j + 1, o["o_draft"][j], 0, ws)
                 if ev is not None:
                     ev["d1"][r * wl.gamma + j].record(stream)
             B.std_kv_append(sess.dims, sess.k_full, sess.v_full, wl.cap_full, sess.len_full, 0,
@@ -386,7 +389,7 @@ def run_std(args, rank, world, local_rank):
             if ev is not None:
                 ev["v0"][r].record(stream)
             B.std_dense_verify_attn(sess.dims, view("q_verify", r), wl.gamma, sess.k_full, sess.v_full,
-                                    sess.len_full, o["o_verify"], sp_v, ws)
+                                    sess.len_full, o["o_verify"], 0, ws)
             if ev is not None:
                 ev["v1"][r].record(stream)
             B.std_accept_prefix(wl.B, wl.gamma, dv["draft_tokens"][r], dv["dense_tokens"][r], o["n_plus_1"],
@@ -500,10 +503,10 @@ def run_std(args, rank, world, local_rank):
         "select_ms": sel_avg,
         "kernels": {
             "dense_verify_attn": {"ms_per_launch": v_avg_ms, "bytes_per_launch": v_bytes_avg,
-                                  "GBps": achieved, "frac_of_8TBps": achieved / 8000.0, "splits": sp_v},
+                                  "GBps": achieved, "frac_of_8TBps": achieved / 8000.0, "ctas": sp_v},
             "sparse_decode_attn": {"us_per_launch": 1e3 * d_avg_ms, "bytes_per_launch": d_bytes_avg,
                                    "GBps": d_bytes_avg / (d_avg_ms / 1e3) / 1e9,
-                                   "frac_of_8TBps": d_bytes_avg / (d_avg_ms / 1e3) / 8e12, "splits": sp_d},
+                                   "frac_of_8TBps": d_bytes_avg / (d_avg_ms / 1e3) / 8e12, "ctas": sp_d},
             "select_topk": {"ms_per_launch": sel_avg, "mma_TFLOPs": select_flops(wl) / (sel_avg / 1e3) / 1e12,
                             "one_pass_TFLOPs": 0.5 * select_flops(wl) / (sel_avg / 1e3) / 1e12},
         },

@@ -140,26 +140,28 @@ int std_topk_from_scores(const float* scores, int rows, int n, int K, int32_t* i
 
 /* ---------------------------------------------------------------- decode attention
  *
- * Split-K flash decoding: the key range of each (layer, sequence, KV head) is
- * cut into `splits` pieces processed by separate CTAs; the G query heads of a
- * KV head (times the query rows) share one tile so each K/V byte is read once.
- * splits = 0 picks a split count from the device's SM count.  Partial results
- * go to the workspace and are merged by a second kernel.
+ * All query rows that read one KV head -- the G grouped query heads times the
+ * query positions -- are processed together, so each K/V byte is read once.
+ * bf16 operands (head dim 64 or 128, G x query rows <= 128, B <= 64) run on a
+ * persistent tensor-core kernel: the 128-key tiles of all (layer, sequence, KV
+ * head) problems form one sequence that the CTAs split into equal slices;
+ * `splits` = 0 launches one CTA per SM, splits = s > 0 launches
+ * s x L x B x Hkv CTAs.  fp32 operands (and bf16 with B > 64) use split-K
+ * kernels with `splits` key ranges per problem (0 = automatic).  Either way
+ * the partial results go to the workspace and a second kernel merges them.
  */
 
 /* Device workspace bytes for a decode-attention call with `q_rows` query rows
  * per query head (1 for the sparse draft, gamma + 1 for the verify) over a
  * cache of `cap` rows (dims->cap_sparse for the draft, dims->cap_full for the
- * verify), and `splits` (0 = the automatic choice, which depends on the number
- * of (layer, sequence, KV head) problems, `cap` and the current device's SM
- * count).  Returns 0 when no workspace is needed or the arguments are invalid. */
+ * verify), and `splits` as above (0 resolves on the current device).  Returns
+ * 0 when the arguments are invalid. */
 size_t std_attn_workspace_size(const std_dims* dims, int q_rows, int64_t cap, int splits);
 
-/* The split count a decode-attention call over a cache of `cap` rows will use
- * for `splits` (0 = automatic; resolved on the current device), or a negative
- * STD_ERR_* code.  With more than one split the call launches a second
- * (merge) kernel. */
-int std_attn_splits(const std_dims* dims, int64_t cap, int splits);
+/* The number of CTAs (tensor-core kernel) or key splits per problem (split-K
+ * kernels) a decode-attention call with these arguments uses, or a negative
+ * STD_ERR_* code. */
+int std_attn_splits(const std_dims* dims, int q_rows, int64_t cap, int splits);
 
 /*
  * Sparse draft attention ("Methodik" item 2: the draft model M_s uses top-K

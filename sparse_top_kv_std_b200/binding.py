@@ -68,7 +68,7 @@ SIGNATURES = {
     "std_select_topk": (_I, [_DP, _P, _I, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "std_topk_from_scores": (_I, [_P, _I, _I, _I, _P, _P]),
     "std_attn_workspace_size": (_SZ, [_DP, _I, _I64, _I]),
-    "std_attn_splits": (_I, [_DP, _I64, _I]),
+    "std_attn_splits": (_I, [_DP, _I, _I64, _I]),
     "std_sparse_decode_attn": (_I, [_DP, _P, _P, _P, _P, _I, _P, _I, _P, _SZ, _P]),
     "std_dense_verify_attn": (_I, [_DP, _P, _I, _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "std_dense_verify_attn_noalloc": (_I, [_DP, _P, _I, _P, _P, _P, _P, _I, _P]),
@@ -183,8 +183,8 @@ def std_attn_workspace_size(d: StdDims, q_rows: int, cap: int, splits: int) -> i
     return lib().std_attn_workspace_size(ctypes.byref(d), q_rows, cap, splits)
 
 
-def std_attn_splits(d: StdDims, cap: int, splits: int = 0) -> int:
-    rc = lib().std_attn_splits(ctypes.byref(d), cap, splits)
+def std_attn_splits(d: StdDims, q_rows: int, cap: int, splits: int = 0) -> int:
+    rc = lib().std_attn_splits(ctypes.byref(d), q_rows, cap, splits)
     if rc < 0:
         _check(rc)
     return rc

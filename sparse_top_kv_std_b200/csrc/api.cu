@@ -107,7 +107,7 @@ int check_ptr(const void* p, size_t align, const char* name) {
 int probs_of(const std_dims* d) { return d->L * d->B * d->Hkv; }
 
 int auto_splits(int probs, int64_t cap, int sm_count) {
-  // about 8 CTAs per SM over the whole grid, at least 256 keys per split
+  // split-K kernels: about 8 CTAs per SM over the whole grid, at least 256 keys per split
   int s = (sm_count * 8 + probs - 1) / probs;
   const int64_t by_len = cap / 256;
   if (s > by_len) s = (int)by_len;
@@ -116,43 +116,62 @@ int auto_splits(int probs, int64_t cap, int sm_count) {
   return s;
 }
 
-int resolve_splits(int splits, int probs, int64_t cap, int* out) {
-  if (splits < 0 || splits > 1024) return fail(STD_ERR_INVALID_ARG, "splits %d out of range [0, 1024]", splits);
-  if (splits > 0) {
-    *out = splits;
-    return STD_OK;
-  }
-  int sms;
-  STD_TRY(device_state(nullptr, &sms));
-  *out = auto_splits(probs, cap, sms);
-  return STD_OK;
-}
+// Launch plan of one decode-attention call: which kernel, how many splits / CTAs,
+// how much workspace.  The same function sizes the workspace and runs the call.
+struct AttnPlan {
+  stdb::AttnArgs a;
+  bool tc;
+  size_t ws_bytes;
+};
 
-size_t attn_ws_bytes(const std_dims* d, int q_rows, int splits) {
-  return stdb::attn_ws_floats(probs_of(d), splits, (d->Hq / d->Hkv) * q_rows, d->d, d->dtype) * sizeof(float);
+int plan_attn(const std_dims* dims, int nq, int64_t cap, int splits, AttnPlan* p) {
+  if (splits < 0 || splits > 1024) return fail(STD_ERR_INVALID_ARG, "splits %d out of range [0, 1024]", splits);
+  const int G = dims->Hq / dims->Hkv;
+  stdb::AttnArgs& a = p->a;
+  a = stdb::AttnArgs{};
+  a.L = dims->L; a.B = dims->B; a.Hq = dims->Hq; a.Hkv = dims->Hkv; a.G = G; a.nq = nq; a.rows = G * nq;
+  a.d = dims->d; a.dtype = dims->dtype; a.cap = cap;
+  if (dims->dtype == STD_BF16 && a.rows > 128)
+    return fail(STD_ERR_UNSUPPORTED, "G * query rows = %d exceeds 128", a.rows);
+  const int probs = probs_of(dims);
+  p->tc = stdb::attn_tc_supported(a);
+  if (p->tc) {
+    int ctas = splits;
+    if (splits > 0) {
+      const int64_t want = (int64_t)splits * probs;
+      ctas = (int)(want > 65535 ? 65535 : want);
+    } else {
+      STD_TRY(device_state(nullptr, &ctas));  // one persistent CTA per SM
+    }
+    a.splits = ctas;
+    p->ws_bytes = stdb::attn_tc_ws_floats(probs, ctas, a.rows, a.d) * sizeof(float);
+  } else {
+    int sp = splits;
+    if (sp == 0) {
+      int sms;
+      STD_TRY(device_state(nullptr, &sms));
+      sp = auto_splits(probs, cap, sms);
+    }
+    a.splits = sp;
+    p->ws_bytes = stdb::attn_ws_floats(probs, sp, a.rows, a.d, a.dtype) * sizeof(float);
+  }
+  return STD_OK;
 }
 
 int run_attn(const std_dims* dims, const void* q, const void* k, const void* v, int64_t cap,
              const int32_t* len, int len_off, int nq, float* o, int splits, void* ws, size_t ws_bytes,
              cudaStream_t stream) {
-  const int G = dims->Hq / dims->Hkv;
-  const int rows = G * nq;
-  if (dims->dtype == STD_BF16 && rows > 128)
-    return fail(STD_ERR_UNSUPPORTED, "G * query rows = %d exceeds 128", rows);
-  int sp;
-  STD_TRY(resolve_splits(splits, probs_of(dims), cap, &sp));
-  const size_t need = attn_ws_bytes(dims, nq, sp);
-  if (need > 0 && (!ws || ws_bytes < need))
-    return fail(STD_ERR_WORKSPACE, "attention workspace: need %zu bytes, got %zu", need, ws ? ws_bytes : 0);
-  if (need > 0) STD_TRY(check_ptr(ws, 16, "ws"));
+  AttnPlan p;
+  STD_TRY(plan_attn(dims, nq, cap, splits, &p));
+  if (p.ws_bytes > 0 && (!ws || ws_bytes < p.ws_bytes))
+    return fail(STD_ERR_WORKSPACE, "attention workspace: need %zu bytes, got %zu", p.ws_bytes, ws ? ws_bytes : 0);
+  if (p.ws_bytes > 0) STD_TRY(check_ptr(ws, 16, "ws"));
   int* err;
   STD_TRY(device_state(&err, nullptr));
-  stdb::AttnArgs a{};
+  stdb::AttnArgs& a = p.a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.len = len; a.len_off = len_off;
-  a.L = dims->L; a.B = dims->B; a.Hq = dims->Hq; a.Hkv = dims->Hkv; a.G = G; a.nq = nq; a.rows = rows;
-  a.d = dims->d; a.dtype = dims->dtype; a.cap = cap; a.splits = sp;
   a.ws = static_cast<float*>(ws); a.err = err;
-  cudaError_t e = stdb::launch_decode_attn(a, stream);
+  cudaError_t e = p.tc ? stdb::launch_decode_attn_tc(a, stream) : stdb::launch_decode_attn(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
   return ok();
 }
@@ -251,18 +270,18 @@ int std_topk_from_scores(const float* scores, int rows, int n, int K, int32_t* i
 
 size_t std_attn_workspace_size(const std_dims* dims, int q_rows, int64_t cap, int splits) {
   if (check_dims(dims) || q_rows < 1 || cap < 1) return 0;
-  int sp;
-  if (resolve_splits(splits, probs_of(dims), cap, &sp)) return 0;
-  return attn_ws_bytes(dims, q_rows, sp);
+  AttnPlan p;
+  if (plan_attn(dims, q_rows, cap, splits, &p)) return 0;
+  return p.ws_bytes;
 }
 
-int std_attn_splits(const std_dims* dims, int64_t cap, int splits) {
+int std_attn_splits(const std_dims* dims, int q_rows, int64_t cap, int splits) {
   STD_TRY(check_dims(dims));
-  if (cap < 1) return fail(STD_ERR_INVALID_ARG, "cap = %lld", (long long)cap);
-  int sp;
-  STD_TRY(resolve_splits(splits, probs_of(dims), cap, &sp));
+  if (cap < 1 || q_rows < 1) return fail(STD_ERR_INVALID_ARG, "cap = %lld, q_rows = %d", (long long)cap, q_rows);
+  AttnPlan p;
+  STD_TRY(plan_attn(dims, q_rows, cap, splits, &p));
   ok();
-  return sp;
+  return p.a.splits;
 }
 
 int std_sparse_decode_attn(const std_dims* dims, const void* q, const void* k_sparse, const void* v_sparse,
@@ -422,14 +441,14 @@ extern "C" int std_dense_verify_attn_noalloc(const std_dims* dims, const void* q
   STD_TRY(check_ptr(len_full, 4, "len_full"));
   STD_TRY(check_ptr(o, 16, "o"));
   if (gamma < 0 || gamma > 31) return fail(STD_ERR_INVALID_ARG, "gamma = %d must be in [0, 31]", gamma);
-  int sp;
-  STD_TRY(resolve_splits(splits, probs_of(dims), dims->cap_full, &sp));
-  const size_t need = attn_ws_bytes(dims, gamma + 1, sp);
+  AttnPlan plan;
+  STD_TRY(plan_attn(dims, gamma + 1, dims->cap_full, splits, &plan));
+  const size_t need = plan.ws_bytes;
   if (need > STD_NOALLOC_SCRATCH_BYTES)
     return fail(STD_ERR_WORKSPACE, "verify partials need %zu bytes of scratch; the built-in array holds %u "
                 "(use fewer splits or std_dense_verify_attn with a workspace)", need, STD_NOALLOC_SCRATCH_BYTES);
   float* scratch = nullptr;
   if (need > 0) STD_TRY(noalloc_scratch(&scratch));
-  return run_attn(dims, q, k_full, v_full, dims->cap_full, len_full, 1, gamma + 1, o, sp, scratch,
+  return run_attn(dims, q, k_full, v_full, dims->cap_full, len_full, 1, gamma + 1, o, splits, scratch,
                   need > 0 ? STD_NOALLOC_SCRATCH_BYTES : 0, stream);
 }

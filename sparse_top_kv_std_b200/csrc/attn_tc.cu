@@ -1,0 +1,539 @@
+// Decode attention on the 5th-generation tensor cores for the sparse draft and
+// the dense verify of Sparse-to-Dense decoding ("Methodik" items 2 and 3 of
+// the gist.science summary: the draft attends to the selected top-K KV, the
+// verifier attends to the whole cache with gamma + 1 query positions in one
+// pass).  bf16 operands, fp32 accumulation, fp32 softmax.
+//
+// Layout of the work.  A problem is one (layer, sequence, KV head); all query
+// rows that read it -- the G grouped query heads times the nq query positions,
+// at most 128 -- form the M = 128 side of every MMA, so each K/V byte crosses
+// HBM once.  The keys of all problems, cut into 128-key tiles, form one flat
+// sequence; a persistent grid of CTAs (one per SM by default) takes equal
+// contiguous slices of it (stream-K), so the load is balanced whatever the
+// lengths.  A CTA writes one partial (m, l, o) per run of tiles of the same
+// problem ("segment"), into slot problem + cta; a merge kernel combines the
+// slots of each problem.
+//
+// Per tile, inside a CTA (warp 0: TMA producer; warp 1: TMEM owner and MMA
+// issuer; warps 2-5: one thread per query row):
+//   TMA        K tile and V tile (128 keys x d, 128-byte swizzle) -> stage ring
+//   MMA        S = Q K^T  -> TMEM S buffer (double-buffered, 128 fp32 columns)
+//   softmax    row max, lazy rescale of O (only when the max grows by more than
+//              2^8), P = 2^(x - m) as bf16 written back over S in TMEM
+//   MMA        O += P V   (A = P from TMEM, B = V from shared memory, MN-major)
+// At the end of a segment the row threads read O from TMEM and write the partial.
+// Every wait is bounded; a timeout flags the device error word and unwinds.
+#include <cuda.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc100.cuh"
+
+namespace stdb {
+namespace {
+
+constexpr int TK = 128;           // keys per tile
+constexpr int kThreads = 192;
+constexpr int STAGES = 3;
+constexpr int kMaxB = 64;         // sequences per call handled by this kernel
+constexpr int kTmemCols = 512;
+constexpr uint32_t kColS = 128;   // TMEM column of S/P buffer 0 (buffer 1 at 256); O at column 0
+constexpr float kTau = 8.f;       // log2 growth of a row max that forces an O rescale
+
+struct Ctl {
+  uint64_t kv_full[STAGES], kv_empty[STAGES];
+  uint64_t q_full, q_empty, done;
+  uint64_t s_full[2], p_full[2], s_free[2];
+  uint64_t o_ready, o_free;
+  uint32_t tmem;
+  int abort_flag;
+  int consumed;
+  int tl;      // tiles per layer
+  int total;   // tiles of the whole call
+  int per;     // tiles per CTA
+  int tiles_b[kMaxB];
+};
+
+// Tiles of sequence b (0 for an invalid length, which is flagged).
+__device__ __forceinline__ int seq_tiles(const AttnArgs& a, int b, bool flag) {
+  const int base = a.len[b] + a.len_off;
+  const int lim_max = base + a.nq - 1;
+  if (base <= 0 || (int64_t)lim_max > a.cap) {
+    if (flag) flag_error(a.err, STD_DEVERR_LENGTH);
+    return 0;
+  }
+  return (lim_max + TK - 1) / TK;
+}
+
+// Walk over this CTA's slice of the flat (problem, tile) sequence.
+struct Iter {
+  int g, g_end;
+  int l, b, h, t, nt;
+  bool first;  // first tile of a segment
+};
+
+__device__ __forceinline__ void iter_seek(Iter& it, const Ctl* c, const AttnArgs& a, int g0, int g1) {
+  it.g = g0;
+  it.g_end = g1;
+  it.first = true;
+  it.l = it.b = it.h = it.t = 0;
+  it.nt = 1;
+  if (g0 >= g1) return;
+  it.l = g0 / c->tl;
+  int r = g0 % c->tl;
+  int b = 0;
+  while (r >= a.Hkv * c->tiles_b[b]) {
+    r -= a.Hkv * c->tiles_b[b];
+    ++b;
+  }
+  it.b = b;
+  it.nt = c->tiles_b[b];
+  it.h = r / it.nt;
+  it.t = r % it.nt;
+}
+
+__device__ __forceinline__ bool iter_last(const Iter& it) { return it.g + 1 == it.g_end || it.t + 1 == it.nt; }
+
+__device__ __forceinline__ void iter_next(Iter& it, const Ctl* c, const AttnArgs& a) {
+  if (++it.g >= it.g_end) return;
+  if (++it.t < it.nt) {
+    it.first = false;
+    return;
+  }
+  it.first = true;
+  it.t = 0;
+  if (++it.h < a.Hkv) return;
+  it.h = 0;
+  do {
+    if (++it.b == a.B) {
+      it.b = 0;
+      ++it.l;
+    }
+    it.nt = c->tiles_b[it.b];
+  } while (it.nt == 0);
+}
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t adr = smem_u32(bar);
+  const uint64_t t0 = tc::globaltimer();
+  while (!tc::mbar_try_wait(adr, parity)) {
+    if (tc::globaltimer() - t0 > tc::kWaitTimeoutNs) return;
+  }
+}
+
+template <int D>
+struct Cfg {
+  static constexpr int KB = D / 64;                   // 128-byte column blocks of a row
+  static constexpr uint32_t Q_BYTES = KB * 128 * 128;  // 128 query rows
+  static constexpr uint32_t T_BYTES = KB * TK * 128;   // one K or V tile
+  static constexpr uint32_t ST_BYTES = 2 * T_BYTES;    // K + V
+  static constexpr uint32_t SMEM = 1024 + Q_BYTES + STAGES * ST_BYTES + sizeof(Ctl);
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sQ = smem_u32(smem);
+  const uint32_t sKV = sQ + C::Q_BYTES;
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::Q_BYTES + STAGES * C::ST_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    int sum = 0;
+    for (int b = 0; b < a.B; ++b) {
+      ctl->tiles_b[b] = seq_tiles(a, b, blockIdx.x == 0);
+      sum += ctl->tiles_b[b];
+    }
+    ctl->tl = a.Hkv * sum;
+    ctl->total = a.L * ctl->tl;
+    ctl->per = ctl->total > 0 ? (ctl->total + gridDim.x - 1) / gridDim.x : 1;
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(&ctl->kv_full[s], 1);
+      tc::mbar_init(&ctl->kv_empty[s], 1);
+    }
+    tc::mbar_init(&ctl->q_full, 1);
+    tc::mbar_init(&ctl->q_empty, 1);
+    tc::mbar_init(&ctl->done, 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&ctl->s_full[i], 1);
+      tc::mbar_init(&ctl->p_full[i], 128);
+      tc::mbar_init(&ctl->s_free[i], 1);
+    }
+    tc::mbar_init(&ctl->o_ready, 1);
+    tc::mbar_init(&ctl->o_free, 128);
+    ctl->abort_flag = 0;
+    ctl->consumed = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tc::tmem_alloc(&ctl->tmem, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = ctl->tmem;
+  volatile int* abort_flag = &ctl->abort_flag;
+  const int g0 = min(ctl->total, (int)blockIdx.x * ctl->per);
+  const int g1 = min(ctl->total, g0 + ctl->per);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && g0 < g1) {
+      tc::prefetch_tmap(&tm_q);
+      tc::prefetch_tmap(&tm_k);
+      tc::prefetch_tmap(&tm_v);
+      Iter it;
+      iter_seek(it, ctl, a, g0, g1);
+      int seg = 0, kv = 0;
+      bool q_pending = false;
+      while (it.g < it.g_end) {
+        const int lb = it.l * a.B + it.b;
+        const int prob = lb * a.Hkv + it.h;
+        if (it.first) {
+          if (!tc::mbar_wait(&ctl->q_empty, (seg & 1) ^ 1, abort_flag, a.err)) break;
+          tc::mbar_expect_tx(&ctl->q_full, C::Q_BYTES);
+          const int qrow = (lb * a.Hq + it.h * a.G) * a.nq;
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb) tc::tma_load_2d(sQ + kb * 128 * 128, &tm_q, kb * 64, qrow, &ctl->q_full);
+          q_pending = true;
+          ++seg;
+        }
+        const int s = kv % STAGES;
+        if (!tc::mbar_wait(&ctl->kv_empty[s], ((kv / STAGES) & 1) ^ 1, abort_flag, a.err)) break;
+        tc::mbar_expect_tx(&ctl->kv_full[s], C::ST_BYTES);
+        const int row = prob * (int)a.cap + it.t * TK;
+        const uint32_t st = sKV + s * C::ST_BYTES;
+#pragma unroll
+        for (int kb = 0; kb < C::KB; ++kb) {
+          tc::tma_load_2d(st + kb * TK * 128, &tm_k, kb * 64, row, &ctl->kv_full[s]);
+          tc::tma_load_2d(st + C::T_BYTES + kb * TK * 128, &tm_v, kb * 64, row, &ctl->kv_full[s]);
+        }
+        ++kv;
+        iter_next(it, ctl, a);
+      }
+      if (*abort_flag) {  // let the copies in flight land
+        if (q_pending) drain_wait(&ctl->q_full, (seg - 1) & 1);
+        for (int k = *(volatile int*)&ctl->consumed; k < kv; ++k) drain_wait(&ctl->kv_full[k % STAGES], (k / STAGES) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && g0 < g1) {
+      constexpr uint32_t idS = tc::idesc_bf16(128, TK);
+      constexpr uint32_t idPV = tc::idesc_bf16(128, D) | (1u << 16);  // B = V, MN-major
+      Iter it;
+      iter_seek(it, ctl, a, g0, g1);
+      int seg = -1, kv = 0, u = 0;
+      int pu = -1, ps = 0, pseg = 0;
+      bool pfirst = false, any = false, ok = true;
+      auto issue_pv = [&](int vu, int vs, bool vfirst, bool vlast, int vseg) -> bool {
+        const int vb = vu & 1;
+        if (!tc::mbar_wait(&ctl->p_full[vb], (vu >> 1) & 1, abort_flag, a.err)) return false;
+        if (vfirst && !tc::mbar_wait(&ctl->o_free, (vseg & 1) ^ 1, abort_flag, a.err)) return false;
+        tc::fence_after_sync();
+        const uint32_t p_tm = tmem + kColS + vb * 128;
+        const uint32_t sv = sKV + vs * C::ST_BYTES + C::T_BYTES;
+#pragma unroll
+        for (int k = 0; k < TK / 16; ++k)
+          tc::umma_bf16_ts(tmem, p_tm + 8 * k, tc::sdesc_sw128_mn(sv + k * 16 * 128, TK * 128), idPV,
+                           (vfirst && k == 0) ? 0u : 1u);
+        tc::umma_commit(&ctl->kv_empty[vs]);
+        tc::umma_commit(&ctl->s_free[vb]);
+        if (vlast) tc::umma_commit(&ctl->o_ready);
+        return true;
+      };
+      while (it.g < it.g_end) {
+        const bool first = it.first, last = iter_last(it);
+        if (first) {
+          ++seg;
+          if (!tc::mbar_wait(&ctl->q_full, seg & 1, abort_flag, a.err)) { ok = false; break; }
+        }
+        const int s = kv % STAGES;
+        if (!tc::mbar_wait(&ctl->kv_full[s], (kv / STAGES) & 1, abort_flag, a.err)) { ok = false; break; }
+        *(volatile int*)&ctl->consumed = kv + 1;
+        const int bu = u & 1;
+        if (!tc::mbar_wait(&ctl->s_free[bu], ((u >> 1) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
+        tc::fence_after_sync();
+        const uint32_t s_tm = tmem + kColS + bu * 128;
+        const uint32_t sk = sKV + s * C::ST_BYTES;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k & 3) * 32;
+          tc::umma_bf16(s_tm, tc::sdesc_sw128(sQ + (k >> 2) * 128 * 128 + off),
+                        tc::sdesc_sw128(sk + (k >> 2) * TK * 128 + off), idS, k > 0 ? 1u : 0u);
+        }
+        any = true;
+        tc::umma_commit(&ctl->s_full[bu]);
+        if (last) tc::umma_commit(&ctl->q_empty);
+        if (pu >= 0) {
+          if (!issue_pv(pu, ps, pfirst, false, pseg)) { ok = false; break; }
+          pu = -1;
+        }
+        if (last) {
+          if (!issue_pv(u, s, first, true, seg)) { ok = false; break; }
+        } else {
+          pu = u;
+          ps = s;
+          pfirst = first;
+          pseg = seg;
+        }
+        ++u;
+        ++kv;
+        iter_next(it, ctl, a);
+      }
+      if (!ok && any) {  // MMAs still in flight must finish before TMEM is freed
+        tc::umma_commit(&ctl->done);
+        drain_wait(&ctl->done, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ one thread per query row
+    const int row = (warp & 3) * 32 + lane;  // = TMEM lane of this thread
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const float sc = kLog2e * rsqrtf((float)D);
+    const int tid = threadIdx.x - 64;
+    Iter it;
+    iter_seek(it, ctl, a, g0, g1);
+    int seg = -1, kv = 0, u = 0;
+    float m = -INFINITY, l = 0.f;
+    int lim = 0, lim_max = 0;
+    while (it.g < it.g_end) {
+      const bool first = it.first, last = iter_last(it);
+      const int lb = it.l * a.B + it.b;
+      const int prob = lb * a.Hkv + it.h;
+      if (first) {
+        ++seg;
+        m = -INFINITY;
+        l = 0.f;
+        const int base = a.len[it.b] + a.len_off;
+        lim = base + (row < a.rows ? row % a.nq : 0);
+        lim_max = base + a.nq - 1;
+      }
+      const int bu = u & 1;
+      const int s = kv % STAGES;
+      const int key0 = it.t * TK;
+      if (!tc::mbar_wait_warp(&ctl->s_full[bu], (u >> 1) & 1, abort_flag, a.err)) break;
+      tc::fence_after_sync();
+      if (key0 + TK > lim_max) {
+        // last tile of the problem: zero V rows past the last query's limit so that
+        // whatever bytes sit there cannot turn 0 * V into NaN
+        if (!tc::mbar_wait_warp(&ctl->kv_full[s], (kv / STAGES) & 1, abort_flag, a.err)) break;
+        const int z0 = max(0, lim_max - key0);
+        uint8_t* vb = smem + C::Q_BYTES + s * C::ST_BYTES + C::T_BYTES;
+        for (int i = tid; i < C::KB * TK * 8; i += 128) {
+          const int r = (i >> 3) % TK;
+          if (r >= z0) *reinterpret_cast<uint4*>(vb + (i / (TK * 8)) * TK * 128 + r * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+        }
+        tc::fence_proxy_async();
+      }
+      // S row of this thread: 128 logits
+      float v[TK];
+      {
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        const uint32_t sa = lane_base + kColS + bu * 128;
+        __syncwarp();
+        tc::tmem_ld_x32(sa, r0);
+        tc::tmem_ld_x32(sa + 32, r1);
+        tc::tmem_ld_x32(sa + 64, r2);
+        tc::tmem_ld_x32(sa + 96, r3);
+        tc::tmem_ld_wait(r0);
+        tc::tmem_ld_wait(r1);
+        tc::tmem_ld_wait(r2);
+        tc::tmem_ld_wait(r3);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          v[j] = __uint_as_float(r0[j]);
+          v[32 + j] = __uint_as_float(r1[j]);
+          v[64 + j] = __uint_as_float(r2[j]);
+          v[96 + j] = __uint_as_float(r3[j]);
+        }
+      }
+      if (key0 + TK > lim) {
+#pragma unroll
+        for (int j = 0; j < TK; ++j)
+          if (key0 + j >= lim) v[j] = -INFINITY;
+      }
+      float mx = v[0];
+#pragma unroll
+      for (int j = 1; j < TK; ++j) mx = fmaxf(mx, v[j]);
+      // lazy rescale: only when the max grows by more than 2^kTau (whole warp, O is warp-collective)
+      const bool resc = (m != -INFINITY) && (mx - m) * sc > kTau;
+      if (__any_sync(0xffffffffu, resc)) {
+        // the previous tile's P V must have landed in O before O is rescaled
+        if (!tc::mbar_wait_warp(&ctl->s_free[(u - 1) & 1], ((u - 1) >> 1) & 1, abort_flag, a.err)) break;
+        tc::fence_after_sync();
+        const float f = resc ? ex2((m - mx) * sc) : 1.f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          __syncwarp();
+          tc::tmem_ld_x32(lane_base + c * 32, o);
+          tc::tmem_ld_wait(o);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
+          tc::tmem_st_x32(lane_base + c * 32, o);
+        }
+        tc::tmem_st_wait();
+        l *= f;
+        if (resc) m = mx;
+      }
+      if (m == -INFINITY) m = mx;  // first key this row may see (stays -inf if none yet)
+      const float msc = m * sc;
+      const bool live = m != -INFINITY;
+      // P = 2^(x - m) as bf16 pairs, written over the S columns already read
+#pragma unroll
+      for (int c = 0; c < TK / 32; ++c) {
+        uint32_t pk[16];
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float p0 = live ? ex2(fmaf(v[c * 32 + 2 * j], sc, -msc)) : 0.f;
+          const float p1 = live ? ex2(fmaf(v[c * 32 + 2 * j + 1], sc, -msc)) : 0.f;
+          s0 += p0;
+          s1 += p1;
+          pk[j] = pack_bf16(p0, p1);
+        }
+        l += s0 + s1;
+        __syncwarp();
+        tc::tmem_st_x16(lane_base + kColS + bu * 128 + c * 16, pk);
+      }
+      tc::tmem_st_wait();
+      tc::fence_before_sync();
+      tc::mbar_arrive(&ctl->p_full[bu]);
+      if (last) {
+        if (!tc::mbar_wait_warp(&ctl->o_ready, seg & 1, abort_flag, a.err)) break;
+        tc::fence_after_sync();
+        const int slot = prob + blockIdx.x;
+        float* po = a.ws + ((size_t)slot * a.rows + row) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          __syncwarp();
+          tc::tmem_ld_x32(lane_base + c * 32, o);
+          tc::tmem_ld_wait(o);
+          if (row < a.rows) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              *reinterpret_cast<float4*>(po + c * 32 + j) =
+                  make_float4(__uint_as_float(o[j]), __uint_as_float(o[j + 1]), __uint_as_float(o[j + 2]),
+                              __uint_as_float(o[j + 3]));
+          }
+        }
+        if (row < a.rows) {
+          float* ml = a.ws + (size_t)(a.L * a.B * a.Hkv + gridDim.x) * a.rows * D;
+          ml[((size_t)slot * a.rows + row) * 2] = msc;
+          ml[((size_t)slot * a.rows + row) * 2 + 1] = l;
+        }
+        tc::fence_before_sync();
+        tc::mbar_arrive(&ctl->o_free);
+      }
+      ++u;
+      ++kv;
+      iter_next(it, ctl, a);
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Merge the partials of each (problem, row): slots problem + c for every CTA c
+// whose slice touched the problem.  One warp per row.
+template <int D>
+__global__ void __launch_bounds__(128) attn_tc_merge_kernel(const AttnArgs a, int grid_ctas) {
+  __shared__ int tiles_b[kMaxB];
+  __shared__ int s_tl;
+  if (threadIdx.x == 0) {
+    int sum = 0;
+    for (int b = 0; b < a.B; ++b) {
+      tiles_b[b] = seq_tiles(a, b, false);
+      sum += tiles_b[b];
+    }
+    s_tl = a.Hkv * sum;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 4 + warp;
+  const int h = blockIdx.y, lb = blockIdx.z, l = lb / a.B, b = lb % a.B;
+  if (row >= a.rows) return;
+  float* dst = a.o + ((size_t)(lb * a.Hq + h * a.G) * a.nq + row) * D;
+  const int nt = tiles_b[b];
+  if (nt == 0) {
+    for (int c = lane; c < D; c += 32) dst[c] = 0.f;
+    return;
+  }
+  const int tl = s_tl;
+  const int total = a.L * tl;
+  const int per = (total + grid_ctas - 1) / grid_ctas;
+  int start = l * tl;
+  for (int bb = 0; bb < b; ++bb) start += a.Hkv * tiles_b[bb];
+  start += h * nt;
+  const int c0 = start / per, c1 = (start + nt - 1) / per;
+  const int prob = lb * a.Hkv + h;
+  const float* ml = a.ws + (size_t)(a.L * a.B * a.Hkv + grid_ctas) * a.rows * D;
+  float M = -INFINITY;
+  for (int c = c0; c <= c1; ++c) M = fmaxf(M, ml[((size_t)(prob + c) * a.rows + row) * 2]);
+  const float ref = M == -INFINITY ? 0.f : M;
+  float L = 0.f;
+  for (int c = c0; c <= c1; ++c) {
+    const size_t k = (size_t)(prob + c) * a.rows + row;
+    L += ex2(ml[k * 2] - ref) * ml[k * 2 + 1];
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  for (int col = lane; col < D; col += 32) {
+    float acc = 0.f;
+    for (int c = c0; c <= c1; ++c) {
+      const size_t k = (size_t)(prob + c) * a.rows + row;
+      acc += ex2(ml[k * 2] - ref) * a.ws[k * D + col];
+    }
+    dst[col] = acc * inv;
+  }
+}
+
+template <int D>
+cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
+  using C = Cfg<D>;
+  const uint64_t qrows = (uint64_t)a.L * a.B * a.Hq * a.nq;
+  const uint64_t krows = (uint64_t)a.L * a.B * a.Hkv * a.cap;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_bf16_2d(&tq, a.q, D, qrows, 128) || !make_tmap_bf16_2d(&tk, a.k, D, krows, TK) ||
+      !make_tmap_bf16_2d(&tv, a.v, D, krows, TK))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  attn_tc_kernel<D><<<a.splits, kThreads, C::SMEM, s>>>(tq, tk, tv, a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  attn_tc_merge_kernel<D><<<dim3((a.rows + 3) / 4, a.Hkv, a.L * a.B), 128, 0, s>>>(a, a.splits);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attn_tc_supported(const AttnArgs& a) {
+  return a.dtype == STD_BF16 && (a.d == 64 || a.d == 128) && a.rows <= 128 && a.B <= kMaxB &&
+         (uint64_t)a.L * a.B * a.Hkv * a.cap + TK < (1ull << 31) &&
+         (uint64_t)a.L * a.B * a.Hq * a.nq + 128 < (1ull << 31);
+}
+
+size_t attn_tc_ws_floats(int probs, int ctas, int rows, int d) {
+  const size_t slots = (size_t)probs + ctas;
+  return slots * rows * d + slots * rows * 2;
+}
+
+// a.splits = number of persistent CTAs.
+cudaError_t launch_decode_attn_tc(const AttnArgs& a, cudaStream_t s) {
+  return a.d == 128 ? launch<128>(a, s) : launch<64>(a, s);
+}
+
+}  // namespace stdb

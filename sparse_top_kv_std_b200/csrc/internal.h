@@ -1,6 +1,7 @@
 // Host-side launchers shared between the C ABI layer and the kernel files.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -23,10 +24,21 @@ struct AttnArgs {
   int* err;
 };
 
+// Split-K kernels (fp32 operands; bf16 when the tensor-core kernel does not apply):
 // rows padded to the kernel's row tile, and the workspace floats for `splits`.
 int attn_rows_pad(int rows, int dtype);
 size_t attn_ws_floats(int probs, int splits, int rows, int d, int dtype);
 cudaError_t launch_decode_attn(const AttnArgs& a, cudaStream_t s);
+
+// Tensor-core kernel (bf16, d in {64, 128}, rows <= 128, B <= 64): persistent
+// stream-K over 128-key tiles, a.splits = number of CTAs; workspace holds
+// (problems + CTAs) partial slots.
+bool attn_tc_supported(const AttnArgs& a);
+size_t attn_tc_ws_floats(int probs, int ctas, int rows, int d);
+cudaError_t launch_decode_attn_tc(const AttnArgs& a, cudaStream_t s);
+
+// 2D bf16 tensor map over `rows` rows of `inner` elements, box 64 x box_rows, 128-byte swizzle.
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows);
 
 struct ScoreArgs {
   const void* q_text;   // [L][B][Hq][T][d]

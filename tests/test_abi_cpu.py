@@ -49,10 +49,15 @@ def test_workspace_queries_host_only(lib):
     d = _dims()
     ws = B.std_select_workspace_size(d, 64, 512)
     assert ws >= (2 * 4 * 7 * 64 * 2 + 2 * 4 * 512) * 4
-    # explicit splits: no device query
+    # explicit splits: no device query.  bf16: tensor-core kernel with splits x problems CTAs
+    # and (problems + CTAs) partial slots of 63 rows x (d + 2) floats
+    probs = 2 * 1 * 4
     a = B.std_attn_workspace_size(d, 9, 1000, 4)
-    assert a == 2 * 4 * 4 * 64 * (128 + 2) * 4      # rows 63 padded to 64
-    assert B.std_attn_workspace_size(d, 9, 1000, 1) == 0
+    assert a == (probs + 4 * probs) * 63 * (128 + 2) * 4
+    # fp32: split-K, no workspace with one split
+    f = _dims(dtype=B.STD_F32, d=64)
+    assert B.std_attn_workspace_size(f, 9, 1000, 1) == 0
+    assert B.std_attn_workspace_size(f, 9, 1000, 4) == probs * 4 * 63 * (64 + 2) * 4
     assert B.std_select_workspace_size(_dims(dtype=7), 64, 512) == 0
     assert B.std_attn_workspace_size(_dims(Hq=5), 1, 1000, 4) == 0
 

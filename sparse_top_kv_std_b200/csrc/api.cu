@@ -5,6 +5,7 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <atomic>
 #include <mutex>
 #include <string>
 
@@ -14,6 +15,7 @@
 namespace {
 
 thread_local std::string g_last_error;
+std::atomic<uint32_t> g_epoch{0};  // tags the in-kernel merge counters of each attention call
 
 int fail(int code, const char* fmt, ...) {
   char buf[512];
@@ -171,6 +173,7 @@ int run_attn(const std_dims* dims, const void* q, const void* k, const void* v, 
   stdb::AttnArgs& a = p.a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.len = len; a.len_off = len_off;
   a.ws = static_cast<float*>(ws); a.err = err;
+  a.epoch = g_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
   cudaError_t e = p.tc ? stdb::launch_decode_attn_tc(a, stream) : stdb::launch_decode_attn(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
   return ok();

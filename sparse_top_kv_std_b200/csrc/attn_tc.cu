@@ -10,12 +10,14 @@
 // HBM once.  The keys of all problems, cut into 128-key tiles, form one flat
 // sequence; a persistent grid of CTAs (one per SM by default) takes equal
 // contiguous slices of it (stream-K), so the load is balanced whatever the
-// lengths.  A CTA writes one partial (m, l, o) per run of tiles of the same
-// problem ("segment"), into slot problem + cta; a merge kernel combines the
-// slots of each problem.
+// lengths.  A CTA that covers a whole problem writes its output directly;
+// otherwise it writes one partial (m, l, o) per run of tiles of the same
+// problem ("segment") into slot problem + cta, and the last CTA to finish a
+// problem (an epoch-tagged arrival counter per problem, no waiting) merges the
+// partials of that problem.
 //
-// Per tile, inside a CTA (warp 0: TMA producer; warp 1: TMEM owner and MMA
-// issuer; warps 2-5: one thread per query row):
+// Per tile, inside a CTA (warp 0: TMA producers, lane 0 for K/V and lane 1 for
+// Q; warp 1: TMEM owner and MMA issuer; warps 2-5: one thread per query row):
 //   TMA        K tile and V tile (128 keys x d, 128-byte swizzle) -> stage ring
 //   MMA        S = Q K^T  -> TMEM S buffer (double-buffered, 128 fp32 columns)
 //   softmax    row max, lazy rescale of O (only when the max grows by more than
@@ -46,14 +48,33 @@ struct Ctl {
   uint64_t q_full, q_empty, done;
   uint64_t s_full[2], p_full[2], s_free[2];
   uint64_t o_ready, o_free;
+  uint64_t pub, flag;  // partial published by all 128 row threads / merge decision made
   uint32_t tmem;
   int abort_flag;
   int consumed;
   int tl;      // tiles per layer
   int total;   // tiles of the whole call
   int per;     // tiles per CTA
+  int last_flag;
   int tiles_b[kMaxB];
+  int pre_b[kMaxB];  // Hkv * (tiles of sequences before b)
 };
+
+// Arrival on the merge counter of one problem: the counter holds (epoch << 32) |
+// arrivals; a stale epoch (an earlier call, or uninitialised memory) restarts the
+// count.  Returns true for the arrival that completes `need`.  Lock-free: a CAS
+// retry loop, never a wait on another CTA.
+__device__ __forceinline__ bool arrive_last(unsigned long long* ctr, uint32_t epoch, int need) {
+  unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(ctr);
+  for (;;) {
+    const unsigned long long want =
+        (uint32_t)(old >> 32) == epoch ? old + 1 : (((unsigned long long)epoch << 32) | 1ull);
+    const unsigned long long prev = atomicCAS(ctr, old, want);
+    if (prev == old) return (int)(want & 0xffffffffull) == need;
+    old = prev;
+  }
+}
+
 
 // Tiles of sequence b (0 for an invalid length, which is flagged).
 __device__ __forceinline__ int seq_tiles(const AttnArgs& a, int b, bool flag) {
@@ -147,6 +168,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     int sum = 0;
     for (int b = 0; b < a.B; ++b) {
       ctl->tiles_b[b] = seq_tiles(a, b, blockIdx.x == 0);
+      ctl->pre_b[b] = a.Hkv * sum;
       sum += ctl->tiles_b[b];
     }
     ctl->tl = a.Hkv * sum;
@@ -166,6 +188,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     tc::mbar_init(&ctl->o_ready, 1);
     tc::mbar_init(&ctl->o_free, 128);
+    tc::mbar_init(&ctl->pub, 128);
+    tc::mbar_init(&ctl->flag, 1);
     ctl->abort_flag = 0;
     ctl->consumed = 0;
     tc::fence_mbar_init();
@@ -184,27 +208,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int g1 = min(ctl->total, g0 + ctl->per);
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producers
     if (lane == 0 && g0 < g1) {
-      tc::prefetch_tmap(&tm_q);
       tc::prefetch_tmap(&tm_k);
       tc::prefetch_tmap(&tm_v);
       Iter it;
       iter_seek(it, ctl, a, g0, g1);
-      int seg = 0, kv = 0;
-      bool q_pending = false;
+      int kv = 0;
       while (it.g < it.g_end) {
-        const int lb = it.l * a.B + it.b;
-        const int prob = lb * a.Hkv + it.h;
-        if (it.first) {
-          if (!tc::mbar_wait(&ctl->q_empty, (seg & 1) ^ 1, abort_flag, a.err)) break;
-          tc::mbar_expect_tx(&ctl->q_full, C::Q_BYTES);
-          const int qrow = (lb * a.Hq + it.h * a.G) * a.nq;
-#pragma unroll
-          for (int kb = 0; kb < C::KB; ++kb) tc::tma_load_2d(sQ + kb * 128 * 128, &tm_q, kb * 64, qrow, &ctl->q_full);
-          q_pending = true;
-          ++seg;
-        }
+        const int prob = (it.l * a.B + it.b) * a.Hkv + it.h;
         const int s = kv % STAGES;
         if (!tc::mbar_wait(&ctl->kv_empty[s], ((kv / STAGES) & 1) ^ 1, abort_flag, a.err)) break;
         tc::mbar_expect_tx(&ctl->kv_full[s], C::ST_BYTES);
@@ -219,9 +231,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         iter_next(it, ctl, a);
       }
       if (*abort_flag) {  // let the copies in flight land
-        if (q_pending) drain_wait(&ctl->q_full, (seg - 1) & 1);
         for (int k = *(volatile int*)&ctl->consumed; k < kv; ++k) drain_wait(&ctl->kv_full[k % STAGES], (k / STAGES) & 1);
       }
+    } else if (lane == 1 && g0 < g1) {
+      tc::prefetch_tmap(&tm_q);
+      Iter it;
+      iter_seek(it, ctl, a, g0, g1);
+      int seg = 0;
+      while (it.g < it.g_end) {
+        if (it.first) {
+          if (!tc::mbar_wait(&ctl->q_empty, (seg & 1) ^ 1, abort_flag, a.err)) break;
+          tc::mbar_expect_tx(&ctl->q_full, C::Q_BYTES);
+          const int qrow = ((it.l * a.B + it.b) * a.Hq + it.h * a.G) * a.nq;
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb) tc::tma_load_2d(sQ + kb * 128 * 128, &tm_q, kb * 64, qrow, &ctl->q_full);
+          ++seg;
+        }
+        iter_next(it, ctl, a);
+      }
+      if (*abort_flag && seg > 0) drain_wait(&ctl->q_full, (seg - 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -301,7 +329,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int tid = threadIdx.x - 64;
     Iter it;
     iter_seek(it, ctl, a, g0, g1);
-    int seg = -1, kv = 0, u = 0;
+    int seg = -1, kv = 0, u = 0, npub = 0;
     float m = -INFINITY, l = 0.f;
     int lim = 0, lim_max = 0;
     while (it.g < it.g_end) {
@@ -410,29 +438,98 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (last) {
         if (!tc::mbar_wait_warp(&ctl->o_ready, seg & 1, abort_flag, a.err)) break;
         tc::fence_after_sync();
-        const int slot = prob + blockIdx.x;
-        float* po = a.ws + ((size_t)slot * a.rows + row) * D;
+        // CTAs whose slices touch this problem
+        const int start = it.l * ctl->tl + ctl->pre_b[it.b] + it.h * it.nt;
+        const int c0 = start / ctl->per, c1 = (start + it.nt - 1) / ctl->per;
+        const size_t orow = (size_t)(lb * a.Hq + it.h * a.G) * a.nq + row;
+        if (c0 == c1) {
+          // this CTA saw the whole problem: normalised output straight from TMEM
+          const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          __syncwarp();
-          tc::tmem_ld_x32(lane_base + c * 32, o);
-          tc::tmem_ld_wait(o);
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            __syncwarp();
+            tc::tmem_ld_x32(lane_base + c * 32, o);
+            tc::tmem_ld_wait(o);
+            if (row < a.rows) {
+              float* dst = a.o + orow * D + c * 32;
+#pragma unroll
+              for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(dst + j) =
+                    make_float4(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv,
+                                __uint_as_float(o[j + 2]) * inv, __uint_as_float(o[j + 3]) * inv);
+            }
+          }
+          tc::fence_before_sync();
+          tc::mbar_arrive(&ctl->o_free);
+        } else {
+          const size_t nslots = (size_t)a.L * a.B * a.Hkv + gridDim.x;
+          float* ml = a.ws + nslots * a.rows * D;
+          unsigned long long* ctr = reinterpret_cast<unsigned long long*>(ml + nslots * a.rows * 2);
+          const int slot = prob + blockIdx.x;
+          float* po = a.ws + ((size_t)slot * a.rows + row) * D;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            __syncwarp();
+            tc::tmem_ld_x32(lane_base + c * 32, o);
+            tc::tmem_ld_wait(o);
+            if (row < a.rows) {
+#pragma unroll
+              for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(po + c * 32 + j) =
+                    make_float4(__uint_as_float(o[j]), __uint_as_float(o[j + 1]), __uint_as_float(o[j + 2]),
+                                __uint_as_float(o[j + 3]));
+            }
+          }
           if (row < a.rows) {
-#pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              *reinterpret_cast<float4*>(po + c * 32 + j) =
-                  make_float4(__uint_as_float(o[j]), __uint_as_float(o[j + 1]), __uint_as_float(o[j + 2]),
-                              __uint_as_float(o[j + 3]));
+            ml[((size_t)slot * a.rows + row) * 2] = msc;
+            ml[((size_t)slot * a.rows + row) * 2 + 1] = l;
+          }
+          tc::fence_before_sync();
+          tc::mbar_arrive(&ctl->o_free);  // O may be reused: the rest reads global memory only
+          // publish the partial, count the arrival; the last CTA merges every slot of the problem
+          __threadfence();
+          tc::mbar_arrive(&ctl->pub);
+          if (tid == 0) {
+            if (!tc::mbar_wait(&ctl->pub, npub & 1, abort_flag, a.err)) break;
+            __threadfence();
+            ctl->last_flag = arrive_last(ctr + prob, a.epoch, c1 - c0 + 1) ? 1 : 0;
+            tc::mbar_arrive(&ctl->flag);
+          }
+          if (!tc::mbar_wait(&ctl->flag, npub & 1, abort_flag, a.err)) break;
+          ++npub;
+          if (ctl->last_flag) {
+            __threadfence();
+            // all 128 row threads share the merge: one item = 4 columns of one query row
+            const int nseg = c1 - c0 + 1;
+            for (int item = tid; item < a.rows * (D / 4); item += 128) {
+              const int r = item / (D / 4), col = (item % (D / 4)) * 4;
+              const size_t k0 = (size_t)(prob + c0) * a.rows + r;
+              float M = -INFINITY;
+              for (int c = 0; c < nseg; ++c) M = fmaxf(M, __ldcg(ml + (k0 + (size_t)c * a.rows) * 2));
+              const float ref = M == -INFINITY ? 0.f : M;
+              float L = 0.f;
+              float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+              for (int c = 0; c < nseg; ++c) {
+                const size_t k = k0 + (size_t)c * a.rows;
+                const float2 mlk = __ldcg(reinterpret_cast<const float2*>(ml + k * 2));
+                const float w = ex2(mlk.x - ref);
+                L += w * mlk.y;
+                const float4 x = __ldcg(reinterpret_cast<const float4*>(a.ws + k * D + col));
+                acc.x += w * x.x;
+                acc.y += w * x.y;
+                acc.z += w * x.z;
+                acc.w += w * x.w;
+              }
+              const float inv = L > 0.f ? 1.f / L : 0.f;
+              const size_t orow_r = (size_t)(lb * a.Hq + it.h * a.G) * a.nq + r;
+              *reinterpret_cast<float4*>(a.o + orow_r * D + col) =
+                  make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+            }
+            if (tid == 0) atomicExch(ctr + prob, (unsigned long long)a.epoch << 32);  // ready for a replay
           }
         }
-        if (row < a.rows) {
-          float* ml = a.ws + (size_t)(a.L * a.B * a.Hkv + gridDim.x) * a.rows * D;
-          ml[((size_t)slot * a.rows + row) * 2] = msc;
-          ml[((size_t)slot * a.rows + row) * 2 + 1] = l;
-        }
-        tc::fence_before_sync();
-        tc::mbar_arrive(&ctl->o_free);
       }
       ++u;
       ++kv;
@@ -448,59 +545,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   }
 }
 
-// Merge the partials of each (problem, row): slots problem + c for every CTA c
-// whose slice touched the problem.  One warp per row.
-template <int D>
-__global__ void __launch_bounds__(128) attn_tc_merge_kernel(const AttnArgs a, int grid_ctas) {
-  __shared__ int tiles_b[kMaxB];
-  __shared__ int s_tl;
-  if (threadIdx.x == 0) {
-    int sum = 0;
-    for (int b = 0; b < a.B; ++b) {
-      tiles_b[b] = seq_tiles(a, b, false);
-      sum += tiles_b[b];
-    }
-    s_tl = a.Hkv * sum;
-  }
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 4 + warp;
-  const int h = blockIdx.y, lb = blockIdx.z, l = lb / a.B, b = lb % a.B;
-  if (row >= a.rows) return;
-  float* dst = a.o + ((size_t)(lb * a.Hq + h * a.G) * a.nq + row) * D;
-  const int nt = tiles_b[b];
-  if (nt == 0) {
-    for (int c = lane; c < D; c += 32) dst[c] = 0.f;
-    return;
-  }
-  const int tl = s_tl;
-  const int total = a.L * tl;
-  const int per = (total + grid_ctas - 1) / grid_ctas;
-  int start = l * tl;
-  for (int bb = 0; bb < b; ++bb) start += a.Hkv * tiles_b[bb];
-  start += h * nt;
-  const int c0 = start / per, c1 = (start + nt - 1) / per;
-  const int prob = lb * a.Hkv + h;
-  const float* ml = a.ws + (size_t)(a.L * a.B * a.Hkv + grid_ctas) * a.rows * D;
-  float M = -INFINITY;
-  for (int c = c0; c <= c1; ++c) M = fmaxf(M, ml[((size_t)(prob + c) * a.rows + row) * 2]);
-  const float ref = M == -INFINITY ? 0.f : M;
-  float L = 0.f;
-  for (int c = c0; c <= c1; ++c) {
-    const size_t k = (size_t)(prob + c) * a.rows + row;
-    L += ex2(ml[k * 2] - ref) * ml[k * 2 + 1];
-  }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  for (int col = lane; col < D; col += 32) {
-    float acc = 0.f;
-    for (int c = c0; c <= c1; ++c) {
-      const size_t k = (size_t)(prob + c) * a.rows + row;
-      acc += ex2(ml[k * 2] - ref) * a.ws[k * D + col];
-    }
-    dst[col] = acc * inv;
-  }
-}
-
 template <int D>
 cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   using C = Cfg<D>;
@@ -513,8 +557,6 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   attn_tc_kernel<D><<<a.splits, kThreads, C::SMEM, s>>>(tq, tk, tv, a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  attn_tc_merge_kernel<D><<<dim3((a.rows + 3) / 4, a.Hkv, a.L * a.B), 128, 0, s>>>(a, a.splits);
   return cudaGetLastError();
 }
 
@@ -526,9 +568,10 @@ bool attn_tc_supported(const AttnArgs& a) {
          (uint64_t)a.L * a.B * a.Hq * a.nq + 128 < (1ull << 31);
 }
 
+// partial o, partial (m, l), then one 64-bit merge counter per problem
 size_t attn_tc_ws_floats(int probs, int ctas, int rows, int d) {
   const size_t slots = (size_t)probs + ctas;
-  return slots * rows * d + slots * rows * 2;
+  return slots * rows * d + slots * rows * 2 + (size_t)probs * 2;
 }
 
 // a.splits = number of persistent CTAs.

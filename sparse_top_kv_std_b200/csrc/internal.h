@@ -22,6 +22,7 @@ struct AttnArgs {
   int splits;
   float* ws;  // partials: [prob][split][rows_pad][d] then [prob][split][rows_pad][2]
   int* err;
+  uint32_t epoch;  // per-call tag of the merge counters (tensor-core kernel)
 };
 
 // Split-K kernels (fp32 operands; bf16 when the tensor-core kernel does not apply):

@@ -50,10 +50,10 @@ def test_workspace_queries_host_only(lib):
     ws = B.std_select_workspace_size(d, 64, 512)
     assert ws >= (2 * 4 * 7 * 64 * 2 + 2 * 4 * 512) * 4
     # explicit splits: no device query.  bf16: tensor-core kernel with splits x problems CTAs
-    # and (problems + CTAs) partial slots of 63 rows x (d + 2) floats
+    # (problems + CTAs) partial slots of 63 rows x (d + 2) floats and a merge counter per problem
     probs = 2 * 1 * 4
     a = B.std_attn_workspace_size(d, 9, 1000, 4)
-    assert a == (probs + 4 * probs) * 63 * (128 + 2) * 4
+    assert a == (probs + 4 * probs) * 63 * (128 + 2) * 4 + probs * 8   # + one merge counter per problem
     # fp32: split-K, no workspace with one split
     f = _dims(dtype=B.STD_F32, d=64)
     assert B.std_attn_workspace_size(f, 9, 1000, 1) == 0

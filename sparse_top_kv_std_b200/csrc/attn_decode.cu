@@ -78,6 +78,8 @@ __device__ __forceinline__ void store_pair(const AttnArgs& a, int prob, int lb, 
 template <int D, int RT, int KS>
 __global__ void __launch_bounds__(Cfg<D, RT, KS>::NT)
 attn_bf16_kernel(const AttnArgs a) {
+  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
+  pdl_trigger();
   using C = Cfg<D, RT, KS>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int split = blockIdx.x, h = blockIdx.y, lb = blockIdx.z;
@@ -281,6 +283,8 @@ attn_bf16_kernel(const AttnArgs a) {
 // dot products and an online softmax with the accurate exp2f.
 template <int D>
 __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnArgs a) {
+  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
+  pdl_trigger();
   constexpr int PER = D / 32;
   const int split = blockIdx.x, h = blockIdx.y, lb = blockIdx.z;
   const int b = lb % a.B;
@@ -334,6 +338,8 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnArgs a) {
 
 // Merge split partials: m = max m_s, l = sum l_s 2^(m_s - m), o = sum o_s 2^(m_s - m) / l.
 __global__ void __launch_bounds__(128) attn_reduce_kernel(const AttnArgs a, int rows_pad) {
+  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 4 + warp;
   const int h = blockIdx.y, lb = blockIdx.z;
@@ -368,8 +374,7 @@ cudaError_t launch_bf16(const AttnArgs& a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid(a.splits, a.Hkv, a.L * a.B);
-  kern<<<grid, C::NT, C::SMEM, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(C::NT), C::SMEM, s, a);
 }
 
 template <int D>
@@ -404,18 +409,16 @@ cudaError_t launch_decode_attn(const AttnArgs& a, cudaStream_t s) {
   } else {
     dim3 grid(a.splits, a.Hkv, a.L * a.B);
     switch (a.d) {
-      case 32: attn_f32_kernel<32><<<grid, 128, 0, s>>>(a); break;
-      case 64: attn_f32_kernel<64><<<grid, 128, 0, s>>>(a); break;
-      case 96: attn_f32_kernel<96><<<grid, 128, 0, s>>>(a); break;
-      case 128: attn_f32_kernel<128><<<grid, 128, 0, s>>>(a); break;
+      case 32: e = launch_pdl(attn_f32_kernel<32>, grid, dim3(128), 0, s, a); break;
+      case 64: e = launch_pdl(attn_f32_kernel<64>, grid, dim3(128), 0, s, a); break;
+      case 96: e = launch_pdl(attn_f32_kernel<96>, grid, dim3(128), 0, s, a); break;
+      case 128: e = launch_pdl(attn_f32_kernel<128>, grid, dim3(128), 0, s, a); break;
       default: return cudaErrorInvalidValue;
     }
-    e = cudaGetLastError();
   }
   if (e != cudaSuccess || a.splits == 1) return e;
   dim3 rgrid((a.rows + 3) / 4, a.Hkv, a.L * a.B);
-  attn_reduce_kernel<<<rgrid, 128, 0, s>>>(a, attn_rows_pad(a.rows, a.dtype));
-  return cudaGetLastError();
+  return launch_pdl(attn_reduce_kernel, rgrid, dim3(128), 0, s, a, attn_rows_pad(a.rows, a.dtype));
 }
 
 }  // namespace stdb

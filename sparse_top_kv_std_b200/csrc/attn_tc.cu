@@ -156,6 +156,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
+  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
+  pdl_trigger();
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -556,8 +558,7 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<D><<<a.splits, kThreads, C::SMEM, s>>>(tq, tk, tv, a);
-  return cudaGetLastError();
+  return launch_pdl(attn_tc_kernel<D>, dim3(a.splits), dim3(kThreads), C::SMEM, s, tq, tk, tv, a);
 }
 
 }  // namespace

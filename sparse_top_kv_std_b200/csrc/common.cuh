@@ -16,6 +16,13 @@ __device__ __forceinline__ void flag_error(int* err, int bits) {
   if (err) atomicOr(err, bits);
 }
 
+// Programmatic dependent launch: every kernel of the library is launched so
+// that it may start while the previous kernel in the stream finishes.  It must
+// call pdl_wait() before touching memory a previous kernel writes or reads, and
+// calls pdl_trigger() to let the next kernel start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- loads
 template <typename T>
 __device__ __forceinline__ float to_f32(T x);

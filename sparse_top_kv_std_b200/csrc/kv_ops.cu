@@ -18,6 +18,8 @@ __device__ __forceinline__ void copy_row(uint8_t* dst, const uint8_t* src, int b
 
 // Sparse cache rows [0, K) <- full rows idx[0..K); rows [K, K + T) <- text rows.
 __global__ void __launch_bounds__(ROWS_PER_CTA * 32) gather_kernel(const GatherArgs a) {
+  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
+  pdl_trigger();
   const int h = blockIdx.y, lb = blockIdx.z, b = lb % a.B;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.x * ROWS_PER_CTA + warp;
@@ -49,6 +51,8 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) gather_kernel(const GatherA
 __global__ void __launch_bounds__(ROWS_PER_CTA * 32)
 append_kernel(uint8_t* kc, uint8_t* vc, int64_t cap, const int32_t* len, int off,
               const uint8_t* kn, const uint8_t* vn, int n_new, int B, int Hkv, int row_bytes, int* err) {
+  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
+  pdl_trigger();
   const int h = blockIdx.y, lb = blockIdx.z, b = lb % B;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * ROWS_PER_CTA + warp;
@@ -70,6 +74,8 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32)
 commit_copy_kernel(const uint8_t* kf, const uint8_t* vf, uint8_t* ks, uint8_t* vs, const int32_t* len_full,
                    const int32_t* len_sp, const int32_t* n_plus_1, int max_n, int B, int Hkv,
                    int row_bytes, int64_t cap_full, int64_t cap_sparse, int* err) {
+  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
+  pdl_trigger();
   const int h = blockIdx.y, lb = blockIdx.z, b = lb % B;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * ROWS_PER_CTA + warp;
@@ -91,6 +97,8 @@ commit_copy_kernel(const uint8_t* kf, const uint8_t* vf, uint8_t* ks, uint8_t* v
 // Both lengths advance by n + 1 (after every copy of the commit has read them).
 __global__ void commit_len_kernel(int32_t* len_full, int32_t* len_sp, const int32_t* n_plus_1, int max_n,
                                   int B, int64_t cap_full, int64_t cap_sparse) {
+  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
+  pdl_trigger();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= B) return;
   const int n = n_plus_1[b];
@@ -104,6 +112,8 @@ __global__ void commit_len_kernel(int32_t* len_full, int32_t* len_sp, const int3
 // One warp per sequence: n = index of the first mismatch (gamma if none).
 __global__ void accept_kernel(int B, int gamma, const int32_t* draft, const int32_t* dense,
                               int32_t* n_plus_1, int32_t* accepted) {
+  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
+  pdl_trigger();
   const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (b >= B) return;
@@ -118,8 +128,7 @@ __global__ void accept_kernel(int B, int gamma, const int32_t* draft, const int3
 
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s) {
   dim3 grid((a.K + a.T + ROWS_PER_CTA - 1) / ROWS_PER_CTA, a.Hkv, a.L * a.B);
-  gather_kernel<<<grid, ROWS_PER_CTA * 32, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(gather_kernel, grid, dim3(ROWS_PER_CTA * 32), 0, s, a);
 }
 
 cudaError_t launch_append(void* k_cache, void* v_cache, int64_t cap, const int32_t* len, int off,
@@ -127,10 +136,9 @@ cudaError_t launch_append(void* k_cache, void* v_cache, int64_t cap, const int32
                           int row_bytes, int* err, cudaStream_t s) {
   if (n_new <= 0) return cudaSuccess;
   dim3 grid((n_new + ROWS_PER_CTA - 1) / ROWS_PER_CTA, Hkv, L * B);
-  append_kernel<<<grid, ROWS_PER_CTA * 32, 0, s>>>(
-      static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache), cap, len, off,
-      static_cast<const uint8_t*>(k_new), static_cast<const uint8_t*>(v_new), n_new, B, Hkv, row_bytes, err);
-  return cudaGetLastError();
+  return launch_pdl(append_kernel, grid, dim3(ROWS_PER_CTA * 32), 0, s, static_cast<uint8_t*>(k_cache),
+                    static_cast<uint8_t*>(v_cache), cap, len, off, static_cast<const uint8_t*>(k_new),
+                    static_cast<const uint8_t*>(v_new), n_new, B, Hkv, row_bytes, err);
 }
 
 cudaError_t launch_commit(void* k_full, void* v_full, void* k_sp, void* v_sp, int32_t* len_full,
@@ -138,19 +146,17 @@ cudaError_t launch_commit(void* k_full, void* v_full, void* k_sp, void* v_sp, in
                           int Hkv, int row_bytes, int64_t cap_full, int64_t cap_sparse, int* err,
                           cudaStream_t s) {
   dim3 grid((max_n + ROWS_PER_CTA - 1) / ROWS_PER_CTA, Hkv, L * B);
-  commit_copy_kernel<<<grid, ROWS_PER_CTA * 32, 0, s>>>(
-      static_cast<const uint8_t*>(k_full), static_cast<const uint8_t*>(v_full), static_cast<uint8_t*>(k_sp),
-      static_cast<uint8_t*>(v_sp), len_full, len_sp, n_plus_1, max_n, B, Hkv, row_bytes, cap_full, cap_sparse, err);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(commit_copy_kernel, grid, dim3(ROWS_PER_CTA * 32), 0, s, static_cast<const uint8_t*>(k_full),
+                             static_cast<const uint8_t*>(v_full), static_cast<uint8_t*>(k_sp), static_cast<uint8_t*>(v_sp),
+                             len_full, len_sp, n_plus_1, max_n, B, Hkv, row_bytes, cap_full, cap_sparse, err);
   if (e != cudaSuccess) return e;
-  commit_len_kernel<<<(B + 127) / 128, 128, 0, s>>>(len_full, len_sp, n_plus_1, max_n, B, cap_full, cap_sparse);
-  return cudaGetLastError();
+  return launch_pdl(commit_len_kernel, dim3((B + 127) / 128), dim3(128), 0, s, len_full, len_sp, n_plus_1, max_n, B,
+                    cap_full, cap_sparse);
 }
 
 cudaError_t launch_accept(int B, int gamma, const int32_t* draft, const int32_t* dense,
                           int32_t* n_plus_1, int32_t* accepted, cudaStream_t s) {
-  accept_kernel<<<(B + 3) / 4, 128, 0, s>>>(B, gamma, draft, dense, n_plus_1, accepted);
-  return cudaGetLastError();
+  return launch_pdl(accept_kernel, dim3((B + 3) / 4), dim3(128), 0, s, B, gamma, draft, dense, n_plus_1, accepted);
 }
 
 }  // namespace stdb

@@ -82,6 +82,8 @@ __device__ __forceinline__ void load_ktile(uint32_t sk, const __nv_bfloat16* kp,
 // streams every visual key of the head through a 3-stage pipeline.
 template <int D>
 __global__ void __launch_bounds__(128) rowstats_bf16_kernel(const ScoreArgs a) {
+  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
+  pdl_trigger();
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int TILE = TKS * D * 2;
   const int h = blockIdx.y, lb = blockIdx.z, b = lb % a.B;
@@ -156,6 +158,8 @@ __global__ void __launch_bounds__(128) rowstats_bf16_kernel(const ScoreArgs a) {
 // in shared memory while the 4 warps sweep all M text rows 16 at a time.
 template <int D>
 __global__ void __launch_bounds__(128) colsum_bf16_kernel(const ScoreArgs a) {
+  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
+  pdl_trigger();
   extern __shared__ __align__(128) uint8_t smem[];
   const int h = blockIdx.y, lb = blockIdx.z, b = lb % a.B;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
@@ -228,6 +232,8 @@ __global__ void __launch_bounds__(128) colsum_bf16_kernel(const ScoreArgs a) {
 // fp32 operands: pass 1 with one thread per text row.
 template <int D>
 __global__ void __launch_bounds__(128) rowstats_f32_kernel(const ScoreArgs a) {
+  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
+  pdl_trigger();
   const int h = blockIdx.y, lb = blockIdx.z, b = lb % a.B;
   const int prob = lb * a.Hkv + h;
   const int M = a.G * a.T;
@@ -261,6 +267,8 @@ __global__ void __launch_bounds__(128) rowstats_f32_kernel(const ScoreArgs a) {
 // fp32 operands: pass 2 with one thread per visual key.
 template <int D>
 __global__ void __launch_bounds__(128) colsum_f32_kernel(const ScoreArgs a) {
+  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
+  pdl_trigger();
   const int h = blockIdx.y, lb = blockIdx.z, b = lb % a.B;
   const int prob = lb * a.Hkv + h;
   const int M = a.G * a.T;
@@ -290,21 +298,17 @@ cudaError_t launch_bf16_scores(const ScoreArgs& a, cudaStream_t s) {
   constexpr int smem1 = P1_STAGES * TKS * D * 2;
   cudaError_t e = cudaFuncSetAttribute(rowstats_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
   if (e != cudaSuccess) return e;
-  rowstats_bf16_kernel<D><<<dim3((M + 63) / 64, a.Hkv, a.L * a.B), 128, smem1, s>>>(a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_pdl(rowstats_bf16_kernel<D>, dim3((M + 63) / 64, a.Hkv, a.L * a.B), dim3(128), smem1, s, a)) != cudaSuccess) return e;
   constexpr int smem2 = TKS * D * 2;
-  colsum_bf16_kernel<D><<<dim3((a.nvis_max + TKS - 1) / TKS, a.Hkv, a.L * a.B), 128, smem2, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(colsum_bf16_kernel<D>, dim3((a.nvis_max + TKS - 1) / TKS, a.Hkv, a.L * a.B), dim3(128), smem2, s, a);
 }
 
 template <int D>
 cudaError_t launch_f32_scores(const ScoreArgs& a, cudaStream_t s) {
   const int M = a.G * a.T;
-  rowstats_f32_kernel<D><<<dim3((M + 127) / 128, a.Hkv, a.L * a.B), 128, 0, s>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(rowstats_f32_kernel<D>, dim3((M + 127) / 128, a.Hkv, a.L * a.B), dim3(128), 0, s, a);
   if (e != cudaSuccess) return e;
-  colsum_f32_kernel<D><<<dim3((a.nvis_max + 127) / 128, a.Hkv, a.L * a.B), 128, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(colsum_f32_kernel<D>, dim3((a.nvis_max + 127) / 128, a.Hkv, a.L * a.B), dim3(128), 0, s, a);
 }
 
 }  // namespace

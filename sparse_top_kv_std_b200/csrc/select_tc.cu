@@ -158,6 +158,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 rowstats_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const ScoreArgs a) {
+  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
+  pdl_trigger();
   using C = P1<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -319,6 +321,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const ScoreArgs a) {
+  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
+  pdl_trigger();
   using C = P2<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -523,10 +527,11 @@ static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s) {
   e = cudaFuncSetAttribute(colsum_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, P2<D>::SMEM);
   if (e != cudaSuccess) return e;
   const int M = a.G * a.T;
-  rowstats_tc_kernel<D><<<dim3((M + BM - 1) / BM, a.Hkv, a.L * a.B), kThreads, P1<D>::SMEM, s>>>(tq128, tk, a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  colsum_tc_kernel<D><<<dim3((a.nvis_max + 255) / 256, a.Hkv, a.L * a.B), kThreads, P2<D>::SMEM, s>>>(tq256, tk, a);
-  return cudaGetLastError();
+  e = launch_pdl(rowstats_tc_kernel<D>, dim3((M + BM - 1) / BM, a.Hkv, a.L * a.B), dim3(kThreads), P1<D>::SMEM, s,
+                 tq128, tk, a);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(colsum_tc_kernel<D>, dim3((a.nvis_max + 255) / 256, a.Hkv, a.L * a.B), dim3(kThreads),
+                    P2<D>::SMEM, s, tq256, tk, a);
 }
 
 // tcgen05 path for bf16 operands; cudaErrorNotSupported for shapes it does not cover.

@@ -29,6 +29,8 @@ __device__ __forceinline__ uint32_t order_key(float x) {
 __global__ void __launch_bounds__(TOPK_THREADS)
 topk_kernel(const float* scores, int64_t stride, const int32_t* n_dev, int n_const, int n_div,
             int n_mod, int K, int32_t* idx, int* err) {
+  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
+  pdl_trigger();
   __shared__ uint32_t hist[256];
   __shared__ uint32_t s_prefix, s_mask;
   __shared__ int s_remaining;
@@ -132,8 +134,8 @@ cudaError_t launch_topk(const float* scores, int64_t stride, int rows, const int
                         int n_const, int n_div, int n_mod, int K, int32_t* idx, int* err,
                         cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
-  topk_kernel<<<rows, TOPK_THREADS, 0, s>>>(scores, stride, n_dev, n_const, n_div, n_mod, K, idx, err);
-  return cudaGetLastError();
+  return launch_pdl(topk_kernel, dim3(rows), dim3(TOPK_THREADS), 0, s, scores, stride, n_dev, n_const, n_div, n_mod, K,
+                    idx, err);
 }
 
 }  // namespace stdb

@@ -326,6 +326,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   } else {
     // ------------------------------------------------------------ one thread per query row
     const int row = (warp & 3) * 32 + lane;  // = TMEM lane of this thread
+    const bool wactive = (warp & 3) * 32 < a.rows;  // warp holds at least one real query row
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const float sc = kLog2e * rsqrtf((float)D);
     const int tid = threadIdx.x - 64;
@@ -363,78 +364,80 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         tc::fence_proxy_async();
       }
-      // S row of this thread: 128 logits
-      float v[TK];
-      {
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        const uint32_t sa = lane_base + kColS + bu * 128;
-        __syncwarp();
-        tc::tmem_ld_x32(sa, r0);
-        tc::tmem_ld_x32(sa + 32, r1);
-        tc::tmem_ld_x32(sa + 64, r2);
-        tc::tmem_ld_x32(sa + 96, r3);
-        tc::tmem_ld_wait(r0);
-        tc::tmem_ld_wait(r1);
-        tc::tmem_ld_wait(r2);
-        tc::tmem_ld_wait(r3);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          v[j] = __uint_as_float(r0[j]);
-          v[32 + j] = __uint_as_float(r1[j]);
-          v[64 + j] = __uint_as_float(r2[j]);
-          v[96 + j] = __uint_as_float(r3[j]);
-        }
-      }
-      if (key0 + TK > lim) {
-#pragma unroll
-        for (int j = 0; j < TK; ++j)
-          if (key0 + j >= lim) v[j] = -INFINITY;
-      }
-      float mx = v[0];
-#pragma unroll
-      for (int j = 1; j < TK; ++j) mx = fmaxf(mx, v[j]);
-      // lazy rescale: only when the max grows by more than 2^kTau (whole warp, O is warp-collective)
-      const bool resc = (m != -INFINITY) && (mx - m) * sc > kTau;
-      if (__any_sync(0xffffffffu, resc)) {
-        // the previous tile's P V must have landed in O before O is rescaled
-        if (!tc::mbar_wait_warp(&ctl->s_free[(u - 1) & 1], ((u - 1) >> 1) & 1, abort_flag, a.err)) break;
-        tc::fence_after_sync();
-        const float f = resc ? ex2((m - mx) * sc) : 1.f;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
+      if (wactive) {
+        // S row of this thread: 128 logits
+        float v[TK];
+        {
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          const uint32_t sa = lane_base + kColS + bu * 128;
           __syncwarp();
-          tc::tmem_ld_x32(lane_base + c * 32, o);
-          tc::tmem_ld_wait(o);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
-          tc::tmem_st_x32(lane_base + c * 32, o);
+          tc::tmem_ld_x32(sa, r0);
+          tc::tmem_ld_x32(sa + 32, r1);
+          tc::tmem_ld_x32(sa + 64, r2);
+          tc::tmem_ld_x32(sa + 96, r3);
+          tc::tmem_ld_wait(r0);
+          tc::tmem_ld_wait(r1);
+          tc::tmem_ld_wait(r2);
+          tc::tmem_ld_wait(r3);
+  #pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            v[j] = __uint_as_float(r0[j]);
+            v[32 + j] = __uint_as_float(r1[j]);
+            v[64 + j] = __uint_as_float(r2[j]);
+            v[96 + j] = __uint_as_float(r3[j]);
+          }
+        }
+        if (key0 + TK > lim) {
+  #pragma unroll
+          for (int j = 0; j < TK; ++j)
+            if (key0 + j >= lim) v[j] = -INFINITY;
+        }
+        float mx = v[0];
+  #pragma unroll
+        for (int j = 1; j < TK; ++j) mx = fmaxf(mx, v[j]);
+        // lazy rescale: only when the max grows by more than 2^kTau (whole warp, O is warp-collective)
+        const bool resc = (m != -INFINITY) && (mx - m) * sc > kTau;
+        if (__any_sync(0xffffffffu, resc)) {
+          // the previous tile's P V must have landed in O before O is rescaled
+          if (!tc::mbar_wait_warp(&ctl->s_free[(u - 1) & 1], ((u - 1) >> 1) & 1, abort_flag, a.err)) break;
+          tc::fence_after_sync();
+          const float f = resc ? ex2((m - mx) * sc) : 1.f;
+  #pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            __syncwarp();
+            tc::tmem_ld_x32(lane_base + c * 32, o);
+            tc::tmem_ld_wait(o);
+  #pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
+            tc::tmem_st_x32(lane_base + c * 32, o);
+          }
+          tc::tmem_st_wait();
+          l *= f;
+          if (resc) m = mx;
+        }
+        if (m == -INFINITY) m = mx;  // first key this row may see (stays -inf if none yet)
+        const float msc = m * sc;
+        const bool live = m != -INFINITY;
+        // P = 2^(x - m) as bf16 pairs, written over the S columns already read
+  #pragma unroll
+        for (int c = 0; c < TK / 32; ++c) {
+          uint32_t pk[16];
+          float s0 = 0.f, s1 = 0.f;
+  #pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float p0 = live ? ex2(fmaf(v[c * 32 + 2 * j], sc, -msc)) : 0.f;
+            const float p1 = live ? ex2(fmaf(v[c * 32 + 2 * j + 1], sc, -msc)) : 0.f;
+            s0 += p0;
+            s1 += p1;
+            pk[j] = pack_bf16(p0, p1);
+          }
+          l += s0 + s1;
+          __syncwarp();
+          tc::tmem_st_x16(lane_base + kColS + bu * 128 + c * 16, pk);
         }
         tc::tmem_st_wait();
-        l *= f;
-        if (resc) m = mx;
       }
-      if (m == -INFINITY) m = mx;  // first key this row may see (stays -inf if none yet)
-      const float msc = m * sc;
-      const bool live = m != -INFINITY;
-      // P = 2^(x - m) as bf16 pairs, written over the S columns already read
-#pragma unroll
-      for (int c = 0; c < TK / 32; ++c) {
-        uint32_t pk[16];
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float p0 = live ? ex2(fmaf(v[c * 32 + 2 * j], sc, -msc)) : 0.f;
-          const float p1 = live ? ex2(fmaf(v[c * 32 + 2 * j + 1], sc, -msc)) : 0.f;
-          s0 += p0;
-          s1 += p1;
-          pk[j] = pack_bf16(p0, p1);
-        }
-        l += s0 + s1;
-        __syncwarp();
-        tc::tmem_st_x16(lane_base + kColS + bu * 128 + c * 16, pk);
-      }
-      tc::tmem_st_wait();
       tc::fence_before_sync();
       tc::mbar_arrive(&ctl->p_full[bu]);
       if (last) {
@@ -485,7 +488,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
           }
           if (row < a.rows) {
-            ml[((size_t)slot * a.rows + row) * 2] = msc;
+            ml[((size_t)slot * a.rows + row) * 2] = m * sc;
             ml[((size_t)slot * a.rows + row) * 2 + 1] = l;
           }
           tc::fence_before_sync();

@@ -71,26 +71,61 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x <= 0 (used beside ex2() to split the exponential
-// work between the special-function unit and the FP32 pipe).  Method: round
-// x to the nearest integer j with the 1.5 * 2^23 shifter (Cody-Waite style
-// reduction, f = x - j in [-1/2, 1/2]), evaluate 2^f = e^(f ln 2) with its
-// Taylor series to degree 6 (truncation error below 1.2e-7 relative), then add
-// j to the exponent field.  Inputs below -125 are clamped (result ~2e-38, far
-// below anything that matters next to the row maximum's 2^0).
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;
-  const float j = t - 12582912.f;
-  const float f = x - j;
-  float p = 1.5403530393381606e-4f;
-  p = fmaf(p, f, 1.3333558146428441e-3f);
-  p = fmaf(p, f, 9.618129107628477e-3f);
-  p = fmaf(p, f, 5.5504108664821576e-2f);
-  p = fmaf(p, f, 2.402265069591007e-1f);
-  p = fmaf(p, f, 6.931471805599453e-1f);
-  p = fmaf(p, f, 1.f);
-  return __int_as_float(__float_as_int(p) + (int)((uint32_t)(__float_as_int(t) - 0x4B400000) << 23));
+// ---------------------------------------------------------------- packed fp32 pairs (sm_100)
+// Two fp32 lanes in one 64-bit register: one instruction does both.
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 f2_make(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(f32x2 v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair of x <= 0 on the FMA pipe (used beside ex2() to split the
+// exponential work between the special-function unit and the FP32 pipe).
+// Method: round x to the nearest integer j with the 1.5 * 2^23 shifter
+// (Cody-Waite style reduction, f = x - j in [-1/2, 1/2]), evaluate
+// 2^f = e^(f ln 2) with its Taylor series to degree 6 (truncation error below
+// 1.2e-7 relative), then add j to the exponent field.  That last step uses
+// (t_bits - bits(1.5 * 2^23)) << 23 == t_bits << 23 (mod 2^32), since the
+// shifter's low nine bits are zero.  Inputs below -125 are clamped (result
+// ~2e-38, negligible next to the row maximum's 2^0).
+__device__ __forceinline__ f32x2 exp2_fma2(f32x2 x) {
+  float x0, x1;
+  f2_split(x, x0, x1);
+  x = f2_make(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const f32x2 t = f2_add(x, f2_make(12582912.f, 12582912.f));
+  const f32x2 j = f2_add(t, f2_make(-12582912.f, -12582912.f));
+  const f32x2 f = f2_fma(j, f2_make(-1.f, -1.f), x);
+  f32x2 p = f2_make(1.5403530393381606e-4f, 1.5403530393381606e-4f);
+  p = f2_fma(p, f, f2_make(1.3333558146428441e-3f, 1.3333558146428441e-3f));
+  p = f2_fma(p, f, f2_make(9.618129107628477e-3f, 9.618129107628477e-3f));
+  p = f2_fma(p, f, f2_make(5.5504108664821576e-2f, 5.5504108664821576e-2f));
+  p = f2_fma(p, f, f2_make(2.402265069591007e-1f, 2.402265069591007e-1f));
+  p = f2_fma(p, f, f2_make(6.931471805599453e-1f, 6.931471805599453e-1f));
+  p = f2_fma(p, f, f2_make(1.f, 1.f));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  return f2_make(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
+                 __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {

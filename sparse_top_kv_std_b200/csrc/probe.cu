@@ -3,11 +3,18 @@
 #include "common.cuh"
 
 namespace {
+// Each thread evaluates a pair (2i, 2i + 1) through the packed polynomial.
 __global__ void probe_exp2_kernel(const float* x, float* y_fma, float* y_sfu, int n) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) {
-    y_fma[i] = stdb::exp2_fma(x[i]);
-    y_sfu[i] = stdb::ex2(x[i]);
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float x0 = x[i], x1 = i + 1 < n ? x[i + 1] : 0.f;
+  float e0, e1;
+  stdb::f2_split(stdb::exp2_fma2(stdb::f2_make(x0, x1)), e0, e1);
+  y_fma[i] = e0;
+  y_sfu[i] = stdb::ex2(x0);
+  if (i + 1 < n) {
+    y_fma[i + 1] = e1;
+    y_sfu[i + 1] = stdb::ex2(x1);
   }
 }
 }  // namespace
@@ -15,6 +22,6 @@ __global__ void probe_exp2_kernel(const float* x, float* y_fma, float* y_sfu, in
 extern "C" int std_probe_exp2(const float* x, float* y_fma, float* y_sfu, int n, std_stream_t stream) {
   if (!x || !y_fma || !y_sfu || n < 0) return STD_ERR_INVALID_ARG;
   if (n == 0) return STD_OK;
-  probe_exp2_kernel<<<(n + 255) / 256, 256, 0, stream>>>(x, y_fma, y_sfu, n);
+  probe_exp2_kernel<<<(n + 511) / 512, 256, 0, stream>>>(x, y_fma, y_sfu, n);
   return cudaGetLastError() == cudaSuccess ? STD_OK : STD_ERR_CUDA;
 }

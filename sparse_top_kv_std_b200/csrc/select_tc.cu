@@ -43,7 +43,7 @@ constexpr int BN = 256;      // MMA N (keys in pass 1, text rows in pass 2)
 constexpr int kMaxRows = 2048;  // G * T supported by pass 2 (row statistics kept in shared memory)
 constexpr int kTmemCols = 512;
 constexpr int kHalf = BN / 2;   // accumulator columns per epilogue warpgroup
-constexpr int kPolyLanes = 8;   // of every 32 exponentials, this many on the FMA pipe
+constexpr int kPolyPairs = 6;   // of every 16 pairs of exponentials, this many on the FMA pipe
 
 struct Ctl {
   uint64_t full[8], empty[8];
@@ -74,6 +74,8 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Pass-1 epilogue on 32 logits of one row: online max / sum of 2^(x - m).
+// Pairs of logits go through packed fp32 instructions; kPolyPairs of the 16
+// pairs take their exponential on the FMA pipe, the rest on the SFU.
 template <bool TAIL>
 __device__ __forceinline__ void p1_chunk(const uint32_t (&r)[32], int key, int nv, float sc, float& m, float& l) {
   float v[32];
@@ -84,42 +86,64 @@ __device__ __forceinline__ void p1_chunk(const uint32_t (&r)[32], int key, int n
   }
   float cm = v[0];
 #pragma unroll
-  for (int j = 1; j < 32; ++j) cm = fmaxf(cm, v[j]);
+  for (int j = 1; j < 31; j += 2) cm = max3f(cm, v[j], v[j + 1]);
+  cm = fmaxf(cm, v[31]);
   if (cm == -INFINITY) return;  // every key of the chunk is past the visual tokens
   if (cm > m) {
     l *= ex2((m - cm) * sc);
     m = cm;
   }
   const float msc = m * sc;
-  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+  const f32x2 scc = f2_make(sc, sc), nm = f2_make(-msc, -msc);
+  f32x2 a0 = f2_make(0.f, 0.f), a1 = a0;
 #pragma unroll
-  for (int j = 0; j < kPolyLanes; j += 2) {
-    s0 += exp2_fma(fmaf(v[j], sc, -msc));
-    s1 += exp2_fma(fmaf(v[j + 1], sc, -msc));
+  for (int p = 0; p < 16; ++p) {
+    const f32x2 x = f2_fma(f2_make(v[2 * p], v[2 * p + 1]), scc, nm);
+    f32x2 e;
+    if (p < kPolyPairs) {
+      e = exp2_fma2(x);
+    } else {
+      float x0, x1;
+      f2_split(x, x0, x1);
+      e = f2_make(ex2(x0), ex2(x1));
+    }
+    if (p & 1) a1 = f2_add(a1, e); else a0 = f2_add(a0, e);
   }
-#pragma unroll
-  for (int j = kPolyLanes; j < 32; j += 2) {
-    s2 += ex2(fmaf(v[j], sc, -msc));
-    s3 += ex2(fmaf(v[j + 1], sc, -msc));
-  }
+  float s0, s1, s2, s3;
+  f2_split(a0, s0, s1);
+  f2_split(a1, s2, s3);
   l += (s0 + s1) + (s2 + s3);
 }
 
-// Pass-2 epilogue on 32 logits of one key: sum_r 2^(x_r - m_r) w_r, (m, w) from shared memory.
-__device__ __forceinline__ float p2_chunk(const uint32_t (&r)[32], const float2* mw, float sc) {
-  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+// Pass-2 epilogue on 32 logits of one key: sum_r 2^(x_r - m_r) w_r with -m_r and
+// w_r = 1 / l_r from shared memory (separate arrays, so pairs load directly).
+__device__ __forceinline__ float p2_chunk(const uint32_t (&r)[32], const float* negm, const float* w, float sc) {
+  const f32x2 scc = f2_make(sc, sc);
+  f32x2 a0 = f2_make(0.f, 0.f), a1 = a0;
 #pragma unroll
-  for (int j = 0; j < kPolyLanes; j += 2) {
-    const float4 p = *reinterpret_cast<const float4*>(mw + j);
-    s0 += exp2_fma(fmaf(__uint_as_float(r[j]), sc, -p.x)) * p.y;
-    s1 += exp2_fma(fmaf(__uint_as_float(r[j + 1]), sc, -p.z)) * p.w;
-  }
+  for (int q = 0; q < 8; ++q) {  // 4 rows at a time
+    const float4 nm4 = *reinterpret_cast<const float4*>(negm + 4 * q);
+    const float4 w4 = *reinterpret_cast<const float4*>(w + 4 * q);
 #pragma unroll
-  for (int j = kPolyLanes; j < 32; j += 2) {
-    const float4 p = *reinterpret_cast<const float4*>(mw + j);
-    s2 += ex2(fmaf(__uint_as_float(r[j]), sc, -p.x)) * p.y;
-    s3 += ex2(fmaf(__uint_as_float(r[j + 1]), sc, -p.z)) * p.w;
+    for (int h = 0; h < 2; ++h) {
+      const int p = 2 * q + h;
+      const f32x2 nm = h ? f2_make(nm4.z, nm4.w) : f2_make(nm4.x, nm4.y);
+      const f32x2 ww = h ? f2_make(w4.z, w4.w) : f2_make(w4.x, w4.y);
+      const f32x2 x = f2_fma(f2_make(__uint_as_float(r[2 * p]), __uint_as_float(r[2 * p + 1])), scc, nm);
+      f32x2 e;
+      if (p < kPolyPairs) {
+        e = exp2_fma2(x);
+      } else {
+        float x0, x1;
+        f2_split(x, x0, x1);
+        e = f2_make(ex2(x0), ex2(x1));
+      }
+      if (p & 1) a1 = f2_fma(e, ww, a1); else a0 = f2_fma(e, ww, a0);
+    }
   }
+  float s0, s1, s2, s3;
+  f2_split(a0, s0, s1);
+  f2_split(a1, s2, s3);
   return (s0 + s1) + (s2 + s3);
 }
 
@@ -328,7 +352,8 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sK = smem_u32(smem);
   const uint32_t sQ = sK + C::K_BYTES;
-  float2* mw = reinterpret_cast<float2*>(smem + C::K_BYTES + C::QSTAGES * C::QC_BYTES);
+  float* negm = reinterpret_cast<float*>(smem + C::K_BYTES + C::QSTAGES * C::QC_BYTES);  // -m_r
+  float* wr = negm + kMaxRows;                                                               // 1 / l_r
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::K_BYTES + C::QSTAGES * C::QC_BYTES + C::MW_BYTES);
 
   const int h = blockIdx.y, lb = blockIdx.z, b = lb % a.B;
@@ -341,11 +366,11 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int key0 = blockIdx.x * 256;
   if (key0 >= nv) return;
 
-  // row statistics of this head: (m_r, 1 / l_r); padding rows contribute 2^-inf * 0 = 0
+  // row statistics of this head: -m_r and 1 / l_r; padding rows contribute 2^(-inf or -125) * 0 = 0
   for (int r = threadIdx.x; r < nch * BN; r += kThreads) {
     const bool in = r < M;
-    mw[r] = in ? make_float2(a.row_m[(size_t)prob * M + r], 1.f / a.row_l[(size_t)prob * M + r])
-               : make_float2(INFINITY, 0.f);
+    negm[r] = in ? -a.row_m[(size_t)prob * M + r] : -INFINITY;
+    wr[r] = in ? 1.f / a.row_l[(size_t)prob * M + r] : 0.f;
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::QSTAGES; ++s) {
@@ -451,9 +476,9 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         tc::fence_after_sync();
         const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + blk * BN + g * kHalf;
-        const float2* mwc = mw + c * BN + g * kHalf;
+        const int r0 = c * BN + g * kHalf;
         float s = 0.f;
-        tmem_sweep4(base, [&](const uint32_t(&r)[32], int cc) { s += p2_chunk(r, mwc + cc * 32, sc); });
+        tmem_sweep4(base, [&](const uint32_t(&r)[32], int cc) { s += p2_chunk(r, negm + r0 + cc * 32, wr + r0 + cc * 32, sc); });
         acc[blk] += s;
         tc::fence_before_sync();
         tc::mbar_arrive(&ctl->accempty[blk]);

@@ -3,7 +3,7 @@
 // Same quantities as select_score.cu ("Methodik" item 4 of the gist.science
 // summary: average text-to-visual attention per (layer, KV head)):
 //   pass 1  m_r = max_n x_rn,  l_r = sum_n 2^(x_rn - m_r)        x = log2(e) q_r . k_n / sqrt(d)
-//   pass 2  score_n = 1/M sum_r 2^(x_rn - m_r) / l_r
+//   pass 2  score_n = 1/M sum_r 2^(x_rn - m_r) / l_r  = 1/M sum_r 2^(x_rn - m_r - log2 l_r)
 //
 // Pass 1: CTA = 128 text rows (the MMA M axis) of one (layer, seq, KV head);
 //   keys stream through a 3-stage TMA ring in 256-key tiles; S = Q K^T lands
@@ -115,20 +115,19 @@ __device__ __forceinline__ void p1_chunk(const uint32_t (&r)[32], int key, int n
   l += (s0 + s1) + (s2 + s3);
 }
 
-// Pass-2 epilogue on 32 logits of one key: sum_r 2^(x_r - m_r) w_r with -m_r and
-// w_r = 1 / l_r from shared memory (separate arrays, so pairs load directly).
-__device__ __forceinline__ float p2_chunk(const uint32_t (&r)[32], const float* negm, const float* w, float sc) {
+// Pass-2 epilogue on 32 logits of one key: sum_r 2^(x_r - m'_r), where
+// m'_r = m_r + log2 l_r folds the row normalisation 1 / l_r into the exponent
+// (shared memory holds -m'_r).
+__device__ __forceinline__ float p2_chunk(const uint32_t (&r)[32], const float* negm, float sc) {
   const f32x2 scc = f2_make(sc, sc);
   f32x2 a0 = f2_make(0.f, 0.f), a1 = a0;
 #pragma unroll
   for (int q = 0; q < 8; ++q) {  // 4 rows at a time
     const float4 nm4 = *reinterpret_cast<const float4*>(negm + 4 * q);
-    const float4 w4 = *reinterpret_cast<const float4*>(w + 4 * q);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int p = 2 * q + h;
       const f32x2 nm = h ? f2_make(nm4.z, nm4.w) : f2_make(nm4.x, nm4.y);
-      const f32x2 ww = h ? f2_make(w4.z, w4.w) : f2_make(w4.x, w4.y);
       const f32x2 x = f2_fma(f2_make(__uint_as_float(r[2 * p]), __uint_as_float(r[2 * p + 1])), scc, nm);
       f32x2 e;
       if (p < kPolyPairs) {
@@ -138,7 +137,7 @@ __device__ __forceinline__ float p2_chunk(const uint32_t (&r)[32], const float* 
         f2_split(x, x0, x1);
         e = f2_make(ex2(x0), ex2(x1));
       }
-      if (p & 1) a1 = f2_fma(e, ww, a1); else a0 = f2_fma(e, ww, a0);
+      if (p & 1) a1 = f2_add(a1, e); else a0 = f2_add(a0, e);
     }
   }
   float s0, s1, s2, s3;
@@ -337,7 +336,7 @@ struct P2 {
   static constexpr int QSTAGES = 2;
   static constexpr uint32_t K_BYTES = KB * 256 * 128;   // 256 keys = two 128-key MMA tiles
   static constexpr uint32_t QC_BYTES = KB * BN * 128;   // one chunk of 256 text rows
-  static constexpr uint32_t MW_BYTES = kMaxRows * 8;
+  static constexpr uint32_t MW_BYTES = kMaxRows * 4;
   static constexpr uint32_t SMEM = 1024 + K_BYTES + QSTAGES * QC_BYTES + MW_BYTES + sizeof(Ctl);
 };
 
@@ -352,8 +351,7 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sK = smem_u32(smem);
   const uint32_t sQ = sK + C::K_BYTES;
-  float* negm = reinterpret_cast<float*>(smem + C::K_BYTES + C::QSTAGES * C::QC_BYTES);  // -m_r
-  float* wr = negm + kMaxRows;                                                               // 1 / l_r
+  float* negm = reinterpret_cast<float*>(smem + C::K_BYTES + C::QSTAGES * C::QC_BYTES);  // -(m_r + log2 l_r)
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::K_BYTES + C::QSTAGES * C::QC_BYTES + C::MW_BYTES);
 
   const int h = blockIdx.y, lb = blockIdx.z, b = lb % a.B;
@@ -366,12 +364,10 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int key0 = blockIdx.x * 256;
   if (key0 >= nv) return;
 
-  // row statistics of this head: -m_r and 1 / l_r; padding rows contribute 2^(-inf or -125) * 0 = 0
-  for (int r = threadIdx.x; r < nch * BN; r += kThreads) {
-    const bool in = r < M;
-    negm[r] = in ? -a.row_m[(size_t)prob * M + r] : -INFINITY;
-    wr[r] = in ? 1.f / a.row_l[(size_t)prob * M + r] : 0.f;
-  }
+  // row statistics of this head as -(m_r + log2 l_r); padding rows get -inf (2^-inf = 0 on the
+  // SFU, 2^-125 ~ 2e-38 on the FMA pipe: negligible)
+  for (int r = threadIdx.x; r < nch * BN; r += kThreads)
+    negm[r] = r < M ? -(a.row_m[(size_t)prob * M + r] + log2f(a.row_l[(size_t)prob * M + r])) : -INFINITY;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::QSTAGES; ++s) {
       tc::mbar_init(&ctl->full[s], 1);
@@ -478,7 +474,7 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + blk * BN + g * kHalf;
         const int r0 = c * BN + g * kHalf;
         float s = 0.f;
-        tmem_sweep4(base, [&](const uint32_t(&r)[32], int cc) { s += p2_chunk(r, negm + r0 + cc * 32, wr + r0 + cc * 32, sc); });
+        tmem_sweep4(base, [&](const uint32_t(&r)[32], int cc) { s += p2_chunk(r, negm + r0 + cc * 32, sc); });
         acc[blk] += s;
         tc::fence_before_sync();
         tc::mbar_arrive(&ctl->accempty[blk]);

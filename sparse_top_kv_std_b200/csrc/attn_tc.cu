@@ -150,6 +150,7 @@ struct Cfg {
   static constexpr uint32_t T_BYTES = KB * TK * 128;   // one K or V tile
   static constexpr uint32_t ST_BYTES = 2 * T_BYTES;    // K + V
   static constexpr uint32_t SMEM = 1024 + Q_BYTES + STAGES * ST_BYTES + sizeof(Ctl);
+  static_assert(SMEM <= 232448, "dynamic shared memory above the 227 KB a CTA may use");
 };
 
 template <int D>

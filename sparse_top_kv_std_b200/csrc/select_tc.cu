@@ -175,6 +175,7 @@ struct P1 {
   static constexpr uint32_t Q_BYTES = KB * BM * 128;
   static constexpr uint32_t KT_BYTES = KB * BN * 128;
   static constexpr uint32_t SMEM = 1024 + Q_BYTES + STAGES * KT_BYTES + sizeof(Ctl);
+  static_assert(SMEM <= 232448, "dynamic shared memory above the 227 KB a CTA may use");
 };
 
 template <int D>
@@ -338,6 +339,7 @@ struct P2 {
   static constexpr uint32_t QC_BYTES = KB * BN * 128;   // one chunk of 256 text rows
   static constexpr uint32_t MW_BYTES = kMaxRows * 4;
   static constexpr uint32_t SMEM = 1024 + K_BYTES + QSTAGES * QC_BYTES + MW_BYTES + sizeof(Ctl);
+  static_assert(SMEM <= 232448, "dynamic shared memory above the 227 KB a CTA may use");
 };
 
 template <int D>

@@ -92,6 +92,21 @@ def attention_bytes(wl, rounds, accepted):
     return draft, verify, per_round_verify
 
 
+def dist_max(x, pg, device):
+    """Max of a per-rank float over all ranks (pg: torch.distributed or None)."""
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if pg is not None:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(bytes_per_step, steps, world, elapsed_ms):
+    """Whole-job GB/s: every rank processed `steps` steps of `bytes_per_step` in `elapsed_ms`
+    (the max over ranks)."""
+    return bytes_per_step * steps * world / (elapsed_ms / 1e3) / 1e9
+
+
 def select_flops(wl):
     """Executed MMA flops of the selection (2 passes over the M x Nv logits)."""
     M = wl.G * wl.T
@@ -446,10 +461,7 @@ def run_std(args, rank, world, local_rank):
     step(dev_ev, draft_ev=True)
     torch.cuda.synchronize()
     d_ms = [dev_ev["d0"][k].elapsed_time(dev_ev["d1"][k]) for k in range(R * wl.gamma)]
-    mx = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if pg:
-        pg.all_reduce(mx, op=pg.ReduceOp.MAX)
-    elapsed_ms = float(mx.item())
+    elapsed_ms = dist_max(elapsed_ms, pg, dev)
 
     # ---- e2e through the public API with host buffers (H2D of inputs, D2H of the accepted tokens)
     e2e = None
@@ -475,13 +487,10 @@ def run_std(args, rank, world, local_rank):
             e2e_step()
         a1.record(stream)
         torch.cuda.synchronize()
-        e_ms = torch.tensor([a0.elapsed_time(a1)], dtype=torch.float64, device=dev)
-        if pg:
-            pg.all_reduce(e_ms, op=pg.ReduceOp.MAX)
-        e_ms = float(e_ms.item())
+        e_ms = dist_max(a0.elapsed_time(a1), pg, dev)
         h2d = pin_k.numel() * pin_k.element_size() * 2 + sum(t.numel() * t.element_size() for t in pin.values())
         d2h = acc_host.numel() * 4
-        e2e = {"value": step_attn * args.e2e_steps * world / (e_ms / 1e3) / 1e9, "unit": "GB/s",
+        e2e = {"value": weak_scaling_value(step_attn, args.e2e_steps, world, e_ms), "unit": "GB/s",
                "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
@@ -491,7 +500,7 @@ def run_std(args, rank, world, local_rank):
         return 0
 
     peaks, peak_src = load_peaks()
-    value = step_attn * args.steps * world / (elapsed_ms / 1e3) / 1e9
+    value = weak_scaling_value(step_attn, args.steps, world, elapsed_ms)
     v_avg_ms = statistics.mean(v_ms)
     v_bytes_avg = verify_b / R
     achieved = v_bytes_avg / (v_avg_ms / 1e3) / 1e9

@@ -395,7 +395,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         float mx = v[0];
   #pragma unroll
-        for (int j = 1; j < TK; ++j) mx = fmaxf(mx, v[j]);
+        for (int j = 1; j + 1 < TK; j += 2) mx = max3f(mx, v[j], v[j + 1]);
+        mx = fmaxf(mx, v[TK - 1]);
         // lazy rescale: only when the max grows by more than 2^kTau (whole warp, O is warp-collective)
         const bool resc = (m != -INFINITY) && (mx - m) * sc > kTau;
         if (__any_sync(0xffffffffu, resc)) {
@@ -424,16 +425,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   #pragma unroll
         for (int c = 0; c < TK / 32; ++c) {
           uint32_t pk[16];
-          float s0 = 0.f, s1 = 0.f;
+          f32x2 sacc = f2_make(0.f, 0.f);
+          const f32x2 scc = f2_make(sc, sc), nm = f2_make(-msc, -msc);
   #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const float p0 = live ? ex2(fmaf(v[c * 32 + 2 * j], sc, -msc)) : 0.f;
-            const float p1 = live ? ex2(fmaf(v[c * 32 + 2 * j + 1], sc, -msc)) : 0.f;
-            s0 += p0;
-            s1 += p1;
+            float x0, x1;
+            f2_split(f2_fma(f2_make(v[c * 32 + 2 * j], v[c * 32 + 2 * j + 1]), scc, nm), x0, x1);
+            const float p0 = live ? ex2(x0) : 0.f;
+            const float p1 = live ? ex2(x1) : 0.f;
+            sacc = f2_add(sacc, f2_make(p0, p1));
             pk[j] = pack_bf16(p0, p1);
           }
-          l += s0 + s1;
+          float sl, sh;
+          f2_split(sacc, sl, sh);
+          l += sl + sh;
           __syncwarp();
           tc::tmem_st_x16(lane_base + kColS + bu * 128 + c * 16, pk);
         }

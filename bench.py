@@ -556,22 +556,37 @@ def gpu_uuid(dev):
         return None
 
 
-def load_traffic(kernel, workload):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged since."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(p):
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_dense_verify_attn_video_140k.txt")
+
+
+def sources_sha256(paths):
+    """sha256 over the concatenated bytes of the given repo-relative files."""
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def load_traffic(kernel, workload, path=TRAFFIC_FILE):
+    """DRAM bytes per launch from a committed ncu summary ("key: value" lines), or None when the
+    summary is missing, is for another kernel or workload, or its kernel sources changed since."""
+    if not os.path.exists(path):
         return None
-    with open(p) as f:
-        d = json.load(f)
-    e = d.get(kernel, {})
-    if e.get("workload") != workload:
+    kv = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith((" ", "#")):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+    if kv.get("kernel") != kernel or kv.get("workload") != workload:
         return None
-    src = os.path.join(ROOT, e.get("source", ""))
-    if not os.path.exists(src):
+    srcs = kv.get("sources", "").split()
+    if not srcs or not all(os.path.exists(os.path.join(ROOT, r)) for r in srcs):
         return None
-    with open(src, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()
-    return e.get("dram_bytes_per_launch") if sha == e.get("source_sha256") else None
+    if sources_sha256(srcs) != kv.get("sources_sha256"):
+        return None
+    return float(kv["dram_bytes_per_launch"])
 
 
 def main(argv=None):

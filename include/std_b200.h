@@ -33,7 +33,11 @@
  *    Conditions that depend on device-resident lengths are checked by the
  *    kernels: the offending (sequence, head) is skipped and a bit is OR-ed
  *    into a per-device error word, read with std_get_device_error().
- *  - No kernel waits on another kernel, CTA or device; nothing spins.
+ *  - No kernel waits on another kernel, CTA or device.  The tensor-core kernels
+ *    wait only on their own CTA's mbarriers (TMA arrivals, MMA commits, warp
+ *    hand-offs); every such wait gives up after 0.5 s, sets
+ *    STD_DEVERR_TIMEOUT, drains its copies in flight, frees its tensor memory
+ *    and returns.
  */
 #ifndef STD_B200_H
 #define STD_B200_H
@@ -55,7 +59,7 @@ enum std_status {
   STD_ERR_CAPACITY = -3,    /* a host-checkable size exceeds a cache capacity */
   STD_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed */
   STD_ERR_DEVICE = -5,      /* std_get_device_error found flags set */
-  STD_ERR_TIMEOUT = -6,     /* reserved: a bounded wait gave up (no current kernel waits) */
+  STD_ERR_TIMEOUT = -6,     /* reserved; a timed-out wait inside a kernel shows as STD_DEVERR_TIMEOUT */
   STD_ERR_WORKSPACE = -7    /* workspace missing or smaller than the size query returned */
 };
 
@@ -148,7 +152,10 @@ int std_topk_from_scores(const float* scores, int rows, int n, int K, int32_t* i
  * `splits` = 0 launches one CTA per SM, splits = s > 0 launches
  * s x L x B x Hkv CTAs.  fp32 operands (and bf16 with B > 64) use split-K
  * kernels with `splits` key ranges per problem (0 = automatic).  Either way
- * the partial results go to the workspace and a second kernel merges them.
+ * the partial results go to the workspace.  The tensor-core kernel merges them
+ * itself: the last CTA to finish a slice of a problem (an arrival counter per
+ * problem, no waiting) combines that problem's partials; the split-K kernels
+ * leave the merge to a second kernel.
  */
 
 /* Device workspace bytes for a decode-attention call with `q_rows` query rows

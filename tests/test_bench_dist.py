@@ -61,3 +61,19 @@ def test_reference_arm_runs_on_rank_zero_only():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_traffic_summary_is_used_only_while_its_sources_are_unchanged(tmp_path):
+    sys.path.insert(0, ROOT)
+    import bench
+    srcs = "sparse_top_kv_std_b200/csrc/attn_tc.cu sparse_top_kv_std_b200/csrc/tc100.cuh"
+    sha = bench.sources_sha256(srcs.split())
+    p = tmp_path / "t.txt"
+    body = ("# header\nkernel: dense_verify_attn\nworkload: video_140k\nsources: %s\nsources_sha256: %s\n"
+            "dram_bytes_per_launch: 8.3e9\ncommand: x: y\n")
+    p.write_text(body % (srcs, sha))
+    assert bench.load_traffic("dense_verify_attn", "video_140k", str(p)) == 8.3e9
+    assert bench.load_traffic("dense_verify_attn", "layer_16k", str(p)) is None
+    p.write_text(body % (srcs, "0" * 64))
+    assert bench.load_traffic("dense_verify_attn", "video_140k", str(p)) is None
+    assert bench.load_traffic("dense_verify_attn", "video_140k", str(tmp_path / "missing.txt")) is None

@@ -18,7 +18,7 @@
 // each accumulator's columns (TMEM lane quarter = warp % 4), so every SM
 // sub-partition has two epilogue warps to hide the TMEM-load latency, which
 // is pipelined one 32-column chunk ahead.  A quarter of the exponentials run
-// as a polynomial on the FMA pipe (exp2_fma) beside the special-function unit.
+// as a polynomial on the FMA pipe (exp2_fma2) beside the special-function unit.
 // Every wait is bounded; on a timeout the CTA raises its abort flag, records
 // the error, lets in-flight copies and MMAs finish (bounded), frees TMEM and
 // returns.  No multicast loads are used.
@@ -43,7 +43,10 @@ constexpr int BN = 256;      // MMA N (keys in pass 1, text rows in pass 2)
 constexpr int kMaxRows = 2048;  // G * T supported by pass 2 (row statistics kept in shared memory)
 constexpr int kTmemCols = 512;
 constexpr int kHalf = BN / 2;   // accumulator columns per epilogue warpgroup
-constexpr int kPolyPairs = 6;   // of every 16 pairs of exponentials, this many on the FMA pipe
+// Of every 16 pairs of exponentials, these 4 (spread through the chunk so both
+// pipes have work at every point of it) run as a polynomial on the FMA pipe,
+// the other 12 on the special-function unit.
+__host__ __device__ constexpr bool poly_pair(int p) { return (p & 3) == 1; }
 
 struct Ctl {
   uint64_t full[8], empty[8];
@@ -74,8 +77,8 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Pass-1 epilogue on 32 logits of one row: online max / sum of 2^(x - m).
-// Pairs of logits go through packed fp32 instructions; kPolyPairs of the 16
-// pairs take their exponential on the FMA pipe, the rest on the SFU.
+// Pairs of logits go through packed fp32 instructions; the pairs poly_pair()
+// picks take their exponential on the FMA pipe, the rest on the SFU.
 template <bool TAIL>
 __device__ __forceinline__ void p1_chunk(const uint32_t (&r)[32], int key, int nv, float sc, float& m, float& l) {
   float v[32];
@@ -100,7 +103,7 @@ __device__ __forceinline__ void p1_chunk(const uint32_t (&r)[32], int key, int n
   for (int p = 0; p < 16; ++p) {
     const f32x2 x = f2_fma(f2_make(v[2 * p], v[2 * p + 1]), scc, nm);
     f32x2 e;
-    if (p < kPolyPairs) {
+    if (poly_pair(p)) {
       e = exp2_fma2(x);
     } else {
       float x0, x1;
@@ -130,7 +133,7 @@ __device__ __forceinline__ float p2_chunk(const uint32_t (&r)[32], const float* 
       const f32x2 nm = h ? f2_make(nm4.z, nm4.w) : f2_make(nm4.x, nm4.y);
       const f32x2 x = f2_fma(f2_make(__uint_as_float(r[2 * p]), __uint_as_float(r[2 * p + 1])), scc, nm);
       f32x2 e;
-      if (p < kPolyPairs) {
+      if (poly_pair(p)) {
         e = exp2_fma2(x);
       } else {
         float x0, x1;

@@ -50,7 +50,34 @@ SELECT_CASES = {
 @pytest.mark.parametrize("name", sorted(SELECT_CASES))
 def test_select_topk_matches_oracle(name):
     wl = SELECT_CASES[name]
+    _check_select(wl, synth.host_inputs(wl, seed=0))
+
+
+def test_select_row_max_jumps_and_ramps():
+    """A per-key logit bias shared by every text row: all queries get +8 on component 0
+    and visual key n gets component 0 = t_n, which adds 8 t_n / sqrt(d) (about t_n in the
+    exp2 domain) to every row's logit of key n.  t jumps 0 -> 80, ramps 80 -> 110, drops
+    to 20, jumps to 118, so each row's running maximum rises within a tile by more than
+    the online-softmax rescale thresholds (2^8 and 2^64), while the softmax inside each
+    group of keys stays smooth (scores are not saturated)."""
+    wl = small_wl("max_jumps", nvis=(1500,), T=40, K=16, wl_id=104)
     x = synth.host_inputs(wl, seed=0)
+    nv = wl.nvis[0]
+    t = np.zeros(nv)
+    t[300:600] = 80.0
+    t[600:900] = 80.0 + 0.1 * np.arange(300)
+    t[900:1100] = 20.0
+    t[1100:] = 118.0
+    q = H.f64(x["q_text"], wl)
+    q[..., 0] += 8.0
+    k = H.f64(x["k_full"], wl)
+    k[:, :, :, :nv, 0] = t
+    x["q_text"] = synth.storage(q.astype(np.float32), wl.dtype)
+    x["k_full"] = synth.storage(k.astype(np.float32), wl.dtype)
+    _check_select(wl, x)
+
+
+def _check_select(wl, x):
     s = H.session_for(wl)
     s.k_full.copy_(H.to_dev(x["k_full"]))
     s.v_full.copy_(H.to_dev(x["v_full"]))

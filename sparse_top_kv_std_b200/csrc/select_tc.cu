@@ -10,15 +10,18 @@
 //   in a double-buffered TMEM accumulator (2 x 256 fp32 columns); each of the
 //   128 epilogue threads owns one row and keeps its running max / sum, so no
 //   cross-thread reduction is needed.
-// Pass 2: transposed.  CTA = 256 keys (two 128-key MMA tiles, M axis) kept in
-//   shared memory; the text rows stream through as 256-row chunks (N axis);
-//   each epilogue thread owns one key and sums its column in registers.
+// Pass 2: transposed.  CTA = four consecutive 256-key blocks of one head; each
+//   block's two 128-key halves (M axis) stay in shared memory while the text
+//   rows stream through as 128-row chunks (N axis); epilogue warpgroup g owns
+//   key half g through a double-buffered TMEM accumulator, so each thread sums
+//   the column of one key in registers and writes its score, with no merge.
 // Warp roles (320 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
-// issuer (one elected lane), warps 2-9 epilogue in two warpgroups that split
-// each accumulator's columns (TMEM lane quarter = warp % 4), so every SM
-// sub-partition has two epilogue warps to hide the TMEM-load latency, which
-// is pipelined one 32-column chunk ahead.  A quarter of the exponentials run
-// as a polynomial on the FMA pipe (exp2_fma2) beside the special-function unit.
+// issuer (one elected lane), warps 2-9 epilogue in two warpgroups (TMEM lane
+// quarter = warp % 4; pass 1 splits each accumulator's columns between them),
+// so every SM sub-partition has two epilogue warps to hide the TMEM-load
+// latency, which is pipelined one 32-column chunk ahead.  A quarter of the
+// exponentials run as a polynomial on the FMA pipe (exp2_fma2) beside the
+// special-function unit.
 // Every wait is bounded; on a timeout the CTA raises its abort flag, records
 // the error, lets in-flight copies and MMAs finish (bounded), frees TMEM and
 // returns.  No multicast loads are used.
@@ -50,11 +53,11 @@ __host__ __device__ constexpr bool poly_pair(int p) { return (p & 3) == 1; }
 
 struct Ctl {
   uint64_t full[8], empty[8];
-  uint64_t qfull, kfull, done;
-  uint64_t accfull[2], accempty[2];
+  uint64_t qfull, kfull, kempty, done;
+  uint64_t accfull[4], accempty[4];
   uint32_t tmem;
   int abort_flag;
-  int consumed;
+  int consumed, kconsumed;
 };
 
 __device__ __forceinline__ bool visual_ok(const ScoreArgs& a, int b, int* nv_out) {
@@ -149,26 +152,27 @@ __device__ __forceinline__ float p2_chunk(const uint32_t (&r)[32], const float* 
   return (s0 + s1) + (s2 + s3);
 }
 
-// Four 32-column TMEM chunks at `base`, each load issued one chunk ahead of its use.
-template <typename F>
-__device__ __forceinline__ void tmem_sweep4(uint32_t base, F&& use) {
+// NCH consecutive 32-column TMEM chunks at `base`, each load issued one chunk ahead of its use.
+template <int NCH, typename F>
+__device__ __forceinline__ void tmem_sweep(uint32_t base, F&& use) {
+  static_assert(NCH % 2 == 0, "chunks go in pairs");
   uint32_t ra[32], rb[32];
   __syncwarp();
   tc::tmem_ld_x32(base, ra);
   tc::tmem_ld_wait(ra);
-  __syncwarp();
-  tc::tmem_ld_x32(base + 32, rb);
-  use(ra, 0);
-  tc::tmem_ld_wait(rb);
-  __syncwarp();
-  tc::tmem_ld_x32(base + 64, ra);
-  use(rb, 1);
-  tc::tmem_ld_wait(ra);
-  __syncwarp();
-  tc::tmem_ld_x32(base + 96, rb);
-  use(ra, 2);
-  tc::tmem_ld_wait(rb);
-  use(rb, 3);
+#pragma unroll
+  for (int c = 0; c < NCH; c += 2) {
+    __syncwarp();
+    tc::tmem_ld_x32(base + (c + 1) * 32, rb);
+    use(ra, c);
+    tc::tmem_ld_wait(rb);
+    if (c + 2 < NCH) {
+      __syncwarp();
+      tc::tmem_ld_x32(base + (c + 2) * 32, ra);
+    }
+    use(rb, c + 1);
+    if (c + 2 < NCH) tc::tmem_ld_wait(ra);
+  }
 }
 
 template <int D>
@@ -302,9 +306,9 @@ rowstats_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + buf * BN + g * kHalf;
       const int key0 = t * BN + g * kHalf;
       if (t * BN + BN > nv) {
-        tmem_sweep4(base, [&](const uint32_t(&r)[32], int c) { p1_chunk<true>(r, key0 + c * 32, nv, sc, m, l); });
+        tmem_sweep<4>(base, [&](const uint32_t(&r)[32], int c) { p1_chunk<true>(r, key0 + c * 32, nv, sc, m, l); });
       } else {
-        tmem_sweep4(base, [&](const uint32_t(&r)[32], int c) { p1_chunk<false>(r, key0 + c * 32, nv, sc, m, l); });
+        tmem_sweep<4>(base, [&](const uint32_t(&r)[32], int c) { p1_chunk<false>(r, key0 + c * 32, nv, sc, m, l); });
       }
       tc::fence_before_sync();
       tc::mbar_arrive(&ctl->accempty[buf]);
@@ -334,17 +338,26 @@ rowstats_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   }
 }
 
+constexpr int BN2 = 128;       // text rows per pass-2 chunk (MMA N)
+constexpr int kKeyBlocks = 4;  // 256-key blocks one pass-2 CTA walks through
+
 template <int D>
 struct P2 {
   static constexpr int KB = D / 64;
-  static constexpr int QSTAGES = 2;
+  static constexpr int QSTAGES = 4;
   static constexpr uint32_t K_BYTES = KB * 256 * 128;   // 256 keys = two 128-key MMA tiles
-  static constexpr uint32_t QC_BYTES = KB * BN * 128;   // one chunk of 256 text rows
+  static constexpr uint32_t QC_BYTES = KB * BN2 * 128;  // one chunk of 128 text rows
   static constexpr uint32_t MW_BYTES = kMaxRows * 4;
   static constexpr uint32_t SMEM = 1024 + K_BYTES + QSTAGES * QC_BYTES + MW_BYTES + sizeof(Ctl);
   static_assert(SMEM <= 232448, "dynamic shared memory above the 227 KB a CTA may use");
 };
 
+// Pass 2.  CTA = kKeyBlocks consecutive 256-key blocks of one (layer, seq, KV head);
+// each block's two 128-key halves are the M axis of two MMAs per 128-row chunk of
+// text queries.  Epilogue warpgroup g owns key half g: its TMEM accumulator is
+// double-buffered over the chunks (columns (2g + chunk parity) * 128), so every
+// thread sums the whole column of one key in registers and writes its score
+// directly.  The next block's keys load while the last chunks are summed.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -362,16 +375,17 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int h = blockIdx.y, lb = blockIdx.z, b = lb % a.B;
   const int prob = lb * a.Hkv + h;
   const int M = a.G * a.T;
-  const int nch = (M + BN - 1) / BN;
+  const int nch = (M + BN2 - 1) / BN2;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int nv;
   if (!visual_ok(a, b, &nv)) return;  // pass 1 flagged it
-  const int key0 = blockIdx.x * 256;
-  if (key0 >= nv) return;
+  const int key_base = blockIdx.x * (kKeyBlocks * 256);
+  if (key_base >= nv) return;
+  const int nkb = min(kKeyBlocks, (nv - key_base + 255) / 256);
 
   // row statistics of this head as -(m_r + log2 l_r); padding rows get -inf (2^-inf = 0 on the
   // SFU, 2^-125 ~ 2e-38 on the FMA pipe: negligible)
-  for (int r = threadIdx.x; r < nch * BN; r += kThreads)
+  for (int r = threadIdx.x; r < nch * BN2; r += kThreads)
     negm[r] = r < M ? -(a.row_m[(size_t)prob * M + r] + log2f(a.row_l[(size_t)prob * M + r])) : -INFINITY;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::QSTAGES; ++s) {
@@ -379,13 +393,15 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tc::mbar_init(&ctl->empty[s], 1);
     }
     tc::mbar_init(&ctl->kfull, 1);
+    tc::mbar_init(&ctl->kempty, 1);
     tc::mbar_init(&ctl->done, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       tc::mbar_init(&ctl->accfull[i], 1);
-      tc::mbar_init(&ctl->accempty[i], kEpiThreads);
+      tc::mbar_init(&ctl->accempty[i], 128);
     }
     ctl->abort_flag = 0;
     ctl->consumed = 0;
+    ctl->kconsumed = 0;
     tc::fence_mbar_init();
   }
   if (warp == 1) {
@@ -403,92 +419,112 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (lane == 0) {
       tc::prefetch_tmap(&tm_q);
       tc::prefetch_tmap(&tm_k);
-      tc::mbar_expect_tx(&ctl->kfull, C::K_BYTES);
-#pragma unroll
-      for (int kb = 0; kb < C::KB; ++kb)
-        tc::tma_load_2d(sK + kb * 256 * 128, &tm_k, kb * 64, prob * (int)a.cap + key0, &ctl->kfull);
       const int qrow = (lb * a.Hq + h * a.G) * a.T;
-      int issued = 0;
-      for (int c = 0; c < nch; ++c) {
-        const int s = c % C::QSTAGES;
-        const uint32_t ph = (c / C::QSTAGES) & 1;
-        if (!tc::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag, a.err)) break;
-        tc::mbar_expect_tx(&ctl->full[s], C::QC_BYTES);
+      int issued = 0, kissued = 0;
+      bool ok = true;
+      for (int kbi = 0; ok && kbi < nkb; ++kbi) {
+        // the key buffer is free once every MMA of the previous block has completed
+        if (kbi > 0 && !tc::mbar_wait(&ctl->kempty, (kbi - 1) & 1, abort_flag, a.err)) break;
+        tc::mbar_expect_tx(&ctl->kfull, C::K_BYTES);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb)
-          tc::tma_load_2d(sQ + s * C::QC_BYTES + kb * BN * 128, &tm_q, kb * 64, qrow + c * BN, &ctl->full[s]);
-        issued = c + 1;
+          tc::tma_load_2d(sK + kb * 256 * 128, &tm_k, kb * 64, prob * (int)a.cap + key_base + kbi * 256,
+                          &ctl->kfull);
+        kissued = kbi + 1;
+        for (int c = 0; c < nch; ++c) {
+          const int qi = kbi * nch + c;
+          const int s = qi % C::QSTAGES;
+          const uint32_t ph = (qi / C::QSTAGES) & 1;
+          if (!tc::mbar_wait(&ctl->empty[s], ph ^ 1, abort_flag, a.err)) {
+            ok = false;
+            break;
+          }
+          tc::mbar_expect_tx(&ctl->full[s], C::QC_BYTES);
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb)
+            tc::tma_load_2d(sQ + s * C::QC_BYTES + kb * BN2 * 128, &tm_q, kb * 64, qrow + c * BN2, &ctl->full[s]);
+          issued = qi + 1;
+        }
       }
-      if (*abort_flag) {
-        drain_wait(&ctl->kfull, 0);
-        for (int c = *(volatile int*)&ctl->consumed; c < issued; ++c)
-          drain_wait(&ctl->full[c % C::QSTAGES], (c / C::QSTAGES) & 1);
+      if (*abort_flag) {  // let the copies still in flight land before the CTA goes away
+        for (int k = *(volatile int*)&ctl->kconsumed; k < kissued; ++k) drain_wait(&ctl->kfull, k & 1);
+        for (int qi = *(volatile int*)&ctl->consumed; qi < issued; ++qi)
+          drain_wait(&ctl->full[qi % C::QSTAGES], (qi / C::QSTAGES) & 1);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = tc::idesc_bf16(BM, BN);
-      bool ok = tc::mbar_wait(&ctl->kfull, 0, abort_flag, a.err);
-      bool issued_any = false;
-      for (int c = 0; ok && c < nch; ++c) {
-        const int s = c % C::QSTAGES;
-        const uint32_t ph = (c / C::QSTAGES) & 1;
-        if (!tc::mbar_wait(&ctl->full[s], ph, abort_flag, a.err)) break;
-        *(volatile int*)&ctl->consumed = c + 1;
-#pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
-          if (!tc::mbar_wait(&ctl->accempty[blk], (c & 1) ^ 1, abort_flag, a.err)) {
+      constexpr uint32_t idesc = tc::idesc_bf16(BM, BN2);
+      bool ok = true, issued_any = false;
+      for (int kbi = 0; ok && kbi < nkb; ++kbi) {
+        if (!tc::mbar_wait(&ctl->kfull, kbi & 1, abort_flag, a.err)) break;
+        *(volatile int*)&ctl->kconsumed = kbi + 1;
+        for (int c = 0; ok && c < nch; ++c) {
+          const int qi = kbi * nch + c;
+          const int s = qi % C::QSTAGES;
+          const uint32_t ph = (qi / C::QSTAGES) & 1;
+          if (!tc::mbar_wait(&ctl->full[s], ph, abort_flag, a.err)) {
             ok = false;
             break;
           }
-          tc::fence_after_sync();
-          const uint32_t d = tmem + blk * BN;
+          *(volatile int*)&ctl->consumed = qi + 1;
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = (k & 3) * 32;
-            const uint32_t ka = sK + (k >> 2) * 256 * 128 + blk * BM * 128 + off;
-            const uint32_t qa = sQ + s * C::QC_BYTES + (k >> 2) * BN * 128 + off;
-            tc::umma_bf16(d, tc::sdesc_sw128(ka), tc::sdesc_sw128(qa), idesc, k > 0 ? 1u : 0u);
+          for (int blk = 0; blk < 2; ++blk) {
+            const int acc = blk * 2 + (qi & 1);
+            if (!tc::mbar_wait(&ctl->accempty[acc], ((qi >> 1) & 1) ^ 1, abort_flag, a.err)) {
+              ok = false;
+              break;
+            }
+            tc::fence_after_sync();
+            const uint32_t d = tmem + acc * BN2;
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              const uint32_t off = (k & 3) * 32;
+              const uint32_t ka = sK + (k >> 2) * 256 * 128 + blk * BM * 128 + off;
+              const uint32_t qa = sQ + s * C::QC_BYTES + (k >> 2) * BN2 * 128 + off;
+              tc::umma_bf16(d, tc::sdesc_sw128(ka), tc::sdesc_sw128(qa), idesc, k > 0 ? 1u : 0u);
+            }
+            issued_any = true;
+            tc::umma_commit(&ctl->accfull[acc]);
           }
-          issued_any = true;
-          tc::umma_commit(&ctl->accfull[blk]);
+          if (!ok) break;
+          tc::umma_commit(&ctl->empty[s]);
         }
-        if (!ok) break;
-        tc::umma_commit(&ctl->empty[s]);
+        if (ok) tc::umma_commit(&ctl->kempty);
       }
-      if (*abort_flag && issued_any) {
+      if (*abort_flag && issued_any) {  // MMAs may still read shared memory / write TMEM
         tc::umma_commit(&ctl->done);
         drain_wait(&ctl->done, 0);
       }
     }
   } else {
-    const int g = (warp - 2) >> 2;
-    const int q = warp & 3;
+    const int g = (warp - 2) >> 2;  // key half (accumulator pair) this warpgroup owns
+    const int q = warp & 3;         // TMEM lane quarter this warp may access
     const int kl = q * 32 + lane;
     const float sc = kLog2e * rsqrtf((float)D);
-    float acc[2] = {0.f, 0.f};
+    const float invM = 1.f / (float)M;
     bool ok = true;
-    for (int c = 0; ok && c < nch; ++c) {
-#pragma unroll
-      for (int blk = 0; blk < 2; ++blk) {
-        if (!tc::mbar_wait_warp(&ctl->accfull[blk], c & 1, abort_flag, a.err)) {
+    for (int kbi = 0; ok && kbi < nkb; ++kbi) {
+      float colsum = 0.f;
+      for (int c = 0; c < nch; ++c) {
+        const int qi = kbi * nch + c;
+        const int acc = g * 2 + (qi & 1);
+        if (!tc::mbar_wait_warp(&ctl->accfull[acc], (qi >> 1) & 1, abort_flag, a.err)) {
           ok = false;
           break;
         }
         tc::fence_after_sync();
-        const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + blk * BN + g * kHalf;
-        const int r0 = c * BN + g * kHalf;
+        const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + acc * BN2;
         float s = 0.f;
-        tmem_sweep4(base, [&](const uint32_t(&r)[32], int cc) { s += p2_chunk(r, negm + r0 + cc * 32, sc); });
-        acc[blk] += s;
+        tmem_sweep<4>(base, [&](const uint32_t(&r)[32], int cc) { s += p2_chunk(r, negm + c * BN2 + cc * 32, sc); });
+        colsum += s;
         tc::fence_before_sync();
-        tc::mbar_arrive(&ctl->accempty[blk]);
+        tc::mbar_arrive(&ctl->accempty[acc]);
       }
+      if (!ok) break;
+      const int n = key_base + kbi * 256 + g * BM + kl;
+      if (n < nv) a.scores[(size_t)prob * a.nvis_max + n] = colsum * invM;
     }
-    // every MMA has completed once the last accumulator was read: the Q stages are free
-    float* part = reinterpret_cast<float*>(smem + C::K_BYTES);
-    part[(g * 2 + 0) * BM + kl] = acc[0];
-    part[(g * 2 + 1) * BM + kl] = acc[1];
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -496,15 +532,6 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncwarp();
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
-  } else if (warp >= 2 && warp < 6 && !*abort_flag) {
-    const int kl = (warp & 3) * 32 + lane;
-    const float* part = reinterpret_cast<const float*>(smem + C::K_BYTES);
-    const float invM = 1.f / (float)M;
-#pragma unroll
-    for (int blk = 0; blk < 2; ++blk) {
-      const int n = key0 + blk * BM + kl;
-      if (n < nv) a.scores[(size_t)prob * a.nvis_max + n] = (part[blk * BM + kl] + part[(2 + blk) * BM + kl]) * invM;
-    }
   }
 }
 
@@ -544,9 +571,8 @@ template <int D>
 static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s) {
   const uint64_t krows = (uint64_t)a.L * a.B * a.Hkv * a.cap;
   const uint64_t qrows = (uint64_t)a.L * a.B * a.Hq * a.T;
-  CUtensorMap tk, tq128, tq256;
-  if (!make_tmap_bf16_2d(&tk, a.k_full, D, krows, BN) || !make_tmap_bf16_2d(&tq128, a.q_text, D, qrows, BM) ||
-      !make_tmap_bf16_2d(&tq256, a.q_text, D, qrows, BN))
+  CUtensorMap tk, tq128;
+  if (!make_tmap_bf16_2d(&tk, a.k_full, D, krows, BN) || !make_tmap_bf16_2d(&tq128, a.q_text, D, qrows, BM))
     return cudaErrorNotSupported;
   cudaError_t e = cudaFuncSetAttribute(rowstats_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, P1<D>::SMEM);
   if (e != cudaSuccess) return e;
@@ -556,8 +582,9 @@ static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s) {
   e = launch_pdl(rowstats_tc_kernel<D>, dim3((M + BM - 1) / BM, a.Hkv, a.L * a.B), dim3(kThreads), P1<D>::SMEM, s,
                  tq128, tk, a);
   if (e != cudaSuccess) return e;
-  return launch_pdl(colsum_tc_kernel<D>, dim3((a.nvis_max + 255) / 256, a.Hkv, a.L * a.B), dim3(kThreads),
-                    P2<D>::SMEM, s, tq256, tk, a);
+  return launch_pdl(colsum_tc_kernel<D>, dim3((a.nvis_max + kKeyBlocks * 256 - 1) / (kKeyBlocks * 256), a.Hkv,
+                                              a.L * a.B),
+                    dim3(kThreads), P2<D>::SMEM, s, tq128, tk, a);
 }
 
 // tcgen05 path for bf16 operands; cudaErrorNotSupported for shapes it does not cover.

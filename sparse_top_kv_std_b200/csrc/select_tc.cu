@@ -7,19 +7,20 @@
 //
 // Pass 1: CTA = 128 text rows (the MMA M axis) of one (layer, seq, KV head);
 //   keys stream through a 3-stage TMA ring in 256-key tiles; S = Q K^T lands
-//   in a double-buffered TMEM accumulator (2 x 256 fp32 columns); each of the
-//   128 epilogue threads owns one row and keeps its running max / sum, so no
-//   cross-thread reduction is needed.
-// Pass 2: transposed.  CTA = four consecutive 256-key blocks of one head; each
+//   in a double-buffered TMEM accumulator (2 x 256 fp32 columns); four
+//   epilogue warpgroups each take 64 of every tile's columns, one row per
+//   thread with its running max / sum, merged once at the end.
+// Pass 2: transposed.  CTA = eight consecutive 256-key blocks of one head; each
 //   block's two 128-key halves (M axis) stay in shared memory while the text
 //   rows stream through as 128-row chunks (N axis); epilogue warpgroup g owns
 //   key half g through a double-buffered TMEM accumulator, so each thread sums
 //   the column of one key in registers and writes its score, with no merge.
-// Warp roles (320 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
-// issuer (one elected lane), warps 2-9 epilogue in two warpgroups (TMEM lane
-// quarter = warp % 4; pass 1 splits each accumulator's columns between them),
-// so every SM sub-partition has two epilogue warps to hide the TMEM-load
-// latency, which is pipelined one 32-column chunk ahead.  A quarter of the
+// Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer (one
+// elected lane), the rest epilogue warpgroups (TMEM lane quarter = warp % 4):
+// four in pass 1 (576 threads, 4 epilogue warps per SM sub-partition), two in
+// pass 2 (320 threads; its epilogue needs ~168 registers), so every SM
+// sub-partition has several epilogue warps to hide the TMEM-load latency,
+// which is pipelined one 32-column chunk ahead.  A quarter of the
 // exponentials run as a polynomial on the FMA pipe (exp2_fma2) beside the
 // special-function unit.
 // Every wait is bounded; on a timeout the CTA raises its abort flag, records
@@ -38,14 +39,14 @@
 namespace stdb {
 namespace {
 
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kThreads = 64 + 32 * 8;  // pass 2: producer, MMA, two epilogue warpgroups
 constexpr int BM = 128;      // MMA M
 constexpr int BN = 256;      // MMA N (keys in pass 1, text rows in pass 2)
 constexpr int kMaxRows = 2048;  // G * T supported by pass 2 (row statistics kept in shared memory)
 constexpr int kTmemCols = 512;
-constexpr int kHalf = BN / 2;   // accumulator columns per epilogue warpgroup
+constexpr int kP1Groups = 4;                      // pass-1 epilogue warpgroups
+constexpr int kP1Threads = 64 + 128 * kP1Groups;  // pass 1 launches 576 threads
+constexpr int kP1Cols = BN / kP1Groups;           // accumulator columns per pass-1 warpgroup
 // Of every 16 pairs of exponentials, these 4 (spread through the chunk so both
 // pipes have work at every point of it) run as a polynomial on the FMA pipe,
 // the other 12 on the special-function unit.
@@ -186,7 +187,7 @@ struct P1 {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kP1Threads, 1)
 rowstats_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const ScoreArgs a) {
   pdl_wait();  // memory of earlier kernels in the stream is visible from here on
@@ -219,7 +220,7 @@ rowstats_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tc::mbar_init(&ctl->done, 1);
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&ctl->accfull[i], 1);
-      tc::mbar_init(&ctl->accempty[i], kEpiThreads);
+      tc::mbar_init(&ctl->accempty[i], 128 * kP1Groups);
     }
     ctl->abort_flag = 0;
     ctl->consumed = 0;
@@ -293,7 +294,7 @@ rowstats_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       }
     }
   } else {
-    const int g = (warp - 2) >> 2;  // warpgroup: which half of the 256 columns
+    const int g = (warp - 2) >> 2;  // warpgroup: which 64 of the 256 columns
     const int q = warp & 3;         // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;
     const float sc = kLog2e * rsqrtf((float)D);
@@ -303,12 +304,12 @@ rowstats_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const uint32_t aph = (t >> 1) & 1;
       if (!tc::mbar_wait_warp(&ctl->accfull[buf], aph, abort_flag, a.err)) break;
       tc::fence_after_sync();
-      const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + buf * BN + g * kHalf;
-      const int key0 = t * BN + g * kHalf;
+      const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + buf * BN + g * kP1Cols;
+      const int key0 = t * BN + g * kP1Cols;
       if (t * BN + BN > nv) {
-        tmem_sweep<4>(base, [&](const uint32_t(&r)[32], int c) { p1_chunk<true>(r, key0 + c * 32, nv, sc, m, l); });
+        tmem_sweep<kP1Cols / 32>(base, [&](const uint32_t(&r)[32], int c) { p1_chunk<true>(r, key0 + c * 32, nv, sc, m, l); });
       } else {
-        tmem_sweep<4>(base, [&](const uint32_t(&r)[32], int c) { p1_chunk<false>(r, key0 + c * 32, nv, sc, m, l); });
+        tmem_sweep<kP1Cols / 32>(base, [&](const uint32_t(&r)[32], int c) { p1_chunk<false>(r, key0 + c * 32, nv, sc, m, l); });
       }
       tc::fence_before_sync();
       tc::mbar_arrive(&ctl->accempty[buf]);
@@ -324,13 +325,18 @@ rowstats_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
   } else if (warp >= 2 && warp < 6 && !*abort_flag) {
-    // merge the two column halves of each row: (m, l) in the exp2 domain
+    // merge the warpgroups' column groups of each row: (m, l) in the exp2 domain
     const int row = (warp & 3) * 32 + lane;
     const int r_glob = blockIdx.x * BM + row;
     const float2* part = reinterpret_cast<const float2*>(smem);
-    const float2 p0 = part[row], p1 = part[BM + row];
-    const float mm = fmaxf(p0.x, p1.x);
-    const float ll = (p0.y > 0.f ? p0.y * ex2(p0.x - mm) : 0.f) + (p1.y > 0.f ? p1.y * ex2(p1.x - mm) : 0.f);
+    float mm = -INFINITY, ll = 0.f;
+#pragma unroll
+    for (int gg = 0; gg < kP1Groups; ++gg) mm = fmaxf(mm, part[gg * BM + row].x);
+#pragma unroll
+    for (int gg = 0; gg < kP1Groups; ++gg) {
+      const float2 p = part[gg * BM + row];
+      if (p.y > 0.f) ll += p.y * ex2(p.x - mm);
+    }
     if (r_glob < M) {
       a.row_m[(size_t)prob * M + r_glob] = mm;
       a.row_l[(size_t)prob * M + r_glob] = ll;
@@ -339,7 +345,7 @@ rowstats_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 }
 
 constexpr int BN2 = 128;       // text rows per pass-2 chunk (MMA N)
-constexpr int kKeyBlocks = 4;  // 256-key blocks one pass-2 CTA walks through
+constexpr int kKeyBlocks = 8;  // 256-key blocks one pass-2 CTA walks through
 
 template <int D>
 struct P2 {
@@ -579,7 +585,7 @@ static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s) {
   e = cudaFuncSetAttribute(colsum_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, P2<D>::SMEM);
   if (e != cudaSuccess) return e;
   const int M = a.G * a.T;
-  e = launch_pdl(rowstats_tc_kernel<D>, dim3((M + BM - 1) / BM, a.Hkv, a.L * a.B), dim3(kThreads), P1<D>::SMEM, s,
+  e = launch_pdl(rowstats_tc_kernel<D>, dim3((M + BM - 1) / BM, a.Hkv, a.L * a.B), dim3(kP1Threads), P1<D>::SMEM, s,
                  tq128, tk, a);
   if (e != cudaSuccess) return e;
   return launch_pdl(colsum_tc_kernel<D>, dim3((a.nvis_max + kKeyBlocks * 256 - 1) / (kKeyBlocks * 256), a.Hkv,

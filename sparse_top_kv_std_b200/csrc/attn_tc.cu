@@ -17,7 +17,11 @@
 // partials of that problem.
 //
 // Per tile, inside a CTA (warp 0: TMA producers, lane 0 for K/V and lane 1 for
-// Q; warp 1: TMEM owner and MMA issuer; warps 2-5: one thread per query row):
+// Q; warp 1: TMEM owner and MMA issuer; warps 2-5: softmax -- one thread per
+// query row when a problem has more than 64 rows (M = 128 MMAs); with at most
+// 64 rows (the draft, and the verify up to gamma + 1 = 64 / G) the MMAs use
+// M = 64, which spreads the rows over all four TMEM lane quarters, so all four
+// SM sub-partitions share the softmax, two threads per row):
 //   TMA        K tile and V tile (128 keys x d, 128-byte swizzle) -> stage ring
 //   MMA        S = Q K^T  -> TMEM S buffer (double-buffered, 128 fp32 columns)
 //   softmax    row max, lazy rescale of O (only when the max grows by more than
@@ -153,7 +157,11 @@ struct Cfg {
   static_assert(SMEM <= 232448, "dynamic shared memory above the 227 KB a CTA may use");
 };
 
-template <int D>
+// HALF: at most 64 query rows per problem.  The MMAs then use M = 64, whose
+// accumulator row i sits in TMEM lane 32 * (i / 16) + i % 16, so the rows are
+// spread over all four lane quarters (and SM sub-partitions) and two softmax
+// threads share a row, each taking 64 of its 128 columns.
+template <int D, bool HALF>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
@@ -257,8 +265,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && g0 < g1) {
-      constexpr uint32_t idS = tc::idesc_bf16(128, TK);
-      constexpr uint32_t idPV = tc::idesc_bf16(128, D) | (1u << 16);  // B = V, MN-major
+      constexpr int MM = HALF ? 64 : 128;  // MMA M: query rows covered
+      constexpr uint32_t idS = tc::idesc_bf16(MM, TK);
+      constexpr uint32_t idPV = tc::idesc_bf16(MM, D) | (1u << 16);  // B = V, MN-major
       Iter it;
       iter_seek(it, ctl, a, g0, g1);
       int seg = -1, kv = 0, u = 0;
@@ -325,10 +334,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
     }
   } else {
-    // ------------------------------------------------------------ one thread per query row
-    const int row = (warp & 3) * 32 + lane;  // = TMEM lane of this thread
-    const bool wactive = (warp & 3) * 32 < a.rows;  // warp holds at least one real query row
-    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    // ------------------------------------------------------------ softmax threads
+    // Full layout: one thread per query row = TMEM lane (warp % 4) * 32 + lane, all 128
+    // columns of S.  HALF layout: query row (warp % 4) * 16 + lane % 16 in TMEM lane
+    // (warp % 4) * 32 + lane % 16; lane < 16 takes columns [0, 64), lane >= 16 [64, 128).
+    constexpr int NC = HALF ? TK / 2 : TK;  // S columns per thread
+    constexpr int OC = HALF ? D / 2 : D;    // O columns per thread
+    const int qd = warp & 3;                // TMEM lane quarter of this warp
+    const int row = HALF ? qd * 16 + (lane & 15) : qd * 32 + lane;  // query row of this thread
+    const int hh = HALF ? lane >> 4 : 0;    // which column half (HALF layout)
+    const bool wactive = (HALF ? qd * 16 : qd * 32) < a.rows;  // warp holds at least one real query row
+    const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
     const float sc = kLog2e * rsqrtf((float)D);
     const int tid = threadIdx.x - 64;
     Iter it;
@@ -366,37 +382,53 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc::fence_proxy_async();
       }
       if (wactive) {
-        // S row of this thread: 128 logits
-        float v[TK];
+        // this thread's logits of the tile: v[j] is key kc0 + j
+        float v[NC];
+        const int kc0 = key0 + hh * NC;
         {
-          uint32_t r0[32], r1[32], r2[32], r3[32];
           const uint32_t sa = lane_base + kColS + bu * 128;
-          __syncwarp();
-          tc::tmem_ld_x32(sa, r0);
-          tc::tmem_ld_x32(sa + 32, r1);
-          tc::tmem_ld_x32(sa + 64, r2);
-          tc::tmem_ld_x32(sa + 96, r3);
-          tc::tmem_ld_wait(r0);
-          tc::tmem_ld_wait(r1);
-          tc::tmem_ld_wait(r2);
-          tc::tmem_ld_wait(r3);
+          if constexpr (HALF) {
+            uint32_t r0[32], r1[32];
+            __syncwarp();
+            tc::tmem_ld16_x32<TK / 2>(sa, r0);
+            tc::tmem_ld16_x32<TK / 2>(sa + 32, r1);
+            tc::tmem_ld_wait(r0);
+            tc::tmem_ld_wait(r1);
   #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            v[j] = __uint_as_float(r0[j]);
-            v[32 + j] = __uint_as_float(r1[j]);
-            v[64 + j] = __uint_as_float(r2[j]);
-            v[96 + j] = __uint_as_float(r3[j]);
+            for (int j = 0; j < 32; ++j) {
+              v[j] = __uint_as_float(r0[j]);
+              v[32 + j] = __uint_as_float(r1[j]);
+            }
+          } else {
+            uint32_t r0[32], r1[32], r2[32], r3[32];
+            __syncwarp();
+            tc::tmem_ld_x32(sa, r0);
+            tc::tmem_ld_x32(sa + 32, r1);
+            tc::tmem_ld_x32(sa + 64, r2);
+            tc::tmem_ld_x32(sa + 96, r3);
+            tc::tmem_ld_wait(r0);
+            tc::tmem_ld_wait(r1);
+            tc::tmem_ld_wait(r2);
+            tc::tmem_ld_wait(r3);
+  #pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              v[j] = __uint_as_float(r0[j]);
+              v[32 + j] = __uint_as_float(r1[j]);
+              v[64 + j] = __uint_as_float(r2[j]);
+              v[96 + j] = __uint_as_float(r3[j]);
+            }
           }
         }
-        if (key0 + TK > lim) {
+        if (kc0 + NC > lim) {
   #pragma unroll
-          for (int j = 0; j < TK; ++j)
-            if (key0 + j >= lim) v[j] = -INFINITY;
+          for (int j = 0; j < NC; ++j)
+            if (kc0 + j >= lim) v[j] = -INFINITY;
         }
         float mx = v[0];
   #pragma unroll
-        for (int j = 1; j + 1 < TK; j += 2) mx = max3f(mx, v[j], v[j + 1]);
-        mx = fmaxf(mx, v[TK - 1]);
+        for (int j = 1; j + 1 < NC; j += 2) mx = max3f(mx, v[j], v[j + 1]);
+        mx = fmaxf(mx, v[NC - 1]);
+        if constexpr (HALF) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));  // both halves of the row
         // lazy rescale: only when the max grows by more than 2^kTau (whole warp, O is warp-collective)
         const bool resc = (m != -INFINITY) && (mx - m) * sc > kTau;
         if (__any_sync(0xffffffffu, resc)) {
@@ -405,14 +437,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           tc::fence_after_sync();
           const float f = resc ? ex2((m - mx) * sc) : 1.f;
   #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < OC / 32; ++c) {  // this thread's O columns
             uint32_t o[32];
             __syncwarp();
-            tc::tmem_ld_x32(lane_base + c * 32, o);
+            if constexpr (HALF) tc::tmem_ld16_x32<D / 2>(lane_base + c * 32, o);
+            else tc::tmem_ld_x32(lane_base + c * 32, o);
             tc::tmem_ld_wait(o);
   #pragma unroll
             for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
-            tc::tmem_st_x32(lane_base + c * 32, o);
+            if constexpr (HALF) tc::tmem_st16_x32<D / 2>(lane_base + c * 32, o);
+            else tc::tmem_st_x32(lane_base + c * 32, o);
           }
           tc::tmem_st_wait();
           l *= f;
@@ -422,11 +456,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const float msc = m * sc;
         const bool live = m != -INFINITY;
         // P = 2^(x - m) as bf16 pairs, written over the S columns already read
+        // (packed column j of the tile holds keys 2j and 2j + 1)
+        uint32_t pk[NC / 2];
+        const f32x2 scc = f2_make(sc, sc), nm = f2_make(-msc, -msc);
   #pragma unroll
-        for (int c = 0; c < TK / 32; ++c) {
-          uint32_t pk[16];
+        for (int c = 0; c < NC / 32; ++c) {
           f32x2 sacc = f2_make(0.f, 0.f);
-          const f32x2 scc = f2_make(sc, sc), nm = f2_make(-msc, -msc);
   #pragma unroll
           for (int j = 0; j < 16; ++j) {
             float x0, x1;
@@ -434,13 +469,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const float p0 = live ? ex2(x0) : 0.f;
             const float p1 = live ? ex2(x1) : 0.f;
             sacc = f2_add(sacc, f2_make(p0, p1));
-            pk[j] = pack_bf16(p0, p1);
+            pk[c * 16 + j] = pack_bf16(p0, p1);
           }
           float sl, sh;
           f2_split(sacc, sl, sh);
-          l += sl + sh;
+          l += sl + sh;  // HALF: this thread's half of the row sum
+          if constexpr (!HALF) {
+            __syncwarp();
+            tc::tmem_st_x16(lane_base + kColS + bu * 128 + c * 16, reinterpret_cast<const uint32_t(&)[16]>(pk[c * 16]));
+          }
+        }
+        if constexpr (HALF) {
           __syncwarp();
-          tc::tmem_st_x16(lane_base + kColS + bu * 128 + c * 16, pk);
+          tc::tmem_st16_x32<TK / 4>(lane_base + kColS + bu * 128, pk);
         }
         tc::tmem_st_wait();
       }
@@ -449,21 +490,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (last) {
         if (!tc::mbar_wait_warp(&ctl->o_ready, seg & 1, abort_flag, a.err)) break;
         tc::fence_after_sync();
+        const float lrow = HALF ? l + __shfl_xor_sync(0xffffffffu, l, 16) : l;  // the whole row's sum
         // CTAs whose slices touch this problem
         const int start = it.l * ctl->tl + ctl->pre_b[it.b] + it.h * it.nt;
         const int c0 = start / ctl->per, c1 = (start + it.nt - 1) / ctl->per;
         const size_t orow = (size_t)(lb * a.Hq + it.h * a.G) * a.nq + row;
         if (c0 == c1) {
           // this CTA saw the whole problem: normalised output straight from TMEM
-          const float inv = l > 0.f ? 1.f / l : 0.f;
+          const float inv = lrow > 0.f ? 1.f / lrow : 0.f;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < OC / 32; ++c) {
             uint32_t o[32];
             __syncwarp();
-            tc::tmem_ld_x32(lane_base + c * 32, o);
+            if constexpr (HALF) tc::tmem_ld16_x32<D / 2>(lane_base + c * 32, o);
+            else tc::tmem_ld_x32(lane_base + c * 32, o);
             tc::tmem_ld_wait(o);
             if (row < a.rows) {
-              float* dst = a.o + orow * D + c * 32;
+              float* dst = a.o + orow * D + hh * OC + c * 32;
 #pragma unroll
               for (int j = 0; j < 32; j += 4)
                 *reinterpret_cast<float4*>(dst + j) =
@@ -478,12 +521,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           float* ml = a.ws + nslots * a.rows * D;
           unsigned long long* ctr = reinterpret_cast<unsigned long long*>(ml + nslots * a.rows * 2);
           const int slot = prob + blockIdx.x;
-          float* po = a.ws + ((size_t)slot * a.rows + row) * D;
+          float* po = a.ws + ((size_t)slot * a.rows + row) * D + hh * OC;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < OC / 32; ++c) {
             uint32_t o[32];
             __syncwarp();
-            tc::tmem_ld_x32(lane_base + c * 32, o);
+            if constexpr (HALF) tc::tmem_ld16_x32<D / 2>(lane_base + c * 32, o);
+            else tc::tmem_ld_x32(lane_base + c * 32, o);
             tc::tmem_ld_wait(o);
             if (row < a.rows) {
 #pragma unroll
@@ -493,9 +537,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                 __uint_as_float(o[j + 3]));
             }
           }
-          if (row < a.rows) {
+          if (row < a.rows && hh == 0) {
             ml[((size_t)slot * a.rows + row) * 2] = m * sc;
-            ml[((size_t)slot * a.rows + row) * 2 + 1] = l;
+            ml[((size_t)slot * a.rows + row) * 2 + 1] = lrow;
           }
           tc::fence_before_sync();
           tc::mbar_arrive(&ctl->o_free);  // O may be reused: the rest reads global memory only
@@ -565,9 +609,12 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   if (!make_tmap_bf16_2d(&tq, a.q, D, qrows, 128) || !make_tmap_bf16_2d(&tk, a.k, D, krows, TK) ||
       !make_tmap_bf16_2d(&tv, a.v, D, krows, TK))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  // at most 64 query rows per problem (the draft's G rows, the verify's G * (gamma + 1)
+  // up to 64): M = 64 MMAs and the spread softmax layout
+  auto kern = a.rows <= 64 ? attn_tc_kernel<D, true> : attn_tc_kernel<D, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  return launch_pdl(attn_tc_kernel<D>, dim3(a.splits), dim3(kThreads), C::SMEM, s, tq, tk, tv, a);
+  return launch_pdl(kern, dim3(a.splits), dim3(kThreads), C::SMEM, s, tq, tk, tv, a);
 }
 
 }  // namespace

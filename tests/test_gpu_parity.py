@@ -149,6 +149,9 @@ ATTN_CASES = {
     "G16_g7": small_wl("G16_g7", Hq=32, Hkv=2, nvis=(700,), T=9, K=64, gamma=7, wl_id=96),
     "f32_d128_g6": small_wl("f32_d128_g6", dtype="f32", Hq=6, Hkv=3, d=128, nvis=(300,), T=11, K=40,
                             gamma=6, wl_id=97),
+    # query rows per problem at the edges of the M = 64 layout: 8 * 8 = 64 (d = 64), 13 * 5 = 65
+    "rows64_d64": small_wl("rows64_d64", Hq=16, Hkv=2, d=64, nvis=(1300,), T=5, K=200, gamma=7, wl_id=105),
+    "rows65": small_wl("rows65", Hq=13, Hkv=1, nvis=(800,), T=6, K=100, gamma=4, wl_id=106),
 }
 
 

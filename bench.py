@@ -18,6 +18,7 @@ the max over ranks.  Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import os
@@ -38,7 +39,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["std", "reference"], default="std")
     ap.add_argument("--workload", default="video_140k")
@@ -116,12 +117,17 @@ def select_flops(wl):
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+    """nvidia-smi samples every 50 ms, started before the warm-up so that the tool is up by
+    the time the timed region starts; stop(window) keeps the samples whose timestamps fall
+    inside the timed region (host wall-clock seconds), or the two nearest ones, marked, if the
+    region was shorter than the sampling interval."""
+    FIELDS = ["timestamp", "index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
               "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
               "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
 
-    def __init__(self, gpu_id):
+    def __init__(self, gpu_id, interval_ms=50):
         self.gpu_id = gpu_id
+        self.interval_ms = interval_ms
         self.proc = None
         self.path = None
 
@@ -131,14 +137,21 @@ class ClockSampler:
             os.close(fd)
             self.f = open(self.path, "w")
             cmd = ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
-                   "-lms", "200"]
+                   "-lms", str(self.interval_ms)]
             if self.gpu_id is not None:
                 cmd += ["-i", str(self.gpu_id)]
             self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
 
-    def stop(self):
+    @staticmethod
+    def _when(ts):
+        try:
+            return datetime.datetime.strptime(ts.strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
+
+    def stop(self, window=None):
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -154,7 +167,22 @@ class ClockSampler:
                 if len(parts) == len(self.FIELDS):
                     rows.append(parts)
         os.unlink(self.path)
-        if not rows:
+        return self.summarise(rows, window)
+
+    @classmethod
+    def summarise(cls, rows, window=None):
+        """Clock summary of nvidia-smi rows (FIELDS order); window = (t0, t1) host seconds."""
+        kept, where = rows, "all"
+        if window is not None:
+            timed = [(cls._when(r[0]), r) for r in rows]
+            timed = [(t, r) for t, r in timed if t is not None]
+            kept = [r for t, r in timed if window[0] <= t <= window[1]]
+            where = "timed region"
+            if not kept and timed:
+                mid = 0.5 * (window[0] + window[1])
+                kept = [r for _, r in sorted(timed, key=lambda tr: abs(tr[0] - mid))[:2]]
+                where = "nearest to the timed region"
+        if not kept:
             return None
 
         def num(x):
@@ -162,18 +190,18 @@ class ClockSampler:
                 return float(x)
             except ValueError:
                 return None
-        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
-        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+        sm = [num(r[2]) for r in kept if num(r[2]) is not None]
+        pw = [num(r[4]) for r in kept if num(r[4]) is not None]
         reasons = set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            for n, v in zip(names, r[5:9]):
+        for r in kept:
+            for n, v in zip(names, r[6:10]):
                 if v.lower() == "active":
                     reasons.add(n)
-        load = [s for s, p in zip(sm, pw) if pw and p >= 0.5 * max(pw)] or sm
+        load = [x for x, p in zip(sm, pw) if pw and p >= 0.5 * max(pw)] or sm
         return {"sm_mhz": statistics.median(load) if load else None,
-                "sm_max_mhz": num(rows[0][2]), "power_w_max": max(pw) if pw else None,
-                "samples": len(rows), "reasons": sorted(reasons)}
+                "sm_max_mhz": num(kept[0][3]), "power_w_max": max(pw) if pw else None,
+                "samples": len(kept), "window": where, "reasons": sorted(reasons)}
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) sample
@@ -421,7 +449,10 @@ def run_std(args, rank, world, local_rank):
                 "d1": [E() for _ in range(R * wl.gamma)], "v0": [E() for _ in range(R)],
                 "v1": [E() for _ in range(R)]}
 
-    # ---- warm-up (also yields the acceptance counts of the byte model)
+    # ---- warm-up (also yields the acceptance counts of the byte model); the clock sampler
+    # starts here so that nvidia-smi is sampling by the time the timed region begins
+    clk = ClockSampler(gpu_uuid(dev))
+    clk.start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -438,14 +469,14 @@ def run_std(args, rank, world, local_rank):
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
-    clk = ClockSampler(gpu_uuid(dev))
-    clk.start()
+    w0 = time.time()
     t0.record(stream)
     for i in range(args.steps):
         step(evs[i])
     t1.record(stream)
     torch.cuda.synchronize()
-    clocks = clk.stop()
+    w1 = time.time()
+    clocks = clk.stop(window=(w0, w1))
     if pg:
         pg.barrier()
     elapsed_ms = t0.elapsed_time(t1)

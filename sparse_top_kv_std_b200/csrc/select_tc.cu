@@ -12,15 +12,15 @@
 //   thread with its running max / sum, merged once at the end.
 // Pass 2: transposed.  CTA = eight consecutive 256-key blocks of one head; each
 //   block's two 128-key halves (M axis) stay in shared memory while the text
-//   rows stream through as 128-row chunks (N axis); epilogue warpgroup g owns
-//   key half g through a double-buffered TMEM accumulator, so each thread sums
-//   the column of one key in registers and writes its score, with no merge.
+//   rows stream through as 128-row chunks (N axis) into four TMEM accumulators
+//   (key half x chunk parity); each of the four epilogue warpgroups owns one,
+//   so each thread sums half of one key's column in registers, and the two
+//   halves meet once per key block in shared memory.
 // Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer (one
 // elected lane), the rest epilogue warpgroups (TMEM lane quarter = warp % 4):
-// four in pass 1 (576 threads, 4 epilogue warps per SM sub-partition), two in
-// pass 2 (320 threads; its epilogue needs ~168 registers), so every SM
-// sub-partition has several epilogue warps to hide the TMEM-load latency,
-// which is pipelined one 32-column chunk ahead.  A quarter of the
+// four in each pass (576 threads, 4 epilogue warps per SM sub-partition), so
+// every SM sub-partition has several epilogue warps to hide the TMEM-load and
+// dependency latency; TMEM loads are pipelined one 32-column chunk ahead.  A quarter of the
 // exponentials run as a polynomial on the FMA pipe (exp2_fma2) beside the
 // special-function unit.
 // Every wait is bounded; on a timeout the CTA raises its abort flag, records
@@ -39,7 +39,7 @@
 namespace stdb {
 namespace {
 
-constexpr int kThreads = 64 + 32 * 8;  // pass 2: producer, MMA, two epilogue warpgroups
+constexpr int kThreads = 64 + 32 * 16;  // pass 2: producer, MMA, four epilogue warpgroups (576)
 constexpr int BM = 128;      // MMA M
 constexpr int BN = 256;      // MMA N (keys in pass 1, text rows in pass 2)
 constexpr int kMaxRows = 2048;  // G * T supported by pass 2 (row statistics kept in shared memory)
@@ -56,6 +56,7 @@ struct Ctl {
   uint64_t full[8], empty[8];
   uint64_t qfull, kfull, kempty, done;
   uint64_t accfull[4], accempty[4];
+  uint64_t xfull[4], xempty[4];
   uint32_t tmem;
   int abort_flag;
   int consumed, kconsumed;
@@ -354,16 +355,19 @@ struct P2 {
   static constexpr uint32_t K_BYTES = KB * 256 * 128;   // 256 keys = two 128-key MMA tiles
   static constexpr uint32_t QC_BYTES = KB * BN2 * 128;  // one chunk of 128 text rows
   static constexpr uint32_t MW_BYTES = kMaxRows * 4;
-  static constexpr uint32_t SMEM = 1024 + K_BYTES + QSTAGES * QC_BYTES + MW_BYTES + sizeof(Ctl);
+  static constexpr uint32_t XCH_BYTES = 4 * 128 * 4;  // partial column sums: [key half][slot][key]
+  static constexpr uint32_t SMEM = 1024 + K_BYTES + QSTAGES * QC_BYTES + MW_BYTES + XCH_BYTES + sizeof(Ctl);
   static_assert(SMEM <= 232448, "dynamic shared memory above the 227 KB a CTA may use");
 };
 
 // Pass 2.  CTA = kKeyBlocks consecutive 256-key blocks of one (layer, seq, KV head);
 // each block's two 128-key halves are the M axis of two MMAs per 128-row chunk of
-// text queries.  Epilogue warpgroup g owns key half g: its TMEM accumulator is
-// double-buffered over the chunks (columns (2g + chunk parity) * 128), so every
-// thread sums the whole column of one key in registers and writes its score
-// directly.  The next block's keys load while the last chunks are summed.
+// text queries.  The accumulator of (key half h, chunk parity p) sits at TMEM
+// columns (2h + p) * 128, and epilogue warpgroup 2p + h owns it: each thread sums
+// one key's column over the chunks of its parity in registers; per key block the
+// parity-1 warpgroup leaves its sums in a double-buffered shared-memory slot and
+// the parity-0 warpgroup adds them and writes the scores.  The next block's keys
+// load while the last chunks are summed.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -376,7 +380,8 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const uint32_t sK = smem_u32(smem);
   const uint32_t sQ = sK + C::K_BYTES;
   float* negm = reinterpret_cast<float*>(smem + C::K_BYTES + C::QSTAGES * C::QC_BYTES);  // -(m_r + log2 l_r)
-  Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::K_BYTES + C::QSTAGES * C::QC_BYTES + C::MW_BYTES);
+  float* xch = reinterpret_cast<float*>(smem + C::K_BYTES + C::QSTAGES * C::QC_BYTES + C::MW_BYTES);
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::K_BYTES + C::QSTAGES * C::QC_BYTES + C::MW_BYTES + C::XCH_BYTES);
 
   const int h = blockIdx.y, lb = blockIdx.z, b = lb % a.B;
   const int prob = lb * a.Hkv + h;
@@ -404,6 +409,8 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     for (int i = 0; i < 4; ++i) {
       tc::mbar_init(&ctl->accfull[i], 1);
       tc::mbar_init(&ctl->accempty[i], 128);
+      tc::mbar_init(&ctl->xfull[i], 128);
+      tc::mbar_init(&ctl->xempty[i], 128);
     }
     ctl->abort_flag = 0;
     ctl->consumed = 0;
@@ -504,8 +511,11 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
     }
   } else {
-    const int g = (warp - 2) >> 2;  // key half (accumulator pair) this warpgroup owns
-    const int q = warp & 3;         // TMEM lane quarter this warp may access
+    const int wg = (warp - 2) >> 2;  // epilogue warpgroup 0..3
+    const int blk = wg & 1;          // key half it owns
+    const int par = wg >> 1;         // chunk parity it sums (its accumulator: blk * 2 + par)
+    const int acc = blk * 2 + par;
+    const int q = warp & 3;          // TMEM lane quarter this warp may access
     const int kl = q * 32 + lane;
     const float sc = kLog2e * rsqrtf((float)D);
     const float invM = 1.f / (float)M;
@@ -514,7 +524,7 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       float colsum = 0.f;
       for (int c = 0; c < nch; ++c) {
         const int qi = kbi * nch + c;
-        const int acc = g * 2 + (qi & 1);
+        if ((qi & 1) != par) continue;
         if (!tc::mbar_wait_warp(&ctl->accfull[acc], (qi >> 1) & 1, abort_flag, a.err)) {
           ok = false;
           break;
@@ -528,8 +538,21 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc::mbar_arrive(&ctl->accempty[acc]);
       }
       if (!ok) break;
-      const int n = key_base + kbi * 256 + g * BM + kl;
-      if (n < nv) a.scores[(size_t)prob * a.nvis_max + n] = colsum * invM;
+      // the two parities of a key half meet in a double-buffered shared-memory slot
+      const int slot = kbi & 1;
+      const uint32_t use = (uint32_t)(kbi >> 1) & 1;
+      float* x = xch + (blk * 2 + slot) * 128;
+      if (par == 1) {
+        if (!tc::mbar_wait_warp(&ctl->xempty[blk * 2 + slot], use ^ 1, abort_flag, a.err)) break;
+        x[kl] = colsum;
+        tc::mbar_arrive(&ctl->xfull[blk * 2 + slot]);
+      } else {
+        if (!tc::mbar_wait_warp(&ctl->xfull[blk * 2 + slot], use, abort_flag, a.err)) break;
+        const float total = colsum + x[kl];
+        tc::mbar_arrive(&ctl->xempty[blk * 2 + slot]);
+        const int n = key_base + kbi * 256 + blk * BM + kl;
+        if (n < nv) a.scores[(size_t)prob * a.nvis_max + n] = total * invM;
+      }
     }
   }
   tc::fence_before_sync();

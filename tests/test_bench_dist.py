@@ -77,3 +77,24 @@ def test_traffic_summary_is_used_only_while_its_sources_are_unchanged(tmp_path):
     p.write_text(body % (srcs, "0" * 64))
     assert bench.load_traffic("dense_verify_attn", "video_140k", str(p)) is None
     assert bench.load_traffic("dense_verify_attn", "video_140k", str(tmp_path / "missing.txt")) is None
+
+
+def test_clock_summary_keeps_samples_of_the_timed_region():
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import bench
+
+    def row(t, mhz, reason="Not Active", power="600.0"):
+        ts = datetime.datetime.fromtimestamp(t).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return [ts, "0", str(mhz), "1965", power, "0x0", "Not Active", "Not Active", "Not Active", reason]
+
+    t = 1_800_000_000.0
+    rows = [row(t, 1000), row(t + 1.0, 1600, "Active"), row(t + 1.1, 1700), row(t + 2.0, 900)]
+    s = bench.ClockSampler.summarise(rows, window=(t + 0.95, t + 1.15))
+    assert s["samples"] == 2 and s["window"] == "timed region"
+    assert s["sm_mhz"] == 1650 and s["reasons"] == ["sw_power_cap"] and s["sm_max_mhz"] == 1965
+    # a region shorter than the sampling interval: the two nearest samples, marked
+    s = bench.ClockSampler.summarise(rows, window=(t + 1.5, t + 1.52))
+    assert s["samples"] == 2 and s["window"] == "nearest to the timed region"
+    assert bench.ClockSampler.summarise([], window=(t, t + 1)) is None

@@ -12,6 +12,7 @@ from .std_oracle import (  # noqa: F401
     kv_commit,
     select_topk,
     selection_scores,
+    selection_scores_causal,
     softmax,
     sparse_decode_attn,
     topk_indices,

@@ -76,6 +76,30 @@ def selection_scores(q_text: np.ndarray, k_vis: np.ndarray) -> np.ndarray:
     return total / q.shape[0]
 
 
+def selection_scores_causal(q_text: np.ndarray, k_vis: np.ndarray, k_text: np.ndarray) -> np.ndarray:
+    """The causal full-row reading of the selection score [P-M4] (the pages do not say
+    which keys the text queries' softmax runs over; this variant lets each text query see
+    what it sees in the prompt's causal attention: every visual key and the text keys up to
+    its own position).
+
+    q_text: [G, T, d]; k_vis: [Nv, d]; k_text: [T, d], the text keys of the prompt.
+    Row (g, t) takes the softmax over [k_vis; k_text[0..t]] of q[g, t] . k / sqrt(d);
+    score[n] = mean over (g, t) of that row's probability at visual key n, fp64.
+    The scores sum to 1 minus the mean probability mass the rows put on text keys.
+    """
+    q = np.asarray(q_text, np.float64)
+    kv = np.asarray(k_vis, np.float64)
+    kt = np.asarray(k_text, np.float64)
+    G, T, d = q.shape
+    scale = 1.0 / math.sqrt(d)
+    total = np.zeros(kv.shape[0], np.float64)
+    for g in range(G):
+        for t in range(T):
+            keys = np.concatenate([kv, kt[:t + 1]], axis=0)
+            total += softmax(scale * (keys @ q[g, t]))[:kv.shape[0]]
+    return total / (G * T)
+
+
 def topk_indices(scores: np.ndarray, K: int) -> np.ndarray:
     """The K highest scores' positions, ties to the lower position, ascending. int32."""
     s = np.asarray(scores)
@@ -87,8 +111,11 @@ def topk_indices(scores: np.ndarray, K: int) -> np.ndarray:
 
 
 def select_topk(q_text: np.ndarray, k_full: np.ndarray, v_full: np.ndarray, nvis: np.ndarray,
-                T: int, K: int, cap_sparse: int):
+                T: int, K: int, cap_sparse: int, causal_text: bool = False):
     """Prefill selection for every (layer, batch, KV head) [P-M4], [P-M2].
+
+    causal_text: score with selection_scores_causal (text keys join each row's softmax)
+    instead of selection_scores (visual keys only).
 
     q_text [L][B][Hq][T][d]; k_full, v_full [L][B][Hkv][cap_full][d] (visual rows
     [0, nvis_b), text rows [nvis_b, nvis_b + T)).  Returns
@@ -110,7 +137,11 @@ def select_topk(q_text: np.ndarray, k_full: np.ndarray, v_full: np.ndarray, nvis
         for b in range(B):
             nv = int(nvis[b])
             for h in range(Hkv):
-                s = selection_scores(q_text[l, b, h * G:(h + 1) * G], k_full[l, b, h, :nv])
+                qh = q_text[l, b, h * G:(h + 1) * G]
+                if causal_text:
+                    s = selection_scores_causal(qh, k_full[l, b, h, :nv], k_full[l, b, h, nv:nv + T])
+                else:
+                    s = selection_scores(qh, k_full[l, b, h, :nv])
                 scores[l, b, h, :nv] = s
                 ix = topk_indices(s, K)
                 idx[l, b, h] = ix

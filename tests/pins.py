@@ -133,6 +133,41 @@ def check_selection_invariants(orc, seed: int = 5) -> None:
     assert int(np.argmax(s2)) == 17
 
 
+
+def check_selection_causal(orc, seed: int = 11) -> None:
+    """The causal full-row reading of the selection score, against (1) the prompt's full
+    causal attention matrix for the text rows, masked and normalised by torch in float64;
+    (2) a closed form; (3) invariants."""
+    import torch
+    rng = np.random.default_rng(seed)
+    G, T, d, nv = 3, 6, 8, 11
+    q = rng.standard_normal((G, T, d)) * 2
+    kv = rng.standard_normal((nv, d))
+    kt = rng.standard_normal((T, d))
+    s = orc.selection_scores_causal(q, kv, kt)
+    # (1) logits of every text query against [visual keys, text keys], mask text key j > t
+    keys = torch.from_numpy(np.concatenate([kv, kt]))
+    qt = torch.from_numpy(q.reshape(G * T, d))
+    logits = (qt @ keys.T) / math.sqrt(d)
+    t_of_row = torch.arange(G * T) % T
+    mask = torch.arange(nv + T)[None, :] >= (nv + t_of_row[:, None] + 1)
+    p = torch.softmax(logits.masked_fill(mask, float("-inf")), dim=-1)
+    np.testing.assert_allclose(s, p[:, :nv].mean(dim=0).numpy(), rtol=1e-12, atol=1e-15)
+    # (2) one visual key, one text key, d = 1: score = logistic((b - c) a), written via tanh
+    a, b, c = 0.7, 1.9, -0.4
+    s1 = orc.selection_scores_causal(np.array([[[a]]]), np.array([[b]]), np.array([[c]]))
+    assert abs(s1[0] - 0.5 * (1 + math.tanh(0.5 * (b - c) * a))) < 1e-15
+    # (3) text keys can only take mass away; with text logits far below, the visual-only score
+    sv = orc.selection_scores(q, kv)
+    assert (s <= sv + 1e-15).all() and s.sum() < 1.0
+    q2 = q.copy()
+    q2[..., 0] = 5.0
+    kt2 = kt.copy()
+    kt2[:, 0] = -1000.0
+    np.testing.assert_allclose(orc.selection_scores_causal(q2, kv, kt2), orc.selection_scores(q2, kv),
+                               rtol=0, atol=1e-12)
+
+
 def _brute_topk(s, K):
     """The unique K-subset whose members all beat all non-members under (score desc, pos asc)."""
     n = len(s)
@@ -260,7 +295,7 @@ def check_round_lossless_extremes(orc, seed: int = 10) -> None:
 
 ALL_CHECKS = [
     check_golden_attention, check_golden_verify, check_attention_vs_sdpa,
-    check_attention_closed_forms, check_golden_selection, check_selection_invariants,
+    check_attention_closed_forms, check_golden_selection, check_selection_invariants, check_selection_causal,
     check_topk_bruteforce, check_topk_special, check_full_k_sparse_equals_dense,
     check_golden_accept, check_accept_bruteforce, check_commit, check_round_lossless_extremes,
 ]

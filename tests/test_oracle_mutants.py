@@ -40,6 +40,19 @@ def _select_interleaved_groups(q_text, k_full, v_full, nvis, T, K, cap_sparse):
     return (idx, scores) + tuple(res[2:])
 
 
+
+def _causal_text_off_by_one(q_text, k_vis, k_text):
+    # row t sees text keys 0..t-1 only (row 0 sees none)
+    q = np.asarray(q_text, np.float64)
+    G, T, d = q.shape
+    total = np.zeros(k_vis.shape[0])
+    for g in range(G):
+        for t in range(T):
+            keys = np.concatenate([k_vis, k_text[:t]], axis=0)
+            total += oracle.softmax(keys @ q[g, t] / math.sqrt(d))[:k_vis.shape[0]]
+    return total / (G * T)
+
+
 def _topk_ties_high(scores, K):
     s = np.asarray(scores)
     order = np.lexsort((-np.arange(len(s)), -s))
@@ -82,6 +95,8 @@ def _commit_shifted(k_full, v_full, k_sp, v_sp, len_full, len_sp, n_plus_1):
 MUTANTS = {
     "attention scale 1/d": _mutant(attend=_attend_scale_1_over_d),
     "selection sum not mean": _mutant(selection_scores=_scores_sum_not_mean),
+    "causal text mask off by one": _mutant(selection_scores_causal=_causal_text_off_by_one),
+    "causal variant ignores text keys": _mutant(selection_scores_causal=lambda q, kv, kt: oracle.selection_scores(q, kv)),
     "GQA grouping hq % Hkv": _mutant(select_topk=_select_interleaved_groups),
     "top-K ties to higher position": _mutant(topk_indices=_topk_ties_high),
     "verify mask off by one": _mutant(dense_verify_attn=_verify_off_by_one),

@@ -135,6 +135,26 @@ int std_select_topk(const std_dims* dims, const void* q_text, int T, const void*
                     int32_t* idx_out, void* k_sparse, void* v_sparse, int32_t* len_sparse,
                     float* scores_out, void* ws, size_t ws_bytes, std_stream_t stream);
 
+/* Flags of std_select_topk_ex. */
+enum std_select_flags {
+  /* Causal full-row score: the softmax of text row (g, t) runs over the visual keys
+   * and the text keys [nvis[b], nvis[b] + t] -- the keys that query sees in the
+   * prompt's causal attention -- instead of the visual keys only.  The score of
+   * visual key n is still the mean over the G * T rows of that row's probability
+   * at n, so the scores sum to 1 minus the rows' mean mass on text keys.  The
+   * summary's "average attention from text to visual tokens" ("Methodik" item 4)
+   * does not say which keys the softmax covers; this is the other plain reading. */
+  STD_SELECT_CAUSAL_TEXT = 1
+};
+
+/* std_select_topk with flags (a bitwise OR of std_select_flags; 0 gives
+ * std_select_topk).  Same arguments, workspace and results otherwise; unknown
+ * flag bits are rejected with STD_ERR_INVALID_ARG. */
+int std_select_topk_ex(const std_dims* dims, const void* q_text, int T, const void* k_full,
+                       const void* v_full, const int32_t* nvis, int nvis_max, int K, int flags,
+                       int32_t* idx_out, void* k_sparse, void* v_sparse, int32_t* len_sparse,
+                       float* scores_out, void* ws, size_t ws_bytes, std_stream_t stream);
+
 /* The selection's top-K step alone, on caller-supplied float32 scores:
  * `rows` independent rows of `n` scores each (row stride n), K <= n.
  * idx_out [rows][K] receives the K highest positions of each row, ties to the

@@ -66,6 +66,7 @@ SIGNATURES = {
     "std_get_device_error": (_I, [ctypes.POINTER(ctypes.c_int32), _I, _P]),
     "std_select_workspace_size": (_SZ, [_DP, _I, _I]),
     "std_select_topk": (_I, [_DP, _P, _I, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "std_select_topk_ex": (_I, [_DP, _P, _I, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "std_topk_from_scores": (_I, [_P, _I, _I, _I, _P, _P]),
     "std_attn_workspace_size": (_SZ, [_DP, _I, _I64, _I]),
     "std_attn_splits": (_I, [_DP, _I, _I64, _I]),
@@ -173,6 +174,16 @@ def std_select_topk(d: StdDims, q_text, T, k_full, v_full, nvis, nvis_max, K, id
     _check(lib().std_select_topk(ctypes.byref(d), _ptr(q_text), T, _ptr(k_full), _ptr(v_full), _ptr(nvis),
                                  nvis_max, K, _ptr(idx_out), _ptr(k_sparse), _ptr(v_sparse), _ptr(len_sparse),
                                  _ptr(scores_out), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+STD_SELECT_CAUSAL_TEXT = 1
+
+
+def std_select_topk_ex(d: StdDims, q_text, T, k_full, v_full, nvis, nvis_max, K, flags, idx_out, k_sparse,
+                       v_sparse, len_sparse, scores_out, ws, stream=None) -> None:
+    _check(lib().std_select_topk_ex(ctypes.byref(d), _ptr(q_text), T, _ptr(k_full), _ptr(v_full), _ptr(nvis),
+                                    nvis_max, K, flags, _ptr(idx_out), _ptr(k_sparse), _ptr(v_sparse),
+                                    _ptr(len_sparse), _ptr(scores_out), _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
 def std_topk_from_scores(scores, rows, n, K, idx_out, stream=None) -> None:

@@ -211,7 +211,16 @@ int std_select_topk(const std_dims* dims, const void* q_text, int T, const void*
                     const void* v_full, const int32_t* nvis, int nvis_max, int K, int32_t* idx_out,
                     void* k_sparse, void* v_sparse, int32_t* len_sparse, float* scores_out, void* ws,
                     size_t ws_bytes, std_stream_t stream) {
+  return std_select_topk_ex(dims, q_text, T, k_full, v_full, nvis, nvis_max, K, 0, idx_out, k_sparse, v_sparse,
+                            len_sparse, scores_out, ws, ws_bytes, stream);
+}
+
+int std_select_topk_ex(const std_dims* dims, const void* q_text, int T, const void* k_full,
+                       const void* v_full, const int32_t* nvis, int nvis_max, int K, int flags,
+                       int32_t* idx_out, void* k_sparse, void* v_sparse, int32_t* len_sparse,
+                       float* scores_out, void* ws, size_t ws_bytes, std_stream_t stream) {
   STD_TRY(check_dims(dims));
+  if (flags & ~STD_SELECT_CAUSAL_TEXT) return fail(STD_ERR_INVALID_ARG, "unknown selection flags %#x", flags);
   STD_TRY(check_ptr(q_text, 16, "q_text"));
   STD_TRY(check_ptr(k_full, 16, "k_full"));
   STD_TRY(check_ptr(v_full, 16, "v_full"));
@@ -245,6 +254,7 @@ int std_select_topk(const std_dims* dims, const void* q_text, int T, const void*
   s.q_text = q_text; s.k_full = k_full; s.nvis = nvis; s.nvis_max = nvis_max;
   s.L = dims->L; s.B = dims->B; s.Hq = dims->Hq; s.Hkv = dims->Hkv; s.G = G; s.T = T; s.d = dims->d;
   s.dtype = dims->dtype; s.cap = dims->cap_full; s.row_m = row_m; s.row_l = row_l; s.scores = scores; s.err = err;
+  s.causal_text = (flags & STD_SELECT_CAUSAL_TEXT) ? 1 : 0;
   cudaError_t e = stdb::launch_select_scores(s, stream);
   if (e != cudaSuccess) return cuda_fail(e, "selection score launch");
   e = stdb::launch_topk(scores, nvis_max, probs, nvis, 0, dims->Hkv, dims->B, K, idx_out, err, stream);

@@ -72,8 +72,11 @@ struct ScoreArgs {
   float* row_l;   // [prob][G*T]  sum of 2^(x - m)
   float* scores;  // [prob][nvis_max]
   int* err;
+  int causal_text;  // nonzero: text keys 0..t join row (g, t)'s softmax (launch_text_rowstats after pass 1)
 };
 cudaError_t launch_select_scores(const ScoreArgs& a, cudaStream_t s);
+// Causal full-row variant: merge each text row's visible text keys into pass 1's (row_m, row_l).
+cudaError_t launch_text_rowstats(const ScoreArgs& a, cudaStream_t s);
 // tcgen05 version for bf16 operands; cudaErrorNotSupported for shapes it does not cover.
 cudaError_t launch_select_scores_tc(const ScoreArgs& a, cudaStream_t s);
 

@@ -299,6 +299,7 @@ cudaError_t launch_bf16_scores(const ScoreArgs& a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(rowstats_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
   if (e != cudaSuccess) return e;
   if ((e = launch_pdl(rowstats_bf16_kernel<D>, dim3((M + 63) / 64, a.Hkv, a.L * a.B), dim3(128), smem1, s, a)) != cudaSuccess) return e;
+  if (a.causal_text && (e = launch_text_rowstats(a, s)) != cudaSuccess) return e;
   constexpr int smem2 = TKS * D * 2;
   return launch_pdl(colsum_bf16_kernel<D>, dim3((a.nvis_max + TKS - 1) / TKS, a.Hkv, a.L * a.B), dim3(128), smem2, s, a);
 }
@@ -308,6 +309,7 @@ cudaError_t launch_f32_scores(const ScoreArgs& a, cudaStream_t s) {
   const int M = a.G * a.T;
   cudaError_t e = launch_pdl(rowstats_f32_kernel<D>, dim3((M + 127) / 128, a.Hkv, a.L * a.B), dim3(128), 0, s, a);
   if (e != cudaSuccess) return e;
+  if (a.causal_text && (e = launch_text_rowstats(a, s)) != cudaSuccess) return e;
   return launch_pdl(colsum_f32_kernel<D>, dim3((a.nvis_max + 127) / 128, a.Hkv, a.L * a.B), dim3(128), 0, s, a);
 }
 

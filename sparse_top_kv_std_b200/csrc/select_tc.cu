@@ -611,6 +611,7 @@ static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s) {
   e = launch_pdl(rowstats_tc_kernel<D>, dim3((M + BM - 1) / BM, a.Hkv, a.L * a.B), dim3(kP1Threads), P1<D>::SMEM, s,
                  tq128, tk, a);
   if (e != cudaSuccess) return e;
+  if (a.causal_text && (e = launch_text_rowstats(a, s)) != cudaSuccess) return e;
   return launch_pdl(colsum_tc_kernel<D>, dim3((a.nvis_max + kKeyBlocks * 256 - 1) / (kKeyBlocks * 256), a.Hkv,
                                               a.L * a.B),
                     dim3(kThreads), P2<D>::SMEM, s, tq128, tk, a);

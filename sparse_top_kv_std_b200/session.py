@@ -8,7 +8,7 @@ as calls into ``libstd_b200.so``:
     s = DecodeSession(L=28, B=1, Hq=28, Hkv=4, d=128, dtype=STD_BF16, ...)
     s.k_full[...] = prompt keys; s.v_full[...] = prompt values
     s.start(nvis)            # committed context = nvis + T
-    s.select(q_text)         # prefill top-K selection + gather  (std_select_topk)
+    s.select(q_text)         # prefill top-K selection + gather  (std_select_topk_ex)
     s.round(io)              # gamma drafts + verify + accept + commit  (std_decode_round)
 """
 from __future__ import annotations
@@ -57,10 +57,11 @@ class DecodeSession:
         self.nvis.copy_(nv, non_blocking=True)
         self.len_full.copy_(self.nvis + self.T, non_blocking=True)
 
-    def select(self, q_text: torch.Tensor, stream=None, keep_scores: bool = True) -> None:
-        B_.std_select_topk(self.dims, q_text, self.T, self.k_full, self.v_full, self.nvis, self.nvis_max,
-                           self.K, self.idx, self.k_sparse, self.v_sparse, self.len_sparse,
-                           self.scores if keep_scores else None, self.ws_select, stream)
+    def select(self, q_text: torch.Tensor, stream=None, keep_scores: bool = True, flags: int = 0) -> None:
+        """Prefill selection; flags = binding.STD_SELECT_CAUSAL_TEXT for the causal full-row score."""
+        B_.std_select_topk_ex(self.dims, q_text, self.T, self.k_full, self.v_full, self.nvis, self.nvis_max,
+                              self.K, flags, self.idx, self.k_sparse, self.v_sparse, self.len_sparse,
+                              self.scores if keep_scores else None, self.ws_select, stream)
 
     # -- decoding
     def round(self, io: Dict[str, torch.Tensor], stream=None) -> None:

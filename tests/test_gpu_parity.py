@@ -77,19 +77,30 @@ def test_select_row_max_jumps_and_ramps():
     _check_select(wl, x)
 
 
-def _check_select(wl, x):
+CAUSAL_CASES = ["tiny_f32", "ragged_bf16", "d64_bf16_G1", "f32_G4_K1", "rows2100_fallback", "tc_ragged_rows"]
+
+
+@pytest.mark.parametrize("name", CAUSAL_CASES)
+def test_select_causal_text_matches_oracle(name):
+    """The causal full-row score (text keys 0..t join row (g, t)'s softmax) on the
+    tensor-core, bf16 fallback and fp32 paths."""
+    wl = SELECT_CASES[name]
+    _check_select(wl, synth.host_inputs(wl, seed=3), flags=B.STD_SELECT_CAUSAL_TEXT)
+
+
+def _check_select(wl, x, flags=0):
     s = H.session_for(wl)
     s.k_full.copy_(H.to_dev(x["k_full"]))
     s.v_full.copy_(H.to_dev(x["v_full"]))
     s.start(x["nvis"])
     q_text = H.to_dev(x["q_text"])
-    s.select(q_text)
+    s.select(q_text, flags=flags)
     torch.cuda.synchronize()
     assert B.std_get_device_error() == 0
 
     idx_o, sc_o, ksp_o, vsp_o, lsp_o = oracle.select_topk(
         H.f64(x["q_text"], wl), H.f64(x["k_full"], wl), H.f64(x["v_full"], wl), x["nvis"], wl.T, wl.K,
-        wl.cap_sparse)
+        wl.cap_sparse, causal_text=bool(flags))
     sc_g = s.scores.cpu().numpy().astype(np.float64)
     idx_g = s.idx.cpu().numpy()
     rtol = H.score_rtol(wl)

@@ -8,6 +8,7 @@ from .std_oracle import (  # noqa: F401
     attend,
     decode_round,
     dense_verify_attn,
+    gather_sparse,
     kv_append,
     kv_commit,
     select_topk,
@@ -15,5 +16,6 @@ from .std_oracle import (  # noqa: F401
     selection_scores_causal,
     softmax,
     sparse_decode_attn,
+    streaming_indices,
     topk_indices,
 )

@@ -152,6 +152,38 @@ def select_topk(q_text: np.ndarray, k_full: np.ndarray, v_full: np.ndarray, nvis
     return idx, scores, k_sp, v_sp, np.full(B, K + T, np.int32)
 
 
+# --------------------------------------------------------------------------- streaming draft baseline
+
+def streaming_indices(nv: int, K: int, n_sink: int) -> np.ndarray:
+    """Index set of the "Streaming" draft baseline (gist.science summary, "Experimentelle
+    Ergebnisse", item "Vergleich": a baseline that drafts with streaming attention; no
+    detail printed).  Read as attention sinks plus a recent window: the first n_sink
+    visual positions and the last K - n_sink, ascending.  int32."""
+    if not (0 <= n_sink <= K <= nv):
+        raise ValueError("need 0 <= n_sink <= K <= nv")
+    return np.concatenate([np.arange(n_sink), np.arange(nv - (K - n_sink), nv)]).astype(np.int32)
+
+
+def gather_sparse(k_full: np.ndarray, v_full: np.ndarray, nvis: np.ndarray, idx: np.ndarray, T: int,
+                  cap_sparse: int):
+    """Sparse cache from given indices [P-M2]: rows [0, K) = full rows idx[l, b, h, j] in the
+    given order, rows [K, K + T) = the text rows [nvis_b, nvis_b + T).  Returns
+    (k_sparse, v_sparse [L][B][Hkv][cap_sparse][d], len_sparse [B] = K + T)."""
+    L, B, Hkv, K = idx.shape
+    d = k_full.shape[4]
+    k_sp = np.zeros((L, B, Hkv, cap_sparse, d), np.float64)
+    v_sp = np.zeros((L, B, Hkv, cap_sparse, d), np.float64)
+    for l in range(L):
+        for b in range(B):
+            nv = int(nvis[b])
+            for h in range(Hkv):
+                k_sp[l, b, h, :K] = k_full[l, b, h, idx[l, b, h]]
+                v_sp[l, b, h, :K] = v_full[l, b, h, idx[l, b, h]]
+                k_sp[l, b, h, K:K + T] = k_full[l, b, h, nv:nv + T]
+                v_sp[l, b, h, K:K + T] = v_full[l, b, h, nv:nv + T]
+    return k_sp, v_sp, np.full(B, K + T, np.int32)
+
+
 # --------------------------------------------------------------------------- attention [P-M2]
 
 def attend(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> np.ndarray:

@@ -168,6 +168,34 @@ def check_selection_causal(orc, seed: int = 11) -> None:
                                rtol=0, atol=1e-12)
 
 
+
+def check_streaming_and_gather(orc, seed: int = 12) -> None:
+    """Streaming index sets written out by hand; gather_sparse on the top-K indices equals
+    select_topk's own sparse cache, and on a hand-made index set copies the named rows."""
+    assert orc.streaming_indices(10, 4, 1).tolist() == [0, 7, 8, 9]
+    assert orc.streaming_indices(10, 4, 0).tolist() == [6, 7, 8, 9]
+    assert orc.streaming_indices(10, 4, 4).tolist() == [0, 1, 2, 3]
+    assert orc.streaming_indices(5, 5, 2).tolist() == [0, 1, 2, 3, 4]
+    rng = np.random.default_rng(seed)
+    L, B, Hq, Hkv, d, T, K = 2, 2, 4, 2, 8, 3, 5
+    nvis = np.array([12, 9])
+    cap = 12 + T
+    q = rng.standard_normal((L, B, Hq, T, d))
+    kf = rng.standard_normal((L, B, Hkv, cap, d))
+    vf = rng.standard_normal((L, B, Hkv, cap, d))
+    idx, _, ksp, vsp, lsp = orc.select_topk(q, kf, vf, nvis, T, K, K + T + 2)
+    k2, v2, l2 = orc.gather_sparse(kf, vf, nvis, idx, T, K + T + 2)
+    np.testing.assert_array_equal(k2, ksp)
+    np.testing.assert_array_equal(v2, vsp)
+    np.testing.assert_array_equal(l2, lsp)
+    mine = np.zeros((L, B, Hkv, 2), np.int32)
+    mine[..., 0], mine[..., 1] = 3, 0
+    k3, v3, _ = orc.gather_sparse(kf, vf, nvis, mine, T, 2 + T)
+    np.testing.assert_array_equal(k3[1, 1, 0, 0], kf[1, 1, 0, 3])
+    np.testing.assert_array_equal(v3[0, 1, 1, 1], vf[0, 1, 1, 0])
+    np.testing.assert_array_equal(k3[0, 1, 1, 2:2 + T], kf[0, 1, 1, 9:9 + T])
+
+
 def _brute_topk(s, K):
     """The unique K-subset whose members all beat all non-members under (score desc, pos asc)."""
     n = len(s)
@@ -296,6 +324,7 @@ def check_round_lossless_extremes(orc, seed: int = 10) -> None:
 ALL_CHECKS = [
     check_golden_attention, check_golden_verify, check_attention_vs_sdpa,
     check_attention_closed_forms, check_golden_selection, check_selection_invariants, check_selection_causal,
+    check_streaming_and_gather,
     check_topk_bruteforce, check_topk_special, check_full_k_sparse_equals_dense,
     check_golden_accept, check_accept_bruteforce, check_commit, check_round_lossless_extremes,
 ]

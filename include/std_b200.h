@@ -162,6 +162,31 @@ int std_select_topk_ex(const std_dims* dims, const void* q_text, int T, const vo
 int std_topk_from_scores(const float* scores, int rows, int n, int K, int32_t* idx_out,
                          std_stream_t stream);
 
+/* ---------------------------------------------------------------- streaming draft baseline
+ *
+ * Not the method's selection.  The gist.science summary ("Experimentelle
+ * Ergebnisse", item "Vergleich") compares Sparse-to-Dense with a baseline named
+ * Streaming that drafts with streaming attention, without details.  Read plainly,
+ * it keeps fixed positions instead of the top-K by attention: the first n_sink
+ * visual positions (attention sinks) and the most recent K - n_sink.  These two
+ * calls build such a sparse cache so that the draft / verify / commit calls run
+ * on it unchanged; std_gather_sparse also serves any caller-chosen index set.
+ */
+
+/* idx_out [L][B][Hkv][K] (device int32) <- for sequence b: j for j < n_sink, then
+ * nvis[b] - K + j (ascending).  Requires 0 <= n_sink <= K; K <= nvis[b] is checked
+ * on the device (STD_DEVERR_K_RANGE, that sequence skipped). */
+int std_streaming_indices(const std_dims* dims, const int32_t* nvis, int K, int n_sink, int32_t* idx_out,
+                          std_stream_t stream);
+
+/* The gather step of std_select_topk on caller-given indices: sparse rows [0, K)
+ * <- full rows idx[l][b][h][j] (any order, each in [0, nvis[b]); an index outside
+ * it flags STD_DEVERR_K_RANGE and leaves that row), rows [K, K + T) <- the text
+ * rows [nvis[b], nvis[b] + T), len_sparse[b] <- K + T.  K + T <= cap_sparse. */
+int std_gather_sparse(const std_dims* dims, const void* k_full, const void* v_full, const int32_t* nvis,
+                      const int32_t* idx, int K, int T, void* k_sparse, void* v_sparse, int32_t* len_sparse,
+                      std_stream_t stream);
+
 /* ---------------------------------------------------------------- decode attention
  *
  * All query rows that read one KV head -- the G grouped query heads times the

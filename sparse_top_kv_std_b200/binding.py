@@ -68,6 +68,8 @@ SIGNATURES = {
     "std_select_topk": (_I, [_DP, _P, _I, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "std_select_topk_ex": (_I, [_DP, _P, _I, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "std_topk_from_scores": (_I, [_P, _I, _I, _I, _P, _P]),
+    "std_streaming_indices": (_I, [_DP, _P, _I, _I, _P, _P]),
+    "std_gather_sparse": (_I, [_DP, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P]),
     "std_attn_workspace_size": (_SZ, [_DP, _I, _I64, _I]),
     "std_attn_splits": (_I, [_DP, _I, _I64, _I]),
     "std_sparse_decode_attn": (_I, [_DP, _P, _P, _P, _P, _I, _P, _I, _P, _SZ, _P]),
@@ -188,6 +190,16 @@ def std_select_topk_ex(d: StdDims, q_text, T, k_full, v_full, nvis, nvis_max, K,
 
 def std_topk_from_scores(scores, rows, n, K, idx_out, stream=None) -> None:
     _check(lib().std_topk_from_scores(_ptr(scores), rows, n, K, _ptr(idx_out), _stream(stream)))
+
+
+def std_streaming_indices(d: StdDims, nvis, K, n_sink, idx_out, stream=None) -> None:
+    _check(lib().std_streaming_indices(ctypes.byref(d), _ptr(nvis), K, n_sink, _ptr(idx_out), _stream(stream)))
+
+
+def std_gather_sparse(d: StdDims, k_full, v_full, nvis, idx, K, T, k_sparse, v_sparse, len_sparse,
+                      stream=None) -> None:
+    _check(lib().std_gather_sparse(ctypes.byref(d), _ptr(k_full), _ptr(v_full), _ptr(nvis), _ptr(idx), K, T,
+                                   _ptr(k_sparse), _ptr(v_sparse), _ptr(len_sparse), _stream(stream)))
 
 
 def std_attn_workspace_size(d: StdDims, q_rows: int, cap: int, splits: int) -> int:

@@ -269,6 +269,46 @@ int std_select_topk_ex(const std_dims* dims, const void* q_text, int T, const vo
   return ok();
 }
 
+int std_streaming_indices(const std_dims* dims, const int32_t* nvis, int K, int n_sink, int32_t* idx_out,
+                          std_stream_t stream) {
+  STD_TRY(check_dims(dims));
+  STD_TRY(check_ptr(nvis, 4, "nvis"));
+  STD_TRY(check_ptr(idx_out, 4, "idx_out"));
+  if (K < 1) return fail(STD_ERR_INVALID_ARG, "K = %d must be >= 1", K);
+  if (n_sink < 0 || n_sink > K) return fail(STD_ERR_INVALID_ARG, "n_sink = %d must be in [0, K = %d]", n_sink, K);
+  int* err;
+  STD_TRY(device_state(&err, nullptr));
+  cudaError_t e = stdb::launch_streaming_indices(nvis, dims->L, dims->B, dims->Hkv, K, n_sink, idx_out, err, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "streaming index launch");
+  return ok();
+}
+
+int std_gather_sparse(const std_dims* dims, const void* k_full, const void* v_full, const int32_t* nvis,
+                      const int32_t* idx, int K, int T, void* k_sparse, void* v_sparse, int32_t* len_sparse,
+                      std_stream_t stream) {
+  STD_TRY(check_dims(dims));
+  STD_TRY(check_ptr(k_full, 16, "k_full"));
+  STD_TRY(check_ptr(v_full, 16, "v_full"));
+  STD_TRY(check_ptr(nvis, 4, "nvis"));
+  STD_TRY(check_ptr(idx, 4, "idx"));
+  STD_TRY(check_ptr(k_sparse, 16, "k_sparse"));
+  STD_TRY(check_ptr(v_sparse, 16, "v_sparse"));
+  STD_TRY(check_ptr(len_sparse, 4, "len_sparse"));
+  if (K < 1 || T < 0) return fail(STD_ERR_INVALID_ARG, "K = %d, T = %d", K, T);
+  if ((int64_t)K + T > dims->cap_sparse)
+    return fail(STD_ERR_CAPACITY, "K + T = %d exceeds cap_sparse = %lld", K + T, (long long)dims->cap_sparse);
+  int* err;
+  STD_TRY(device_state(&err, nullptr));
+  stdb::GatherArgs g{};
+  g.k_full = k_full; g.v_full = v_full; g.k_sp = k_sparse; g.v_sp = v_sparse; g.idx = idx; g.nvis = nvis;
+  g.len_sparse = len_sparse; g.L = dims->L; g.B = dims->B; g.Hkv = dims->Hkv; g.T = T; g.K = K;
+  g.row_bytes = dims->d * elem_bytes(dims->dtype); g.cap_full = dims->cap_full; g.cap_sparse = dims->cap_sparse;
+  g.err = err;
+  cudaError_t e = stdb::launch_gather(g, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+  return ok();
+}
+
 int std_topk_from_scores(const float* scores, int rows, int n, int K, int32_t* idx_out, std_stream_t stream) {
   STD_TRY(check_ptr(scores, 4, "scores"));
   STD_TRY(check_ptr(idx_out, 4, "idx_out"));

@@ -99,6 +99,9 @@ struct GatherArgs {
   int* err;
 };
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s);
+// Sink + recent-window index set: idx[prob][j] = j (j < n_sink), else nvis[b] - K + j.
+cudaError_t launch_streaming_indices(const int32_t* nvis, int L, int B, int Hkv, int K, int n_sink, int32_t* idx,
+                                     int* err, cudaStream_t s);
 
 cudaError_t launch_append(void* k_cache, void* v_cache, int64_t cap, const int32_t* len, int off,
                           const void* k_new, const void* v_new, int n_new, int L, int B, int Hkv,

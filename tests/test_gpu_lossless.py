@@ -73,3 +73,20 @@ def test_full_selection_drafts_are_accepted():
     assert got == want
     full = sum(n == 9 for n in counts[:-1])
     assert full >= 0.8 * (len(counts) - 1), counts
+
+
+def test_streaming_baseline_is_lossless_and_compared_with_topk():
+    """The streaming draft baseline (sinks + recent window, same kernels) is lossless too:
+    any index set only changes how many drafts are accepted.  Prints the mean tokens per
+    round of both index sets at equal K."""
+    rows = []
+    for seed, K, gamma in [(1, 512, 6), (2, 512, 6), (6, 256, 8), (1, 128, 6)]:
+        m, want, kf, vf, qt, first = _model(seed)
+        got_t, cnt_t = std_decode(m, kf, vf, qt, first, K, gamma, N_TOKENS)
+        got_s, cnt_s = std_decode(m, kf, vf, qt, first, K, gamma, N_TOKENS, select="stream")
+        assert got_t == want, _first_diff(got_t, want)
+        assert got_s == want, _first_diff(got_s, want)
+        rows.append((seed, K, gamma, sum(cnt_t) / len(cnt_t), sum(cnt_s) / len(cnt_s)))
+    print("\nseed  K  gamma  tokens/round top-K  tokens/round streaming")
+    for r in rows:
+        print("%4d %4d %5d %12.2f %18.2f" % r)

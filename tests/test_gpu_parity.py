@@ -5,6 +5,8 @@ operands and 2e-2 for bf16 operands with fp32 accumulation; top-K indices on
 identical fp32 scores and acceptance results bit-exact; cache copies
 byte-exact.  Selection scores use the relative tolerance in harness.score_rtol.
 """
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -410,3 +412,82 @@ def test_exp2_polynomial_error_bound():
     assert rel_f.max() < 4e-7, rel_f.max()
     assert rel_f.mean() < 1e-7
     assert rel_s.max() < 4e-7     # the SFU reference the polynomial stands beside
+
+
+# ----------------------------------------------------------------------------- streaming baseline
+
+@pytest.mark.parametrize("name,n_sink", [("ragged_bf16", 4), ("tiny_f32", 0), ("d64_bf16_G1", 300)])
+def test_streaming_indices_and_gather(name, n_sink):
+    wl = SELECT_CASES[name]
+    x = synth.host_inputs(wl, seed=4)
+    d = B.dims(wl.L, wl.B, wl.Hq, wl.Hkv, wl.d, H.dtype_code(wl), wl.cap_full, wl.cap_sparse)
+    nvis = torch.tensor(wl.nvis, dtype=torch.int32, device="cuda")
+    idx = torch.full((wl.L, wl.B, wl.Hkv, wl.K), -1, dtype=torch.int32, device="cuda")
+    st = torch.float32 if wl.dtype == "f32" else torch.int16
+    ksp = torch.zeros((wl.L, wl.B, wl.Hkv, wl.cap_sparse, wl.d), dtype=st, device="cuda")
+    vsp = torch.zeros_like(ksp)
+    lsp = torch.zeros(wl.B, dtype=torch.int32, device="cuda")
+    B.std_streaming_indices(d, nvis, wl.K, n_sink, idx)
+    B.std_gather_sparse(d, H.to_dev(x["k_full"]), H.to_dev(x["v_full"]), nvis, idx, wl.K, wl.T, ksp, vsp, lsp)
+    torch.cuda.synchronize()
+    assert B.std_get_device_error() == 0
+    idx_h = idx.cpu().numpy()
+    for b in range(wl.B):
+        want = oracle.streaming_indices(wl.nvis[b], wl.K, n_sink)
+        for l in range(wl.L):
+            for h in range(wl.Hkv):
+                np.testing.assert_array_equal(idx_h[l, b, h], want)
+    kw, vw, lw = oracle.gather_sparse(x["k_full"], x["v_full"], np.array(wl.nvis), idx_h, wl.T, wl.cap_sparse)
+    n = wl.K + wl.T
+    got_k = ksp.cpu().numpy().view(x["k_full"].dtype)[..., :n, :]
+    got_v = vsp.cpu().numpy().view(x["v_full"].dtype)[..., :n, :]
+    np.testing.assert_array_equal(got_k, kw[..., :n, :].astype(x["k_full"].dtype))
+    np.testing.assert_array_equal(got_v, vw[..., :n, :].astype(x["v_full"].dtype))
+    assert lsp.cpu().tolist() == lw.tolist()
+
+
+def test_streaming_window_larger_than_the_sequence_is_flagged():
+    wl = SELECT_CASES["ragged_bf16"]  # nvis (777, 1500, 64)
+    d = B.dims(wl.L, wl.B, wl.Hq, wl.Hkv, wl.d, H.dtype_code(wl), wl.cap_full, wl.cap_sparse)
+    nvis = torch.tensor(wl.nvis, dtype=torch.int32, device="cuda")
+    idx = torch.full((wl.L, wl.B, wl.Hkv, 65), -7, dtype=torch.int32, device="cuda")
+    B.std_streaming_indices(d, nvis, 65, 4, idx)
+    torch.cuda.synchronize()
+    assert B.std_get_device_error() == B.STD_DEVERR_K_RANGE
+    h = idx.cpu().numpy()
+    assert (h[:, 2] == -7).all()                              # the 64-token sequence was skipped
+    assert h[0, 0, 0].tolist() == list(range(4)) + list(range(777 - 61, 777))
+
+
+def test_topk_keeps_more_attention_mass_than_the_streaming_window():
+    """Selection quality on the generator's long-video layer: the share of each draft
+    query's dense softmax mass (over the prompt) that falls on the sparse cache's rows.
+    The method's top-K (chosen from the text queries) keeps more of it than the sink +
+    recent window of the same size.  The mass is computed in torch from the library's
+    own index sets (test-side arithmetic only)."""
+    wl = synth.workload("layer_16k")
+    x = synth.host_inputs(wl, seed=0)
+    s = H.session_for(wl)
+    s.k_full.copy_(H.to_dev(x["k_full"]))
+    s.v_full.copy_(H.to_dev(x["v_full"]))
+    s.start(x["nvis"])
+    s.select(H.to_dev(x["q_text"]))
+    idx_top = s.idx.clone()
+    idx_str = torch.empty_like(s.idx)
+    B.std_streaming_indices(s.dims, s.nvis, wl.K, 4, idx_str)
+    torch.cuda.synchronize()
+    assert B.std_get_device_error() == 0
+    nv, G, N = wl.nvis[0], wl.G, wl.nvis[0] + wl.T
+    keys = s.k_full[:, 0, :, :N].float()                                   # [L, Hkv, N, d]
+    q = H.to_dev(np.ascontiguousarray(x["q_draft"][0, 0])).float()[:, 0, :, 0]   # [L, Hq, d]
+    q = q.reshape(wl.L, wl.Hkv, G, wl.d)
+    p = torch.softmax(torch.einsum("lhgd,lhnd->lhgn", q, keys) / math.sqrt(wl.d), dim=-1)
+    text = p[..., nv:].sum(-1)
+
+    def kept(idx):
+        ix = idx[:, 0].long()[:, :, None, :].expand(-1, -1, G, -1)             # [L, Hkv, G, K]
+        return float((torch.gather(p, 3, ix).sum(-1) + text).mean())
+    m_top, m_str = kept(idx_top), kept(idx_str)
+    print(f"\nmean dense attention mass kept by K = {wl.K} of {nv} visual rows + {wl.T} text rows: "
+          f"top-K {m_top:.3f}, sink + window {m_str:.3f}")
+    assert m_top > 1.5 * m_str, (m_top, m_str)

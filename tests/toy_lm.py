@@ -162,8 +162,13 @@ def dense_decode_gpu(m: ToyLM, k_full, v_full, first: int, n_tokens: int):
     return out
 
 
-def std_decode(m: ToyLM, k_full, v_full, q_text, first: int, K: int, gamma: int, n_tokens: int):
-    """Sparse-to-Dense decoding through the library.  Returns (tokens, n + 1 of every round)."""
+def std_decode(m: ToyLM, k_full, v_full, q_text, first: int, K: int, gamma: int, n_tokens: int,
+               select: str = "topk", n_sink: int = 4):
+    """Sparse-to-Dense decoding through the library.  Returns (tokens, n + 1 of every round).
+
+    select: "topk" -- the method's selection (std_select_topk); "stream" -- the streaming
+    draft baseline (n_sink attention sinks + the most recent visual positions, through
+    std_streaming_indices and std_gather_sparse)."""
     from sparse_top_kv_std_b200 import binding as B
     c, W = m.cfg, m.dev()
     k_full, v_full = k_full.clone(), v_full.clone()
@@ -176,8 +181,12 @@ def std_decode(m: ToyLM, k_full, v_full, q_text, first: int, K: int, gamma: int,
     len_sp = torch.zeros(1, dtype=torch.int32, device="cuda")
     nvis = torch.tensor([c.nvis], dtype=torch.int32, device="cuda")
     idx = torch.zeros((c.L, 1, c.Hkv, K), dtype=torch.int32, device="cuda")
-    ws_sel = torch.empty(B.std_select_workspace_size(dims, c.T, c.nvis), dtype=torch.uint8, device="cuda")
-    B.std_select_topk(dims, q_text, c.T, k_full, v_full, nvis, c.nvis, K, idx, k_sp, v_sp, len_sp, None, ws_sel)
+    if select == "topk":
+        ws_sel = torch.empty(B.std_select_workspace_size(dims, c.T, c.nvis), dtype=torch.uint8, device="cuda")
+        B.std_select_topk(dims, q_text, c.T, k_full, v_full, nvis, c.nvis, K, idx, k_sp, v_sp, len_sp, None, ws_sel)
+    else:
+        B.std_streaming_indices(dims, nvis, K, n_sink, idx)
+        B.std_gather_sparse(dims, k_full, v_full, nvis, idx, K, c.T, k_sp, v_sp, len_sp)
     d1 = B.dims(1, 1, c.Hq, c.Hkv, c.d, B.STD_BF16, cap_full, cap_sp)
     ws = torch.empty(max(16, B.std_round_workspace_size(d1, gamma)), dtype=torch.uint8, device="cuda")
     n1 = torch.zeros(1, dtype=torch.int32, device="cuda")

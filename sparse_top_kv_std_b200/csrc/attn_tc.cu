@@ -32,6 +32,8 @@
 #include <cuda.h>
 #include <math.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 #include "tc100.cuh"
@@ -46,6 +48,7 @@ constexpr int kMaxB = 64;         // sequences per call handled by this kernel
 constexpr int kTmemCols = 512;
 constexpr uint32_t kColS = 128;   // TMEM column of S/P buffer 0 (buffer 1 at 256); O at column 0
 constexpr float kTau = 8.f;       // log2 growth of a row max that forces an O rescale
+constexpr int kMergeSegs = 4;     // segments a merge holds in registers (more: one at a time)
 
 struct Ctl {
   uint64_t kv_full[STAGES], kv_empty[STAGES];
@@ -144,6 +147,81 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = tc::globaltimer();
   while (!tc::mbar_try_wait(adr, parity)) {
     if (tc::globaltimer() - t0 > tc::kWaitTimeoutNs) return;
+  }
+}
+
+// Merge of a problem's segment partials (m, l, o) into its output, by the 128 softmax
+// threads of the last CTA to finish the problem.  One item = 4 columns of one query row.
+// BATCHED (up to kMergeSegs segments): every load of an item is issued before any is
+// used, so an item costs one L2 round trip instead of two; the M = 128 kernel, already
+// near the register limit, keeps the two-pass form.  Partial k of row r sits
+// at slot0 + k * rows + r; output row r at orow0 + r.
+template <int D, bool BATCHED>
+__device__ __forceinline__ void merge_problem(float* out, const float* ws, const float* ml, int rows, size_t slot0,
+                                           int nseg, size_t orow0, int tid) {
+  const int nitems = rows * (D / 4);
+  auto write = [&](int r, int col, float L, float4 acc) {
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    *reinterpret_cast<float4*>(out + (orow0 + r) * D + col) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  };
+  auto finish = [&](const float2* mlv, const float4* xv, int r, int col) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kMergeSegs; ++c)
+      if (c < nseg) M = fmaxf(M, mlv[c].x);
+    const float ref = M == -INFINITY ? 0.f : M;
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < kMergeSegs; ++c) {
+      if (c >= nseg) break;
+      const float w = ex2(mlv[c].x - ref);
+      L += w * mlv[c].y;
+      acc.x += w * xv[c].x;
+      acc.y += w * xv[c].y;
+      acc.z += w * xv[c].z;
+      acc.w += w * xv[c].w;
+    }
+    write(r, col, L, acc);
+  };
+  auto slow = [&](int item) {  // more segments than registers: one segment at a time
+    const int r = item / (D / 4), col = (item % (D / 4)) * 4;
+    float M = -INFINITY;
+    for (int c = 0; c < nseg; ++c) M = fmaxf(M, __ldcg(ml + (slot0 + (size_t)c * rows + r) * 2));
+    const float ref = M == -INFINITY ? 0.f : M;
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < nseg; ++c) {
+      const size_t k = slot0 + (size_t)c * rows + r;
+      const float2 mlk = __ldcg(reinterpret_cast<const float2*>(ml + k * 2));
+      const float w = ex2(mlk.x - ref);
+      L += w * mlk.y;
+      const float4 x = __ldcg(reinterpret_cast<const float4*>(ws + k * D + col));
+      acc.x += w * x.x;
+      acc.y += w * x.y;
+      acc.z += w * x.z;
+      acc.w += w * x.w;
+    }
+    write(r, col, L, acc);
+  };
+  for (int item = tid; item < nitems; item += 128) {
+    if (!BATCHED || nseg > kMergeSegs) {
+      slow(item);
+      continue;
+    }
+    const int r = item / (D / 4), col = (item % (D / 4)) * 4;
+    float2 mlv[kMergeSegs];
+    float4 xv[kMergeSegs];
+#pragma unroll
+    for (int c = 0; c < kMergeSegs; ++c) {
+      if (c < nseg) {
+        const size_t k = slot0 + (size_t)c * rows + r;
+        mlv[c] = __ldcg(reinterpret_cast<const float2*>(ml + k * 2));
+        xv[c] = __ldcg(reinterpret_cast<const float4*>(ws + k * D + col));
+      }
+    }
+    finish(mlv, xv, r, col);
   }
 }
 
@@ -252,7 +330,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       while (it.g < it.g_end) {
         if (it.first) {
           if (!tc::mbar_wait(&ctl->q_empty, (seg & 1) ^ 1, abort_flag, a.err)) break;
-          tc::mbar_expect_tx(&ctl->q_full, C::Q_BYTES);
+          tc::mbar_expect_tx(&ctl->q_full, HALF ? C::Q_BYTES / 2 : C::Q_BYTES);  // HALF: 64-row boxes
           const int qrow = ((it.l * a.B + it.b) * a.Hq + it.h * a.G) * a.nq;
 #pragma unroll
           for (int kb = 0; kb < C::KB; ++kb) tc::tma_load_2d(sQ + kb * 128 * 128, &tm_q, kb * 64, qrow, &ctl->q_full);
@@ -556,32 +634,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           ++npub;
           if (ctl->last_flag) {
             __threadfence();
-            // all 128 row threads share the merge: one item = 4 columns of one query row
-            const int nseg = c1 - c0 + 1;
-            for (int item = tid; item < a.rows * (D / 4); item += 128) {
-              const int r = item / (D / 4), col = (item % (D / 4)) * 4;
-              const size_t k0 = (size_t)(prob + c0) * a.rows + r;
-              float M = -INFINITY;
-              for (int c = 0; c < nseg; ++c) M = fmaxf(M, __ldcg(ml + (k0 + (size_t)c * a.rows) * 2));
-              const float ref = M == -INFINITY ? 0.f : M;
-              float L = 0.f;
-              float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-              for (int c = 0; c < nseg; ++c) {
-                const size_t k = k0 + (size_t)c * a.rows;
-                const float2 mlk = __ldcg(reinterpret_cast<const float2*>(ml + k * 2));
-                const float w = ex2(mlk.x - ref);
-                L += w * mlk.y;
-                const float4 x = __ldcg(reinterpret_cast<const float4*>(a.ws + k * D + col));
-                acc.x += w * x.x;
-                acc.y += w * x.y;
-                acc.z += w * x.z;
-                acc.w += w * x.w;
-              }
-              const float inv = L > 0.f ? 1.f / L : 0.f;
-              const size_t orow_r = (size_t)(lb * a.Hq + it.h * a.G) * a.nq + r;
-              *reinterpret_cast<float4*>(a.o + orow_r * D + col) =
-                  make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-            }
+            // all 128 softmax threads share the merge
+            merge_problem<D, HALF>(a.o, a.ws, ml, a.rows, (size_t)(prob + c0) * a.rows, c1 - c0 + 1,
+                             (size_t)(lb * a.Hq + it.h * a.G) * a.nq, tid);
             if (tid == 0) atomicExch(ctr + prob, (unsigned long long)a.epoch << 32);  // ready for a replay
           }
         }
@@ -603,17 +658,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 template <int D>
 cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   using C = Cfg<D>;
+  // at most 64 query rows per problem (the draft's G rows, the verify's G * (gamma + 1)
+  // up to 64): M = 64 MMAs, the spread softmax layout, and 64-row query boxes
+  const bool half = a.rows <= 64;
   const uint64_t qrows = (uint64_t)a.L * a.B * a.Hq * a.nq;
   const uint64_t krows = (uint64_t)a.L * a.B * a.Hkv * a.cap;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap_bf16_2d(&tq, a.q, D, qrows, 128) || !make_tmap_bf16_2d(&tk, a.k, D, krows, TK) ||
+  if (!make_tmap_bf16_2d(&tq, a.q, D, qrows, half ? 64 : 128) || !make_tmap_bf16_2d(&tk, a.k, D, krows, TK) ||
       !make_tmap_bf16_2d(&tv, a.v, D, krows, TK))
     return cudaErrorInvalidValue;
-  // at most 64 query rows per problem (the draft's G rows, the verify's G * (gamma + 1)
-  // up to 64): M = 64 MMAs and the spread softmax layout
-  auto kern = a.rows <= 64 ? attn_tc_kernel<D, true> : attn_tc_kernel<D, false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  auto kern = half ? attn_tc_kernel<D, true> : attn_tc_kernel<D, false>;
+  // the shared-memory size is a per-device attribute of each kernel: set it once per device
+  static std::atomic<uint64_t> attr_done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << ((dev & 31) * 2 + (half ? 1 : 0));
+  if (!(attr_done.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_done.fetch_or(bit, std::memory_order_release);
+  }
   return launch_pdl(kern, dim3(a.splits), dim3(kThreads), C::SMEM, s, tq, tk, tv, a);
 }
 

@@ -194,7 +194,9 @@ int std_gather_sparse(const std_dims* dims, const void* k_full, const void* v_fu
  * bf16 operands (head dim 64 or 128, G x query rows <= 128, B <= 64) run on a
  * persistent tensor-core kernel: the 128-key tiles of all (layer, sequence, KV
  * head) problems form one sequence that the CTAs split into equal slices;
- * `splits` = 0 launches one CTA per SM, splits = s > 0 launches
+ * `splits` = 0 launches one CTA per SM -- or one CTA per problem when there are
+ * between half and all as many problems as SMs and `cap` is short (at most 2048
+ * keys for up to 16 query rows, 8192 otherwise) -- and splits = s > 0 launches
  * s x L x B x Hkv CTAs.  fp32 operands (and bf16 with B > 64) use split-K
  * kernels with `splits` key ranges per problem (0 = automatic).  Either way
  * the partial results go to the workspace.  The tensor-core kernel merges them

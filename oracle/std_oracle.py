@@ -76,27 +76,31 @@ def selection_scores(q_text: np.ndarray, k_vis: np.ndarray) -> np.ndarray:
     return total / q.shape[0]
 
 
-def selection_scores_causal(q_text: np.ndarray, k_vis: np.ndarray, k_text: np.ndarray) -> np.ndarray:
+def selection_scores_causal(q_text: np.ndarray, k_vis: np.ndarray, k_text: np.ndarray,
+                            k_prefix: np.ndarray = None) -> np.ndarray:
     """The causal full-row reading of the selection score [P-M4] (the pages do not say
     which keys the text queries' softmax runs over; this variant lets each text query see
     what it sees in the prompt's causal attention: every visual key and the text keys up to
     its own position).
 
-    q_text: [G, T, d]; k_vis: [Nv, d]; k_text: [T, d], the text keys of the prompt.
-    Row (g, t) takes the softmax over [k_vis; k_text[0..t]] of q[g, t] . k / sqrt(d);
+    q_text: [G, T, d]; k_vis: [Nv, d]; k_text: [T, d], the text keys of the prompt;
+    k_prefix: [P, d], keys of a prompt prefix before the video (a system prompt), or None.
+    Row (g, t) takes the softmax over [k_prefix; k_vis; k_text[0..t]] of q[g, t] . k / sqrt(d);
     score[n] = mean over (g, t) of that row's probability at visual key n, fp64.
-    The scores sum to 1 minus the mean probability mass the rows put on text keys.
+    The scores sum to 1 minus the mean probability mass the rows put on other keys.
     """
     q = np.asarray(q_text, np.float64)
     kv = np.asarray(k_vis, np.float64)
     kt = np.asarray(k_text, np.float64)
+    kp = np.zeros((0, kv.shape[1])) if k_prefix is None else np.asarray(k_prefix, np.float64)
     G, T, d = q.shape
+    P, nv = kp.shape[0], kv.shape[0]
     scale = 1.0 / math.sqrt(d)
-    total = np.zeros(kv.shape[0], np.float64)
+    total = np.zeros(nv, np.float64)
     for g in range(G):
         for t in range(T):
-            keys = np.concatenate([kv, kt[:t + 1]], axis=0)
-            total += softmax(scale * (keys @ q[g, t]))[:kv.shape[0]]
+            keys = np.concatenate([kp, kv, kt[:t + 1]], axis=0)
+            total += softmax(scale * (keys @ q[g, t]))[P:P + nv]
     return total / (G * T)
 
 
@@ -111,11 +115,15 @@ def topk_indices(scores: np.ndarray, K: int) -> np.ndarray:
 
 
 def select_topk(q_text: np.ndarray, k_full: np.ndarray, v_full: np.ndarray, nvis: np.ndarray,
-                T: int, K: int, cap_sparse: int, causal_text: bool = False):
+                T: int, K: int, cap_sparse: int, causal_text: bool = False, n_prefix: int = 0):
     """Prefill selection for every (layer, batch, KV head) [P-M4], [P-M2].
 
     causal_text: score with selection_scores_causal (text keys join each row's softmax)
     instead of selection_scores (visual keys only).
+    n_prefix: rows of a prompt prefix (a system prompt) before the visual block; the
+    cache is then [prefix | visual | text], the indices stay positions within the visual
+    block, and the sparse cache is [prefix | K selected visual | text] (length
+    n_prefix + K + T).  With causal_text the prefix keys join every text row's softmax.
 
     q_text [L][B][Hq][T][d]; k_full, v_full [L][B][Hkv][cap_full][d] (visual rows
     [0, nvis_b), text rows [nvis_b, nvis_b + T)).  Returns
@@ -138,18 +146,16 @@ def select_topk(q_text: np.ndarray, k_full: np.ndarray, v_full: np.ndarray, nvis
             nv = int(nvis[b])
             for h in range(Hkv):
                 qh = q_text[l, b, h * G:(h + 1) * G]
+                P = n_prefix
+                kvis = k_full[l, b, h, P:P + nv]
                 if causal_text:
-                    s = selection_scores_causal(qh, k_full[l, b, h, :nv], k_full[l, b, h, nv:nv + T])
+                    s = selection_scores_causal(qh, kvis, k_full[l, b, h, P + nv:P + nv + T], k_full[l, b, h, :P])
                 else:
-                    s = selection_scores(qh, k_full[l, b, h, :nv])
+                    s = selection_scores(qh, kvis)
                 scores[l, b, h, :nv] = s
-                ix = topk_indices(s, K)
-                idx[l, b, h] = ix
-                k_sp[l, b, h, :K] = k_full[l, b, h, ix]
-                v_sp[l, b, h, :K] = v_full[l, b, h, ix]
-                k_sp[l, b, h, K:K + T] = k_full[l, b, h, nv:nv + T]
-                v_sp[l, b, h, K:K + T] = v_full[l, b, h, nv:nv + T]
-    return idx, scores, k_sp, v_sp, np.full(B, K + T, np.int32)
+                idx[l, b, h] = topk_indices(s, K)
+    k_sp, v_sp, lsp = gather_sparse(k_full, v_full, nvis, idx, T, cap_sparse, n_prefix)
+    return idx, scores, k_sp, v_sp, lsp
 
 
 # --------------------------------------------------------------------------- streaming draft baseline
@@ -165,23 +171,26 @@ def streaming_indices(nv: int, K: int, n_sink: int) -> np.ndarray:
 
 
 def gather_sparse(k_full: np.ndarray, v_full: np.ndarray, nvis: np.ndarray, idx: np.ndarray, T: int,
-                  cap_sparse: int):
-    """Sparse cache from given indices [P-M2]: rows [0, K) = full rows idx[l, b, h, j] in the
-    given order, rows [K, K + T) = the text rows [nvis_b, nvis_b + T).  Returns
-    (k_sparse, v_sparse [L][B][Hkv][cap_sparse][d], len_sparse [B] = K + T)."""
+                  cap_sparse: int, n_prefix: int = 0):
+    """Sparse cache from given indices [P-M2].  The full cache holds [P prefix rows |
+    nvis_b visual rows | T text rows] with P = n_prefix; the sparse cache gets the P
+    prefix rows, then the visual rows P + idx[l, b, h, j] in the given order, then the
+    text rows.  Returns (k_sparse, v_sparse [L][B][Hkv][cap_sparse][d],
+    len_sparse [B] = P + K + T)."""
     L, B, Hkv, K = idx.shape
     d = k_full.shape[4]
+    P = n_prefix
     k_sp = np.zeros((L, B, Hkv, cap_sparse, d), np.float64)
     v_sp = np.zeros((L, B, Hkv, cap_sparse, d), np.float64)
     for l in range(L):
         for b in range(B):
             nv = int(nvis[b])
             for h in range(Hkv):
-                k_sp[l, b, h, :K] = k_full[l, b, h, idx[l, b, h]]
-                v_sp[l, b, h, :K] = v_full[l, b, h, idx[l, b, h]]
-                k_sp[l, b, h, K:K + T] = k_full[l, b, h, nv:nv + T]
-                v_sp[l, b, h, K:K + T] = v_full[l, b, h, nv:nv + T]
-    return k_sp, v_sp, np.full(B, K + T, np.int32)
+                for dst, src in ((k_sp, k_full), (v_sp, v_full)):
+                    dst[l, b, h, :P] = src[l, b, h, :P]
+                    dst[l, b, h, P:P + K] = src[l, b, h, P + idx[l, b, h]]
+                    dst[l, b, h, P + K:P + K + T] = src[l, b, h, P + nv:P + nv + T]
+    return k_sp, v_sp, np.full(B, P + K + T, np.int32)
 
 
 # --------------------------------------------------------------------------- attention [P-M2]

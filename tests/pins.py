@@ -166,6 +166,40 @@ def check_selection_causal(orc, seed: int = 11) -> None:
     kt2[:, 0] = -1000.0
     np.testing.assert_allclose(orc.selection_scores_causal(q2, kv, kt2), orc.selection_scores(q2, kv),
                                rtol=0, atol=1e-12)
+    # (4) a prompt prefix (system prompt) before the video: its keys are visible to every row
+    P = 4
+    kp = rng.standard_normal((P, d))
+    sp = orc.selection_scores_causal(q, kv, kt, kp)
+    keys = torch.from_numpy(np.concatenate([kp, kv, kt]))
+    logits = (qt @ keys.T) / math.sqrt(d)
+    mask = torch.arange(P + nv + T)[None, :] >= (P + nv + t_of_row[:, None] + 1)
+    p = torch.softmax(logits.masked_fill(mask, float("-inf")), dim=-1)
+    np.testing.assert_allclose(sp, p[:, P:P + nv].mean(dim=0).numpy(), rtol=1e-12, atol=1e-15)
+    assert (sp <= s + 1e-15).all()
+
+
+def check_selection_prefix(orc, seed: int = 13) -> None:
+    """A prompt prefix before the visual block: the visual-only scores and indices are those
+    of the same prompt without it (softmax over the visual keys, which did not change), and
+    the sparse cache is [prefix rows | selected visual rows | text rows]."""
+    rng = np.random.default_rng(seed)
+    L, B, Hq, Hkv, d, T, K, P = 1, 2, 4, 2, 8, 3, 4, 5
+    nvis = np.array([11, 7])
+    cap = P + 11 + T
+    q = rng.standard_normal((L, B, Hq, T, d)) * 2
+    kf = rng.standard_normal((L, B, Hkv, cap, d))
+    vf = rng.standard_normal((L, B, Hkv, cap, d))
+    idx_p, sc_p, ksp, vsp, lsp = orc.select_topk(q, kf, vf, nvis, T, K, P + K + T, n_prefix=P)
+    idx_0, sc_0, k0, _, _ = orc.select_topk(q, kf[:, :, :, P:], vf[:, :, :, P:], nvis, T, K, K + T)
+    np.testing.assert_array_equal(idx_p, idx_0)
+    np.testing.assert_allclose(sc_p, sc_0, rtol=0, atol=0)
+    assert lsp.tolist() == [P + K + T] * B
+    for b in range(B):
+        nv = nvis[b]
+        np.testing.assert_array_equal(ksp[0, b, 1, :P], kf[0, b, 1, :P])
+        np.testing.assert_array_equal(ksp[0, b, 1, P:P + K], kf[0, b, 1, P + idx_p[0, b, 1]])
+        np.testing.assert_array_equal(vsp[0, b, 0, P + K:P + K + T], vf[0, b, 0, P + nv:P + nv + T])
+        np.testing.assert_array_equal(ksp[0, b, 1, P:P + K + T], k0[0, b, 1, :K + T])
 
 
 
@@ -324,7 +358,7 @@ def check_round_lossless_extremes(orc, seed: int = 10) -> None:
 ALL_CHECKS = [
     check_golden_attention, check_golden_verify, check_attention_vs_sdpa,
     check_attention_closed_forms, check_golden_selection, check_selection_invariants, check_selection_causal,
-    check_streaming_and_gather,
+    check_selection_prefix, check_streaming_and_gather,
     check_topk_bruteforce, check_topk_special, check_full_k_sparse_equals_dense,
     check_golden_accept, check_accept_bruteforce, check_commit, check_round_lossless_extremes,
 ]

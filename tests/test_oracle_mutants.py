@@ -27,14 +27,14 @@ def _scores_sum_not_mean(q_text, k_vis):
     return so.selection_scores(q_text, k_vis) * (q_text.shape[0] * q_text.shape[1])
 
 
-def _select_interleaved_groups(q_text, k_full, v_full, nvis, T, K, cap_sparse):
+def _select_interleaved_groups(q_text, k_full, v_full, nvis, T, K, cap_sparse, causal_text=False, n_prefix=0):
     L, B, Hq = q_text.shape[:3]
     Hkv = k_full.shape[2]
-    res = so.select_topk(q_text, k_full, v_full, nvis, T, K, cap_sparse)
+    res = so.select_topk(q_text, k_full, v_full, nvis, T, K, cap_sparse, causal_text, n_prefix)
     idx, scores = res[0].copy(), res[1].copy()
     for h in range(Hkv):
         q = q_text[0, 0, h::Hkv]                               # hq % Hkv grouping
-        s = so.selection_scores(q, k_full[0, 0, h, :int(nvis[0])])
+        s = so.selection_scores(q, k_full[0, 0, h, n_prefix:n_prefix + int(nvis[0])])
         scores[0, 0, h, :len(s)] = s
         idx[0, 0, h] = so.topk_indices(s, K)
     return (idx, scores) + tuple(res[2:])

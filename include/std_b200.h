@@ -147,12 +147,22 @@ enum std_select_flags {
   STD_SELECT_CAUSAL_TEXT = 1
 };
 
-/* std_select_topk with flags (a bitwise OR of std_select_flags; 0 gives
- * std_select_topk).  Same arguments, workspace and results otherwise; unknown
- * flag bits are rejected with STD_ERR_INVALID_ARG. */
+/* std_select_topk for prompts with a prefix and with flags (n_prefix = 0 and
+ * flags = 0 give std_select_topk; same workspace).
+ * n_prefix  prompt rows before the video (a system prompt), the same for every
+ *           sequence: the full cache holds [n_prefix rows | nvis[b] visual rows |
+ *           T text rows].  idx_out and scores_out stay positions within the visual
+ *           block; the sparse cache becomes [n_prefix rows | K selected visual rows |
+ *           T text rows] and len_sparse n_prefix + K + T.  Requires
+ *           n_prefix + nvis_max + T <= cap_full and n_prefix + K + T <= cap_sparse.
+ *           The default score ignores the prefix rows (the softmax runs over the
+ *           visual keys); with STD_SELECT_CAUSAL_TEXT they join every text row's
+ *           softmax, as they precede it.
+ * flags     a bitwise OR of std_select_flags; unknown bits are rejected with
+ *           STD_ERR_INVALID_ARG. */
 int std_select_topk_ex(const std_dims* dims, const void* q_text, int T, const void* k_full,
-                       const void* v_full, const int32_t* nvis, int nvis_max, int K, int flags,
-                       int32_t* idx_out, void* k_sparse, void* v_sparse, int32_t* len_sparse,
+                       const void* v_full, const int32_t* nvis, int nvis_max, int K, int n_prefix,
+                       int flags, int32_t* idx_out, void* k_sparse, void* v_sparse, int32_t* len_sparse,
                        float* scores_out, void* ws, size_t ws_bytes, std_stream_t stream);
 
 /* The selection's top-K step alone, on caller-supplied float32 scores:
@@ -179,13 +189,15 @@ int std_topk_from_scores(const float* scores, int rows, int n, int K, int32_t* i
 int std_streaming_indices(const std_dims* dims, const int32_t* nvis, int K, int n_sink, int32_t* idx_out,
                           std_stream_t stream);
 
-/* The gather step of std_select_topk on caller-given indices: sparse rows [0, K)
- * <- full rows idx[l][b][h][j] (any order, each in [0, nvis[b]); an index outside
- * it flags STD_DEVERR_K_RANGE and leaves that row), rows [K, K + T) <- the text
- * rows [nvis[b], nvis[b] + T), len_sparse[b] <- K + T.  K + T <= cap_sparse. */
+/* The gather step of std_select_topk_ex on caller-given indices, for a full
+ * cache of [P = n_prefix rows | nvis[b] visual rows | T text rows]: sparse rows
+ * [0, P) <- the prefix rows, rows [P, P + K) <- visual rows idx[l][b][h][j] (any
+ * order, each a position in [0, nvis[b]); one outside it flags
+ * STD_DEVERR_K_RANGE and leaves that row), rows [P + K, P + K + T) <- the text
+ * rows, len_sparse[b] <- P + K + T.  P + K + T <= cap_sparse. */
 int std_gather_sparse(const std_dims* dims, const void* k_full, const void* v_full, const int32_t* nvis,
-                      const int32_t* idx, int K, int T, void* k_sparse, void* v_sparse, int32_t* len_sparse,
-                      std_stream_t stream);
+                      const int32_t* idx, int K, int T, int n_prefix, void* k_sparse, void* v_sparse,
+                      int32_t* len_sparse, std_stream_t stream);
 
 /* ---------------------------------------------------------------- decode attention
  *

@@ -66,10 +66,10 @@ SIGNATURES = {
     "std_get_device_error": (_I, [ctypes.POINTER(ctypes.c_int32), _I, _P]),
     "std_select_workspace_size": (_SZ, [_DP, _I, _I]),
     "std_select_topk": (_I, [_DP, _P, _I, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
-    "std_select_topk_ex": (_I, [_DP, _P, _I, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "std_select_topk_ex": (_I, [_DP, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "std_topk_from_scores": (_I, [_P, _I, _I, _I, _P, _P]),
     "std_streaming_indices": (_I, [_DP, _P, _I, _I, _P, _P]),
-    "std_gather_sparse": (_I, [_DP, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P]),
+    "std_gather_sparse": (_I, [_DP, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P]),
     "std_attn_workspace_size": (_SZ, [_DP, _I, _I64, _I]),
     "std_attn_splits": (_I, [_DP, _I, _I64, _I]),
     "std_sparse_decode_attn": (_I, [_DP, _P, _P, _P, _P, _I, _P, _I, _P, _SZ, _P]),
@@ -181,10 +181,10 @@ def std_select_topk(d: StdDims, q_text, T, k_full, v_full, nvis, nvis_max, K, id
 STD_SELECT_CAUSAL_TEXT = 1
 
 
-def std_select_topk_ex(d: StdDims, q_text, T, k_full, v_full, nvis, nvis_max, K, flags, idx_out, k_sparse,
-                       v_sparse, len_sparse, scores_out, ws, stream=None) -> None:
+def std_select_topk_ex(d: StdDims, q_text, T, k_full, v_full, nvis, nvis_max, K, n_prefix, flags, idx_out,
+                       k_sparse, v_sparse, len_sparse, scores_out, ws, stream=None) -> None:
     _check(lib().std_select_topk_ex(ctypes.byref(d), _ptr(q_text), T, _ptr(k_full), _ptr(v_full), _ptr(nvis),
-                                    nvis_max, K, flags, _ptr(idx_out), _ptr(k_sparse), _ptr(v_sparse),
+                                    nvis_max, K, n_prefix, flags, _ptr(idx_out), _ptr(k_sparse), _ptr(v_sparse),
                                     _ptr(len_sparse), _ptr(scores_out), _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
@@ -197,9 +197,9 @@ def std_streaming_indices(d: StdDims, nvis, K, n_sink, idx_out, stream=None) -> 
 
 
 def std_gather_sparse(d: StdDims, k_full, v_full, nvis, idx, K, T, k_sparse, v_sparse, len_sparse,
-                      stream=None) -> None:
+                      n_prefix=0, stream=None) -> None:
     _check(lib().std_gather_sparse(ctypes.byref(d), _ptr(k_full), _ptr(v_full), _ptr(nvis), _ptr(idx), K, T,
-                                   _ptr(k_sparse), _ptr(v_sparse), _ptr(len_sparse), _stream(stream)))
+                                   n_prefix, _ptr(k_sparse), _ptr(v_sparse), _ptr(len_sparse), _stream(stream)))
 
 
 def std_attn_workspace_size(d: StdDims, q_rows: int, cap: int, splits: int) -> int:

@@ -220,16 +220,17 @@ int std_select_topk(const std_dims* dims, const void* q_text, int T, const void*
                     const void* v_full, const int32_t* nvis, int nvis_max, int K, int32_t* idx_out,
                     void* k_sparse, void* v_sparse, int32_t* len_sparse, float* scores_out, void* ws,
                     size_t ws_bytes, std_stream_t stream) {
-  return std_select_topk_ex(dims, q_text, T, k_full, v_full, nvis, nvis_max, K, 0, idx_out, k_sparse, v_sparse,
-                            len_sparse, scores_out, ws, ws_bytes, stream);
+  return std_select_topk_ex(dims, q_text, T, k_full, v_full, nvis, nvis_max, K, 0, 0, idx_out, k_sparse,
+                            v_sparse, len_sparse, scores_out, ws, ws_bytes, stream);
 }
 
 int std_select_topk_ex(const std_dims* dims, const void* q_text, int T, const void* k_full,
-                       const void* v_full, const int32_t* nvis, int nvis_max, int K, int flags,
-                       int32_t* idx_out, void* k_sparse, void* v_sparse, int32_t* len_sparse,
+                       const void* v_full, const int32_t* nvis, int nvis_max, int K, int n_prefix,
+                       int flags, int32_t* idx_out, void* k_sparse, void* v_sparse, int32_t* len_sparse,
                        float* scores_out, void* ws, size_t ws_bytes, std_stream_t stream) {
   STD_TRY(check_dims(dims));
   if (flags & ~STD_SELECT_CAUSAL_TEXT) return fail(STD_ERR_INVALID_ARG, "unknown selection flags %#x", flags);
+  if (n_prefix < 0) return fail(STD_ERR_INVALID_ARG, "n_prefix = %d must be >= 0", n_prefix);
   STD_TRY(check_ptr(q_text, 16, "q_text"));
   STD_TRY(check_ptr(k_full, 16, "k_full"));
   STD_TRY(check_ptr(v_full, 16, "v_full"));
@@ -242,10 +243,12 @@ int std_select_topk_ex(const std_dims* dims, const void* q_text, int T, const vo
   if (T < 1) return fail(STD_ERR_INVALID_ARG, "T = %d must be >= 1", T);
   if (nvis_max < 1) return fail(STD_ERR_INVALID_ARG, "nvis_max = %d must be >= 1", nvis_max);
   if (K < 1 || K > nvis_max) return fail(STD_ERR_INVALID_ARG, "K = %d must be in [1, nvis_max = %d]", K, nvis_max);
-  if ((int64_t)K + T > dims->cap_sparse)
-    return fail(STD_ERR_CAPACITY, "K + T = %d exceeds cap_sparse = %lld", K + T, (long long)dims->cap_sparse);
-  if ((int64_t)nvis_max + T > dims->cap_full)
-    return fail(STD_ERR_CAPACITY, "nvis_max + T = %d exceeds cap_full = %lld", nvis_max + T, (long long)dims->cap_full);
+  if ((int64_t)n_prefix + K + T > dims->cap_sparse)
+    return fail(STD_ERR_CAPACITY, "n_prefix + K + T = %lld exceeds cap_sparse = %lld", (long long)n_prefix + K + T,
+                (long long)dims->cap_sparse);
+  if ((int64_t)n_prefix + nvis_max + T > dims->cap_full)
+    return fail(STD_ERR_CAPACITY, "n_prefix + nvis_max + T = %lld exceeds cap_full = %lld",
+                (long long)n_prefix + nvis_max + T, (long long)dims->cap_full);
   const size_t need = std_select_workspace_size(dims, T, nvis_max);
   if (!ws || ws_bytes < need) return fail(STD_ERR_WORKSPACE, "select workspace: need %zu bytes, got %zu", need, ws ? ws_bytes : 0);
   STD_TRY(check_ptr(ws, 16, "ws"));
@@ -264,6 +267,7 @@ int std_select_topk_ex(const std_dims* dims, const void* q_text, int T, const vo
   s.L = dims->L; s.B = dims->B; s.Hq = dims->Hq; s.Hkv = dims->Hkv; s.G = G; s.T = T; s.d = dims->d;
   s.dtype = dims->dtype; s.cap = dims->cap_full; s.row_m = row_m; s.row_l = row_l; s.scores = scores; s.err = err;
   s.causal_text = (flags & STD_SELECT_CAUSAL_TEXT) ? 1 : 0;
+  s.prefix = n_prefix;
   cudaError_t e = stdb::launch_select_scores(s, stream);
   if (e != cudaSuccess) return cuda_fail(e, "selection score launch");
   e = stdb::launch_topk(scores, nvis_max, probs, nvis, 0, dims->Hkv, dims->B, K, idx_out, err, stream);
@@ -272,7 +276,7 @@ int std_select_topk_ex(const std_dims* dims, const void* q_text, int T, const vo
   g.k_full = k_full; g.v_full = v_full; g.k_sp = k_sparse; g.v_sp = v_sparse; g.idx = idx_out; g.nvis = nvis;
   g.len_sparse = len_sparse; g.L = dims->L; g.B = dims->B; g.Hkv = dims->Hkv; g.T = T; g.K = K;
   g.row_bytes = dims->d * elem_bytes(dims->dtype); g.cap_full = dims->cap_full; g.cap_sparse = dims->cap_sparse;
-  g.err = err;
+  g.prefix = n_prefix; g.err = err;
   e = stdb::launch_gather(g, stream);
   if (e != cudaSuccess) return cuda_fail(e, "gather launch");
   return ok();
@@ -293,8 +297,8 @@ int std_streaming_indices(const std_dims* dims, const int32_t* nvis, int K, int 
 }
 
 int std_gather_sparse(const std_dims* dims, const void* k_full, const void* v_full, const int32_t* nvis,
-                      const int32_t* idx, int K, int T, void* k_sparse, void* v_sparse, int32_t* len_sparse,
-                      std_stream_t stream) {
+                      const int32_t* idx, int K, int T, int n_prefix, void* k_sparse, void* v_sparse,
+                      int32_t* len_sparse, std_stream_t stream) {
   STD_TRY(check_dims(dims));
   STD_TRY(check_ptr(k_full, 16, "k_full"));
   STD_TRY(check_ptr(v_full, 16, "v_full"));
@@ -303,16 +307,17 @@ int std_gather_sparse(const std_dims* dims, const void* k_full, const void* v_fu
   STD_TRY(check_ptr(k_sparse, 16, "k_sparse"));
   STD_TRY(check_ptr(v_sparse, 16, "v_sparse"));
   STD_TRY(check_ptr(len_sparse, 4, "len_sparse"));
-  if (K < 1 || T < 0) return fail(STD_ERR_INVALID_ARG, "K = %d, T = %d", K, T);
-  if ((int64_t)K + T > dims->cap_sparse)
-    return fail(STD_ERR_CAPACITY, "K + T = %d exceeds cap_sparse = %lld", K + T, (long long)dims->cap_sparse);
+  if (K < 1 || T < 0 || n_prefix < 0) return fail(STD_ERR_INVALID_ARG, "K = %d, T = %d, n_prefix = %d", K, T, n_prefix);
+  if ((int64_t)n_prefix + K + T > dims->cap_sparse)
+    return fail(STD_ERR_CAPACITY, "n_prefix + K + T = %lld exceeds cap_sparse = %lld", (long long)n_prefix + K + T,
+                (long long)dims->cap_sparse);
   int* err;
   STD_TRY(device_state(&err, nullptr));
   stdb::GatherArgs g{};
   g.k_full = k_full; g.v_full = v_full; g.k_sp = k_sparse; g.v_sp = v_sparse; g.idx = idx; g.nvis = nvis;
   g.len_sparse = len_sparse; g.L = dims->L; g.B = dims->B; g.Hkv = dims->Hkv; g.T = T; g.K = K;
   g.row_bytes = dims->d * elem_bytes(dims->dtype); g.cap_full = dims->cap_full; g.cap_sparse = dims->cap_sparse;
-  g.err = err;
+  g.prefix = n_prefix; g.err = err;
   cudaError_t e = stdb::launch_gather(g, stream);
   if (e != cudaSuccess) return cuda_fail(e, "gather launch");
   return ok();

@@ -73,6 +73,7 @@ struct ScoreArgs {
   float* scores;  // [prob][nvis_max]
   int* err;
   int causal_text;  // nonzero: text keys 0..t join row (g, t)'s softmax (launch_text_rowstats after pass 1)
+  int prefix;       // prompt rows before the visual block (a system prompt): cache = [prefix | visual | text]
 };
 cudaError_t launch_select_scores(const ScoreArgs& a, cudaStream_t s);
 // Causal full-row variant: merge each text row's visible text keys into pass 1's (row_m, row_l).
@@ -95,6 +96,7 @@ struct GatherArgs {
   const int32_t* nvis;
   int32_t* len_sparse;
   int L, B, Hkv, T, K, row_bytes;
+  int prefix;  // prompt rows before the visual block, copied first
   int64_t cap_full, cap_sparse;
   int* err;
 };

@@ -25,26 +25,29 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) gather_kernel(const GatherA
   const int j = blockIdx.x * ROWS_PER_CTA + warp;
   const int prob = lb * a.Hkv + h;
   const int nv = a.nvis[b];
-  if (a.K > nv || (int64_t)nv + a.T > a.cap_full) {
+  if (a.K > nv || (int64_t)a.prefix + nv + a.T > a.cap_full) {
     if (j == 0 && h == 0 && lane == 0) flag_error(a.err, STD_DEVERR_K_RANGE);
     return;
   }
-  if (j >= a.K + a.T) return;
-  int src;
-  if (j < a.K) {
-    src = a.idx[(size_t)prob * a.K + j];
-    if (src < 0 || src >= nv) {  // only possible if the top-K step was skipped
+  if (j >= a.prefix + a.K + a.T) return;
+  int src;  // full-cache row: [prefix | visual | text] -> sparse [prefix | K selected | text]
+  if (j < a.prefix) {
+    src = j;
+  } else if (j < a.prefix + a.K) {
+    src = a.idx[(size_t)prob * a.K + (j - a.prefix)];
+    if (src < 0 || src >= nv) {  // an index outside the visual block
       if (lane == 0) flag_error(a.err, STD_DEVERR_K_RANGE);
       return;
     }
+    src += a.prefix;
   } else {
-    src = nv + (j - a.K);
+    src = a.prefix + nv + (j - a.prefix - a.K);
   }
   const size_t so = ((size_t)prob * a.cap_full + src) * a.row_bytes;
   const size_t dof = ((size_t)prob * a.cap_sparse + j) * a.row_bytes;
   copy_row(static_cast<uint8_t*>(a.k_sp) + dof, static_cast<const uint8_t*>(a.k_full) + so, a.row_bytes, lane);
   copy_row(static_cast<uint8_t*>(a.v_sp) + dof, static_cast<const uint8_t*>(a.v_full) + so, a.row_bytes, lane);
-  if (blockIdx.x == 0 && h == 0 && blockIdx.z / a.B == 0 && threadIdx.x == 0) a.len_sparse[b] = a.K + a.T;
+  if (blockIdx.x == 0 && h == 0 && blockIdx.z / a.B == 0 && threadIdx.x == 0) a.len_sparse[b] = a.prefix + a.K + a.T;
 }
 
 // cache rows len[b] + off + r <- new rows r (r < n_new).
@@ -127,7 +130,7 @@ __global__ void accept_kernel(int B, int gamma, const int32_t* draft, const int3
 }  // namespace
 
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s) {
-  dim3 grid((a.K + a.T + ROWS_PER_CTA - 1) / ROWS_PER_CTA, a.Hkv, a.L * a.B);
+  dim3 grid((a.prefix + a.K + a.T + ROWS_PER_CTA - 1) / ROWS_PER_CTA, a.Hkv, a.L * a.B);
   return launch_pdl(gather_kernel, grid, dim3(ROWS_PER_CTA * 32), 0, s, a);
 }
 

@@ -28,7 +28,7 @@ constexpr int P1_STAGES = 3;
 __device__ __forceinline__ bool visual_ok(const ScoreArgs& a, int b, int* nv_out) {
   const int nv = a.nvis[b];
   *nv_out = nv;
-  return nv >= 1 && nv <= a.nvis_max && (int64_t)nv + a.T <= a.cap;
+  return nv >= 1 && nv <= a.nvis_max && (int64_t)a.prefix + nv + a.T <= a.cap;
 }
 
 // Q fragments (m16n8k16 A operand) of 16 text rows starting at r_base.
@@ -95,7 +95,8 @@ __global__ void __launch_bounds__(128) rowstats_bf16_kernel(const ScoreArgs a) {
     if (blockIdx.x == 0 && tid == 0) flag_error(a.err, nv > a.nvis_max ? STD_DEVERR_NVIS_MAX : STD_DEVERR_K_RANGE);
     return;
   }
-  const __nv_bfloat16* kp = reinterpret_cast<const __nv_bfloat16*>(a.k_full) + (size_t)prob * a.cap * D;
+  const __nv_bfloat16* kp = reinterpret_cast<const __nv_bfloat16*>(a.k_full) +
+                               ((size_t)prob * a.cap + a.prefix) * D;  // visual key 0
   const __nv_bfloat16* qp = reinterpret_cast<const __nv_bfloat16*>(a.q_text) + (size_t)(lb * a.Hq + h * a.G) * a.T * D;
   const int r_base = blockIdx.x * 64 + warp * 16;
   uint32_t qf[D / 16][4];
@@ -169,7 +170,8 @@ __global__ void __launch_bounds__(128) colsum_bf16_kernel(const ScoreArgs a) {
   if (!visual_ok(a, b, &nv)) return;  // pass 1 flagged it
   const int key0 = blockIdx.x * TKS;
   if (key0 >= nv) return;
-  const __nv_bfloat16* kp = reinterpret_cast<const __nv_bfloat16*>(a.k_full) + (size_t)prob * a.cap * D;
+  const __nv_bfloat16* kp = reinterpret_cast<const __nv_bfloat16*>(a.k_full) +
+                               ((size_t)prob * a.cap + a.prefix) * D;  // visual key 0
   const __nv_bfloat16* qp = reinterpret_cast<const __nv_bfloat16*>(a.q_text) + (size_t)(lb * a.Hq + h * a.G) * a.T * D;
   const uint32_t sk = smem_u32(smem);
   load_ktile<D>(sk, kp, key0, nv, tid, 128);
@@ -244,7 +246,7 @@ __global__ void __launch_bounds__(128) rowstats_f32_kernel(const ScoreArgs a) {
   }
   const int r = blockIdx.x * 128 + threadIdx.x;
   if (r >= M) return;
-  const float* kp = reinterpret_cast<const float*>(a.k_full) + (size_t)prob * a.cap * D;
+  const float* kp = reinterpret_cast<const float*>(a.k_full) + ((size_t)prob * a.cap + a.prefix) * D;  // visual key 0
   const float* qp = reinterpret_cast<const float*>(a.q_text) + ((size_t)(lb * a.Hq + h * a.G) * a.T + r) * D;
   float q[D];
 #pragma unroll
@@ -276,7 +278,7 @@ __global__ void __launch_bounds__(128) colsum_f32_kernel(const ScoreArgs a) {
   if (!visual_ok(a, b, &nv)) return;
   const int n = blockIdx.x * 128 + threadIdx.x;
   if (n >= nv) return;
-  const float* kp = reinterpret_cast<const float*>(a.k_full) + ((size_t)prob * a.cap + n) * D;
+  const float* kp = reinterpret_cast<const float*>(a.k_full) + ((size_t)prob * a.cap + a.prefix + n) * D;
   const float* qp = reinterpret_cast<const float*>(a.q_text) + (size_t)(lb * a.Hq + h * a.G) * a.T * D;
   float k[D];
 #pragma unroll

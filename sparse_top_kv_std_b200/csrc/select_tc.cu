@@ -65,7 +65,7 @@ struct Ctl {
 __device__ __forceinline__ bool visual_ok(const ScoreArgs& a, int b, int* nv_out) {
   const int nv = a.nvis[b];
   *nv_out = nv;
-  return nv >= 1 && nv <= a.nvis_max && (int64_t)nv + a.T <= a.cap;
+  return nv >= 1 && nv <= a.nvis_max && (int64_t)a.prefix + nv + a.T <= a.cap;
 }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -246,7 +246,7 @@ rowstats_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tc::mbar_expect_tx(&ctl->qfull, C::Q_BYTES);
 #pragma unroll
       for (int kb = 0; kb < C::KB; ++kb) tc::tma_load_2d(sQ + kb * BM * 128, &tm_q, kb * 64, qrow, &ctl->qfull);
-      const int krow = prob * (int)a.cap;
+      const int krow = prob * (int)a.cap + a.prefix;  // visual key 0
       int issued = 0;
       for (int t = 0; t < ntiles; ++t) {
         const int s = t % C::STAGES;
@@ -441,7 +441,7 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc::mbar_expect_tx(&ctl->kfull, C::K_BYTES);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb)
-          tc::tma_load_2d(sK + kb * 256 * 128, &tm_k, kb * 64, prob * (int)a.cap + key_base + kbi * 256,
+          tc::tma_load_2d(sK + kb * 256 * 128, &tm_k, kb * 64, prob * (int)a.cap + a.prefix + key_base + kbi * 256,
                           &ctl->kfull);
         kissued = kbi + 1;
         for (int c = 0; c < nch; ++c) {

@@ -3,17 +3,19 @@
 // "Methodik" item 4 of the gist.science summary averages the attention from the
 // text tokens to the visual tokens but does not say which keys that softmax runs
 // over.  The default reading takes the visual keys only; this variant lets each
-// text query see what it sees in the prompt's causal attention: every visual key
-// and the text keys up to its own position.  The visual-key probabilities then
-// carry the text keys' share of each row's denominator.
+// text query see what it sees in the prompt's causal attention: the prompt prefix
+// before the video (a system prompt, if any), every visual key and the text keys
+// up to its own position.  The visual-key probabilities then carry the other
+// keys' share of each row's denominator.
 //
 // Pass 1 of the selection leaves, per text row r, statistics of its visual logits
 // in the exp2 domain: m_r = max_n x_rn and l_r = sum_n 2^(x_rn - m_r), with
-// x = log2(e) q . k / sqrt(d).  This kernel adds the text keys 0..t of row
-// r = (g, t) to (m_r, l_r); pass 2 then turns the merged statistics into
-// visual-key probabilities unchanged.  The text keys are a few hundred per row
-// (well under 1% of the visual work at the long-video shapes), so plain fp32 dot
-// products suffice.
+// x = log2(e) q . k / sqrt(d).  This kernel adds the keys row r = (g, t) sees
+// besides the visual ones -- the rows of a prompt prefix before the video (a
+// system prompt), if any, and the text keys 0..t -- to (m_r, l_r); pass 2 then
+// turns the merged statistics into visual-key probabilities unchanged.  These
+// are a few hundred keys per row (well under 1% of the visual work at the
+// long-video shapes), so plain fp32 dot products suffice.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -26,7 +28,7 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kRowsPerWarp = 4;
 constexpr int kRows = kWarps * kRowsPerWarp;  // text rows per CTA
-constexpr int kKeys = 32;                     // text keys per shared-memory tile: one per lane
+constexpr int kKeys = 32;                     // extra keys per shared-memory tile: one per lane
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -41,13 +43,15 @@ __global__ void __launch_bounds__(kWarps * 32) text_rowstats_kernel(const ScoreA
   const int prob = lb * a.Hkv + h;
   const int M = a.G * a.T;
   const int nv = a.nvis[b];
-  if (nv < 1 || nv > a.nvis_max || (int64_t)nv + a.T > a.cap) return;  // pass 1 flagged it
+  if (nv < 1 || nv > a.nvis_max || (int64_t)a.prefix + nv + a.T > a.cap) return;  // pass 1 flagged it
   const int r0 = blockIdx.x * kRows;
   if (r0 >= M) return;
   const int nrows = min(kRows, M - r0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // text key 0 of this head, and query row r0 of the head's G x T text rows
-  const E* kbase = static_cast<const E*>(a.k_full) + ((size_t)prob * a.cap + nv) * D;
+  // key j of the extra keys: prefix row j (j < prefix), else text key j - prefix; and
+  // query row r0 of the head's G x T text rows
+  const E* kpre = static_cast<const E*>(a.k_full) + (size_t)prob * a.cap * D;
+  const E* ktext = kpre + ((size_t)a.prefix + nv) * D;
   const E* qbase = static_cast<const E*>(a.q_text) + ((size_t)(lb * a.Hq + h * a.G) * a.T + r0) * D;
   for (int i = threadIdx.x; i < kRows * D; i += blockDim.x) {
     const int r = i / D;
@@ -55,28 +59,31 @@ __global__ void __launch_bounds__(kWarps * 32) text_rowstats_kernel(const ScoreA
   }
   int tmax = 0;  // last text position any of the CTA's rows sees
   for (int r = 0; r < nrows; ++r) tmax = max(tmax, (r0 + r) % a.T);
+  const int jend = a.prefix + tmax;  // last extra key any row sees
 
   const float sc = kLog2e * rsqrtf((float)D);
   float m[kRowsPerWarp], l[kRowsPerWarp];
-  int tpos[kRowsPerWarp];  // text position of the warp's i-th row, -1 past the rows
+  int tpos[kRowsPerWarp];  // last extra key (prefix + t) the warp's i-th row sees, -1 past the rows
 #pragma unroll
   for (int i = 0; i < kRowsPerWarp; ++i) {
     const int r = warp + kWarps * i;
     m[i] = -INFINITY;
     l[i] = 0.f;
-    tpos[i] = r < nrows ? (r0 + r) % a.T : -1;
+    tpos[i] = r < nrows ? a.prefix + (r0 + r) % a.T : -1;
   }
-  for (int k0 = 0; k0 <= tmax; k0 += kKeys) {
+  for (int k0 = 0; k0 <= jend; k0 += kKeys) {
     __syncthreads();  // the previous tile is consumed (and the query rows are written)
     for (int i = threadIdx.x; i < kKeys * D; i += blockDim.x) {
       const int j = i / D;
-      ks[j][i % D] = k0 + j <= tmax ? to_f(kbase[(size_t)(k0 + j) * D + i % D]) : 0.f;
+      const int jj = k0 + j;
+      const E* row = jj < a.prefix ? kpre + (size_t)jj * D : ktext + (size_t)(jj - a.prefix) * D;
+      ks[j][i % D] = jj <= jend ? to_f(row[i % D]) : 0.f;
     }
     __syncthreads();
-    const int j = k0 + lane;  // this lane's text key
+    const int j = k0 + lane;  // this lane's extra key
 #pragma unroll
     for (int i = 0; i < kRowsPerWarp; ++i) {
-      if (j > tpos[i]) continue;  // causal: row (g, t) sees text keys 0..t (and none past the rows)
+      if (j > tpos[i]) continue;  // causal: row (g, t) sees the prefix and text keys 0..t
       const float* qr = qs[warp + kWarps * i];
       float acc = 0.f;
 #pragma unroll 8

@@ -57,10 +57,12 @@ class DecodeSession:
         self.nvis.copy_(nv, non_blocking=True)
         self.len_full.copy_(self.nvis + self.T, non_blocking=True)
 
-    def select(self, q_text: torch.Tensor, stream=None, keep_scores: bool = True, flags: int = 0) -> None:
-        """Prefill selection; flags = binding.STD_SELECT_CAUSAL_TEXT for the causal full-row score."""
+    def select(self, q_text: torch.Tensor, stream=None, keep_scores: bool = True, flags: int = 0,
+               n_prefix: int = 0) -> None:
+        """Prefill selection; flags = binding.STD_SELECT_CAUSAL_TEXT for the causal full-row score,
+        n_prefix = prompt rows (a system prompt) before the visual block of the full cache."""
         B_.std_select_topk_ex(self.dims, q_text, self.T, self.k_full, self.v_full, self.nvis, self.nvis_max,
-                              self.K, flags, self.idx, self.k_sparse, self.v_sparse, self.len_sparse,
+                              self.K, n_prefix, flags, self.idx, self.k_sparse, self.v_sparse, self.len_sparse,
                               self.scores if keep_scores else None, self.ws_select, stream)
 
     # -- decoding

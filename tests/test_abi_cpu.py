@@ -76,14 +76,19 @@ FAKE = 1 << 40  # a 16-byte aligned non-null "pointer": never dereferenced, chec
     (lambda: lib_().std_select_topk(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, FAKE, 512, 256, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_CAPACITY),
     (lambda: lib_().std_select_topk(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, FAKE, 990, 16, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_CAPACITY),
     (lambda: lib_().std_select_topk(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, FAKE, 512, 16, FAKE, FAKE, FAKE, FAKE, None, FAKE, 16, None), B.STD_ERR_WORKSPACE),
-    (lambda: lib_().std_select_topk_ex(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, FAKE, 512, 16, 2, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_INVALID_ARG),
-    (lambda: lib_().std_select_topk_ex(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, FAKE, 512, 256, 1, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_CAPACITY),
+    (lambda: lib_().std_select_topk_ex(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, FAKE, 512, 16, 0, 2, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_select_topk_ex(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, FAKE, 512, 256, 0, 1, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_CAPACITY),
+    (lambda: lib_().std_select_topk_ex(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, FAKE, 512, 16, -1, 0, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_select_topk_ex(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, FAKE, 512, 16, 425, 0, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_CAPACITY),
+    (lambda: lib_().std_select_topk_ex(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, FAKE, 800, 16, 200, 0, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_CAPACITY),
     (lambda: lib_().std_topk_from_scores(FAKE, 4, 100, 101, FAKE, None), B.STD_ERR_INVALID_ARG),
     (lambda: lib_().std_streaming_indices(ctypes.byref(_dims()), FAKE, 16, 17, FAKE, None), B.STD_ERR_INVALID_ARG),
     (lambda: lib_().std_streaming_indices(ctypes.byref(_dims()), FAKE, 0, 0, FAKE, None), B.STD_ERR_INVALID_ARG),
     (lambda: lib_().std_streaming_indices(ctypes.byref(_dims()), None, 16, 4, FAKE, None), B.STD_ERR_INVALID_ARG),
-    (lambda: lib_().std_gather_sparse(ctypes.byref(_dims()), FAKE, FAKE, FAKE, FAKE, 256, 64, FAKE, FAKE, FAKE, None), B.STD_ERR_CAPACITY),
-    (lambda: lib_().std_gather_sparse(ctypes.byref(_dims()), FAKE, FAKE, FAKE, None, 16, 64, FAKE, FAKE, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_gather_sparse(ctypes.byref(_dims()), FAKE, FAKE, FAKE, FAKE, 256, 64, 0, FAKE, FAKE, FAKE, None), B.STD_ERR_CAPACITY),
+    (lambda: lib_().std_gather_sparse(ctypes.byref(_dims()), FAKE, FAKE, FAKE, FAKE, 200, 64, 37, FAKE, FAKE, FAKE, None), B.STD_ERR_CAPACITY),
+    (lambda: lib_().std_gather_sparse(ctypes.byref(_dims()), FAKE, FAKE, FAKE, FAKE, 16, 64, -1, FAKE, FAKE, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_gather_sparse(ctypes.byref(_dims()), FAKE, FAKE, FAKE, None, 16, 64, 0, FAKE, FAKE, FAKE, None), B.STD_ERR_INVALID_ARG),
     (lambda: lib_().std_topk_from_scores(None, 4, 100, 10, FAKE, None), B.STD_ERR_INVALID_ARG),
     (lambda: lib_().std_dense_verify_attn(ctypes.byref(_dims()), FAKE, 32, FAKE, FAKE, FAKE, FAKE, 1, None, 0, None), B.STD_ERR_INVALID_ARG),
     (lambda: lib_().std_dense_verify_attn(ctypes.byref(_dims()), FAKE, -1, FAKE, FAKE, FAKE, FAKE, 1, None, 0, None), B.STD_ERR_INVALID_ARG),

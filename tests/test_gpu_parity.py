@@ -90,42 +90,67 @@ def test_select_causal_text_matches_oracle(name):
     _check_select(wl, synth.host_inputs(wl, seed=3), flags=B.STD_SELECT_CAUSAL_TEXT)
 
 
-def _check_select(wl, x, flags=0):
-    s = H.session_for(wl)
+PREFIX_CASES = [("ragged_bf16", 0), ("ragged_bf16", 1), ("tiny_f32", 0), ("tiny_f32", 1),
+                ("rows2100_fallback", 0), ("tc_ragged_rows", 1)]
+
+
+@pytest.mark.parametrize("name,causal", PREFIX_CASES)
+def test_select_with_prompt_prefix(name, causal):
+    """A system prompt of 13 rows before the video in the full cache: scores, indices and the
+    sparse layout [prefix | selected visual | text], on the tensor-core, bf16 and fp32 paths,
+    with both readings of the score."""
+    wl = SELECT_CASES[name]
+    x = synth.host_inputs(wl, seed=5)
+    P = 13
+    rng = np.random.default_rng(17)
+    for key in ("k_full", "v_full"):
+        pre = rng.standard_normal(x[key].shape[:3] + (P, wl.d)).astype(np.float32)
+        x[key] = np.concatenate([synth.storage(pre, wl.dtype), x[key]], axis=3)
+    _check_select(wl, x, flags=B.STD_SELECT_CAUSAL_TEXT if causal else 0, n_prefix=P)
+
+
+def _check_select(wl, x, flags=0, n_prefix=0):
+    """Selection through the library against the oracle; x["k_full"] / x["v_full"] hold
+    [n_prefix rows | visual | text] per (layer, sequence, KV head)."""
+    from sparse_top_kv_std_b200.session import DecodeSession
+    P = n_prefix
+    cap_full, cap_sparse = x["k_full"].shape[3], wl.cap_sparse + P
+    s = DecodeSession(wl.L, wl.B, wl.Hq, wl.Hkv, wl.d, H.dtype_code(wl), cap_full, cap_sparse, wl.T, wl.K,
+                      wl.gamma, wl.nvis_max)
     s.k_full.copy_(H.to_dev(x["k_full"]))
     s.v_full.copy_(H.to_dev(x["v_full"]))
     s.start(x["nvis"])
     q_text = H.to_dev(x["q_text"])
-    s.select(q_text, flags=flags)
+    s.select(q_text, flags=flags, n_prefix=P)
     torch.cuda.synchronize()
     assert B.std_get_device_error() == 0
 
     idx_o, sc_o, ksp_o, vsp_o, lsp_o = oracle.select_topk(
         H.f64(x["q_text"], wl), H.f64(x["k_full"], wl), H.f64(x["v_full"], wl), x["nvis"], wl.T, wl.K,
-        wl.cap_sparse, causal_text=bool(flags))
+        cap_sparse, causal_text=bool(flags), n_prefix=P)
     sc_g = s.scores.cpu().numpy().astype(np.float64)
     idx_g = s.idx.cpu().numpy()
     rtol = H.score_rtol(wl)
-    kf = x["k_full"]
+    kf, vf = x["k_full"], x["v_full"]
     ksp_g = H.to_host_bits(s.k_sparse)
     vsp_g = H.to_host_bits(s.v_sparse)
-    assert s.len_sparse.cpu().tolist() == [wl.K + wl.T] * wl.B
+    K, T = wl.K, wl.T
+    assert s.len_sparse.cpu().tolist() == [P + K + T] * wl.B
     for l in range(wl.L):
         for b in range(wl.B):
             nv = wl.nvis[b]
             for h in range(wl.Hkv):
                 o_s, g_s = sc_o[l, b, h, :nv], sc_g[l, b, h, :nv]
                 np.testing.assert_allclose(g_s, o_s, rtol=rtol, atol=rtol * 1e-3 * o_s.max())
-                H.assert_topk_boundary(idx_g[l, b, h], idx_o[l, b, h], o_s, wl.K, rtol)
-                # gather: byte-exact rows at the GPU's own indices, then the text rows
+                H.assert_topk_boundary(idx_g[l, b, h], idx_o[l, b, h], o_s, K, rtol)
+                # gather: byte-exact prefix rows, rows at the GPU's own indices, then the text rows
                 ix = idx_g[l, b, h]
-                np.testing.assert_array_equal(ksp_g[l, b, h, :wl.K], kf[l, b, h, ix])
-                np.testing.assert_array_equal(vsp_g[l, b, h, :wl.K], x["v_full"][l, b, h, ix])
-                np.testing.assert_array_equal(ksp_g[l, b, h, wl.K:wl.K + wl.T], kf[l, b, h, nv:nv + wl.T])
-                np.testing.assert_array_equal(vsp_g[l, b, h, wl.K:wl.K + wl.T],
-                                              x["v_full"][l, b, h, nv:nv + wl.T])
+                for got, full in ((ksp_g, kf), (vsp_g, vf)):
+                    np.testing.assert_array_equal(got[l, b, h, :P], full[l, b, h, :P])
+                    np.testing.assert_array_equal(got[l, b, h, P:P + K], full[l, b, h, P + ix])
+                    np.testing.assert_array_equal(got[l, b, h, P + K:P + K + T], full[l, b, h, P + nv:P + nv + T])
                 # top-K step bit-exact on the GPU's own fp32 scores
-                want = oracle.topk_indices(s.scores[l, b, h, :nv].cpu().numpy(), wl.K)
+                want = oracle.topk_indices(s.scores[l, b, h, :nv].cpu().numpy(), K)
                 np.testing.assert_array_equal(ix, want)
 
 
@@ -416,19 +441,26 @@ def test_exp2_polynomial_error_bound():
 
 # ----------------------------------------------------------------------------- streaming baseline
 
-@pytest.mark.parametrize("name,n_sink", [("ragged_bf16", 4), ("tiny_f32", 0), ("d64_bf16_G1", 300)])
-def test_streaming_indices_and_gather(name, n_sink):
+@pytest.mark.parametrize("name,n_sink,P", [("ragged_bf16", 4, 0), ("tiny_f32", 0, 0), ("d64_bf16_G1", 300, 0),
+                                            ("ragged_bf16", 4, 9)])
+def test_streaming_indices_and_gather(name, n_sink, P):
     wl = SELECT_CASES[name]
     x = synth.host_inputs(wl, seed=4)
-    d = B.dims(wl.L, wl.B, wl.Hq, wl.Hkv, wl.d, H.dtype_code(wl), wl.cap_full, wl.cap_sparse)
+    if P:  # a prompt prefix before the visual block
+        for key in ("k_full", "v_full"):
+            pre = np.random.default_rng(3).standard_normal(x[key].shape[:3] + (P, wl.d)).astype(np.float32)
+            x[key] = np.concatenate([synth.storage(pre, wl.dtype), x[key]], axis=3)
+    cap_sparse = wl.cap_sparse + P
+    d = B.dims(wl.L, wl.B, wl.Hq, wl.Hkv, wl.d, H.dtype_code(wl), x["k_full"].shape[3], cap_sparse)
     nvis = torch.tensor(wl.nvis, dtype=torch.int32, device="cuda")
     idx = torch.full((wl.L, wl.B, wl.Hkv, wl.K), -1, dtype=torch.int32, device="cuda")
     st = torch.float32 if wl.dtype == "f32" else torch.int16
-    ksp = torch.zeros((wl.L, wl.B, wl.Hkv, wl.cap_sparse, wl.d), dtype=st, device="cuda")
+    ksp = torch.zeros((wl.L, wl.B, wl.Hkv, cap_sparse, wl.d), dtype=st, device="cuda")
     vsp = torch.zeros_like(ksp)
     lsp = torch.zeros(wl.B, dtype=torch.int32, device="cuda")
     B.std_streaming_indices(d, nvis, wl.K, n_sink, idx)
-    B.std_gather_sparse(d, H.to_dev(x["k_full"]), H.to_dev(x["v_full"]), nvis, idx, wl.K, wl.T, ksp, vsp, lsp)
+    B.std_gather_sparse(d, H.to_dev(x["k_full"]), H.to_dev(x["v_full"]), nvis, idx, wl.K, wl.T, ksp, vsp, lsp,
+                        n_prefix=P)
     torch.cuda.synchronize()
     assert B.std_get_device_error() == 0
     idx_h = idx.cpu().numpy()
@@ -437,8 +469,8 @@ def test_streaming_indices_and_gather(name, n_sink):
         for l in range(wl.L):
             for h in range(wl.Hkv):
                 np.testing.assert_array_equal(idx_h[l, b, h], want)
-    kw, vw, lw = oracle.gather_sparse(x["k_full"], x["v_full"], np.array(wl.nvis), idx_h, wl.T, wl.cap_sparse)
-    n = wl.K + wl.T
+    kw, vw, lw = oracle.gather_sparse(x["k_full"], x["v_full"], np.array(wl.nvis), idx_h, wl.T, cap_sparse, P)
+    n = P + wl.K + wl.T
     got_k = ksp.cpu().numpy().view(x["k_full"].dtype)[..., :n, :]
     got_v = vsp.cpu().numpy().view(x["v_full"].dtype)[..., :n, :]
     np.testing.assert_array_equal(got_k, kw[..., :n, :].astype(x["k_full"].dtype))

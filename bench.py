@@ -419,13 +419,12 @@ def run_std(args, rank, world, local_rank):
             ev["sel1"].record(stream)
         for r in range(R):
             o = outs[r]
-            for j in range(wl.gamma):
-                B.std_kv_append(sess.dims, sess.k_sparse, sess.v_sparse, wl.cap_sparse, sess.len_sparse, j,
-                                view("k_draft", r)[j], view("v_draft", r)[j], 1)
+            for j in range(wl.gamma):  # draft step j: append its input's row, attend (one launch)
                 if draft_ev:
                     ev["d0"][r * wl.gamma + j].record(stream)
-                B.std_sparse_decode_attn(sess.dims, view("q_draft", r)[j], sess.k_sparse, sess.v_sparse,
-                                         sess.len_sparse, j + 1, o["o_draft"][j], 0, ws)
+                B.std_sparse_decode_attn_append(sess.dims, view("q_draft", r)[j], sess.k_sparse, sess.v_sparse,
+                                                sess.len_sparse, j + 1, view("k_draft", r)[j], view("v_draft", r)[j],
+                                                o["o_draft"][j], 0, ws)
                 if draft_ev:
                     ev["d1"][r * wl.gamma + j].record(stream)
             B.std_kv_append(sess.dims, sess.k_full, sess.v_full, wl.cap_full, sess.len_full, 0,

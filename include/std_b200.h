@@ -259,6 +259,30 @@ int std_dense_verify_attn(const std_dims* dims, const void* q, int gamma, const 
                           const void* v_full, const int32_t* len_full, float* o, int splits,
                           void* ws, size_t ws_bytes, std_stream_t stream);
 
+/* ---------------------------------------------------------------- append + attention in one launch
+ *
+ * The decode loop appends the K/V rows of its new inputs and then attends over
+ * them ("Methodik" item 3: each draft step, and the verify pass, see the inputs
+ * appended so far).  These calls do both in one launch: the tensor-core kernel
+ * writes the new rows into the cache (each by the CTA that loads its tile) before
+ * reading them; other paths launch std_kv_append's kernel first.  Results equal
+ * std_kv_append followed by the attention call.  Capacity beyond cap shows as
+ * STD_DEVERR_LENGTH (that sequence skipped).
+ */
+
+/* Draft step: k_new/v_new [L][B][Hkv][1][d] go to sparse row len_sparse[b] +
+ * len_offset - 1, then std_sparse_decode_attn with len_offset (>= 1, it counts the
+ * new row). */
+int std_sparse_decode_attn_append(const std_dims* dims, const void* q, void* k_sparse, void* v_sparse,
+                                  const int32_t* len_sparse, int len_offset, const void* k_new, const void* v_new,
+                                  float* o, int splits, void* ws, size_t ws_bytes, std_stream_t stream);
+
+/* Verify: k_new/v_new [L][B][Hkv][gamma + 1][d] go to full rows [len_full[b],
+ * len_full[b] + gamma + 1), then std_dense_verify_attn. */
+int std_dense_verify_attn_append(const std_dims* dims, const void* q, int gamma, void* k_full, void* v_full,
+                                 const int32_t* len_full, const void* k_new, const void* v_new, float* o, int splits,
+                                 void* ws, size_t ws_bytes, std_stream_t stream);
+
 /* ---------------------------------------------------------------- verify attention, no workspace
  *
  * No counterpart in the paper: this entry point exists for callers, not for the method.
@@ -352,8 +376,9 @@ size_t std_round_workspace_size(const std_dims* dims, int gamma, int splits_draf
 
 /*
  * One draft + verify round ("Methodik" item 3), all on `stream`:
- *   for j < gamma: append draft row j to the sparse cache at len_sparse + j,
- *                  sparse attention over len_sparse + j + 1 rows;
+ *   for j < gamma: append draft row j to the sparse cache at len_sparse + j and
+ *                  attend over len_sparse + j + 1 rows (one launch, as
+ *                  std_sparse_decode_attn_append);
  *   append the gamma + 1 verify rows to the full cache at len_full;
  *   dense verify attention; acceptance; commit (lengths advance by n + 1).
  * The token ids of the LM head are inputs here (the language-model layers

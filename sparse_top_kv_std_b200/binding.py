@@ -75,6 +75,8 @@ SIGNATURES = {
     "std_sparse_decode_attn": (_I, [_DP, _P, _P, _P, _P, _I, _P, _I, _P, _SZ, _P]),
     "std_dense_verify_attn": (_I, [_DP, _P, _I, _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "std_dense_verify_attn_noalloc": (_I, [_DP, _P, _I, _P, _P, _P, _P, _I, _P]),
+    "std_sparse_decode_attn_append": (_I, [_DP, _P, _P, _P, _P, _I, _P, _P, _P, _I, _P, _SZ, _P]),
+    "std_dense_verify_attn_append": (_I, [_DP, _P, _I, _P, _P, _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "std_accept_prefix": (_I, [_I, _I, _P, _P, _P, _P, _P]),
     "std_kv_append": (_I, [_DP, _P, _P, _I64, _P, _I, _P, _P, _I, _P]),
     "std_kv_commit": (_I, [_DP, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
@@ -224,6 +226,20 @@ def std_dense_verify_attn(d: StdDims, q, gamma, k_full, v_full, len_full, o, spl
                           stream=None) -> None:
     _check(lib().std_dense_verify_attn(ctypes.byref(d), _ptr(q), gamma, _ptr(k_full), _ptr(v_full),
                                        _ptr(len_full), _ptr(o), splits, _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def std_sparse_decode_attn_append(d: StdDims, q, k_sparse, v_sparse, len_sparse, len_offset, k_new, v_new, o,
+                                  splits=0, ws=None, stream=None) -> None:
+    _check(lib().std_sparse_decode_attn_append(ctypes.byref(d), _ptr(q), _ptr(k_sparse), _ptr(v_sparse),
+                                               _ptr(len_sparse), len_offset, _ptr(k_new), _ptr(v_new), _ptr(o),
+                                               splits, _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def std_dense_verify_attn_append(d: StdDims, q, gamma, k_full, v_full, len_full, k_new, v_new, o, splits=0,
+                                 ws=None, stream=None) -> None:
+    _check(lib().std_dense_verify_attn_append(ctypes.byref(d), _ptr(q), gamma, _ptr(k_full), _ptr(v_full),
+                                              _ptr(len_full), _ptr(k_new), _ptr(v_new), _ptr(o), splits, _ptr(ws),
+                                              _nbytes(ws), _stream(stream)))
 
 
 STD_NOALLOC_SCRATCH_BYTES = 16 << 20

@@ -169,9 +169,12 @@ int plan_attn(const std_dims* dims, int nq, int64_t cap, int splits, AttnPlan* p
   return STD_OK;
 }
 
+// k_new / v_new (optional): rows to append to the cache at len[b] + new_off + r (r < new_rows)
+// before attending -- inside the tensor-core kernel, else as a separate append launch.
 int run_attn(const std_dims* dims, const void* q, const void* k, const void* v, int64_t cap,
              const int32_t* len, int len_off, int nq, float* o, int splits, void* ws, size_t ws_bytes,
-             cudaStream_t stream) {
+             cudaStream_t stream, const void* k_new = nullptr, const void* v_new = nullptr, int new_rows = 0,
+             int new_off = 0) {
   AttnPlan p;
   STD_TRY(plan_attn(dims, nq, cap, splits, &p));
   if (p.ws_bytes > 0 && (!ws || ws_bytes < p.ws_bytes))
@@ -183,6 +186,16 @@ int run_attn(const std_dims* dims, const void* q, const void* k, const void* v, 
   a.q = q; a.k = k; a.v = v; a.o = o; a.len = len; a.len_off = len_off;
   a.ws = static_cast<float*>(ws); a.err = err;
   a.epoch = g_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
+  if (k_new && new_rows > 0) {
+    if (p.tc) {
+      a.k_new = k_new; a.v_new = v_new; a.new_rows = new_rows; a.new_off = new_off;
+    } else {
+      cudaError_t e = stdb::launch_append(const_cast<void*>(k), const_cast<void*>(v), cap, len, new_off, k_new,
+                                          v_new, new_rows, dims->L, dims->B, dims->Hkv,
+                                          dims->d * elem_bytes(dims->dtype), err, stream);
+      if (e != cudaSuccess) return cuda_fail(e, "append launch");
+    }
+  }
   cudaError_t e = p.tc ? stdb::launch_decode_attn_tc(a, stream) : stdb::launch_decode_attn(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
   return ok();
@@ -393,6 +406,40 @@ int std_accept_prefix(int B, int gamma, const int32_t* draft, const int32_t* den
   return ok();
 }
 
+int std_sparse_decode_attn_append(const std_dims* dims, const void* q, void* k_sparse, void* v_sparse,
+                                  const int32_t* len_sparse, int len_offset, const void* k_new, const void* v_new,
+                                  float* o, int splits, void* ws, size_t ws_bytes, std_stream_t stream) {
+  STD_TRY(check_dims(dims));
+  STD_TRY(check_ptr(q, 16, "q"));
+  STD_TRY(check_ptr(k_sparse, 16, "k_sparse"));
+  STD_TRY(check_ptr(v_sparse, 16, "v_sparse"));
+  STD_TRY(check_ptr(len_sparse, 4, "len_sparse"));
+  STD_TRY(check_ptr(k_new, 16, "k_new"));
+  STD_TRY(check_ptr(v_new, 16, "v_new"));
+  STD_TRY(check_ptr(o, 16, "o"));
+  if (len_offset < 1) return fail(STD_ERR_INVALID_ARG, "len_offset = %d must be >= 1 (it counts the new row)", len_offset);
+  if ((int64_t)len_offset > dims->cap_sparse) return fail(STD_ERR_CAPACITY, "len_offset exceeds cap_sparse");
+  return run_attn(dims, q, k_sparse, v_sparse, dims->cap_sparse, len_sparse, len_offset, 1, o, splits, ws,
+                  ws_bytes, stream, k_new, v_new, 1, len_offset - 1);
+}
+
+int std_dense_verify_attn_append(const std_dims* dims, const void* q, int gamma, void* k_full, void* v_full,
+                                 const int32_t* len_full, const void* k_new, const void* v_new, float* o, int splits,
+                                 void* ws, size_t ws_bytes, std_stream_t stream) {
+  STD_TRY(check_dims(dims));
+  STD_TRY(check_ptr(q, 16, "q"));
+  STD_TRY(check_ptr(k_full, 16, "k_full"));
+  STD_TRY(check_ptr(v_full, 16, "v_full"));
+  STD_TRY(check_ptr(len_full, 4, "len_full"));
+  STD_TRY(check_ptr(k_new, 16, "k_new"));
+  STD_TRY(check_ptr(v_new, 16, "v_new"));
+  STD_TRY(check_ptr(o, 16, "o"));
+  if (gamma < 0 || gamma > 31) return fail(STD_ERR_INVALID_ARG, "gamma = %d must be in [0, 31]", gamma);
+  if ((int64_t)gamma + 1 > dims->cap_full) return fail(STD_ERR_CAPACITY, "gamma + 1 exceeds cap_full");
+  return run_attn(dims, q, k_full, v_full, dims->cap_full, len_full, 1, gamma + 1, o, splits, ws, ws_bytes, stream,
+                  k_new, v_new, gamma + 1, 0);
+}
+
 int std_kv_append(const std_dims* dims, void* k_cache, void* v_cache, int64_t cap, const int32_t* len,
                   int pos_offset, const void* k_new, const void* v_new, int n_new, std_stream_t stream) {
   STD_TRY(check_dims(dims));
@@ -448,18 +495,28 @@ int std_decode_round(const std_dims* dims, int gamma, const std_cache* c, const 
   const size_t eb = elem_bytes(dims->dtype);
   const size_t q_step = (size_t)dims->L * dims->B * dims->Hq * dims->d;   // elements per draft query step
   const size_t kv_step = (size_t)dims->L * dims->B * dims->Hkv * dims->d;  // elements per draft K/V step
+  const void* ptrs[] = {c->k_full, c->v_full, c->k_sparse, c->v_sparse, io->q_draft, io->k_draft, io->v_draft,
+                        io->q_verify, io->k_verify, io->v_verify, io->o_draft, io->o_verify};
+  for (const void* ptr : ptrs)
+    if (gamma > 0 || (ptr != io->q_draft && ptr != io->k_draft && ptr != io->v_draft && ptr != io->o_draft))
+      STD_TRY(check_ptr(ptr, 16, "round buffer"));
+  STD_TRY(check_ptr(c->len_full, 4, "len_full"));
+  STD_TRY(check_ptr(c->len_sparse, 4, "len_sparse"));
+  if (gamma > dims->cap_sparse || gamma + 1 > dims->cap_full) return fail(STD_ERR_CAPACITY, "gamma exceeds a cache");
+  // draft step j: append its input's K/V row at len_sparse + j, attend over len_sparse + j + 1 rows
   for (int j = 0; j < gamma; ++j) {
-    STD_TRY(std_kv_append(dims, c->k_sparse, c->v_sparse, dims->cap_sparse, c->len_sparse, j,
-                          static_cast<const uint8_t*>(io->k_draft) + j * kv_step * eb,
-                          static_cast<const uint8_t*>(io->v_draft) + j * kv_step * eb, 1, stream));
-    STD_TRY(std_sparse_decode_attn(dims, static_cast<const uint8_t*>(io->q_draft) + j * q_step * eb, c->k_sparse,
-                                   c->v_sparse, c->len_sparse, j + 1, io->o_draft + j * q_step, splits_draft, ws,
-                                   ws_bytes, stream));
+    STD_TRY(run_attn(dims, static_cast<const uint8_t*>(io->q_draft) + j * q_step * eb, c->k_sparse, c->v_sparse,
+                     dims->cap_sparse, c->len_sparse, j + 1, 1, io->o_draft + j * q_step, splits_draft, ws, ws_bytes,
+                     stream, static_cast<const uint8_t*>(io->k_draft) + j * kv_step * eb,
+                     static_cast<const uint8_t*>(io->v_draft) + j * kv_step * eb, 1, j));
   }
+  // verify: append the gamma + 1 rows at len_full (a separate launch: fused into the verify
+  // kernel it measured ~1% slower on the long-video step, fused into the draft faster), then
+  // row i attends over len_full + i + 1 rows
   STD_TRY(std_kv_append(dims, c->k_full, c->v_full, dims->cap_full, c->len_full, 0, io->k_verify, io->v_verify,
                         gamma + 1, stream));
-  STD_TRY(std_dense_verify_attn(dims, io->q_verify, gamma, c->k_full, c->v_full, c->len_full, io->o_verify,
-                                splits_verify, ws, ws_bytes, stream));
+  STD_TRY(run_attn(dims, io->q_verify, c->k_full, c->v_full, dims->cap_full, c->len_full, 1, gamma + 1, io->o_verify,
+                   splits_verify, ws, ws_bytes, stream));
   STD_TRY(std_accept_prefix(dims->B, gamma, io->draft_tokens, io->dense_tokens, io->n_plus_1, io->accepted,
                             stream));
   STD_TRY(std_kv_commit(dims, c->k_full, c->v_full, c->k_sparse, c->v_sparse, c->len_full, c->len_sparse,

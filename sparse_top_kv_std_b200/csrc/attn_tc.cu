@@ -56,6 +56,7 @@ struct Ctl {
   uint64_t s_full[2], p_full[2], s_free[2];
   uint64_t o_ready, o_free;
   uint64_t pub, flag;  // partial published by all 128 row threads / merge decision made
+  uint64_t nr_ready;   // fused append: the CTA's new cache rows are written (30 copy lanes)
   uint32_t tmem;
   int abort_flag;
   int consumed;
@@ -65,6 +66,7 @@ struct Ctl {
   int last_flag;
   int tiles_b[kMaxB];
   int pre_b[kMaxB];  // Hkv * (tiles of sequences before b)
+  int len_b[kMaxB];  // len[b], read once at setup
 };
 
 // Arrival on the merge counter of one problem: the counter holds (epoch << 32) |
@@ -225,6 +227,49 @@ __device__ __forceinline__ void merge_problem(float* out, const float* ws, const
   }
 }
 
+// Fused append: the 30 idle lanes (index c = 0..29) of the producer warp copy the new
+// cache rows whose tiles lie in the CTA's slice [g0, g1) of the flat tile sequence.  Row r
+// of problem (l, b, h) goes to position len[b] + new_off + r; the rows are 16-byte chunks,
+// K then V, spread over the lanes.
+template <int D>
+__device__ __forceinline__ void copy_new_rows(const AttnArgs& a, const Ctl* ctl, int g0, int g1, int c) {
+  constexpr int kChunks = D * 2 / 16;  // 16-byte chunks per bf16 row
+  const size_t row_bytes = (size_t)D * 2;
+  Iter it;
+  iter_seek(it, ctl, a, g0, g1);
+  int l = it.l, b = it.b, h = it.h, nt = it.nt;
+  int gp = g0 - it.t;  // flat index of tile 0 of the current problem
+  while (gp < g1 && l < a.L) {
+    const int prob = (l * a.B + b) * a.Hkv + h;
+    const int p0 = ctl->len_b[b] + a.new_off;
+    for (int r = 0; r < a.new_rows; ++r) {
+      const int pos = p0 + r;
+      const int flat = gp + pos / TK;
+      if (flat < g0 || flat >= g1 || pos < 0 || (int64_t)pos >= a.cap) continue;
+      for (int i = c; i < 2 * kChunks; i += 30) {
+        const bool isv = i >= kChunks;
+        const size_t off = (size_t)(i % kChunks) * 16;
+        const uint8_t* src = static_cast<const uint8_t*>(isv ? a.v_new : a.k_new) +
+                             ((size_t)prob * a.new_rows + r) * row_bytes + off;
+        uint8_t* dst = static_cast<uint8_t*>(const_cast<void*>(isv ? a.v : a.k)) +
+                       ((size_t)prob * a.cap + pos) * row_bytes + off;
+        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+      }
+    }
+    gp += nt;
+    if (++h == a.Hkv) {  // next sequence (or layer) with tiles
+      h = 0;
+      do {
+        if (++b == a.B) {
+          b = 0;
+          ++l;
+        }
+        nt = ctl->tiles_b[b];
+      } while (nt == 0 && l < a.L);
+    }
+  }
+}
+
 template <int D>
 struct Cfg {
   static constexpr int KB = D / 64;                   // 128-byte column blocks of a row
@@ -257,6 +302,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     int sum = 0;
     for (int b = 0; b < a.B; ++b) {
       ctl->tiles_b[b] = seq_tiles(a, b, blockIdx.x == 0);
+      ctl->len_b[b] = a.len[b];
       ctl->pre_b[b] = a.Hkv * sum;
       sum += ctl->tiles_b[b];
     }
@@ -279,6 +325,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc::mbar_init(&ctl->o_free, 128);
     tc::mbar_init(&ctl->pub, 128);
     tc::mbar_init(&ctl->flag, 1);
+    tc::mbar_init(&ctl->nr_ready, 30);
     ctl->abort_flag = 0;
     ctl->consumed = 0;
     tc::fence_mbar_init();
@@ -304,9 +351,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       Iter it;
       iter_seek(it, ctl, a, g0, g1);
       int kv = 0;
+      bool rows_ready = a.k_new == nullptr;
       while (it.g < it.g_end) {
         const int prob = (it.l * a.B + it.b) * a.Hkv + it.h;
         const int s = kv % STAGES;
+        if (!rows_ready) {  // fused append: a tile holding new rows waits until they are written
+          const int p0 = ctl->len_b[it.b] + a.new_off;
+          if (it.t * TK < p0 + a.new_rows && p0 < (it.t + 1) * TK) {
+            if (!tc::mbar_wait(&ctl->nr_ready, 0, abort_flag, a.err)) break;
+            rows_ready = true;
+          }
+        }
         if (!tc::mbar_wait(&ctl->kv_empty[s], ((kv / STAGES) & 1) ^ 1, abort_flag, a.err)) break;
         tc::mbar_expect_tx(&ctl->kv_full[s], C::ST_BYTES);
         const int row = prob * (int)a.cap + it.t * TK;
@@ -339,6 +394,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         iter_next(it, ctl, a);
       }
       if (*abort_flag && seg > 0) drain_wait(&ctl->q_full, (seg - 1) & 1);
+    } else if (lane >= 2 && g0 < g1 && a.k_new != nullptr) {
+      // fused append: write the new rows whose tiles fall in this CTA's slice (only this
+      // CTA reads those tiles), then order the writes before the TMA loads of them
+      copy_new_rows<D>(a, ctl, g0, g1, lane - 2);
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      tc::mbar_arrive(&ctl->nr_ready);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer

@@ -43,6 +43,12 @@ struct AttnArgs {
   float* ws;  // partials: [prob][split][rows_pad][d] then [prob][split][rows_pad][2]
   int* err;
   uint32_t epoch;  // per-call tag of the merge counters (tensor-core kernel)
+  // Fused append (tensor-core kernel; k_new == nullptr: none): rows r < new_rows of
+  // k_new / v_new [L][B][Hkv][new_rows][d] are written to cache positions
+  // len[b] + new_off + r before those positions are read.
+  const void* k_new;
+  const void* v_new;
+  int new_rows, new_off;
 };
 
 // Split-K kernels (fp32 operands; bf16 when the tensor-core kernel does not apply):

@@ -523,3 +523,44 @@ def test_topk_keeps_more_attention_mass_than_the_streaming_window():
     print(f"\nmean dense attention mass kept by K = {wl.K} of {nv} visual rows + {wl.T} text rows: "
           f"top-K {m_top:.3f}, sink + window {m_str:.3f}")
     assert m_top > 1.5 * m_str, (m_top, m_str)
+
+
+# ----------------------------------------------------------------------------- append + attention
+
+@pytest.mark.parametrize("name", ["layer_16k", "ragged_g10", "d64_G2_g0", "rows64_d64", "f32_d128_g6"])
+def test_append_then_attend_in_one_launch(name):
+    """std_*_attn_append equal std_kv_append followed by the attention call: the caches
+    byte for byte and the outputs exactly (the same kernel reads the same rows)."""
+    wl = ATTN_CASES[name]
+    x = synth.host_inputs(wl, seed=6)
+    d = B.dims(wl.L, wl.B, wl.Hq, wl.Hkv, wl.d, H.dtype_code(wl), wl.cap_full, wl.cap_full)
+    n_ctx = torch.tensor(np.array(wl.nvis) + wl.T, dtype=torch.int32, device="cuda")
+    g = wl.gamma
+    ws = torch.empty(max(16, B.std_attn_workspace_size(d, g + 1, wl.cap_full, 0)), dtype=torch.uint8, device="cuda")
+    kv_new = H.to_dev(x["k_verify"][0]), H.to_dev(x["v_verify"][0])
+    q_ver = H.to_dev(x["q_verify"][0])
+    outs = []
+    for fused in (False, True):
+        kf, vf = H.to_dev(x["k_full"]), H.to_dev(x["v_full"])
+        o_v = torch.full((wl.L, wl.B, wl.Hq, g + 1, wl.d), float("nan"), device="cuda")
+        o_d = torch.full((wl.L, wl.B, wl.Hq, 1, wl.d), float("nan"), device="cuda")
+        k1, v1 = kv_new[0][:, :, :, :1].contiguous(), kv_new[1][:, :, :, :1].contiguous()
+        q1 = q_ver[:, :, :, :1].contiguous()
+        if fused:
+            B.std_dense_verify_attn_append(d, q_ver, g, kf, vf, n_ctx, kv_new[0], kv_new[1], o_v, 0, ws)
+            # a draft-style step on the cache just extended: one more row at n_ctx + g + 1
+            B.std_sparse_decode_attn_append(d, q1, kf, vf, n_ctx, g + 2, k1, v1, o_d, 0, ws)
+        else:
+            B.std_kv_append(d, kf, vf, wl.cap_full, n_ctx, 0, kv_new[0], kv_new[1], g + 1)
+            B.std_dense_verify_attn(d, q_ver, g, kf, vf, n_ctx, o_v, 0, ws)
+            B.std_kv_append(d, kf, vf, wl.cap_full, n_ctx, g + 1, k1, v1, 1)
+            B.std_sparse_decode_attn(d, q1, kf, vf, n_ctx, g + 2, o_d, 0, ws)
+        torch.cuda.synchronize()
+        assert B.std_get_device_error() == 0
+        outs.append((H.to_host_bits(kf), H.to_host_bits(vf), o_v.cpu().numpy(), o_d.cpu().numpy()))
+    for a, b in zip(outs[0], outs[1]):
+        np.testing.assert_array_equal(a, b)
+    # and against the oracle for the verify rows
+    want = oracle.dense_verify_attn(H.f64(x["q_verify"][0], wl), H.f64(outs[1][0], wl), H.f64(outs[1][1], wl),
+                                    np.array(wl.nvis) + wl.T)
+    assert np.abs(outs[1][2] - want).max() <= H.attn_tol(wl)

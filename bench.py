@@ -403,10 +403,6 @@ def run_std(args, rank, world, local_rank):
     sp_v = B.std_attn_splits(sess.dims, wl.gamma + 1, wl.cap_full, 0)
     ws = sess.ws_round
     q_text = view("q_text")
-    # per attention call: the attention kernel plus its merge kernel (none for a single fp32 split)
-    merge_d = 1 if (dt == B.STD_BF16 or sp_d > 1) else 0
-    merge_v = 1 if (dt == B.STD_BF16 or sp_v > 1) else 0
-    launches_per_step = 4 + R * (wl.gamma * (2 + merge_d) + 2 + merge_v + 1 + 2)
 
     def step(ev=None, draft_ev=False):
         """One StD decode: reset lengths, select, R rounds.  ev: dict of event lists to record
@@ -469,12 +465,14 @@ def run_std(args, rank, world, local_rank):
         pg.barrier()
     torch.cuda.synchronize()
     w0 = time.time()
+    launches0 = B.std_launch_count()  # the library's own count of the kernels it launches
     t0.record(stream)
     for i in range(args.steps):
         step(evs[i])
     t1.record(stream)
     torch.cuda.synchronize()
     w1 = time.time()
+    launches = B.std_launch_count() - launches0
     clocks = clk.stop(window=(w0, w1))
     if pg:
         pg.barrier()
@@ -559,7 +557,7 @@ def run_std(args, rank, world, local_rank):
                      "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                      "peak_source": f"{peak_src} HBM copy bandwidth"},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches,
         "clocks": clocks,
         "e2e": e2e,
         "input_gen_s": t_gen,

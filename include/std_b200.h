@@ -86,6 +86,11 @@ typedef struct std_dims {
 /* Library version as major * 10000 + minor * 100 + patch. */
 int std_version(void);
 
+/* Kernel launches this process has issued through the library so far (all
+ * devices and threads), for accounting: the difference around a region counts
+ * the library's kernels launched in it. */
+unsigned long long std_launch_count(void);
+
 /* Message describing the last error returned on this host thread ("" if none). */
 const char* std_last_error(void);
 

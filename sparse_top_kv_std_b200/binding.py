@@ -62,6 +62,7 @@ class StdRoundIO(ctypes.Structure):
 _DP = ctypes.POINTER(StdDims)
 SIGNATURES = {
     "std_version": (_I, []),
+    "std_launch_count": (ctypes.c_ulonglong, []),
     "std_last_error": (ctypes.c_char_p, []),
     "std_get_device_error": (_I, [ctypes.POINTER(ctypes.c_int32), _I, _P]),
     "std_select_workspace_size": (_SZ, [_DP, _I, _I]),
@@ -155,6 +156,10 @@ def dims(L, B, Hq, Hkv, d, dtype, cap_full, cap_sparse) -> StdDims:
 
 def std_version() -> int:
     return lib().std_version()
+
+
+def std_launch_count() -> int:
+    return int(lib().std_launch_count())
 
 
 def std_last_error() -> str:

@@ -203,7 +203,13 @@ int run_attn(const std_dims* dims, const void* q, const void* k, const void* v, 
 
 }  // namespace
 
+namespace stdb {
+std::atomic<unsigned long long> g_launch_count{0};
+}  // namespace stdb
+
 extern "C" {
+
+unsigned long long std_launch_count(void) { return stdb::g_launch_count.load(std::memory_order_relaxed); }
 
 int std_version(void) { return 10000; }
 

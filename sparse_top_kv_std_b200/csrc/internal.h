@@ -1,6 +1,7 @@
 // Host-side launchers shared between the C ABI layer and the kernel files.
 #pragma once
 
+#include <atomic>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -11,6 +12,9 @@ namespace stdb {
 
 // Launch `kern` on `s` with programmatic stream serialization (the kernel may
 // begin while its predecessor finishes; it waits with griddepcontrol.wait).
+// Kernel launches the library has issued (std_launch_count); launch_pdl counts each.
+extern std::atomic<unsigned long long> g_launch_count;
+
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                        Args&&... args) {
@@ -24,7 +28,9 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  if (e == cudaSuccess) g_launch_count.fetch_add(1, std::memory_order_relaxed);
+  return e;
 }
 
 // One decode-attention launch: query row r of a KV head (r = g * nq + i, g the

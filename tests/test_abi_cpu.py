@@ -112,3 +112,11 @@ def test_host_side_rejections(lib, call, code):
 
 def lib_():
     return B.lib()
+
+
+def test_launch_count_ignores_rejected_calls(lib):
+    n0 = B.std_launch_count()
+    assert n0 >= 0
+    rc = lib_().std_accept_prefix(0, 4, FAKE, FAKE, FAKE, FAKE, None)  # rejected before any launch
+    assert rc == B.STD_ERR_INVALID_ARG
+    assert B.std_launch_count() == n0

@@ -564,3 +564,28 @@ def test_append_then_attend_in_one_launch(name):
     want = oracle.dense_verify_attn(H.f64(x["q_verify"][0], wl), H.f64(outs[1][0], wl), H.f64(outs[1][1], wl),
                                     np.array(wl.nvis) + wl.T)
     assert np.abs(outs[1][2] - want).max() <= H.attn_tol(wl)
+
+
+def test_launch_count_matches_the_calls():
+    """std_launch_count counts the library's kernel launches: 4 for a tensor-core selection
+    (two score passes, top-K, gather), gamma + 5 for a round (gamma fused draft attentions,
+    append + verify, acceptance, two commit kernels)."""
+    wl = synth.workload("layer_16k").replace(rounds=1)
+    x = synth.host_inputs(wl, seed=0)
+    s = H.session_for(wl)
+    s.k_full.copy_(H.to_dev(x["k_full"]))
+    s.v_full.copy_(H.to_dev(x["v_full"]))
+    s.start(x["nvis"])
+    torch.cuda.synchronize()
+    n0 = B.std_launch_count()
+    s.select(H.to_dev(x["q_text"]))
+    n1 = B.std_launch_count()
+    io = {k: H.to_dev(x[k][0]) for k in ("q_draft", "k_draft", "v_draft", "q_verify", "k_verify", "v_verify")}
+    io["draft_tokens"] = torch.from_numpy(x["draft_tokens"][0]).cuda()
+    io["dense_tokens"] = torch.from_numpy(x["dense_tokens"][0]).cuda()
+    io.update(s.round_outputs())
+    s.round(io)
+    n2 = B.std_launch_count()
+    torch.cuda.synchronize()
+    assert B.std_get_device_error() == 0
+    assert (n1 - n0, n2 - n1) == (4, wl.gamma + 5)

@@ -413,6 +413,9 @@ def run_std(args, rank, world, local_rank):
         sess.select(q_text, keep_scores=False)
         if ev is not None:
             ev["sel1"].record(stream)
+        rounds(ev, draft_ev)
+
+    def rounds(ev=None, draft_ev=False):
         for r in range(R):
             o = outs[r]
             for j in range(wl.gamma):  # draft step j: append its input's row, attend (one launch)
@@ -497,9 +500,35 @@ def run_std(args, rank, world, local_rank):
         acc_host = torch.zeros((R, wl.B, wl.gamma + 1), dtype=torch.int32, pin_memory=True)
         acc_dev = torch.zeros((R, wl.B, wl.gamma + 1), dtype=torch.int32, device=dev)
 
+        copy_stream = torch.cuda.Stream(device=dev)
+        layer_ev = [torch.cuda.Event() for _ in range(wl.L)]
+        rest_ev = torch.cuda.Event()
+        d1 = B.dims(1, wl.B, wl.Hq, wl.Hkv, wl.d, dt, wl.cap_full, wl.cap_sparse)
+        kf_h, vf_h = sess.k_full.view(host_t), sess.v_full.view(host_t)
+
         def e2e_step():
-            h2d_inputs()
-            step()
+            # the prompt cache and the text queries arrive layer by layer on a copy stream, and
+            # each layer's selection starts as soon as its rows have landed; the rounds need
+            # every layer, so they wait for the whole copy
+            copy_stream.wait_stream(stream)  # the previous step is done with these buffers
+            with torch.cuda.stream(copy_stream):
+                for l in range(wl.L):
+                    kf_h[l].copy_(pin_k[l], non_blocking=True)
+                    vf_h[l].copy_(pin_v[l], non_blocking=True)
+                    dv["q_text"][l].copy_(pin["q_text"][l], non_blocking=True)
+                    layer_ev[l].record(copy_stream)
+                for n in pin:
+                    if n != "q_text":
+                        dv[n].copy_(pin[n], non_blocking=True)
+                rest_ev.record(copy_stream)
+            sess.len_full.copy_(len0, non_blocking=True)
+            for l in range(wl.L):
+                stream.wait_event(layer_ev[l])
+                B.std_select_topk(d1, q_text[l], wl.T, sess.k_full[l], sess.v_full[l], sess.nvis, wl.nvis_max, wl.K,
+                                  sess.idx[l], sess.k_sparse[l], sess.v_sparse[l], sess.len_sparse, None,
+                                  sess.ws_select)
+            stream.wait_event(rest_ev)
+            rounds()
             for r in range(R):
                 acc_dev[r].copy_(outs[r]["accepted"], non_blocking=True)
             acc_host.copy_(acc_dev, non_blocking=True)
@@ -520,6 +549,7 @@ def run_std(args, rank, world, local_rank):
         d2h = acc_host.numel() * 4
         e2e = {"value": weak_scaling_value(step_attn, args.e2e_steps, world, e_ms), "unit": "GB/s",
                "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps,
+               "pipeline": "prompt cache copied layer by layer on a second stream, each layer selected as it lands",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     if rank != 0:

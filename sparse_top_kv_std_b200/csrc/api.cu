@@ -509,6 +509,18 @@ int std_decode_round(const std_dims* dims, int gamma, const std_cache* c, const 
   STD_TRY(check_ptr(c->len_full, 4, "len_full"));
   STD_TRY(check_ptr(c->len_sparse, 4, "len_sparse"));
   if (gamma > dims->cap_sparse || gamma + 1 > dims->cap_full) return fail(STD_ERR_CAPACITY, "gamma exceeds a cache");
+  {  // both attention plans and the workspace are checked before anything is launched
+    AttnPlan pd, pv;
+    size_t need = 0;
+    if (gamma > 0) {
+      STD_TRY(plan_attn(dims, 1, dims->cap_sparse, splits_draft, &pd));
+      need = pd.ws_bytes;
+    }
+    STD_TRY(plan_attn(dims, gamma + 1, dims->cap_full, splits_verify, &pv));
+    if (pv.ws_bytes > need) need = pv.ws_bytes;
+    if (need > 0 && (!ws || ws_bytes < need))
+      return fail(STD_ERR_WORKSPACE, "round workspace: need %zu bytes, got %zu", need, ws ? ws_bytes : 0);
+  }
   // draft step j: append its input's K/V row at len_sparse + j, attend over len_sparse + j + 1 rows
   for (int j = 0; j < gamma; ++j) {
     STD_TRY(run_attn(dims, static_cast<const uint8_t*>(io->q_draft) + j * q_step * eb, c->k_sparse, c->v_sparse,

@@ -55,7 +55,7 @@ typedef struct CUstream_st* std_stream_t;
 enum std_status {
   STD_OK = 0,
   STD_ERR_INVALID_ARG = -1, /* null pointer, bad size or shape */
-  STD_ERR_UNSUPPORTED = -2, /* dtype / head dim / group shape this build has no kernel for */
+  STD_ERR_UNSUPPORTED = -2, /* dtype / head dim / group shape the library has no kernel for */
   STD_ERR_CAPACITY = -3,    /* a host-checkable size exceeds a cache capacity */
   STD_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed */
   STD_ERR_DEVICE = -5,      /* std_get_device_error found flags set */

@@ -228,6 +228,17 @@ def check_streaming_and_gather(orc, seed: int = 12) -> None:
     np.testing.assert_array_equal(k3[1, 1, 0, 0], kf[1, 1, 0, 3])
     np.testing.assert_array_equal(v3[0, 1, 1, 1], vf[0, 1, 1, 0])
     np.testing.assert_array_equal(k3[0, 1, 1, 2:2 + T], kf[0, 1, 1, 9:9 + T])
+    # with a 2-row prompt prefix before the video: [prefix | named visual rows | text]
+    P = 2
+    kp = rng.standard_normal((L, B, Hkv, P + cap, d))
+    vp = rng.standard_normal((L, B, Hkv, P + cap, d))
+    k4, v4, l4 = orc.gather_sparse(kp, vp, nvis, mine, T, P + 2 + T, P)
+    assert l4.tolist() == [P + 2 + T] * B
+    np.testing.assert_array_equal(k4[1, 0, 1, :P], kp[1, 0, 1, :P])
+    np.testing.assert_array_equal(k4[1, 0, 1, P], kp[1, 0, 1, P + 3])
+    np.testing.assert_array_equal(v4[0, 1, 0, P + 1], vp[0, 1, 0, P + 0])
+    np.testing.assert_array_equal(v4[0, 1, 0, P + 2:P + 2 + T], vp[0, 1, 0, P + 9:P + 9 + T])
+    np.testing.assert_array_equal(k4[1, 0, 0, P + 2:P + 2 + T], kp[1, 0, 0, P + 12:P + 12 + T])
 
 
 def _brute_topk(s, K):

@@ -92,7 +92,60 @@ def _commit_shifted(k_full, v_full, k_sp, v_sp, len_full, len_sp, n_plus_1):
         len_sp[b] += n
 
 
+def _streaming_window_early(nv, K, n_sink):
+    # the recent window ends one position before the last visual row
+    return np.concatenate([np.arange(n_sink), np.arange(nv - (K - n_sink) - 1, nv - 1)]).astype(np.int32)
+
+
+def _gather_prefix_after_selected(k_full, v_full, nvis, idx, T, cap_sparse, n_prefix=0):
+    k_sp, v_sp, lsp = so.gather_sparse(k_full, v_full, nvis, idx, T, cap_sparse, n_prefix)
+    K, P = idx.shape[3], n_prefix
+    for t in (k_sp, v_sp):
+        t[..., :P + K, :] = np.concatenate([t[..., P:P + K, :], t[..., :P, :]], axis=-2)
+    return k_sp, v_sp, lsp
+
+
+def _gather_text_at_nvis_max(k_full, v_full, nvis, idx, T, cap_sparse, n_prefix=0):
+    nmax = np.full_like(np.asarray(nvis), int(np.max(nvis)))
+    k_sp, v_sp, _ = so.gather_sparse(k_full, v_full, nmax, idx, T, cap_sparse, n_prefix)
+    return k_sp, v_sp, np.full(idx.shape[1], n_prefix + idx.shape[3] + T, np.int32)
+
+
+def _select_prefix_in_softmax(q_text, k_full, v_full, nvis, T, K, cap_sparse, causal_text=False, n_prefix=0):
+    # the default score's softmax also covers the prompt prefix keys
+    res = so.select_topk(q_text, k_full, v_full, nvis, T, K, cap_sparse, causal_text, n_prefix)
+    if n_prefix == 0 or causal_text:
+        return res
+    L, B, Hq = q_text.shape[:3]
+    Hkv = k_full.shape[2]
+    G = Hq // Hkv
+    idx, scores = res[0].copy(), res[1].copy()
+    for l in range(L):
+        for b in range(B):
+            nv = int(nvis[b])
+            for h in range(Hkv):
+                s = so.selection_scores(q_text[l, b, h * G:(h + 1) * G], k_full[l, b, h, :n_prefix + nv])[n_prefix:]
+                scores[l, b, h, :nv] = s
+                idx[l, b, h] = so.topk_indices(s, K)
+    k_sp, v_sp, lsp = so.gather_sparse(k_full, v_full, nvis, idx, T, cap_sparse, n_prefix)
+    return idx, scores, k_sp, v_sp, lsp
+
+
+def _sparse_attn_one_row_short(q, k_sp, v_sp, length):
+    return so.sparse_decode_attn(q, k_sp, v_sp, np.asarray(length) - 1)
+
+
+def _verify_sees_next_row(q, k_full, v_full, n_ctx):
+    return so.dense_verify_attn(q, k_full, v_full, np.asarray(n_ctx) + 1)
+
+
 MUTANTS = {
+    "streaming window ends one row early": _mutant(streaming_indices=_streaming_window_early),
+    "gather puts the prefix after the selected rows": _mutant(gather_sparse=_gather_prefix_after_selected),
+    "gather reads text rows at the longest visual length": _mutant(gather_sparse=_gather_text_at_nvis_max),
+    "default score's softmax covers the prefix keys": _mutant(select_topk=_select_prefix_in_softmax),
+    "sparse attention one row short": _mutant(sparse_decode_attn=_sparse_attn_one_row_short),
+    "verify row sees the next row": _mutant(dense_verify_attn=_verify_sees_next_row),
     "attention scale 1/d": _mutant(attend=_attend_scale_1_over_d),
     "selection sum not mean": _mutant(selection_scores=_scores_sum_not_mean),
     "causal text mask off by one": _mutant(selection_scores_causal=_causal_text_off_by_one),

@@ -48,6 +48,8 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-draft-modes", action="store_true",
+                    help="skip the draft launch-mode figures (batched / per layer / per-layer CUDA graph)")
     ap.add_argument("--threads", type=int, default=0, help="host threads for input generation")
     return ap.parse_args(argv)
 
@@ -306,6 +308,55 @@ def run_reference(args, rank, world):
     return 0
 
 
+def draft_launch_modes(B, sess, wl, dt, q, k_new, v_new, o, ws, stream, reps=20):
+    """One sparse draft step (the step's row appended in the same launch) issued three ways,
+    each repeated `reps` times after one untimed pass and timed with CUDA events on `stream`:
+    one layer-batched launch (what a decode round issues), one launch per layer issued from
+    the host, and those per-layer launches captured once in a CUDA graph and replayed.
+    Runs outside the timed region on a sparse cache of K + T rows (the length right after the
+    prefill selection); the repeated appends write the same row each time.  Returns
+    microseconds per draft step for each mode, or {"error": ...} if a mode could not run."""
+    import torch
+    try:
+        d1 = B.dims(1, wl.B, wl.Hq, wl.Hkv, wl.d, dt, wl.cap_full, wl.cap_sparse)
+        sess.len_sparse.fill_(wl.K + wl.T)
+
+        def batched():
+            B.std_sparse_decode_attn_append(sess.dims, q, sess.k_sparse, sess.v_sparse, sess.len_sparse, 1,
+                                            k_new, v_new, o, 0, ws)
+
+        def per_layer():
+            for l in range(wl.L):
+                B.std_sparse_decode_attn_append(d1, q[l], sess.k_sparse[l], sess.v_sparse[l], sess.len_sparse, 1,
+                                                k_new[l], v_new[l], o[l], 0, ws)
+
+        def timed(fn):
+            fn()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return 1e3 * e0.elapsed_time(e1) / reps
+
+        res = {"batched_us": timed(batched), "per_layer_eager_us": timed(per_layer)}
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            per_layer()
+        res["per_layer_graph_us"] = timed(g.replay)
+        del g
+        res["launches_per_step"] = {"batched": 1, "per_layer": wl.L}
+        res["reps"] = reps
+        flags = B.std_get_device_error(clear=True)
+        if flags:
+            res["device_error_flags"] = flags
+        return res
+    except Exception as ex:  # an extra figure: never lose the bench line to it
+        return {"error": f"{type(ex).__name__}: {ex}"}
+
+
 def workload_config(wl, R):
     return {"workload": wl.name, "L": wl.L, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
             "nvis": list(wl.nvis) if wl.B > 1 else wl.nvis[0], "T": wl.T, "K": wl.K, "gamma": wl.gamma,
@@ -557,6 +608,11 @@ def run_std(args, rank, world, local_rank):
             pg.destroy_process_group()
         return 0
 
+    draft_modes = None
+    if not args.no_draft_modes and wl.gamma > 0:
+        draft_modes = draft_launch_modes(B, sess, wl, dt, view("q_draft", 0)[0], view("k_draft", 0)[0],
+                                         view("v_draft", 0)[0], outs[0]["o_draft"][0], ws, stream)
+
     peaks, peak_src = load_peaks()
     value = weak_scaling_value(step_attn, args.steps, world, elapsed_ms)
     v_avg_ms = statistics.mean(v_ms)
@@ -579,7 +635,8 @@ def run_std(args, rank, world, local_rank):
             "sparse_decode_attn": {"timing": "one instrumented step outside the timed region",
                                    "us_per_launch": 1e3 * d_avg_ms, "bytes_per_launch": d_bytes_avg,
                                    "GBps": d_bytes_avg / (d_avg_ms / 1e3) / 1e9,
-                                   "frac_of_8TBps": d_bytes_avg / (d_avg_ms / 1e3) / 8e12, "ctas": sp_d},
+                                   "frac_of_8TBps": d_bytes_avg / (d_avg_ms / 1e3) / 8e12, "ctas": sp_d,
+                                   "launch_modes": draft_modes},
             "select_topk": {"ms_per_launch": sel_avg, "mma_TFLOPs": select_flops(wl) / (sel_avg / 1e3) / 1e12,
                             "one_pass_TFLOPs": 0.5 * select_flops(wl) / (sel_avg / 1e3) / 1e12},
         },

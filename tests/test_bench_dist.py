@@ -98,3 +98,77 @@ def test_clock_summary_keeps_samples_of_the_timed_region():
     s = bench.ClockSampler.summarise(rows, window=(t + 1.5, t + 1.52))
     assert s["samples"] == 2 and s["window"] == "nearest to the timed region"
     assert bench.ClockSampler.summarise([], window=(t, t + 1)) is None
+
+
+def test_draft_launch_modes_issue_per_layer_slices(monkeypatch):
+    """The per-layer draft launches get L = 1 dims and the layer's slices of every operand, the
+    CUDA-graph mode captures exactly those launches, and a failure becomes an "error" entry
+    instead of an exception (CUDA events, graphs and the library replaced by fakes)."""
+    import types
+
+    import torch
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class Ev:
+        def __init__(self, **kw):
+            self.t = 0.0
+
+        def record(self, stream=None):
+            pass
+
+        def elapsed_time(self, other):
+            return 2.0
+
+    class Graph:
+        def __init__(self):
+            self.calls = None
+
+        def replay(self):
+            calls.extend(self.calls)
+
+    class Capture:
+        def __init__(self, g, capture_error_mode=None):
+            self.g = g
+
+        def __enter__(self):
+            self.n0 = len(calls)
+
+        def __exit__(self, *exc):
+            self.g.calls = calls[self.n0:]
+            del calls[self.n0:]
+
+    monkeypatch.setattr(torch.cuda, "Event", Ev)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda: None)
+    monkeypatch.setattr(torch.cuda, "CUDAGraph", Graph)
+    monkeypatch.setattr(torch.cuda, "graph", Capture)
+    calls = []
+    L, Bn, Hq, Hkv, d, K, T = 3, 1, 4, 2, 8, 5, 2
+    fake = types.SimpleNamespace(
+        dims=lambda *a: ("dims",) + a,
+        std_get_device_error=lambda clear=True: 0,
+        std_sparse_decode_attn_append=lambda dims, q, k, v, ln, off, kn, vn, o, sp, ws: calls.append(
+            (dims, q, k, v, ln, off, kn, vn, o)))
+    wl = types.SimpleNamespace(L=L, B=Bn, Hq=Hq, Hkv=Hkv, d=d, K=K, T=T, cap_full=20, cap_sparse=12)
+    sess = types.SimpleNamespace(dims="batched-dims", k_sparse=torch.zeros(L, Bn, Hkv, 12, d),
+                                 v_sparse=torch.ones(L, Bn, Hkv, 12, d), len_sparse=torch.zeros(Bn, dtype=torch.int32))
+    q, kn, vn = torch.randn(L, Bn, Hq, 1, d), torch.randn(L, Bn, Hkv, 1, d), torch.randn(L, Bn, Hkv, 1, d)
+    o = torch.zeros(L, Bn, Hq, 1, d)
+    res = bench.draft_launch_modes(fake, sess, wl, 1, q, kn, vn, o, None, None, reps=2)
+    assert "error" not in res, res
+    assert sess.len_sparse.tolist() == [K + T]
+    # batched: 1 + 2 calls; per-layer eager: (1 + 2) x L; graph: capture L, then 1 + 2 replays of L
+    assert len(calls) == 3 + 3 * L + 3 * L
+    assert res["launches_per_step"] == {"batched": 1, "per_layer": L}
+    assert res["batched_us"] == res["per_layer_eager_us"] == res["per_layer_graph_us"] == 1e3
+    first = calls[0]
+    assert first[0] == "batched-dims" and first[1] is q and first[5] == 1
+    for l, c in enumerate(calls[3:3 + L]):
+        assert c[0][:3] == ("dims", 1, Bn)                  # one layer per launch
+        for got, full in zip((c[1], c[2], c[3], c[6], c[7], c[8]), (q, sess.k_sparse, sess.v_sparse, kn, vn, o)):
+            assert got.data_ptr() == full[l].data_ptr() and got.shape == full.shape[1:]
+    replayed = calls[3 + 3 * L:]
+    assert [c[1].data_ptr() for c in replayed] == [q[l].data_ptr() for l in range(L)] * 3
+    # a failing library call is reported, not raised
+    fake.std_sparse_decode_attn_append = lambda *a: (_ for _ in ()).throw(RuntimeError("boom"))
+    assert bench.draft_launch_modes(fake, sess, wl, 1, q, kn, vn, o, None, None)["error"] == "RuntimeError: boom"

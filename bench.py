@@ -116,6 +116,25 @@ def select_flops(wl):
     return 2 * sum(2 * M * n * wl.d for n in wl.nvis) * wl.L * wl.Hkv
 
 
+def select_exps(wl):
+    """Exponentials of the selection: one per logit in each of the 2 passes."""
+    return 2 * sum(wl.G * wl.T * n for n in wl.nvis) * wl.L * wl.Hkv
+
+
+def select_figures(wl, ms, peaks, peak_src):
+    """Rates of one selection call (scores, top-K, gather) that took `ms`: executed MMA flops
+    (both passes) against the bf16 GEMM peaks, the one-pass algorithmic rate, exponentials/s."""
+    s = ms / 1e3
+    mma = select_flops(wl) / s / 1e12
+    out = {"ms_per_launch": ms, "mma_TFLOPs": mma, "one_pass_TFLOPs": 0.5 * mma,
+           "exp2_G_per_s": select_exps(wl) / s / 1e9}
+    for key, name in (("bf16_tflops", "burst"), ("bf16_tflops_sustained", "sustained")):
+        if key in peaks:
+            out[f"frac_of_{name}_bf16"] = mma / peaks[key]
+    out["peak_source"] = f"{peak_src} cuBLAS bf16 GEMM"
+    return out
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -637,8 +656,7 @@ def run_std(args, rank, world, local_rank):
                                    "GBps": d_bytes_avg / (d_avg_ms / 1e3) / 1e9,
                                    "frac_of_8TBps": d_bytes_avg / (d_avg_ms / 1e3) / 8e12, "ctas": sp_d,
                                    "launch_modes": draft_modes},
-            "select_topk": {"ms_per_launch": sel_avg, "mma_TFLOPs": select_flops(wl) / (sel_avg / 1e3) / 1e12,
-                            "one_pass_TFLOPs": 0.5 * select_flops(wl) / (sel_avg / 1e3) / 1e12},
+            "select_topk": select_figures(wl, sel_avg, peaks, peak_src),
         },
         "roofline": {"kernel": "dense_verify_attn (verify attention + split merge)", "bound": "hbm",
                      "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",

@@ -172,3 +172,20 @@ def test_draft_launch_modes_issue_per_layer_slices(monkeypatch):
     # a failing library call is reported, not raised
     fake.std_sparse_decode_attn_append = lambda *a: (_ for _ in ()).throw(RuntimeError("boom"))
     assert bench.draft_launch_modes(fake, sess, wl, 1, q, kn, vn, o, None, None)["error"] == "RuntimeError: boom"
+
+
+def test_selection_figures_at_the_long_video_sizes():
+    """2 passes x 2 x (7 x 256) x 143,360 x 128 flops x 112 heads = 14.73 TFLOP and 2 x 1,792 x
+    143,360 x 112 exponentials per selection; rates and fractions against the given peaks."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    wl = synth.workload("video_140k")
+    assert bench.select_flops(wl) == 2 * 2 * 1792 * 143360 * 128 * 112
+    assert bench.select_exps(wl) == 2 * 1792 * 143360 * 112
+    f = bench.select_figures(wl, 18.0, {"bf16_tflops": 1647.5, "bf16_tflops_sustained": 1399.2}, "measured")
+    assert abs(f["mma_TFLOPs"] - 14.7307e12 / 0.018 / 1e12) < 0.5
+    assert abs(f["one_pass_TFLOPs"] - 0.5 * f["mma_TFLOPs"]) < 1e-9
+    assert abs(f["frac_of_burst_bf16"] - f["mma_TFLOPs"] / 1647.5) < 1e-12
+    assert abs(f["frac_of_sustained_bf16"] - f["mma_TFLOPs"] / 1399.2) < 1e-12
+    assert abs(f["exp2_G_per_s"] - 2 * 1792 * 143360 * 112 / 0.018 / 1e9) < 1e-6

@@ -402,6 +402,16 @@ int std_decode_round(const std_dims* dims, int gamma, const std_cache* cache,
  * error.  Not a step of the method. */
 int std_probe_exp2(const float* x, float* y_fma, float* y_sfu, int n, std_stream_t stream);
 
+/* Test hook for the failure path of the bounded waits.  Launches one CTA whose
+ * thread 0 waits, through the same bounded mbarrier wait the tensor-core kernels
+ * use, on a barrier that no thread ever arrives on.  The wait gives up after its
+ * limit (0.5 s), sets STD_DEVERR_TIMEOUT in the device error word and the kernel
+ * returns, so the context stays usable.  completed: one device int32, set to 0
+ * when the wait gave up (1 would mean it completed).  Asynchronous on `stream`;
+ * STD_ERR_INVALID_ARG for a NULL or unaligned `completed`.  Not a step of the
+ * method. */
+int std_probe_wait_timeout(int32_t* completed, std_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

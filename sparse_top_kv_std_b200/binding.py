@@ -83,6 +83,7 @@ SIGNATURES = {
     "std_kv_commit": (_I, [_DP, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
     "std_round_workspace_size": (_SZ, [_DP, _I, _I, _I]),
     "std_probe_exp2": (_I, [_P, _P, _P, _I, _P]),
+    "std_probe_wait_timeout": (_I, [_P, _P]),
     "std_decode_round": (_I, [_DP, _I, ctypes.POINTER(StdCache), ctypes.POINTER(StdRoundIO), _I, _I,
                               _P, _SZ, _P]),
 }
@@ -288,3 +289,7 @@ def std_decode_round(d: StdDims, gamma, cache: dict, io: dict, splits_draft=0, s
 
 def std_probe_exp2(x, y_fma, y_sfu, stream=None) -> None:
     _check(lib().std_probe_exp2(_ptr(x), _ptr(y_fma), _ptr(y_sfu), x.numel(), _stream(stream)))
+
+
+def std_probe_wait_timeout(completed, stream=None) -> None:
+    _check(lib().std_probe_wait_timeout(_ptr(completed), _stream(stream)))

@@ -205,6 +205,7 @@ int run_attn(const std_dims* dims, const void* q, const void* k, const void* v, 
 
 namespace stdb {
 std::atomic<unsigned long long> g_launch_count{0};
+cudaError_t launch_probe_wait(int* err, int* completed, cudaStream_t s);  // probe.cu
 }  // namespace stdb
 
 extern "C" {
@@ -214,6 +215,15 @@ unsigned long long std_launch_count(void) { return stdb::g_launch_count.load(std
 int std_version(void) { return 10000; }
 
 const char* std_last_error(void) { return g_last_error.c_str(); }
+
+int std_probe_wait_timeout(int32_t* completed, std_stream_t stream) {
+  STD_TRY(check_ptr(completed, 4, "completed"));
+  int* err;
+  STD_TRY(device_state(&err, nullptr));
+  cudaError_t e = stdb::launch_probe_wait(err, completed, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "wait probe launch");
+  return ok();
+}
 
 int std_get_device_error(int32_t* flags, int clear, std_stream_t stream) {
   int* err;

@@ -104,6 +104,8 @@ FAKE = 1 << 40  # a 16-byte aligned non-null "pointer": never dereferenced, chec
     (lambda: lib_().std_kv_append(ctypes.byref(_dims()), FAKE, FAKE, 100, FAKE, -1, FAKE, FAKE, 2, None), B.STD_ERR_INVALID_ARG),
     (lambda: lib_().std_kv_commit(ctypes.byref(_dims()), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 33, None), B.STD_ERR_INVALID_ARG),
     (lambda: lib_().std_decode_round(ctypes.byref(_dims()), 4, None, None, 0, 0, None, 0, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_probe_wait_timeout(None, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_probe_wait_timeout(FAKE + 2, None), B.STD_ERR_INVALID_ARG),
 ])
 def test_host_side_rejections(lib, call, code):
     assert call() == code

@@ -189,3 +189,21 @@ def test_selection_figures_at_the_long_video_sizes():
     assert abs(f["frac_of_burst_bf16"] - f["mma_TFLOPs"] / 1647.5) < 1e-12
     assert abs(f["frac_of_sustained_bf16"] - f["mma_TFLOPs"] / 1399.2) < 1e-12
     assert abs(f["exp2_G_per_s"] - 2 * 1792 * 143360 * 112 / 0.018 / 1e9) < 1e-6
+
+
+def test_attention_byte_model_at_the_long_video_sizes():
+    """K/V bytes the draft and verify calls read: 2 (K, V) x 128 x 2 B x 28 layers x 4 KV heads
+    = 57,344 B per position.  Round 0's verify reads nvis + T + gamma + 1 = 143,625 positions
+    (8.236 GB); draft step j reads K + T + j + 1; accepted tokens advance both caches."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    wl = synth.workload("video_140k")
+    row = 57344
+    d, v, per = bench.attention_bytes(wl, 1, [[9]])
+    assert v == per[0] == 143625 * row == 8_236_032_000
+    assert d == sum(4096 + 256 + j + 1 for j in range(8)) * row
+    d2, v2, per2 = bench.attention_bytes(wl, 3, [[1], [9], [4]])
+    assert per2 == [143625 * row, (143625 + 1) * row, (143625 + 10) * row]
+    assert v2 == sum(per2)
+    assert d2 == sum((4352 + c + j + 1) * row for c in (0, 1, 10) for j in range(8))

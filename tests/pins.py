@@ -113,6 +113,36 @@ def check_golden_selection(orc) -> None:
         assert idx[0, 0].tolist() == g[key], (idx[0, 0].tolist(), g[key])
 
 
+def check_golden_selection_causal(orc) -> None:
+    """Hand-derived causal full-row and visual-only scores, with and without a prompt prefix
+    (exact rationals; derivation in the fixture)."""
+    g = load_golden("selection_causal.json")
+    q = np.array(g["q_text"])[None, None]                          # [1][1][1][T][d]
+    rows, pre = np.array(g["k_rows"]), np.array(g["k_prefix"])
+    nv, T, P = g["nvis"], q.shape[3], pre.shape[0]
+    cases = ((rows, 0, True, "expected_causal"), (rows, 0, False, "expected_visual_only"),
+             (np.concatenate([pre, rows]), P, True, "expected_causal_prefix"),
+             (np.concatenate([pre, rows]), P, False, "expected_visual_only"))
+    for kr, n_prefix, causal, key in cases:
+        kf = kr[None, None, None]
+        vf = kf + 1.0
+        idx, sc, ksp, vsp, lsp = orc.select_topk(q, kf, vf, np.array([nv]), T, 1, n_prefix + 1 + T,
+                                                 causal_text=causal, n_prefix=n_prefix)
+        np.testing.assert_allclose(sc[0, 0, 0], g[key], atol=g["atol"], rtol=0)
+        assert idx[0, 0, 0].tolist() == g["expected_top1"]
+        # sparse cache: [prefix rows | the selected visual row | text rows]
+        want = np.concatenate([kr[:n_prefix], kr[n_prefix:n_prefix + 1], kr[n_prefix + nv:n_prefix + nv + T]])
+        np.testing.assert_array_equal(ksp[0, 0, 0], want)
+        np.testing.assert_array_equal(vsp[0, 0, 0], want + 1.0)
+        assert lsp.tolist() == [n_prefix + 1 + T]
+    # the score functions themselves, on the same rows
+    qg, kv, kt = q[0, 0], rows[:nv], rows[nv:nv + T]
+    np.testing.assert_allclose(orc.selection_scores_causal(qg, kv, kt), g["expected_causal"], atol=g["atol"], rtol=0)
+    np.testing.assert_allclose(orc.selection_scores_causal(qg, kv, kt, pre), g["expected_causal_prefix"],
+                               atol=g["atol"], rtol=0)
+    np.testing.assert_allclose(orc.selection_scores(qg, kv), g["expected_visual_only"], atol=g["atol"], rtol=0)
+
+
 def check_selection_invariants(orc, seed: int = 5) -> None:
     rng = np.random.default_rng(seed)
     G, T, d, nv = 3, 7, 16, 50
@@ -368,7 +398,8 @@ def check_round_lossless_extremes(orc, seed: int = 10) -> None:
 
 ALL_CHECKS = [
     check_golden_attention, check_golden_verify, check_attention_vs_sdpa,
-    check_attention_closed_forms, check_golden_selection, check_selection_invariants, check_selection_causal,
+    check_attention_closed_forms, check_golden_selection, check_golden_selection_causal,
+    check_selection_invariants, check_selection_causal,
     check_selection_prefix, check_streaming_and_gather,
     check_topk_bruteforce, check_topk_special, check_full_k_sparse_equals_dense,
     check_golden_accept, check_accept_bruteforce, check_commit, check_round_lossless_extremes,

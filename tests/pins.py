@@ -396,8 +396,54 @@ def check_round_lossless_extremes(orc, seed: int = 10) -> None:
         np.testing.assert_array_equal(st["k_full"][:, 1, :, 9:9 + gamma + 1], kvv[:, 1])
 
 
+def check_golden_draft_round(orc) -> None:
+    """A whole 2-draft round with hand-derived rational outputs: each draft step's row lands
+    at len_sparse + j and the step attends over len_sparse + j + 1 rows; the verify, the
+    acceptance and the commit (which overwrites the draft rows) follow (derivation in the
+    fixture)."""
+    g = load_golden("draft_round_2step.json")
+    d = 4
+    st = {"k_sp": np.zeros((1, 1, 1, g["cap_sparse"], d)), "v_sp": np.zeros((1, 1, 1, g["cap_sparse"], d)),
+          "k_full": np.zeros((1, 1, 1, g["cap_full"], d)), "v_full": np.zeros((1, 1, 1, g["cap_full"], d)),
+          "len_sp": np.array([g["len_sparse"]]), "len_full": np.array([g["len_full"]])}
+    st["k_sp"][0, 0, 0, :g["len_sparse"]] = g["k_sparse_rows"]
+    st["v_sp"][0, 0, 0, :g["len_sparse"]] = g["v_sparse_rows"]
+    st["k_full"][0, 0, 0, :g["len_full"]] = g["k_full_rows"]
+    st["v_full"][0, 0, 0, :g["len_full"]] = g["v_full_rows"]
+    gamma = len(g["draft_tokens"])
+    per_step = lambda a: np.array(a).reshape(gamma, 1, 1, 1, 1, d)  # noqa: E731  [gamma][L][B][H][1][d]
+    out = orc.decode_round(st, per_step(g["q_draft"]), per_step(g["k_draft"]), per_step(g["v_draft"]),
+                           np.array(g["q_verify"])[None, None, None], np.array(g["k_verify"])[None, None, None],
+                           np.array(g["v_verify"])[None, None, None], np.array([g["draft_tokens"]]),
+                           np.array([g["dense_tokens"]]))
+    np.testing.assert_allclose(out["o_draft"][:, 0, 0, 0, 0], g["expected_o_draft"], atol=g["atol"], rtol=0)
+    np.testing.assert_allclose(out["o_verify"][0, 0, 0], g["expected_o_verify"], atol=g["atol"], rtol=0)
+    assert out["n_plus_1"].tolist() == [g["expected_n_plus_1"]]
+    assert out["accepted"][0].tolist() == g["expected_accepted"]
+    assert st["len_full"].tolist() == [g["expected_len_full"]]
+    assert st["len_sp"].tolist() == [g["expected_len_sparse"]]
+    n = g["expected_len_sparse"]
+    np.testing.assert_allclose(st["k_sp"][0, 0, 0, :n], g["expected_k_sparse_after"], atol=g["atol"], rtol=0)
+    np.testing.assert_array_equal(st["v_sp"][0, 0, 0, :n], g["expected_v_sparse_after"])
+
+
+def check_append_offsets(orc, seed: int = 14) -> None:
+    """kv_append writes row r of sequence b at length[b] + offset + r and nothing else."""
+    rng = np.random.default_rng(seed)
+    L, B, H, cap, d = 2, 3, 2, 12, 3
+    cache = np.zeros((L, B, H, cap, d))
+    length = np.array([0, 4, 7])
+    rows = rng.standard_normal((L, B, H, 2, d))
+    orc.kv_append(cache, length, 3, rows)
+    for b, start in enumerate((3, 7, 10)):
+        np.testing.assert_array_equal(cache[:, b, :, start:start + 2], rows[:, b])
+        untouched = np.delete(cache[:, b], [start, start + 1], axis=2)
+        assert (untouched == 0).all()
+
+
 ALL_CHECKS = [
-    check_golden_attention, check_golden_verify, check_attention_vs_sdpa,
+    check_golden_attention, check_golden_verify, check_golden_draft_round, check_append_offsets,
+    check_attention_vs_sdpa,
     check_attention_closed_forms, check_golden_selection, check_golden_selection_causal,
     check_selection_invariants, check_selection_causal,
     check_selection_prefix, check_streaming_and_gather,

@@ -139,7 +139,35 @@ def _verify_sees_next_row(q, k_full, v_full, n_ctx):
     return so.dense_verify_attn(q, k_full, v_full, np.asarray(n_ctx) + 1)
 
 
+def _round_with_draft(append_offset, attended):
+    """decode_round with the draft leg changed: step j appends at len_sp + append_offset(j)
+    and attends over len_sp + attended(j) rows; verify, accept and commit unchanged."""
+    def decode_round(state, q_draft, k_draft, v_draft, q_verify, k_verify, v_verify, draft_tokens, dense_tokens):
+        o_draft = []
+        for j in range(q_draft.shape[0]):
+            so.kv_append(state["k_sp"], state["len_sp"], append_offset(j), k_draft[j])
+            so.kv_append(state["v_sp"], state["len_sp"], append_offset(j), v_draft[j])
+            o_draft.append(so.sparse_decode_attn(q_draft[j], state["k_sp"], state["v_sp"],
+                                                 state["len_sp"] + attended(j)))
+        so.kv_append(state["k_full"], state["len_full"], 0, k_verify)
+        so.kv_append(state["v_full"], state["len_full"], 0, v_verify)
+        o_verify = so.dense_verify_attn(q_verify, state["k_full"], state["v_full"], state["len_full"])
+        n_plus_1, acc = so.accept_prefix(draft_tokens, dense_tokens)
+        so.kv_commit(state["k_full"], state["v_full"], state["k_sp"], state["v_sp"], state["len_full"],
+                     state["len_sp"], n_plus_1)
+        return {"o_draft": np.stack(o_draft), "o_verify": o_verify, "n_plus_1": n_plus_1, "accepted": acc}
+    return decode_round
+
+
+def _append_offset_ignored(cache, length, offset, rows):
+    so.kv_append(cache, length, 0, rows)
+
+
 MUTANTS = {
+    "draft appends at offset 0 every step": _mutant(decode_round=_round_with_draft(lambda j: 0, lambda j: j + 1)),
+    "draft step attends len_sp + j rows": _mutant(decode_round=_round_with_draft(lambda j: j, lambda j: j)),
+    "draft step attends one row past its own": _mutant(decode_round=_round_with_draft(lambda j: j, lambda j: j + 2)),
+    "append ignores the offset": _mutant(kv_append=_append_offset_ignored),
     "streaming window ends one row early": _mutant(streaming_indices=_streaming_window_early),
     "gather puts the prefix after the selected rows": _mutant(gather_sparse=_gather_prefix_after_selected),
     "gather reads text rows at the longest visual length": _mutant(gather_sparse=_gather_text_at_nvis_max),

@@ -300,9 +300,14 @@ int std_dense_verify_attn_append(const std_dims* dims, const void* q, int gamma,
  * array compiled into the library: STD_NOALLOC_SCRATCH_BYTES on every GPU on
  * which the library is loaded, held until the process exits.  Arguments,
  * layouts, requirements and results are those of std_dense_verify_attn.
- *  - A call whose partials need more than STD_NOALLOC_SCRATCH_BYTES (see
- *    std_attn_workspace_size; splits = 1 needs none) is rejected with
- *    STD_ERR_WORKSPACE before anything is launched.  It never allocates.
+ *  - A call whose partials need more than STD_NOALLOC_SCRATCH_BYTES is
+ *    rejected with STD_ERR_WORKSPACE before anything is launched.  It never
+ *    allocates.  std_attn_workspace_size(dims, gamma + 1, cap_full, splits)
+ *    gives the bytes a call uses; a call touches the shared array exactly when
+ *    that is non-zero.  On the bf16 tensor-core kernel that is every call,
+ *    splits = 1 included (a persistent CTA may cover parts of two problems
+ *    and the merge counters live there too); only the split-K kernels (fp32
+ *    operands, more than 64 sequences) need none at splits = 1.
  *  - The first call on a device looks up the array's device address with that
  *    device current; make that first call before capturing any stream.
  *  - All calls on a device share the one array and it keeps what the last call

@@ -122,3 +122,16 @@ def test_launch_count_ignores_rejected_calls(lib):
     rc = lib_().std_accept_prefix(0, 4, FAKE, FAKE, FAKE, FAKE, None)  # rejected before any launch
     assert rc == B.STD_ERR_INVALID_ARG
     assert B.std_launch_count() == n0
+
+
+def test_binding_constants_match_the_header():
+    """The Python copies of the header's constants (status codes, dtypes, device error bits,
+    the built-in scratch size of the no-alloc verify) have the header's values."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    values = {n: int(v) for n, v in re.findall(r"\b(STD_[A-Z0-9_]+)\s*=\s*(-?\d+)", src)}
+    shift = re.search(r"#define\s+STD_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", src)
+    assert shift, "STD_NOALLOC_SCRATCH_BYTES must stay of the form (a << b)"
+    values["STD_NOALLOC_SCRATCH_BYTES"] = int(shift.group(1)) << int(shift.group(2))
+    assert len(values) >= 15
+    for name, v in values.items():
+        assert getattr(B, name) == v, (name, getattr(B, name), v)

@@ -383,13 +383,20 @@ def test_decode_rounds_match_oracle(name):
     s.v_full.copy_(H.to_dev(x["v_full"]))
     s.start(x["nvis"])
     s.select(H.to_dev(x["q_text"]))
-    idx_o, _, ksp, vsp, lsp = oracle.select_topk(H.f64(x["q_text"], wl), H.f64(x["k_full"], wl),
-                                                 H.f64(x["v_full"], wl), x["nvis"], wl.T, wl.K, wl.cap_sparse)
-    # heads whose index sets agree (a near-tie at the cut may differ, see test_select_topk_matches_oracle)
-    same = (s.idx.cpu().numpy() == idx_o).all(axis=-1)               # [L][B][Hkv]
-    assert same.mean() >= 0.5
-    q_same = np.repeat(same, wl.G, axis=2)                            # [L][B][Hq]
-    state = {"k_full": H.f64(x["k_full"], wl), "v_full": H.f64(x["v_full"], wl), "k_sp": ksp, "v_sp": vsp,
+    kf64, vf64 = H.f64(x["k_full"], wl), H.f64(x["v_full"], wl)
+    idx_o, sc_o, _, _, _ = oracle.select_topk(H.f64(x["q_text"], wl), kf64, vf64, x["nvis"], wl.T, wl.K,
+                                              wl.cap_sparse)
+    # the GPU's index sets may differ from the oracle's only at near-ties of the cut; once that
+    # is checked, the oracle's sparse cache is gathered from the GPU's own indices so every
+    # head's draft attention is compared
+    idx_g = s.idx.cpu().numpy()
+    for l in range(wl.L):
+        for b in range(wl.B):
+            for h in range(wl.Hkv):
+                nv = wl.nvis[b]
+                H.assert_topk_boundary(idx_g[l, b, h], idx_o[l, b, h], sc_o[l, b, h, :nv], wl.K, H.score_rtol(wl))
+    ksp, vsp, lsp = oracle.gather_sparse(kf64, vf64, x["nvis"], idx_g, wl.T, wl.cap_sparse)
+    state = {"k_full": kf64, "v_full": vf64, "k_sp": ksp, "v_sp": vsp,
              "len_full": np.array(wl.nvis) + wl.T, "len_sp": lsp.astype(np.int64)}
     tol = H.attn_tol(wl)
     for r in range(R):
@@ -406,15 +413,13 @@ def test_decode_rounds_match_oracle(name):
         assert B.std_get_device_error() == 0
         np.testing.assert_array_equal(io["n_plus_1"].cpu().numpy(), want["n_plus_1"])
         np.testing.assert_array_equal(io["accepted"].cpu().numpy(), want["accepted"])
-        dr_err = np.abs(io["o_draft"].cpu().numpy() - want["o_draft"]).max(axis=(-1, -2))  # [g][L][B][Hq]
-        assert dr_err[:, q_same].max(initial=0.0) <= tol
+        assert np.abs(io["o_draft"].cpu().numpy() - want["o_draft"]).max(initial=0.0) <= tol
         assert np.abs(io["o_verify"].cpu().numpy() - want["o_verify"]).max() <= tol
         np.testing.assert_array_equal(s.len_full.cpu().numpy(), state["len_full"])
         np.testing.assert_array_equal(s.len_sparse.cpu().numpy(), state["len_sp"])
     # caches after all rounds: byte-exact
-    ksp_g = H.f64(H.to_host_bits(s.k_sparse), wl)
-    np.testing.assert_array_equal(ksp_g[same], state["k_sp"][same])
-    np.testing.assert_array_equal(ksp_g[..., wl.K:, :], state["k_sp"][..., wl.K:, :])
+    np.testing.assert_array_equal(H.f64(H.to_host_bits(s.k_sparse), wl), state["k_sp"])
+    np.testing.assert_array_equal(H.f64(H.to_host_bits(s.v_sparse), wl), state["v_sp"])
     np.testing.assert_array_equal(H.f64(H.to_host_bits(s.v_full), wl), state["v_full"])
 
 

@@ -58,11 +58,28 @@ def test_noalloc_verify_matches_workspace_verify_twice(splits):
 
 
 def test_noalloc_rejects_more_scratch_than_built_in():
+    """A call whose partials would not fit the built-in array is refused before launch.
+    Every buffer is a real device allocation of the size the dims declare, with valid
+    lengths, so the call would be in bounds even if the size check ever let it through."""
     if not torch.cuda.is_available():
         pytest.skip("needs a GPU")
-    # 28 layers x 4 KV heads, 63 rows padded to 64, 64 splits: 112*64*64*130*4 B > 16 MiB
-    d = B.dims(28, 1, 28, 4, 128, B.STD_BF16, 200000, 5000)
-    fake = 1 << 40                                     # never dereferenced: the size check fails first
-    rc = B.lib().std_dense_verify_attn_noalloc(ctypes.byref(d), fake, 8, fake, fake, fake, fake, 64, None)
+    L, Bn, Hq, Hkv, dh, gamma, cap, splits = 1, 1, 28, 4, 128, 8, 4096, 256
+    d = B.dims(L, Bn, Hq, Hkv, dh, B.STD_BF16, cap, 1024)
+    # the tensor-core plan: (probs + splits * probs) partial slots of 63 rows x (128 + 2)
+    # floats, plus one 8-byte merge counter per problem = 1028 * 63 * 130 * 4 + 4 * 8 bytes
+    need = B.std_attn_workspace_size(d, gamma + 1, cap, splits)
+    assert need == (4 + splits * 4) * 63 * 130 * 4 + 4 * 8
+    assert need > B.STD_NOALLOC_SCRATCH_BYTES
+    q = torch.zeros((L, Bn, Hq, gamma + 1, dh), dtype=torch.bfloat16, device="cuda")
+    kf = torch.zeros((L, Bn, Hkv, cap, dh), dtype=torch.bfloat16, device="cuda")
+    vf = torch.zeros_like(kf)
+    ctx = torch.tensor([1000], dtype=torch.int32, device="cuda")
+    o = torch.full((L, Bn, Hq, gamma + 1, dh), 7.0, device="cuda")
+    n0 = B.std_launch_count()
+    rc = B.lib().std_dense_verify_attn_noalloc(ctypes.byref(d), q.data_ptr(), gamma, kf.data_ptr(), vf.data_ptr(),
+                                               ctx.data_ptr(), o.data_ptr(), splits, None)
+    torch.cuda.synchronize()
     assert rc == B.STD_ERR_WORKSPACE
     assert "scratch" in B.std_last_error()
+    assert B.std_launch_count() == n0                  # nothing was launched
+    assert bool((o == 7.0).all())

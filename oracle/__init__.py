@@ -6,11 +6,14 @@ and the CPU-baseline legs of ``bench.py``; never by the library.
 from .std_oracle import (  # noqa: F401
     accept_prefix,
     attend,
+    attend_partial,
+    attn_range_partial,
     decode_round,
     dense_verify_attn,
     gather_sparse,
     kv_append,
     kv_commit,
+    merge_partials,
     select_topk,
     selection_scores,
     selection_scores_causal,

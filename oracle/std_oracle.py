@@ -241,6 +241,73 @@ def dense_verify_attn(q: np.ndarray, k_full: np.ndarray, v_full: np.ndarray,
     return o
 
 
+# --------------------------------------------------------------------------- attention over key ranges
+
+def attend_partial(q: np.ndarray, k: np.ndarray, v: np.ndarray):
+    """Attention of one query q [d] restricted to the rows k, v [n, d], left unnormalised
+    so that ranges of one key sequence can be combined later (the cache split by position
+    over several devices; the pages keep the whole cache on one GPU, "Bedeutung", so this
+    is the plain decomposition of the softmax, not a step the pages describe).
+
+    With logits s_j = q . k_j / sqrt(d): m = max_j s_j, l = sum_j exp(s_j - m),
+    o = sum_j exp(s_j - m) v_j.  An empty range gives (o = 0, m = -inf, l = 0).
+    Returns (o [d], m, l), fp64; attend(q, k, v) = o / l.
+    """
+    q = np.asarray(q, np.float64)
+    if k.shape[0] == 0:
+        return np.zeros(q.shape[-1]), -math.inf, 0.0
+    s = (np.asarray(k, np.float64) @ q) / math.sqrt(q.shape[-1])
+    m = float(s.max())
+    e = np.exp(s - m)
+    return e @ np.asarray(v, np.float64), m, float(e.sum())
+
+
+def merge_partials(o: np.ndarray, m: np.ndarray, l: np.ndarray) -> np.ndarray:
+    """Combine partials (o_k, m_k, l_k), k over the first axis, of disjoint key ranges:
+    M = max_k m_k, weights w_k = exp(m_k - M), result sum_k w_k o_k / sum_k w_k l_k
+    (0 where no range holds a key).  o [n_parts][..., d], m and l [n_parts][...]."""
+    o = np.asarray(o, np.float64)
+    m = np.asarray(m, np.float64)
+    l = np.asarray(l, np.float64)
+    M = m.max(axis=0)
+    ref = np.where(np.isfinite(M), M, 0.0)
+    w = np.exp(m - ref)                                    # exp(-inf) = 0 for empty ranges
+    L = (w * l).sum(axis=0)
+    O = (w[..., None] * o).sum(axis=0)
+    out = np.zeros(O.shape)
+    nz = L > 0
+    out[nz] = O[nz] / L[nz][..., None]
+    return out
+
+
+def attn_range_partial(q: np.ndarray, k: np.ndarray, v: np.ndarray, limit: np.ndarray, pos0: int,
+                       row_begin: int, row_end: int):
+    """Partials of decode attention over one range of cache rows [P-M2], [P-M3].
+
+    q [L][B][Hq][rows][d]; k, v [L][B][Hkv][cap][d] whose row r holds sequence position
+    pos0 + r; limit [B]: query row i of sequence b attends positions j < limit[b] + i
+    (limit = n_ctx + 1 for the dense verify, the sparse length for the draft).  Row i
+    attends cache rows r in [row_begin, row_end) with pos0 + r < limit[b] + i.
+    Returns (o [L][B][Hq][rows][d], m [L][B][Hq][rows], l [L][B][Hq][rows]) as attend_partial.
+    """
+    L, B, Hq, rows, d = q.shape
+    G = Hq // k.shape[2]
+    o = np.zeros(q.shape, np.float64)
+    m = np.full(q.shape[:4], -math.inf)
+    l = np.zeros(q.shape[:4])
+    for li in range(L):
+        for b in range(B):
+            for hq in range(Hq):
+                h = hq // G
+                for i in range(rows):
+                    hi = min(row_end, int(limit[b]) + i - pos0)
+                    lo = row_begin
+                    kk = k[li, b, h, lo:max(lo, hi)]
+                    vv = v[li, b, h, lo:max(lo, hi)]
+                    o[li, b, hq, i], m[li, b, hq, i], l[li, b, hq, i] = attend_partial(q[li, b, hq, i], kk, vv)
+    return o, m, l
+
+
 # --------------------------------------------------------------------------- acceptance [P-M3]
 
 def accept_prefix(draft: np.ndarray, dense: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:

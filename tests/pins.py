@@ -441,6 +441,72 @@ def check_append_offsets(orc, seed: int = 14) -> None:
         assert (untouched == 0).all()
 
 
+# ----------------------------------------------------------------------------- attention over key ranges
+
+def check_golden_partials(orc) -> None:
+    """Hand-derived partials of three key ranges (one empty) and their merge (fixture)."""
+    g = load_golden("attention_partials_3key.json")
+    q, k, v = np.array(g["q"]), np.array(g["k"]), np.array(g["v"])
+    parts = [orc.attend_partial(q, k[a:b], v[a:b]) for a, b in g["ranges"]]
+    for (o, m, l), eo, em, el in zip(parts, g["expected_o"], g["expected_m"], g["expected_l"]):
+        np.testing.assert_allclose(o, eo, atol=g["atol"], rtol=0)
+        assert (m == -math.inf) if em == "-inf" else abs(m - em) <= g["atol"], (m, em)
+        assert abs(l - el) <= g["atol"], (l, el)
+    merged = orc.merge_partials(np.array([p[0] for p in parts]), np.array([p[1] for p in parts]),
+                                np.array([p[2] for p in parts]))
+    np.testing.assert_allclose(merged, g["expected_merged"], atol=g["atol"], rtol=0)
+
+
+def check_range_partials_vs_torch(orc, seed: int = 15) -> None:
+    """attn_range_partial against torch (float64): m is the max of the masked logits, l is
+    exp(logsumexp - m), o / l is SDPA over the range with the causal limit; and merging the
+    partials of any split of the rows into ranges gives dense verify attention."""
+    import torch
+    rng = np.random.default_rng(seed)
+    L, B, Hq, Hkv, d, rows = 2, 2, 4, 2, 8, 3
+    G = Hq // Hkv
+    n_ctx = np.array([13, 6])
+    cap = 20
+    k = rng.standard_normal((L, B, Hkv, cap, d)) * 2
+    v = rng.standard_normal((L, B, Hkv, cap, d))
+    q = rng.standard_normal((L, B, Hq, rows, d)) * 2
+    limit = n_ctx + 1
+    for (r0, r1) in ((0, 20), (4, 11), (7, 7), (9, 16)):
+        o, m, l = orc.attn_range_partial(q, k, v, limit, 0, r0, r1)
+        for li in range(L):
+            for b in range(B):
+                for hq in range(Hq):
+                    kk = torch.from_numpy(k[li, b, hq // G])
+                    logits = torch.from_numpy(q[li, b, hq]) @ kk.T / math.sqrt(d)       # [rows][cap]
+                    j = torch.arange(cap)[None, :]
+                    i = torch.arange(rows)[:, None]
+                    ok = (j >= r0) & (j < r1) & (j < int(limit[b]) + i)
+                    for r in range(rows):
+                        if not bool(ok[r].any()):
+                            assert m[li, b, hq, r] == -math.inf and l[li, b, hq, r] == 0
+                            assert not o[li, b, hq, r].any()
+                            continue
+                        lg = logits[r][ok[r]]
+                        mm = float(lg.max())
+                        assert abs(m[li, b, hq, r] - mm) < 1e-12
+                        assert abs(l[li, b, hq, r] - math.exp(float(torch.logsumexp(lg, 0)) - mm)) < 1e-12
+                        ref = torch.nn.functional.scaled_dot_product_attention(
+                            torch.from_numpy(q[li, b, hq, r])[None], kk, torch.from_numpy(v[li, b, hq // G]),
+                            attn_mask=ok[r][None])
+                        np.testing.assert_allclose(o[li, b, hq, r] / l[li, b, hq, r], ref[0].numpy(), atol=1e-12)
+    dense = orc.dense_verify_attn(q, k, v, n_ctx)
+    for cuts in ((0, 20), (0, 5, 20), (0, 3, 8, 14, 20), (0, 0, 19, 20)):
+        parts = [orc.attn_range_partial(q, k, v, limit, 0, a, b) for a, b in zip(cuts[:-1], cuts[1:])]
+        merged = orc.merge_partials(*(np.array([p[t] for p in parts]) for t in range(3)))
+        np.testing.assert_allclose(merged, dense, atol=1e-12, rtol=0)
+    # a shard that stores positions [pos0, pos0 + n): the same partials as rows [pos0, pos0 + n)
+    o1, m1, l1 = orc.attn_range_partial(q, k[:, :, :, 5:], v[:, :, :, 5:], limit, 5, 0, 10)
+    o2, m2, l2 = orc.attn_range_partial(q, k, v, limit, 0, 5, 15)
+    np.testing.assert_allclose(o1, o2, atol=1e-14)
+    np.testing.assert_array_equal(m1, m2)
+    np.testing.assert_allclose(l1, l2, atol=1e-14)
+
+
 ALL_CHECKS = [
     check_golden_attention, check_golden_verify, check_golden_draft_round, check_append_offsets,
     check_attention_vs_sdpa,
@@ -449,4 +515,5 @@ ALL_CHECKS = [
     check_selection_prefix, check_streaming_and_gather,
     check_topk_bruteforce, check_topk_special, check_full_k_sparse_equals_dense,
     check_golden_accept, check_accept_bruteforce, check_commit, check_round_lossless_extremes,
+    check_golden_partials, check_range_partials_vs_torch,
 ]

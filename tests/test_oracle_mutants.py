@@ -163,7 +163,30 @@ def _append_offset_ignored(cache, length, offset, rows):
     so.kv_append(cache, length, 0, rows)
 
 
+def _merge_without_rescale(o, m, l):
+    o, l = np.asarray(o, np.float64), np.asarray(l, np.float64)
+    L = l.sum(axis=0)
+    return np.where(L[..., None] > 0, o.sum(axis=0) / np.where(L > 0, L, 1.0)[..., None], 0.0)
+
+
+def _partial_normalised(q, k, v):
+    o, m, l = so.attend_partial(q, k, v)
+    return (o / l if l > 0 else o), m, l
+
+
+def _range_end_inclusive(q, k, v, limit, pos0, row_begin, row_end):
+    return so.attn_range_partial(q, k, v, limit, pos0, row_begin, row_end + 1)
+
+
+def _range_ignores_pos0(q, k, v, limit, pos0, row_begin, row_end):
+    return so.attn_range_partial(q, k, v, limit, 0, row_begin, row_end)
+
+
 MUTANTS = {
+    "merge without the exp(m_k - M) rescale": _mutant(merge_partials=_merge_without_rescale),
+    "partial returns the normalised output": _mutant(attend_partial=_partial_normalised),
+    "key range end inclusive": _mutant(attn_range_partial=_range_end_inclusive),
+    "key range ignores the shard's first position": _mutant(attn_range_partial=_range_ignores_pos0),
     "draft appends at offset 0 every step": _mutant(decode_round=_round_with_draft(lambda j: 0, lambda j: j + 1)),
     "draft step attends len_sp + j rows": _mutant(decode_round=_round_with_draft(lambda j: j, lambda j: j)),
     "draft step attends one row past its own": _mutant(decode_round=_round_with_draft(lambda j: j, lambda j: j + 2)),

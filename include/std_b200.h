@@ -71,7 +71,9 @@ enum std_device_error {
   STD_DEVERR_LENGTH = 2,    /* a device length was <= 0 or beyond the capacity in attention */
   STD_DEVERR_K_RANGE = 4,   /* select: K > nvis[b], or nvis[b] + T > cap_full */
   STD_DEVERR_NVIS_MAX = 8,  /* select: nvis[b] > the host-side nvis_max bound */
-  STD_DEVERR_TIMEOUT = 16   /* a bounded wait inside a kernel gave up; that CTA's output is missing */
+  STD_DEVERR_TIMEOUT = 16,  /* a bounded wait inside a kernel gave up; that CTA's output is missing */
+  STD_DEVERR_DEBUG = 32     /* debug build only (libstd_b200_debug.so, compiled with STD_DEBUG): an index
+                               or cache row outside its buffer was caught and that access skipped */
 };
 
 /* Shape of the model slice a call works on.  cap_full / cap_sparse are the row
@@ -282,11 +284,71 @@ int std_sparse_decode_attn_append(const std_dims* dims, const void* q, void* k_s
                                   const int32_t* len_sparse, int len_offset, const void* k_new, const void* v_new,
                                   float* o, int splits, void* ws, size_t ws_bytes, std_stream_t stream);
 
+/* std_sparse_decode_attn_append with `flags`, bits that let the launch start reading
+ * before the kernel just before it in the stream has finished (programmatic dependent
+ * launch; the call still orders every write after that kernel):
+ *   STD_ATTN_EARLY_KV  the previous kernel is one of this library's, launched after every
+ *                      earlier write to this call's buffers, and writes neither len_sparse
+ *                      nor any K/V row below len_sparse[b] + len_offset - 2 (true when it is
+ *                      the previous draft step on the same cache, or attention on other
+ *                      caches); the K/V tiles below that row are fetched early.
+ *   STD_ATTN_EARLY_Q   with STD_ATTN_EARLY_KV: it does not write q either (q is fetched early).
+ * A wrong promise gives wrong results.  The bf16 tensor-core kernel uses the flags; other
+ * paths ignore them.  std_decode_round passes both for its draft steps after the first. */
+#define STD_ATTN_EARLY_KV 1
+#define STD_ATTN_EARLY_Q 2
+int std_sparse_decode_attn_append_ex(const std_dims* dims, const void* q, void* k_sparse, void* v_sparse,
+                                     const int32_t* len_sparse, int len_offset, const void* k_new,
+                                     const void* v_new, float* o, int splits, int flags, void* ws, size_t ws_bytes,
+                                     std_stream_t stream);
+
 /* Verify: k_new/v_new [L][B][Hkv][gamma + 1][d] go to full rows [len_full[b],
  * len_full[b] + gamma + 1), then std_dense_verify_attn. */
 int std_dense_verify_attn_append(const std_dims* dims, const void* q, int gamma, void* k_full, void* v_full,
                                  const int32_t* len_full, const void* k_new, const void* v_new, float* o, int splits,
                                  void* ws, size_t ws_bytes, std_stream_t stream);
+
+/* ---------------------------------------------------------------- attention over a key range
+ *
+ * The summary keeps every KV cache in one GPU's HBM ("Bedeutung"); when a cache
+ * is split by position over several GPUs, each attends its own rows and one
+ * exchange of per-row partials combines them.  These calls are the decode
+ * attention calls above restricted to the cache rows [row_begin, row_end) of
+ * the given buffers, whose row r holds sequence position pos0 + r (pos0 = 0: the
+ * buffers are the whole cache).  Query row i of a sequence attends the positions
+ * j it attends in the full call (j < len_full[b] + 1 + i for the verify,
+ * j < len_sparse[b] + len_offset for the draft) that lie in that row range.
+ * Instead of the normalised output they write, per query row,
+ *     o_part = sum_j exp(s_j - m) v_j       (s_j = q . k_j / sqrt(d))
+ *     ml_part = (m, l),  l = sum_j exp(s_j - m)
+ * where m is a reference value the kernel chose near the row's largest logit
+ * (not necessarily equal to it): o_part / l and m + ln l are the determined
+ * quantities.  A row that attends no key gets o_part = 0, m = -inf, l = 0.
+ * std_merge_partials combines the partials of disjoint ranges into the full
+ * result.  bf16 tensor-core shapes only (STD_ERR_UNSUPPORTED otherwise); the
+ * workspace is that of the full call (std_attn_workspace_size with the same
+ * cap and splits).  Lengths outside the range are not errors here (a range may
+ * hold no attended row).
+ * o_part  float [L][B][Hq][q_rows][d];  ml_part float [L][B][Hq][q_rows][2]
+ * Requires 0 <= row_begin <= row_end <= cap and 0 <= pos0 <= 2^30.
+ */
+int std_dense_verify_attn_partial(const std_dims* dims, const void* q, int gamma, const void* k_full,
+                                  const void* v_full, const int32_t* len_full, int64_t pos0, int64_t row_begin,
+                                  int64_t row_end, float* o_part, float* ml_part, int splits, void* ws,
+                                  size_t ws_bytes, std_stream_t stream);
+
+int std_sparse_decode_attn_partial(const std_dims* dims, const void* q, const void* k_sparse, const void* v_sparse,
+                                   const int32_t* len_sparse, int len_offset, int64_t pos0, int64_t row_begin,
+                                   int64_t row_end, float* o_part, float* ml_part, int splits, void* ws,
+                                   size_t ws_bytes, std_stream_t stream);
+
+/* Merge n_parts partials of the same query rows over disjoint key ranges:
+ *     M = max_k m_k,  w_k = exp(m_k - M),  o = sum_k w_k o_part_k / sum_k w_k l_k
+ * (o = 0 for a row no range attends).  o_parts [n_parts][rows][d] and ml_parts
+ * [n_parts][rows][2] (the layout an all-gather of the per-GPU partials gives),
+ * o [rows][d], all device float; d a multiple of 4.  rows = 0 does nothing. */
+int std_merge_partials(int64_t rows, int d, int n_parts, const float* o_parts, const float* ml_parts, float* o,
+                       std_stream_t stream);
 
 /* ---------------------------------------------------------------- verify attention, no workspace
  *

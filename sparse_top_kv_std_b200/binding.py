@@ -15,7 +15,9 @@ import threading
 from typing import Optional
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libstd_b200.so")
+# STD_B200_DEBUG=1 loads the debug build: the same kernels compiled with device-side
+# bounds checks of every index and cache row (STD_DEVERR_DEBUG), for tests and bug hunts.
+LIB_PATH = os.path.join(PKG, "libstd_b200_debug.so" if os.environ.get("STD_B200_DEBUG") == "1" else "libstd_b200.so")
 
 STD_OK = 0
 STD_ERR_INVALID_ARG = -1
@@ -34,6 +36,7 @@ STD_DEVERR_LENGTH = 2
 STD_DEVERR_K_RANGE = 4
 STD_DEVERR_NVIS_MAX = 8
 STD_DEVERR_TIMEOUT = 16
+STD_DEVERR_DEBUG = 32
 
 # every function the header declares, with (restype, argtypes)
 _P = ctypes.c_void_p
@@ -76,7 +79,11 @@ SIGNATURES = {
     "std_sparse_decode_attn": (_I, [_DP, _P, _P, _P, _P, _I, _P, _I, _P, _SZ, _P]),
     "std_dense_verify_attn": (_I, [_DP, _P, _I, _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "std_dense_verify_attn_noalloc": (_I, [_DP, _P, _I, _P, _P, _P, _P, _I, _P]),
+    "std_dense_verify_attn_partial": (_I, [_DP, _P, _I, _P, _P, _P, _I64, _I64, _I64, _P, _P, _I, _P, _SZ, _P]),
+    "std_sparse_decode_attn_partial": (_I, [_DP, _P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _P, _I, _P, _SZ, _P]),
+    "std_merge_partials": (_I, [_I64, _I, _I, _P, _P, _P, _P]),
     "std_sparse_decode_attn_append": (_I, [_DP, _P, _P, _P, _P, _I, _P, _P, _P, _I, _P, _SZ, _P]),
+    "std_sparse_decode_attn_append_ex": (_I, [_DP, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _P, _SZ, _P]),
     "std_dense_verify_attn_append": (_I, [_DP, _P, _I, _P, _P, _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "std_accept_prefix": (_I, [_I, _I, _P, _P, _P, _P, _P]),
     "std_kv_append": (_I, [_DP, _P, _P, _I64, _P, _I, _P, _P, _I, _P]),
@@ -241,11 +248,40 @@ def std_sparse_decode_attn_append(d: StdDims, q, k_sparse, v_sparse, len_sparse,
                                                splits, _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
+STD_ATTN_EARLY_KV = 1
+STD_ATTN_EARLY_Q = 2
+
+
+def std_sparse_decode_attn_append_ex(d: StdDims, q, k_sparse, v_sparse, len_sparse, len_offset, k_new, v_new, o,
+                                     splits=0, flags=0, ws=None, stream=None) -> None:
+    _check(lib().std_sparse_decode_attn_append_ex(ctypes.byref(d), _ptr(q), _ptr(k_sparse), _ptr(v_sparse),
+                                                  _ptr(len_sparse), len_offset, _ptr(k_new), _ptr(v_new), _ptr(o),
+                                                  splits, flags, _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
 def std_dense_verify_attn_append(d: StdDims, q, gamma, k_full, v_full, len_full, k_new, v_new, o, splits=0,
                                  ws=None, stream=None) -> None:
     _check(lib().std_dense_verify_attn_append(ctypes.byref(d), _ptr(q), gamma, _ptr(k_full), _ptr(v_full),
                                               _ptr(len_full), _ptr(k_new), _ptr(v_new), _ptr(o), splits, _ptr(ws),
                                               _nbytes(ws), _stream(stream)))
+
+
+def std_dense_verify_attn_partial(d: StdDims, q, gamma, k_full, v_full, len_full, pos0, row_begin, row_end, o_part,
+                                  ml_part, splits=0, ws=None, stream=None) -> None:
+    _check(lib().std_dense_verify_attn_partial(ctypes.byref(d), _ptr(q), gamma, _ptr(k_full), _ptr(v_full),
+                                               _ptr(len_full), pos0, row_begin, row_end, _ptr(o_part), _ptr(ml_part),
+                                               splits, _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def std_sparse_decode_attn_partial(d: StdDims, q, k_sparse, v_sparse, len_sparse, len_offset, pos0, row_begin,
+                                   row_end, o_part, ml_part, splits=0, ws=None, stream=None) -> None:
+    _check(lib().std_sparse_decode_attn_partial(ctypes.byref(d), _ptr(q), _ptr(k_sparse), _ptr(v_sparse),
+                                                _ptr(len_sparse), len_offset, pos0, row_begin, row_end, _ptr(o_part),
+                                                _ptr(ml_part), splits, _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def std_merge_partials(rows, d, n_parts, o_parts, ml_parts, o, stream=None) -> None:
+    _check(lib().std_merge_partials(rows, d, n_parts, _ptr(o_parts), _ptr(ml_parts), _ptr(o), _stream(stream)))
 
 
 STD_NOALLOC_SCRATCH_BYTES = 16 << 20

@@ -9,10 +9,22 @@
 #include <mutex>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/std_b200.h"
 #include "internal.h"
 
 namespace {
+
+// An NVTX range around each entry point that launches work, named after it, so that a
+// profiler timeline shows the library's calls (free when no tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define STD_NVTX_RANGE() NvtxRange nvtx_range_(__func__)
 
 thread_local std::string g_last_error;
 std::atomic<uint32_t> g_epoch{0};  // tags the in-kernel merge counters of each attention call
@@ -133,6 +145,7 @@ int plan_attn(const std_dims* dims, int nq, int64_t cap, int splits, AttnPlan* p
   a = stdb::AttnArgs{};
   a.L = dims->L; a.B = dims->B; a.Hq = dims->Hq; a.Hkv = dims->Hkv; a.G = G; a.nq = nq; a.rows = G * nq;
   a.d = dims->d; a.dtype = dims->dtype; a.cap = cap;
+  a.row_begin = 0; a.row_end = (int)cap;
   if (dims->dtype == STD_BF16 && a.rows > 128)
     return fail(STD_ERR_UNSUPPORTED, "G * query rows = %d exceeds 128", a.rows);
   const int probs = probs_of(dims);
@@ -169,14 +182,23 @@ int plan_attn(const std_dims* dims, int nq, int64_t cap, int splits, AttnPlan* p
   return STD_OK;
 }
 
+// Partials over a key range instead of the normalised output (tensor-core kernel only).
+struct RangeOpt {
+  int row_begin, row_end;
+  float* ml;
+};
+
 // k_new / v_new (optional): rows to append to the cache at len[b] + new_off + r (r < new_rows)
 // before attending -- inside the tensor-core kernel, else as a separate append launch.
 int run_attn(const std_dims* dims, const void* q, const void* k, const void* v, int64_t cap,
              const int32_t* len, int len_off, int nq, float* o, int splits, void* ws, size_t ws_bytes,
              cudaStream_t stream, const void* k_new = nullptr, const void* v_new = nullptr, int new_rows = 0,
-             int new_off = 0) {
+             int new_off = 0, int early = 0, const RangeOpt* range = nullptr) {
   AttnPlan p;
   STD_TRY(plan_attn(dims, nq, cap, splits, &p));
+  if (range && !p.tc)
+    return fail(STD_ERR_UNSUPPORTED, "key-range partials need the bf16 tensor-core kernel (d 64 or 128, "
+                "G * query rows <= 128, at most 64 sequences)");
   if (p.ws_bytes > 0 && (!ws || ws_bytes < p.ws_bytes))
     return fail(STD_ERR_WORKSPACE, "attention workspace: need %zu bytes, got %zu", p.ws_bytes, ws ? ws_bytes : 0);
   if (p.ws_bytes > 0) STD_TRY(check_ptr(ws, 16, "ws"));
@@ -186,6 +208,13 @@ int run_attn(const std_dims* dims, const void* q, const void* k, const void* v, 
   a.q = q; a.k = k; a.v = v; a.o = o; a.len = len; a.len_off = len_off;
   a.ws = static_cast<float*>(ws); a.err = err;
   a.epoch = g_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
+  a.early = p.tc ? early : 0;
+  if (range) {
+    a.row_begin = range->row_begin;
+    a.row_end = range->row_end;
+    a.partial = 1;
+    a.ml = range->ml;
+  }
   if (k_new && new_rows > 0) {
     if (p.tc) {
       a.k_new = k_new; a.v_new = v_new; a.new_rows = new_rows; a.new_off = new_off;
@@ -217,6 +246,7 @@ int std_version(void) { return 10000; }
 const char* std_last_error(void) { return g_last_error.c_str(); }
 
 int std_probe_wait_timeout(int32_t* completed, std_stream_t stream) {
+  STD_NVTX_RANGE();
   STD_TRY(check_ptr(completed, 4, "completed"));
   int* err;
   STD_TRY(device_state(&err, nullptr));
@@ -226,6 +256,7 @@ int std_probe_wait_timeout(int32_t* completed, std_stream_t stream) {
 }
 
 int std_get_device_error(int32_t* flags, int clear, std_stream_t stream) {
+  STD_NVTX_RANGE();
   int* err;
   STD_TRY(device_state(&err, nullptr));
   int32_t host = 0;
@@ -242,7 +273,8 @@ size_t std_select_workspace_size(const std_dims* dims, int T, int nvis_max) {
   if (check_dims(dims) || T < 1 || nvis_max < 1) return 0;
   const size_t probs = probs_of(dims);
   const size_t M = (size_t)(dims->Hq / dims->Hkv) * T;
-  return (probs * M * 2 + probs * (size_t)nvis_max) * sizeof(float) + 256;
+  // row max and sum [probs][M] each, scores [probs][nvis_max], top-digit histograms [probs][256]
+  return (probs * M * 2 + probs * (size_t)nvis_max + probs * 256) * sizeof(float) + 256;
 }
 
 int std_select_topk(const std_dims* dims, const void* q_text, int T, const void* k_full,
@@ -257,6 +289,7 @@ int std_select_topk_ex(const std_dims* dims, const void* q_text, int T, const vo
                        const void* v_full, const int32_t* nvis, int nvis_max, int K, int n_prefix,
                        int flags, int32_t* idx_out, void* k_sparse, void* v_sparse, int32_t* len_sparse,
                        float* scores_out, void* ws, size_t ws_bytes, std_stream_t stream) {
+  STD_NVTX_RANGE();
   STD_TRY(check_dims(dims));
   if (flags & ~STD_SELECT_CAUSAL_TEXT) return fail(STD_ERR_INVALID_ARG, "unknown selection flags %#x", flags);
   if (n_prefix < 0) return fail(STD_ERR_INVALID_ARG, "n_prefix = %d must be >= 0", n_prefix);
@@ -290,6 +323,7 @@ int std_select_topk_ex(const std_dims* dims, const void* q_text, int T, const vo
   float* row_m = static_cast<float*>(ws);
   float* row_l = row_m + probs * M;
   float* scores = scores_out ? scores_out : row_l + probs * M;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(row_l + probs * M + (size_t)probs * nvis_max);
 
   stdb::ScoreArgs s{};
   s.q_text = q_text; s.k_full = k_full; s.nvis = nvis; s.nvis_max = nvis_max;
@@ -297,9 +331,12 @@ int std_select_topk_ex(const std_dims* dims, const void* q_text, int T, const vo
   s.dtype = dims->dtype; s.cap = dims->cap_full; s.row_m = row_m; s.row_l = row_l; s.scores = scores; s.err = err;
   s.causal_text = (flags & STD_SELECT_CAUSAL_TEXT) ? 1 : 0;
   s.prefix = n_prefix;
-  cudaError_t e = stdb::launch_select_scores(s, stream);
+  s.hist = hist;
+  bool hist_done = false;
+  cudaError_t e = stdb::launch_select_scores(s, stream, &hist_done);
   if (e != cudaSuccess) return cuda_fail(e, "selection score launch");
-  e = stdb::launch_topk(scores, nvis_max, probs, nvis, 0, dims->Hkv, dims->B, K, idx_out, err, stream);
+  e = stdb::launch_topk(scores, nvis_max, probs, nvis, 0, dims->Hkv, dims->B, K, idx_out, hist_done ? hist : nullptr,
+                        err, stream);
   if (e != cudaSuccess) return cuda_fail(e, "top-K launch");
   stdb::GatherArgs g{};
   g.k_full = k_full; g.v_full = v_full; g.k_sp = k_sparse; g.v_sp = v_sparse; g.idx = idx_out; g.nvis = nvis;
@@ -313,6 +350,7 @@ int std_select_topk_ex(const std_dims* dims, const void* q_text, int T, const vo
 
 int std_streaming_indices(const std_dims* dims, const int32_t* nvis, int K, int n_sink, int32_t* idx_out,
                           std_stream_t stream) {
+  STD_NVTX_RANGE();
   STD_TRY(check_dims(dims));
   STD_TRY(check_ptr(nvis, 4, "nvis"));
   STD_TRY(check_ptr(idx_out, 4, "idx_out"));
@@ -328,6 +366,7 @@ int std_streaming_indices(const std_dims* dims, const int32_t* nvis, int K, int 
 int std_gather_sparse(const std_dims* dims, const void* k_full, const void* v_full, const int32_t* nvis,
                       const int32_t* idx, int K, int T, int n_prefix, void* k_sparse, void* v_sparse,
                       int32_t* len_sparse, std_stream_t stream) {
+  STD_NVTX_RANGE();
   STD_TRY(check_dims(dims));
   STD_TRY(check_ptr(k_full, 16, "k_full"));
   STD_TRY(check_ptr(v_full, 16, "v_full"));
@@ -353,13 +392,14 @@ int std_gather_sparse(const std_dims* dims, const void* k_full, const void* v_fu
 }
 
 int std_topk_from_scores(const float* scores, int rows, int n, int K, int32_t* idx_out, std_stream_t stream) {
+  STD_NVTX_RANGE();
   STD_TRY(check_ptr(scores, 4, "scores"));
   STD_TRY(check_ptr(idx_out, 4, "idx_out"));
   if (rows < 0 || n < 1) return fail(STD_ERR_INVALID_ARG, "rows = %d, n = %d", rows, n);
   if (K < 1 || K > n) return fail(STD_ERR_INVALID_ARG, "K = %d must be in [1, n = %d]", K, n);
   int* err;
   STD_TRY(device_state(&err, nullptr));
-  cudaError_t e = stdb::launch_topk(scores, n, rows, nullptr, n, 1, 1, K, idx_out, err, stream);
+  cudaError_t e = stdb::launch_topk(scores, n, rows, nullptr, n, 1, 1, K, idx_out, nullptr, err, stream);
   if (e != cudaSuccess) return cuda_fail(e, "top-K launch");
   return ok();
 }
@@ -383,6 +423,7 @@ int std_attn_splits(const std_dims* dims, int q_rows, int64_t cap, int splits) {
 int std_sparse_decode_attn(const std_dims* dims, const void* q, const void* k_sparse, const void* v_sparse,
                            const int32_t* len_sparse, int len_offset, float* o, int splits, void* ws,
                            size_t ws_bytes, std_stream_t stream) {
+  STD_NVTX_RANGE();
   STD_TRY(check_dims(dims));
   STD_TRY(check_ptr(q, 16, "q"));
   STD_TRY(check_ptr(k_sparse, 16, "k_sparse"));
@@ -397,6 +438,7 @@ int std_sparse_decode_attn(const std_dims* dims, const void* q, const void* k_sp
 int std_dense_verify_attn(const std_dims* dims, const void* q, int gamma, const void* k_full, const void* v_full,
                           const int32_t* len_full, float* o, int splits, void* ws, size_t ws_bytes,
                           std_stream_t stream) {
+  STD_NVTX_RANGE();
   STD_TRY(check_dims(dims));
   STD_TRY(check_ptr(q, 16, "q"));
   STD_TRY(check_ptr(k_full, 16, "k_full"));
@@ -409,8 +451,76 @@ int std_dense_verify_attn(const std_dims* dims, const void* q, int gamma, const 
                   stream);
 }
 
+// Shared checks of the key-range calls: the range lies in the buffer, and the shift of the
+// causal limit by pos0 fits the kernel's int arithmetic.
+static int check_range(int64_t pos0, int64_t row_begin, int64_t row_end, int64_t cap, const float* o_part,
+                       const float* ml_part) {
+  STD_TRY(check_ptr(o_part, 16, "o_part"));
+  STD_TRY(check_ptr(ml_part, 8, "ml_part"));
+  if (pos0 < 0 || pos0 > (1 << 30))
+    return fail(STD_ERR_INVALID_ARG, "pos0 = %lld must be in [0, 2^30]", (long long)pos0);
+  if (row_begin < 0 || row_begin > row_end || row_end > cap)
+    return fail(STD_ERR_INVALID_ARG, "rows [%lld, %lld) must satisfy 0 <= row_begin <= row_end <= cap = %lld",
+                (long long)row_begin, (long long)row_end, (long long)cap);
+  return STD_OK;
+}
+
+int std_dense_verify_attn_partial(const std_dims* dims, const void* q, int gamma, const void* k_full,
+                                  const void* v_full, const int32_t* len_full, int64_t pos0, int64_t row_begin,
+                                  int64_t row_end, float* o_part, float* ml_part, int splits, void* ws,
+                                  size_t ws_bytes, std_stream_t stream) {
+  STD_NVTX_RANGE();
+  STD_TRY(check_dims(dims));
+  STD_TRY(check_ptr(q, 16, "q"));
+  STD_TRY(check_ptr(k_full, 16, "k_full"));
+  STD_TRY(check_ptr(v_full, 16, "v_full"));
+  STD_TRY(check_ptr(len_full, 4, "len_full"));
+  if (gamma < 0 || gamma > 31) return fail(STD_ERR_INVALID_ARG, "gamma = %d must be in [0, 31]", gamma);
+  STD_TRY(check_range(pos0, row_begin, row_end, dims->cap_full, o_part, ml_part));
+  const RangeOpt rg{(int)row_begin, (int)row_end, ml_part};
+  // row i sees positions j < len_full + 1 + i, i.e. buffer rows r < len_full + 1 - pos0 + i
+  return run_attn(dims, q, k_full, v_full, dims->cap_full, len_full, 1 - (int)pos0, gamma + 1, o_part, splits, ws,
+                  ws_bytes, stream, nullptr, nullptr, 0, 0, 0, &rg);
+}
+
+int std_sparse_decode_attn_partial(const std_dims* dims, const void* q, const void* k_sparse, const void* v_sparse,
+                                   const int32_t* len_sparse, int len_offset, int64_t pos0, int64_t row_begin,
+                                   int64_t row_end, float* o_part, float* ml_part, int splits, void* ws,
+                                   size_t ws_bytes, std_stream_t stream) {
+  STD_NVTX_RANGE();
+  STD_TRY(check_dims(dims));
+  STD_TRY(check_ptr(q, 16, "q"));
+  STD_TRY(check_ptr(k_sparse, 16, "k_sparse"));
+  STD_TRY(check_ptr(v_sparse, 16, "v_sparse"));
+  STD_TRY(check_ptr(len_sparse, 4, "len_sparse"));
+  if (len_offset < 0 || len_offset > (1 << 30))
+    return fail(STD_ERR_INVALID_ARG, "len_offset = %d must be in [0, 2^30]", len_offset);
+  STD_TRY(check_range(pos0, row_begin, row_end, dims->cap_sparse, o_part, ml_part));
+  const RangeOpt rg{(int)row_begin, (int)row_end, ml_part};
+  return run_attn(dims, q, k_sparse, v_sparse, dims->cap_sparse, len_sparse, len_offset - (int)pos0, 1, o_part,
+                  splits, ws, ws_bytes, stream, nullptr, nullptr, 0, 0, 0, &rg);
+}
+
+int std_merge_partials(int64_t rows, int d, int n_parts, const float* o_parts, const float* ml_parts, float* o,
+                       std_stream_t stream) {
+  STD_NVTX_RANGE();
+  if (rows < 0) return fail(STD_ERR_INVALID_ARG, "rows = %lld must be >= 0", (long long)rows);
+  if (d < 4 || d % 4) return fail(STD_ERR_INVALID_ARG, "d = %d must be a positive multiple of 4", d);
+  if (n_parts < 1) return fail(STD_ERR_INVALID_ARG, "n_parts = %d must be >= 1", n_parts);
+  if (rows == 0) return ok();
+  STD_TRY(check_ptr(o_parts, 16, "o_parts"));
+  STD_TRY(check_ptr(ml_parts, 8, "ml_parts"));
+  STD_TRY(check_ptr(o, 16, "o"));
+  int sms;
+  STD_TRY(device_state(nullptr, &sms));
+  cudaError_t e = stdb::launch_merge_partials(rows, d, n_parts, o_parts, ml_parts, o, sms, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return ok();
+}
+
 int std_accept_prefix(int B, int gamma, const int32_t* draft, const int32_t* dense_argmax, int32_t* n_plus_1,
                       int32_t* accepted, std_stream_t stream) {
+  STD_NVTX_RANGE();
   if (B < 1) return fail(STD_ERR_INVALID_ARG, "B = %d must be >= 1", B);
   if (gamma < 0 || gamma > 31) return fail(STD_ERR_INVALID_ARG, "gamma = %d must be in [0, 31]", gamma);
   if (gamma > 0) STD_TRY(check_ptr(draft, 4, "draft"));
@@ -425,6 +535,19 @@ int std_accept_prefix(int B, int gamma, const int32_t* draft, const int32_t* den
 int std_sparse_decode_attn_append(const std_dims* dims, const void* q, void* k_sparse, void* v_sparse,
                                   const int32_t* len_sparse, int len_offset, const void* k_new, const void* v_new,
                                   float* o, int splits, void* ws, size_t ws_bytes, std_stream_t stream) {
+  return std_sparse_decode_attn_append_ex(dims, q, k_sparse, v_sparse, len_sparse, len_offset, k_new, v_new, o, splits,
+                                          0, ws, ws_bytes, stream);
+}
+
+int std_sparse_decode_attn_append_ex(const std_dims* dims, const void* q, void* k_sparse, void* v_sparse,
+                                     const int32_t* len_sparse, int len_offset, const void* k_new,
+                                     const void* v_new, float* o, int splits, int flags, void* ws, size_t ws_bytes,
+                                     std_stream_t stream) {
+  STD_NVTX_RANGE();
+  if (flags & ~(STD_ATTN_EARLY_KV | STD_ATTN_EARLY_Q))
+    return fail(STD_ERR_INVALID_ARG, "unknown attention flags %#x", flags);
+  if ((flags & STD_ATTN_EARLY_Q) && !(flags & STD_ATTN_EARLY_KV))
+    return fail(STD_ERR_INVALID_ARG, "STD_ATTN_EARLY_Q needs STD_ATTN_EARLY_KV");
   STD_TRY(check_dims(dims));
   STD_TRY(check_ptr(q, 16, "q"));
   STD_TRY(check_ptr(k_sparse, 16, "k_sparse"));
@@ -436,12 +559,13 @@ int std_sparse_decode_attn_append(const std_dims* dims, const void* q, void* k_s
   if (len_offset < 1) return fail(STD_ERR_INVALID_ARG, "len_offset = %d must be >= 1 (it counts the new row)", len_offset);
   if ((int64_t)len_offset > dims->cap_sparse) return fail(STD_ERR_CAPACITY, "len_offset exceeds cap_sparse");
   return run_attn(dims, q, k_sparse, v_sparse, dims->cap_sparse, len_sparse, len_offset, 1, o, splits, ws,
-                  ws_bytes, stream, k_new, v_new, 1, len_offset - 1);
+                  ws_bytes, stream, k_new, v_new, 1, len_offset - 1, flags);
 }
 
 int std_dense_verify_attn_append(const std_dims* dims, const void* q, int gamma, void* k_full, void* v_full,
                                  const int32_t* len_full, const void* k_new, const void* v_new, float* o, int splits,
                                  void* ws, size_t ws_bytes, std_stream_t stream) {
+  STD_NVTX_RANGE();
   STD_TRY(check_dims(dims));
   STD_TRY(check_ptr(q, 16, "q"));
   STD_TRY(check_ptr(k_full, 16, "k_full"));
@@ -458,6 +582,7 @@ int std_dense_verify_attn_append(const std_dims* dims, const void* q, int gamma,
 
 int std_kv_append(const std_dims* dims, void* k_cache, void* v_cache, int64_t cap, const int32_t* len,
                   int pos_offset, const void* k_new, const void* v_new, int n_new, std_stream_t stream) {
+  STD_NVTX_RANGE();
   STD_TRY(check_dims(dims));
   STD_TRY(check_ptr(k_cache, 16, "k_cache"));
   STD_TRY(check_ptr(v_cache, 16, "v_cache"));
@@ -478,6 +603,7 @@ int std_kv_append(const std_dims* dims, void* k_cache, void* v_cache, int64_t ca
 int std_kv_commit(const std_dims* dims, void* k_full, void* v_full, void* k_sparse, void* v_sparse,
                   int32_t* len_full, int32_t* len_sparse, const int32_t* n_plus_1, int max_n,
                   std_stream_t stream) {
+  STD_NVTX_RANGE();
   STD_TRY(check_dims(dims));
   STD_TRY(check_ptr(k_full, 16, "k_full"));
   STD_TRY(check_ptr(v_full, 16, "v_full"));
@@ -505,6 +631,7 @@ size_t std_round_workspace_size(const std_dims* dims, int gamma, int splits_draf
 
 int std_decode_round(const std_dims* dims, int gamma, const std_cache* c, const std_round_io* io,
                      int splits_draft, int splits_verify, void* ws, size_t ws_bytes, std_stream_t stream) {
+  STD_NVTX_RANGE();
   STD_TRY(check_dims(dims));
   if (!c || !io) return fail(STD_ERR_INVALID_ARG, "cache or io is NULL");
   if (gamma < 0 || gamma > 31) return fail(STD_ERR_INVALID_ARG, "gamma = %d must be in [0, 31]", gamma);
@@ -531,12 +658,15 @@ int std_decode_round(const std_dims* dims, int gamma, const std_cache* c, const 
     if (need > 0 && (!ws || ws_bytes < need))
       return fail(STD_ERR_WORKSPACE, "round workspace: need %zu bytes, got %zu", need, ws ? ws_bytes : 0);
   }
-  // draft step j: append its input's K/V row at len_sparse + j, attend over len_sparse + j + 1 rows
+  // draft step j: append its input's K/V row at len_sparse + j, attend over len_sparse + j + 1 rows.
+  // Steps j > 0 follow step j - 1, which writes only its output, its partials and sparse row
+  // len_sparse + j - 1, and reads inputs all queued before this call: they start early.
   for (int j = 0; j < gamma; ++j) {
     STD_TRY(run_attn(dims, static_cast<const uint8_t*>(io->q_draft) + j * q_step * eb, c->k_sparse, c->v_sparse,
                      dims->cap_sparse, c->len_sparse, j + 1, 1, io->o_draft + j * q_step, splits_draft, ws, ws_bytes,
                      stream, static_cast<const uint8_t*>(io->k_draft) + j * kv_step * eb,
-                     static_cast<const uint8_t*>(io->v_draft) + j * kv_step * eb, 1, j));
+                     static_cast<const uint8_t*>(io->v_draft) + j * kv_step * eb, 1, j,
+                     j > 0 ? STD_ATTN_EARLY_KV | STD_ATTN_EARLY_Q : 0));
   }
   // verify: append the gamma + 1 rows at len_full (a separate launch: fused into the verify
   // kernel it measured ~1% slower on the long-video step, fused into the draft faster), then
@@ -586,6 +716,7 @@ int noalloc_scratch(float** out) {
 extern "C" int std_dense_verify_attn_noalloc(const std_dims* dims, const void* q, int gamma, const void* k_full,
                                              const void* v_full, const int32_t* len_full, float* o, int splits,
                                              std_stream_t stream) {
+  STD_NVTX_RANGE();
   STD_TRY(check_dims(dims));
   STD_TRY(check_ptr(q, 16, "q"));
   STD_TRY(check_ptr(k_full, 16, "k_full"));

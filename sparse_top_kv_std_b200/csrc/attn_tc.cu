@@ -48,7 +48,8 @@ constexpr int kMaxB = 64;         // sequences per call handled by this kernel
 constexpr int kTmemCols = 512;
 constexpr uint32_t kColS = 128;   // TMEM column of S/P buffer 0 (buffer 1 at 256); O at column 0
 constexpr float kTau = 8.f;       // log2 growth of a row max that forces an O rescale
-constexpr int kMergeSegs = 4;     // segments a merge holds in registers (more: one at a time)
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kMergeSegs = 4;     // segments a merge loads per L2 round trip
 
 struct Ctl {
   uint64_t kv_full[STAGES], kv_empty[STAGES];
@@ -57,10 +58,14 @@ struct Ctl {
   uint64_t o_ready, o_free;
   uint64_t pub, flag;  // partial published by all 128 row threads / merge decision made
   uint64_t nr_ready;   // fused append: the CTA's new cache rows are written (30 copy lanes)
+  uint64_t xb1, xb2, xb3;  // SPLIT layout: a segment's quarter (m, l) published / O halves summed / summed
+  float xml[4][16][2];  // SPLIT layout: per quarter and query row, (m in log2 units, l)
+  float xrow[16][2];    // SPLIT layout: per query row, the combined (M, L)
   uint32_t tmem;
   int abort_flag;
   int consumed;
   int tl;      // tiles per layer
+  int tb;      // first tile of every problem (row_begin / TK)
   int total;   // tiles of the whole call
   int per;     // tiles per CTA
   int last_flag;
@@ -85,15 +90,17 @@ __device__ __forceinline__ bool arrive_last(unsigned long long* ctr, uint32_t ep
 }
 
 
-// Tiles of sequence b (0 for an invalid length, which is flagged).
+// Tiles of sequence b from tile row_begin / TK on (0 for an invalid length, which is
+// flagged, and, for partials, for a sequence with no key in the range).
 __device__ __forceinline__ int seq_tiles(const AttnArgs& a, int b, bool flag) {
   const int base = a.len[b] + a.len_off;
   const int lim_max = base + a.nq - 1;
-  if (base <= 0 || (int64_t)lim_max > a.cap) {
+  if (!a.partial && (base <= 0 || (int64_t)lim_max > a.cap)) {
     if (flag) flag_error(a.err, STD_DEVERR_LENGTH);
     return 0;
   }
-  return (lim_max + TK - 1) / TK;
+  const int end = min(lim_max, a.row_end);
+  return end > a.row_begin ? (end + TK - 1) / TK - a.row_begin / TK : 0;
 }
 
 // Walk over this CTA's slice of the flat (problem, tile) sequence.
@@ -154,40 +161,29 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 
 // Merge of a problem's segment partials (m, l, o) into its output, by the 128 softmax
 // threads of the last CTA to finish the problem.  One item = 4 columns of one query row.
-// BATCHED (up to kMergeSegs segments): every load of an item is issued before any is
-// used, so an item costs one L2 round trip instead of two; the M = 128 kernel, already
-// near the register limit, keeps the two-pass form.  Partial k of row r sits
-// at slot0 + k * rows + r; output row r at orow0 + r.
+// BATCHED: the segments are taken kMergeSegs at a time, every load of a batch issued
+// before any is used (one L2 round trip per batch instead of one per segment), and the
+// batches are combined with an online rescale (running max M, sum L, accumulator), so a
+// problem split over many CTAs costs ceil(nseg / kMergeSegs) round trips.  The M = 128
+// kernel, already near the register limit, keeps the two-pass form (max over all
+// segments, then the weighted sums).  Partial k of row r sits at slot0 + k * rows + r;
+// output row r at orow0 + r.
 template <int D, bool BATCHED>
-__device__ __forceinline__ void merge_problem(float* out, const float* ws, const float* ml, int rows, size_t slot0,
-                                           int nseg, size_t orow0, int tid) {
+__device__ __forceinline__ void merge_problem(float* out, float* ml_out, const float* ws, const float* ml, int rows,
+                                           size_t slot0, int nseg, size_t orow0, int tid) {
   const int nitems = rows * (D / 4);
-  auto write = [&](int r, int col, float L, float4 acc) {
-    const float inv = L > 0.f ? 1.f / L : 0.f;
+  // ml_out == nullptr: normalised output; else the merged partial, unnormalised, and its
+  // (m, l) with m converted from log2 to natural-log units
+  auto write = [&](int r, int col, float M, float L, float4 acc) {
+    const float inv = ml_out ? 1.f : (L > 0.f ? 1.f / L : 0.f);
     *reinterpret_cast<float4*>(out + (orow0 + r) * D + col) =
         make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  };
-  auto finish = [&](const float2* mlv, const float4* xv, int r, int col) {
-    float M = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < kMergeSegs; ++c)
-      if (c < nseg) M = fmaxf(M, mlv[c].x);
-    const float ref = M == -INFINITY ? 0.f : M;
-    float L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int c = 0; c < kMergeSegs; ++c) {
-      if (c >= nseg) break;
-      const float w = ex2(mlv[c].x - ref);
-      L += w * mlv[c].y;
-      acc.x += w * xv[c].x;
-      acc.y += w * xv[c].y;
-      acc.z += w * xv[c].z;
-      acc.w += w * xv[c].w;
+    if (ml_out && col == 0) {
+      ml_out[(orow0 + r) * 2] = M * kLn2;
+      ml_out[(orow0 + r) * 2 + 1] = L;
     }
-    write(r, col, L, acc);
   };
-  auto slow = [&](int item) {  // more segments than registers: one segment at a time
+  auto two_pass = [&](int item) {
     const int r = item / (D / 4), col = (item % (D / 4)) * 4;
     float M = -INFINITY;
     for (int c = 0; c < nseg; ++c) M = fmaxf(M, __ldcg(ml + (slot0 + (size_t)c * rows + r) * 2));
@@ -205,25 +201,51 @@ __device__ __forceinline__ void merge_problem(float* out, const float* ws, const
       acc.z += w * x.z;
       acc.w += w * x.w;
     }
-    write(r, col, L, acc);
+    write(r, col, M, L, acc);
   };
   for (int item = tid; item < nitems; item += 128) {
-    if (!BATCHED || nseg > kMergeSegs) {
-      slow(item);
+    if (!BATCHED) {
+      two_pass(item);
       continue;
     }
     const int r = item / (D / 4), col = (item % (D / 4)) * 4;
-    float2 mlv[kMergeSegs];
-    float4 xv[kMergeSegs];
+    float M = -INFINITY, L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = 0; c0 < nseg; c0 += kMergeSegs) {
+      float2 mlv[kMergeSegs];
+      float4 xv[kMergeSegs];
 #pragma unroll
-    for (int c = 0; c < kMergeSegs; ++c) {
-      if (c < nseg) {
-        const size_t k = slot0 + (size_t)c * rows + r;
-        mlv[c] = __ldcg(reinterpret_cast<const float2*>(ml + k * 2));
-        xv[c] = __ldcg(reinterpret_cast<const float4*>(ws + k * D + col));
+      for (int c = 0; c < kMergeSegs; ++c) {
+        if (c0 + c < nseg) {
+          const size_t k = slot0 + (size_t)(c0 + c) * rows + r;
+          mlv[c] = __ldcg(reinterpret_cast<const float2*>(ml + k * 2));
+          xv[c] = __ldcg(reinterpret_cast<const float4*>(ws + k * D + col));
+        }
       }
+      float Mn = M;
+#pragma unroll
+      for (int c = 0; c < kMergeSegs; ++c)
+        if (c0 + c < nseg) Mn = fmaxf(Mn, mlv[c].x);
+      const float ref = Mn == -INFINITY ? 0.f : Mn;
+      const float f = ex2(M - ref);  // rescale of the batches so far (0 while M is -inf)
+      L *= f;
+      acc.x *= f;
+      acc.y *= f;
+      acc.z *= f;
+      acc.w *= f;
+#pragma unroll
+      for (int c = 0; c < kMergeSegs; ++c) {
+        if (c0 + c >= nseg) break;
+        const float w = ex2(mlv[c].x - ref);
+        L += w * mlv[c].y;
+        acc.x += w * xv[c].x;
+        acc.y += w * xv[c].y;
+        acc.z += w * xv[c].z;
+        acc.w += w * xv[c].w;
+      }
+      M = Mn;
     }
-    finish(mlv, xv, r, col);
+    write(r, col, M, L, acc);
   }
 }
 
@@ -244,7 +266,7 @@ __device__ __forceinline__ void copy_new_rows(const AttnArgs& a, const Ctl* ctl,
     const int p0 = ctl->len_b[b] + a.new_off;
     for (int r = 0; r < a.new_rows; ++r) {
       const int pos = p0 + r;
-      const int flat = gp + pos / TK;
+      const int flat = gp + pos / TK - ctl->tb;
       if (flat < g0 || flat >= g1 || pos < 0 || (int64_t)pos >= a.cap) continue;
       for (int i = c; i < 2 * kChunks; i += 30) {
         const bool isv = i >= kChunks;
@@ -284,12 +306,20 @@ struct Cfg {
 // accumulator row i sits in TMEM lane 32 * (i / 16) + i % 16, so the rows are
 // spread over all four lane quarters (and SM sub-partitions) and two softmax
 // threads share a row, each taking 64 of its 128 columns.
-template <int D, bool HALF>
+// SPLIT (with HALF; at most 16 query rows, the draft's case): the 16 query rows are
+// loaded four times, to MMA rows q * 16 + i for q = 0..3, so every lane quarter holds
+// a copy of every row and every softmax warp has work.  Quarter q takes 32 of each
+// tile's 128 keys (keys 16q..16q+15 and 64+16q..64+16q+15; the thread pair of a row
+// 16 each) and keeps its own running max, sum and O row -- zeros in P elsewhere keep
+// the other quarters' keys out of its O; at the end of a segment the four (m, l, O)
+// are combined in shared memory in a fixed order ((q0 + q2) + (q1 + q3)), so results
+// do not depend on scheduling.  Each softmax thread then handles 16 keys of a tile
+// instead of 64: the per-tile latency that bounds a CTA with few query rows drops.
+template <int D, bool HALF, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
-  pdl_wait();  // memory of earlier kernels in the stream is visible from here on
-  pdl_trigger();
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k16,
+               const __grid_constant__ CUtensorMap tm_v16, const AttnArgs a) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -299,16 +329,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    int sum = 0;
-    for (int b = 0; b < a.B; ++b) {
-      ctl->tiles_b[b] = seq_tiles(a, b, blockIdx.x == 0);
-      ctl->len_b[b] = a.len[b];
-      ctl->pre_b[b] = a.Hkv * sum;
-      sum += ctl->tiles_b[b];
-    }
-    ctl->tl = a.Hkv * sum;
-    ctl->total = a.L * ctl->tl;
-    ctl->per = ctl->total > 0 ? (ctl->total + gridDim.x - 1) / gridDim.x : 1;
     for (int s = 0; s < STAGES; ++s) {
       tc::mbar_init(&ctl->kv_full[s], 1);
       tc::mbar_init(&ctl->kv_empty[s], 1);
@@ -326,6 +346,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc::mbar_init(&ctl->pub, 128);
     tc::mbar_init(&ctl->flag, 1);
     tc::mbar_init(&ctl->nr_ready, 30);
+    tc::mbar_init(&ctl->xb1, 128);
+    tc::mbar_init(&ctl->xb2, 128);
+    tc::mbar_init(&ctl->xb3, 128);
     ctl->abort_flag = 0;
     ctl->consumed = 0;
     tc::fence_mbar_init();
@@ -334,6 +357,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __syncwarp();
     tc::tmem_alloc(&ctl->tmem, kTmemCols);
     tc::tmem_relinquish();
+  }
+  // The barrier and TMEM set-up above touch no global memory and may overlap the previous
+  // kernel.  Without the early start, everything below waits for it; with it (a.early),
+  // the lengths are read now and each role waits just before it needs to (below).
+  if (!a.early) {
+    pdl_wait();
+    pdl_trigger();  // only after this CTA's wait: the next kernel may start early itself
+  }
+  if (threadIdx.x == 0) {
+    int sum = 0;
+    for (int b = 0; b < a.B; ++b) {
+      ctl->tiles_b[b] = seq_tiles(a, b, blockIdx.x == 0);
+      ctl->len_b[b] = a.len[b];
+      ctl->pre_b[b] = a.Hkv * sum;
+      sum += ctl->tiles_b[b];
+    }
+    ctl->tl = a.Hkv * sum;
+    ctl->tb = a.row_begin / TK;
+    ctl->total = a.L * ctl->tl;
+    ctl->per = ctl->total > 0 ? (ctl->total + gridDim.x - 1) / gridDim.x : 1;
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -348,28 +391,54 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (lane == 0 && g0 < g1) {
       tc::prefetch_tmap(&tm_k);
       tc::prefetch_tmap(&tm_v);
+      tc::prefetch_tmap(&tm_k16);
+      tc::prefetch_tmap(&tm_v16);
       Iter it;
       iter_seek(it, ctl, a, g0, g1);
       int kv = 0;
       bool rows_ready = a.k_new == nullptr;
+      bool waited = !a.early;
       while (it.g < it.g_end) {
         const int prob = (it.l * a.B + it.b) * a.Hkv + it.h;
         const int s = kv % STAGES;
+        const int tabs = it.t + ctl->tb;  // tile index within the problem
+        // early start: rows from len[b] + new_off - 1 on may still be written by the previous kernel
+        if (!waited && (tabs + 1) * TK > ctl->len_b[it.b] + a.new_off - 1) {
+          pdl_wait();
+          waited = true;
+        }
         if (!rows_ready) {  // fused append: a tile holding new rows waits until they are written
           const int p0 = ctl->len_b[it.b] + a.new_off;
-          if (it.t * TK < p0 + a.new_rows && p0 < (it.t + 1) * TK) {
+          if (tabs * TK < p0 + a.new_rows && p0 < (tabs + 1) * TK) {
             if (!tc::mbar_wait(&ctl->nr_ready, 0, abort_flag, a.err)) break;
             rows_ready = true;
           }
         }
         if (!tc::mbar_wait(&ctl->kv_empty[s], ((kv / STAGES) & 1) ^ 1, abort_flag, a.err)) break;
-        tc::mbar_expect_tx(&ctl->kv_full[s], C::ST_BYTES);
-        const int row = prob * (int)a.cap + it.t * TK;
+        if (!STD_DCHECK(tabs * TK < a.cap && prob < a.L * a.B * a.Hkv, a.err)) break;
+        const int row = prob * (int)a.cap + tabs * TK;
         const uint32_t st = sKV + s * C::ST_BYTES;
+        // keys any query row of the problem attends to in this tile; a short last tile is
+        // fetched in 16-row boxes (the rows past them are masked and their V zeroed)
+        const int nvalid = min(ctl->len_b[it.b] + a.len_off + a.nq - 1, a.row_end) - tabs * TK;
+        if (nvalid >= TK) {
+          tc::mbar_expect_tx(&ctl->kv_full[s], C::ST_BYTES);
 #pragma unroll
-        for (int kb = 0; kb < C::KB; ++kb) {
-          tc::tma_load_2d(st + kb * TK * 128, &tm_k, kb * 64, row, &ctl->kv_full[s]);
-          tc::tma_load_2d(st + C::T_BYTES + kb * TK * 128, &tm_v, kb * 64, row, &ctl->kv_full[s]);
+          for (int kb = 0; kb < C::KB; ++kb) {
+            tc::tma_load_2d(st + kb * TK * 128, &tm_k, kb * 64, row, &ctl->kv_full[s]);
+            tc::tma_load_2d(st + C::T_BYTES + kb * TK * 128, &tm_v, kb * 64, row, &ctl->kv_full[s]);
+          }
+        } else {
+          const int nb = (nvalid + 15) >> 4;  // 1..8 boxes of 16 rows
+          tc::mbar_expect_tx(&ctl->kv_full[s], (uint32_t)nb * 16 * 128 * C::KB * 2);
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb) {
+            for (int i = 0; i < nb; ++i) {
+              tc::tma_load_2d(st + kb * TK * 128 + i * 16 * 128, &tm_k16, kb * 64, row + i * 16, &ctl->kv_full[s]);
+              tc::tma_load_2d(st + C::T_BYTES + kb * TK * 128 + i * 16 * 128, &tm_v16, kb * 64, row + i * 16,
+                              &ctl->kv_full[s]);
+            }
+          }
         }
         ++kv;
         iter_next(it, ctl, a);
@@ -382,14 +451,33 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       Iter it;
       iter_seek(it, ctl, a, g0, g1);
       int seg = 0;
+      bool waited = !a.early;
       while (it.g < it.g_end) {
         if (it.first) {
+          if (!waited && !(a.early & STD_ATTN_EARLY_Q)) {  // Q may still be written by the previous kernel
+            pdl_wait();
+            pdl_trigger();
+            waited = true;
+          }
           if (!tc::mbar_wait(&ctl->q_empty, (seg & 1) ^ 1, abort_flag, a.err)) break;
           tc::mbar_expect_tx(&ctl->q_full, HALF ? C::Q_BYTES / 2 : C::Q_BYTES);  // HALF: 64-row boxes
           const int qrow = ((it.l * a.B + it.b) * a.Hq + it.h * a.G) * a.nq;
 #pragma unroll
-          for (int kb = 0; kb < C::KB; ++kb) tc::tma_load_2d(sQ + kb * 128 * 128, &tm_q, kb * 64, qrow, &ctl->q_full);
+          for (int kb = 0; kb < C::KB; ++kb) {
+            if constexpr (SPLIT) {  // the same 16 rows at MMA rows 0, 16, 32, 48 (tm_q: 16-row boxes)
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                tc::tma_load_2d(sQ + kb * 128 * 128 + q * 16 * 128, &tm_q, kb * 64, qrow, &ctl->q_full);
+            } else {
+              tc::tma_load_2d(sQ + kb * 128 * 128, &tm_q, kb * 64, qrow, &ctl->q_full);
+            }
+          }
           ++seg;
+          if (!waited) {  // this CTA's wait, off every other role's path
+            pdl_wait();
+            pdl_trigger();
+            waited = true;
+          }
         }
         iter_next(it, ctl, a);
       }
@@ -397,6 +485,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     } else if (lane >= 2 && g0 < g1 && a.k_new != nullptr) {
       // fused append: write the new rows whose tiles fall in this CTA's slice (only this
       // CTA reads those tiles), then order the writes before the TMA loads of them
+      if (a.early) pdl_wait();  // the previous kernel may still read the tile these rows land in
       copy_new_rows<D>(a, ctl, g0, g1, lane - 2);
       asm volatile("fence.proxy.async.global;" ::: "memory");
       tc::mbar_arrive(&ctl->nr_ready);
@@ -477,18 +566,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // Full layout: one thread per query row = TMEM lane (warp % 4) * 32 + lane, all 128
     // columns of S.  HALF layout: query row (warp % 4) * 16 + lane % 16 in TMEM lane
     // (warp % 4) * 32 + lane % 16; lane < 16 takes columns [0, 64), lane >= 16 [64, 128).
-    constexpr int NC = HALF ? TK / 2 : TK;  // S columns per thread
+    // SPLIT layout: query row lane % 16, copy of quarter (warp % 4); the thread takes keys
+    // 16 (warp % 4) + 64 (lane / 16) + [0, 16) of each tile.
+    constexpr int NC = SPLIT ? 16 : (HALF ? TK / 2 : TK);  // S columns (keys) per thread
     constexpr int OC = HALF ? D / 2 : D;    // O columns per thread
     const int qd = warp & 3;                // TMEM lane quarter of this warp
-    const int row = HALF ? qd * 16 + (lane & 15) : qd * 32 + lane;  // query row of this thread
+    const int row = SPLIT ? (lane & 15) : HALF ? qd * 16 + (lane & 15) : qd * 32 + lane;  // query row
     const int hh = HALF ? lane >> 4 : 0;    // which column half (HALF layout)
-    const bool wactive = (HALF ? qd * 16 : qd * 32) < a.rows;  // warp holds at least one real query row
+    const bool wactive = SPLIT || (HALF ? qd * 16 : qd * 32) < a.rows;  // warp holds a real query row
+    // SPLIT: two [16][D] fp32 sums of the quarters' O rows (quarters 0 + 2 and 1 + 3), in the
+    // parts of the Q area that the 64-row query tile leaves unused (8 KB at 8 KB, and 8 KB at
+    // 24 KB for D = 128 or 4 KB at 12 KB for D = 64)
+    float* redA = reinterpret_cast<float*>(smem + 8192);
+    float* redB = reinterpret_cast<float*>(smem + (D == 128 ? 24576 : 12288));
     const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
     const float sc = kLog2e * rsqrtf((float)D);
     const int tid = threadIdx.x - 64;
     Iter it;
     iter_seek(it, ctl, a, g0, g1);
-    int seg = -1, kv = 0, u = 0, npub = 0;
+    int seg = -1, kv = 0, u = 0, npub = 0, nx = 0;
     float m = -INFINITY, l = 0.f;
     int lim = 0, lim_max = 0;
     while (it.g < it.g_end) {
@@ -500,33 +596,43 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         m = -INFINITY;
         l = 0.f;
         const int base = a.len[it.b] + a.len_off;
-        lim = base + (row < a.rows ? row % a.nq : 0);
-        lim_max = base + a.nq - 1;
+        lim = min(base + (row < a.rows ? row % a.nq : 0), a.row_end);
+        lim_max = min(base + a.nq - 1, a.row_end);
       }
       const int bu = u & 1;
       const int s = kv % STAGES;
-      const int key0 = it.t * TK;
+      const int key0 = (it.t + ctl->tb) * TK;
       if (!tc::mbar_wait_warp(&ctl->s_full[bu], (u >> 1) & 1, abort_flag, a.err)) break;
       tc::fence_after_sync();
-      if (key0 + TK > lim_max) {
-        // last tile of the problem: zero V rows past the last query's limit so that
-        // whatever bytes sit there cannot turn 0 * V into NaN
+      if (key0 + TK > lim_max || key0 < a.row_begin) {
+        // last tile of the problem (or first tile of a key range): zero the V rows past
+        // the last query's limit and before the range, so that whatever bytes sit there
+        // cannot turn 0 * V into NaN
         if (!tc::mbar_wait_warp(&ctl->kv_full[s], (kv / STAGES) & 1, abort_flag, a.err)) break;
         const int z0 = max(0, lim_max - key0);
+        const int zb = a.row_begin - key0;
         uint8_t* vb = smem + C::Q_BYTES + s * C::ST_BYTES + C::T_BYTES;
         for (int i = tid; i < C::KB * TK * 8; i += 128) {
           const int r = (i >> 3) % TK;
-          if (r >= z0) *reinterpret_cast<uint4*>(vb + (i / (TK * 8)) * TK * 128 + r * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+          if (r >= z0 || r < zb)
+            *reinterpret_cast<uint4*>(vb + (i / (TK * 8)) * TK * 128 + r * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
         }
         tc::fence_proxy_async();
       }
       if (wactive) {
         // this thread's logits of the tile: v[j] is key kc0 + j
         float v[NC];
-        const int kc0 = key0 + hh * NC;
+        const int kc0 = key0 + hh * (TK / 2) + (SPLIT ? 16 * qd : 0);
         {
           const uint32_t sa = lane_base + kColS + bu * 128;
-          if constexpr (HALF) {
+          if constexpr (SPLIT) {
+            uint32_t r0[16];
+            __syncwarp();
+            tc::tmem_ld16_x16<TK / 2>(sa + 16 * qd, r0);
+            tc::tmem_ld_wait16(r0);
+  #pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r0[j]);
+          } else if constexpr (HALF) {
             uint32_t r0[32], r1[32];
             __syncwarp();
             tc::tmem_ld16_x32<TK / 2>(sa, r0);
@@ -563,6 +669,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           for (int j = 0; j < NC; ++j)
             if (kc0 + j >= lim) v[j] = -INFINITY;
         }
+        if (kc0 < a.row_begin) {  // key range: keys before it are not attended
+  #pragma unroll
+          for (int j = 0; j < NC; ++j)
+            if (kc0 + j < a.row_begin) v[j] = -INFINITY;
+        }
         float mx = v[0];
   #pragma unroll
         for (int j = 1; j + 1 < NC; j += 2) mx = max3f(mx, v[j], v[j + 1]);
@@ -598,6 +709,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // (packed column j of the tile holds keys 2j and 2j + 1)
         uint32_t pk[NC / 2];
         const f32x2 scc = f2_make(sc, sc), nm = f2_make(-msc, -msc);
+        if constexpr (SPLIT) {
+          f32x2 sacc = f2_make(0.f, 0.f);
+  #pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float x0, x1;
+            f2_split(f2_fma(f2_make(v[2 * j], v[2 * j + 1]), scc, nm), x0, x1);
+            const float p0 = live ? ex2(x0) : 0.f;
+            const float p1 = live ? ex2(x1) : 0.f;
+            sacc = f2_add(sacc, f2_make(p0, p1));
+            pk[j] = pack_bf16(p0, p1);
+          }
+          float sl, sh;
+          f2_split(sacc, sl, sh);
+          l += sl + sh;
+          // this thread's half of the P row: its 8 packed columns, zeros for the other quarters' keys
+          uint32_t prow[32];
+  #pragma unroll
+          for (int c = 0; c < 32; ++c) prow[c] = (c >> 3) == qd ? pk[c & 7] : 0u;
+          __syncwarp();
+          tc::tmem_st16_x32<TK / 4>(lane_base + kColS + bu * 128, prow);
+        }
   #pragma unroll
         for (int c = 0; c < NC / 32; ++c) {
           f32x2 sacc = f2_make(0.f, 0.f);
@@ -618,7 +750,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tc::tmem_st_x16(lane_base + kColS + bu * 128 + c * 16, reinterpret_cast<const uint32_t(&)[16]>(pk[c * 16]));
           }
         }
-        if constexpr (HALF) {
+        if constexpr (HALF && !SPLIT) {
           __syncwarp();
           tc::tmem_st16_x32<TK / 4>(lane_base + kColS + bu * 128, pk);
         }
@@ -629,14 +761,105 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (last) {
         if (!tc::mbar_wait_warp(&ctl->o_ready, seg & 1, abort_flag, a.err)) break;
         tc::fence_after_sync();
-        const float lrow = HALF ? l + __shfl_xor_sync(0xffffffffu, l, 16) : l;  // the whole row's sum
+        if (a.early) pdl_wait();  // outputs, partials and merge counters: after the previous kernel
+        const float lrow = HALF ? l + __shfl_xor_sync(0xffffffffu, l, 16) : l;  // the row's (quarter's) sum
         // CTAs whose slices touch this problem
         const int start = it.l * ctl->tl + ctl->pre_b[it.b] + it.h * it.nt;
         const int c0 = start / ctl->per, c1 = (start + it.nt - 1) / ctl->per;
-        const size_t orow = (size_t)(lb * a.Hq + it.h * a.G) * a.nq + row;
-        if (c0 == c1) {
-          // this CTA saw the whole problem: normalised output straight from TMEM
-          const float inv = lrow > 0.f ? 1.f / lrow : 0.f;
+        const size_t orow0 = (size_t)(lb * a.Hq + it.h * a.G) * a.nq;  // output row of query row 0
+        const size_t orow = orow0 + row;
+        // segment partials: slot prob + blockIdx.x of [slots][rows][D], then (m, l), then counters
+        const size_t nslots = (size_t)a.L * a.B * a.Hkv + gridDim.x;
+        float* wml = a.ws + nslots * a.rows * D;
+        unsigned long long* ctr = reinterpret_cast<unsigned long long*>(wml + nslots * a.rows * 2);
+        const int slot = prob + blockIdx.x;
+        if constexpr (SPLIT) {
+          // combine the four quarters' (m, l, O) of every query row: publish (m, l), weigh each
+          // quarter's O row by 2^(m_q - M) into the shared sum, then write from the sum
+          if (hh == 0) {
+            ctl->xml[qd][row][0] = m * sc;
+            ctl->xml[qd][row][1] = lrow;
+          }
+          tc::mbar_arrive(&ctl->xb1);
+          if (!tc::mbar_wait_warp(&ctl->xb1, nx & 1, abort_flag, a.err)) break;
+          float M = -INFINITY;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) M = fmaxf(M, ctl->xml[q][row][0]);
+          const float ref = M == -INFINITY ? 0.f : M;
+          if (qd == 0 && hh == 0) {
+            float L = 0.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) L += ex2(ctl->xml[q][row][0] - ref) * ctl->xml[q][row][1];
+            ctl->xrow[row][0] = M;
+            ctl->xrow[row][1] = L;
+          }
+          const float w = ex2(m * sc - ref);  // 0 for a quarter that saw no key
+          // quarters 0 and 1 store w O into redA / redB, then quarters 2 and 3 add theirs: every
+          // element is written by one thread at a time, in a fixed order
+          float* red = (qd & 1) ? redB : redA;
+          if (qd < 2) {
+#pragma unroll
+            for (int c = 0; c < OC / 32; ++c) {
+              uint32_t o[32];
+              __syncwarp();
+              tc::tmem_ld16_x32<D / 2>(lane_base + c * 32, o);
+              tc::tmem_ld_wait(o);
+              if (row < a.rows) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) red[row * D + hh * OC + c * 32 + j] = w * __uint_as_float(o[j]);
+              }
+            }
+          }
+          tc::mbar_arrive(&ctl->xb2);
+          if (!tc::mbar_wait_warp(&ctl->xb2, nx & 1, abort_flag, a.err)) break;
+          if (qd >= 2) {
+#pragma unroll
+            for (int c = 0; c < OC / 32; ++c) {
+              uint32_t o[32];
+              __syncwarp();
+              tc::tmem_ld16_x32<D / 2>(lane_base + c * 32, o);
+              tc::tmem_ld_wait(o);
+              if (row < a.rows) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) red[row * D + hh * OC + c * 32 + j] += w * __uint_as_float(o[j]);
+              }
+            }
+          }
+          tc::fence_before_sync();
+          tc::mbar_arrive(&ctl->o_free);  // O may be reused
+          tc::mbar_arrive(&ctl->xb3);
+          if (!tc::mbar_wait_warp(&ctl->xb3, nx & 1, abort_flag, a.err)) break;
+          ++nx;
+          for (int e = tid; e < a.rows * (D / 4); e += 128) {
+            const int r = e / (D / 4), col = (e % (D / 4)) * 4;
+            const float4 xa = *reinterpret_cast<const float4*>(redA + r * D + col);
+            const float4 xb = *reinterpret_cast<const float4*>(redB + r * D + col);
+            const float4 x = make_float4(xa.x + xb.x, xa.y + xb.y, xa.z + xb.z, xa.w + xb.w);
+            const float Mr = ctl->xrow[r][0], Lr = ctl->xrow[r][1];
+            if (c0 == c1) {
+              const float inv = a.partial ? 1.f : (Lr > 0.f ? 1.f / Lr : 0.f);
+              *reinterpret_cast<float4*>(a.o + (orow0 + r) * D + col) =
+                  make_float4(x.x * inv, x.y * inv, x.z * inv, x.w * inv);
+              if (a.partial && col == 0) {
+                a.ml[(orow0 + r) * 2] = Mr * kLn2;
+                a.ml[(orow0 + r) * 2 + 1] = Lr;
+              }
+            } else {
+              *reinterpret_cast<float4*>(a.ws + ((size_t)slot * a.rows + r) * D + col) = x;
+              if (col == 0) {
+                wml[((size_t)slot * a.rows + r) * 2] = Mr;
+                wml[((size_t)slot * a.rows + r) * 2 + 1] = Lr;
+              }
+            }
+          }
+        } else if (c0 == c1) {
+          // this CTA saw the whole problem: normalised output straight from TMEM (partials:
+          // unnormalised, with (m, l) beside it)
+          const float inv = a.partial ? 1.f : (lrow > 0.f ? 1.f / lrow : 0.f);
+          if (a.partial && row < a.rows && hh == 0) {
+            a.ml[orow * 2] = m * rsqrtf((float)D);
+            a.ml[orow * 2 + 1] = lrow;
+          }
 #pragma unroll
           for (int c = 0; c < OC / 32; ++c) {
             uint32_t o[32];
@@ -656,10 +879,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           tc::fence_before_sync();
           tc::mbar_arrive(&ctl->o_free);
         } else {
-          const size_t nslots = (size_t)a.L * a.B * a.Hkv + gridDim.x;
-          float* ml = a.ws + nslots * a.rows * D;
-          unsigned long long* ctr = reinterpret_cast<unsigned long long*>(ml + nslots * a.rows * 2);
-          const int slot = prob + blockIdx.x;
           float* po = a.ws + ((size_t)slot * a.rows + row) * D + hh * OC;
 #pragma unroll
           for (int c = 0; c < OC / 32; ++c) {
@@ -677,11 +896,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
           }
           if (row < a.rows && hh == 0) {
-            ml[((size_t)slot * a.rows + row) * 2] = m * sc;
-            ml[((size_t)slot * a.rows + row) * 2 + 1] = lrow;
+            wml[((size_t)slot * a.rows + row) * 2] = m * sc;
+            wml[((size_t)slot * a.rows + row) * 2 + 1] = lrow;
           }
           tc::fence_before_sync();
           tc::mbar_arrive(&ctl->o_free);  // O may be reused: the rest reads global memory only
+        }
+        if (c0 != c1) {
           // publish the partial, count the arrival; the last CTA merges every slot of the problem
           __threadfence();
           tc::mbar_arrive(&ctl->pub);
@@ -693,11 +914,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
           if (!tc::mbar_wait(&ctl->flag, npub & 1, abort_flag, a.err)) break;
           ++npub;
-          if (ctl->last_flag) {
+          if (ctl->last_flag && STD_DCHECK((size_t)prob + c1 < nslots && c0 <= c1, a.err)) {
             __threadfence();
             // all 128 softmax threads share the merge
-            merge_problem<D, HALF>(a.o, a.ws, ml, a.rows, (size_t)(prob + c0) * a.rows, c1 - c0 + 1,
-                             (size_t)(lb * a.Hq + it.h * a.G) * a.nq, tid);
+            merge_problem<D, HALF>(a.o, a.partial ? a.ml : nullptr, a.ws, wml, a.rows, (size_t)(prob + c0) * a.rows,
+                                   c1 - c0 + 1, orow0, tid);
             if (tid == 0) atomicExch(ctr + prob, (unsigned long long)a.epoch << 32);  // ready for a replay
           }
         }
@@ -705,6 +926,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       ++u;
       ++kv;
       iter_next(it, ctl, a);
+    }
+    if (a.partial && blockIdx.x == 0) {
+      // partials of a sequence with no key in the range: o = 0, m = -inf, l = 0
+      const int per_b = a.Hq * a.nq;  // output rows of one (layer, sequence)
+      for (int b = 0; b < a.B; ++b) {
+        if (ctl->tiles_b[b] != 0) continue;
+        for (int i = tid; i < a.L * per_b * (D / 4); i += 128) {
+          const int l_ = i / (per_b * (D / 4)), rem = i % (per_b * (D / 4));
+          const size_t orow = (size_t)(l_ * a.B + b) * per_b + rem / (D / 4);
+          *reinterpret_cast<float4*>(a.o + orow * D + (rem % (D / 4)) * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (rem % (D / 4) == 0) {
+            a.ml[orow * 2] = -INFINITY;
+            a.ml[orow * 2 + 1] = 0.f;
+          }
+        }
+      }
     }
   }
   tc::fence_before_sync();
@@ -720,27 +957,32 @@ template <int D>
 cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   using C = Cfg<D>;
   // at most 64 query rows per problem (the draft's G rows, the verify's G * (gamma + 1)
-  // up to 64): M = 64 MMAs, the spread softmax layout, and 64-row query boxes
+  // up to 64): M = 64 MMAs, the spread softmax layout, and 64-row query boxes; at most 16
+  // (the draft): every row copied to all four lane quarters, 16-row query boxes
   const bool half = a.rows <= 64;
+  const bool split = a.rows <= 16;
   const uint64_t qrows = (uint64_t)a.L * a.B * a.Hq * a.nq;
   const uint64_t krows = (uint64_t)a.L * a.B * a.Hkv * a.cap;
-  CUtensorMap tq, tk, tv;
-  if (!make_tmap_bf16_2d(&tq, a.q, D, qrows, half ? 64 : 128) || !make_tmap_bf16_2d(&tk, a.k, D, krows, TK) ||
-      !make_tmap_bf16_2d(&tv, a.v, D, krows, TK))
+  CUtensorMap tq, tk, tv, tk16, tv16;
+  if (!make_tmap_bf16_2d(&tq, a.q, D, qrows, split ? 16 : half ? 64 : 128) ||
+      !make_tmap_bf16_2d(&tk, a.k, D, krows, TK) || !make_tmap_bf16_2d(&tv, a.v, D, krows, TK) ||
+      !make_tmap_bf16_2d(&tk16, a.k, D, krows, 16) || !make_tmap_bf16_2d(&tv16, a.v, D, krows, 16))
     return cudaErrorInvalidValue;
-  auto kern = half ? attn_tc_kernel<D, true> : attn_tc_kernel<D, false>;
+  const int variant = split ? 2 : half ? 1 : 0;
+  auto kern = split ? attn_tc_kernel<D, true, true> : half ? attn_tc_kernel<D, true, false>
+                                                            : attn_tc_kernel<D, false, false>;
   // the shared-memory size is a per-device attribute of each kernel: set it once per device
   static std::atomic<uint64_t> attr_done{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const uint64_t bit = 1ull << ((dev & 31) * 2 + (half ? 1 : 0));
+  const uint64_t bit = 1ull << ((dev & 15) * 4 + variant);
   if (!(attr_done.load(std::memory_order_acquire) & bit)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(bit, std::memory_order_release);
   }
-  return launch_pdl(kern, dim3(a.splits), dim3(kThreads), C::SMEM, s, tq, tk, tv, a);
+  return launch_pdl(kern, dim3(a.splits), dim3(kThreads), C::SMEM, s, tq, tk, tv, tk16, tv16, a);
 }
 
 }  // namespace

@@ -16,12 +16,34 @@ __device__ __forceinline__ void flag_error(int* err, int bits) {
   if (err) atomicOr(err, bits);
 }
 
+// Debug builds (compiled with -DSTD_DEBUG into libstd_b200_debug.so) check, on the device,
+// that every index and cache row a kernel is about to use lies inside its buffer: a failed
+// check sets STD_DEVERR_DEBUG and the caller skips the access.  Never a trap.  In the
+// product build the check is the constant true and costs nothing.
+#ifdef STD_DEBUG
+__device__ __forceinline__ bool std_dcheck(bool ok, int* err) {
+  if (!ok) flag_error(err, STD_DEVERR_DEBUG);
+  return ok;
+}
+#define STD_DCHECK(cond, err) ::stdb::std_dcheck((cond), (err))
+#else
+#define STD_DCHECK(cond, err) true
+#endif
+
 // Programmatic dependent launch: every kernel of the library is launched so
 // that it may start while the previous kernel in the stream finishes.  It must
 // call pdl_wait() before touching memory a previous kernel writes or reads, and
 // calls pdl_trigger() to let the next kernel start launching.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Order-preserving 32-bit key of a float (larger float -> larger key; -0.0 maps like
+// +0.0): the radix of the top-K select, and the digit the selection's score pass counts.
+__device__ __forceinline__ uint32_t score_order_key(float x) {
+  uint32_t u = __float_as_uint(x);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
 
 // ---------------------------------------------------------------- loads
 template <typename T>

@@ -55,6 +55,22 @@ struct AttnArgs {
   const void* k_new;
   const void* v_new;
   int new_rows, new_off;
+  // Early start (tensor-core kernel), bits of STD_ATTN_EARLY_*: the kernel just before
+  // this one in the stream is one of this library's (launched after every earlier write
+  // to these buffers) and writes neither len nor any K/V row below len[b] + new_off - 1
+  // (bit 1), nor q (bit 2).  The kernel then reads the lengths, loads the K/V tiles
+  // below that row (and Q) and runs their softmax before griddepcontrol.wait, overlapping
+  // the previous kernel's tail, and waits only before the tiles above that row, before
+  // Q (without bit 2) and before its first global write.
+  int early;
+  // Key range (tensor-core kernel): only cache rows [row_begin, row_end) are attended
+  // (plan_attn sets 0 and cap).  partial != 0: instead of the normalised output, write
+  // o = sum_j 2^(x_j - m) v_j unnormalised to `o` and (m, l) to `ml` [rows][2] (m in
+  // natural-log units of the scaled logits, l = sum_j 2^(x_j - m)); a query row that
+  // attends no key gets o = 0, m = -inf, l = 0, and no length check is flagged.
+  int row_begin, row_end;
+  int partial;
+  float* ml;
 };
 
 // Split-K kernels (fp32 operands; bf16 when the tensor-core kernel does not apply):
@@ -86,8 +102,12 @@ struct ScoreArgs {
   int* err;
   int causal_text;  // nonzero: text keys 0..t join row (g, t)'s softmax (launch_text_rowstats after pass 1)
   int prefix;       // prompt rows before the visual block (a system prompt): cache = [prefix | visual | text]
+  // [prob][256]: counts of the top 8 bits of score_order_key over each problem's scores,
+  // made by the tensor-core score pass as it writes the scores (the top-K's first radix pass)
+  uint32_t* hist;
 };
-cudaError_t launch_select_scores(const ScoreArgs& a, cudaStream_t s);
+// *hist_done: whether the path that ran filled a.hist (the tensor-core path does).
+cudaError_t launch_select_scores(const ScoreArgs& a, cudaStream_t s, bool* hist_done);
 // Causal full-row variant: merge each text row's visible text keys into pass 1's (row_m, row_l).
 cudaError_t launch_text_rowstats(const ScoreArgs& a, cudaStream_t s);
 // tcgen05 version for bf16 operands; cudaErrorNotSupported for shapes it does not cover.
@@ -95,8 +115,9 @@ cudaError_t launch_select_scores_tc(const ScoreArgs& a, cudaStream_t s);
 
 // Top-K of `rows` rows of scores at scores + p * stride.  Row p has
 // n_dev[(p / n_div) % n_mod] valid entries (n_const if n_dev is NULL).  idx [rows][K].
+// hist0: NULL, or each row's histogram of the top 8 key bits (ScoreArgs::hist).
 cudaError_t launch_topk(const float* scores, int64_t stride, int rows, const int32_t* n_dev,
-                        int n_const, int n_div, int n_mod, int K, int32_t* idx, int* err,
+                        int n_const, int n_div, int n_mod, int K, int32_t* idx, const uint32_t* hist0, int* err,
                         cudaStream_t s);
 
 struct GatherArgs {
@@ -125,6 +146,10 @@ cudaError_t launch_commit(void* k_full, void* v_full, void* k_sp, void* v_sp, in
                           int32_t* len_sp, const int32_t* n_plus_1, int max_n, int L, int B,
                           int Hkv, int row_bytes, int64_t cap_full, int64_t cap_sparse, int* err,
                           cudaStream_t s);
+
+// o[r] = merge of n_parts partials (o_parts [n_parts][rows][d], ml_parts [n_parts][rows][2]).
+cudaError_t launch_merge_partials(int64_t rows, int d, int n_parts, const float* o_parts, const float* ml_parts,
+                                  float* o, int sms, cudaStream_t s);
 
 cudaError_t launch_accept(int B, int gamma, const int32_t* draft, const int32_t* dense,
                           int32_t* n_plus_1, int32_t* accepted, cudaStream_t s);

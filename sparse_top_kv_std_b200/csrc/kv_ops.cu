@@ -43,6 +43,7 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) gather_kernel(const GatherA
   } else {
     src = a.prefix + nv + (j - a.prefix - a.K);
   }
+  if (!STD_DCHECK(src >= 0 && src < a.cap_full && j < a.cap_sparse, a.err)) return;
   const size_t so = ((size_t)prob * a.cap_full + src) * a.row_bytes;
   const size_t dof = ((size_t)prob * a.cap_sparse + j) * a.row_bytes;
   copy_row(static_cast<uint8_t*>(a.k_sp) + dof, static_cast<const uint8_t*>(a.k_full) + so, a.row_bytes, lane);
@@ -66,6 +67,7 @@ append_kernel(uint8_t* kc, uint8_t* vc, int64_t cap, const int32_t* len, int off
     return;
   }
   const int prob = lb * Hkv + h;
+  if (!STD_DCHECK(pos0 + r < cap, err)) return;
   const size_t dof = ((size_t)prob * cap + pos0 + r) * row_bytes;
   const size_t so = ((size_t)prob * n_new + r) * row_bytes;
   copy_row(kc + dof, kn + so, row_bytes, lane);
@@ -91,6 +93,7 @@ commit_copy_kernel(const uint8_t* kf, const uint8_t* vf, uint8_t* ks, uint8_t* v
   }
   if (r >= n) return;
   const int prob = lb * Hkv + h;
+  if (!STD_DCHECK(a0 + r < cap_full && s0 + r < cap_sparse, err)) return;
   const size_t so = ((size_t)prob * cap_full + a0 + r) * row_bytes;
   const size_t dof = ((size_t)prob * cap_sparse + s0 + r) * row_bytes;
   copy_row(ks + dof, kf + so, row_bytes, lane);

@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(128) colsum_bf16_kernel(const ScoreArgs a) {
     const int n = key0 + tid;
     if (n < nv) {
       const float tot = (cbuf[tid] + cbuf[64 + tid]) + (cbuf[128 + tid] + cbuf[192 + tid]);
-      a.scores[(size_t)prob * a.nvis_max + n] = tot / (float)M;
+      if (STD_DCHECK(n < a.nvis_max, a.err)) a.scores[(size_t)prob * a.nvis_max + n] = tot / (float)M;
     }
   }
 }
@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(128) colsum_f32_kernel(const ScoreArgs a) {
     for (int j = 0; j < D; ++j) x = fmaf(qp[(size_t)r * D + j], k[j], x);
     acc += exp2f(x * sc - a.row_m[(size_t)prob * M + r]) / a.row_l[(size_t)prob * M + r];
   }
-  a.scores[(size_t)prob * a.nvis_max + n] = acc / (float)M;
+  if (STD_DCHECK(n < a.nvis_max, a.err)) a.scores[(size_t)prob * a.nvis_max + n] = acc / (float)M;
 }
 
 template <int D>
@@ -317,10 +317,14 @@ cudaError_t launch_f32_scores(const ScoreArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_select_scores(const ScoreArgs& a, cudaStream_t s) {
+cudaError_t launch_select_scores(const ScoreArgs& a, cudaStream_t s, bool* hist_done) {
+  *hist_done = false;
   if (a.dtype == STD_BF16) {
     const cudaError_t e = launch_select_scores_tc(a, s);  // tensor-core path
-    if (e != cudaErrorNotSupported) return e;
+    if (e != cudaErrorNotSupported) {
+      *hist_done = e == cudaSuccess && a.hist != nullptr;
+      return e;
+    }
     if (a.d == 128) return launch_bf16_scores<128>(a, s);
     if (a.d == 64) return launch_bf16_scores<64>(a, s);
   } else {

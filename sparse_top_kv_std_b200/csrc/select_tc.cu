@@ -204,6 +204,8 @@ rowstats_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const int prob = lb * a.Hkv + h;
   const int M = a.G * a.T;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // pass 2 counts the top digit of every score into this problem's histogram: clear it
+  if (a.hist && blockIdx.x == 0 && threadIdx.x < 256) a.hist[(size_t)prob * 256 + threadIdx.x] = 0u;
   int nv;
   if (!visual_ok(a, b, &nv)) {
     if (blockIdx.x == 0 && threadIdx.x == 0)
@@ -383,6 +385,9 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   float* xch = reinterpret_cast<float*>(smem + C::K_BYTES + C::QSTAGES * C::QC_BYTES + C::MW_BYTES);
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::K_BYTES + C::QSTAGES * C::QC_BYTES + C::MW_BYTES + C::XCH_BYTES);
 
+  // this CTA's counts of the top 8 bits of its scores' order keys (the top-K's first radix
+  // pass, done here while the scores are in registers), added to the problem's histogram
+  __shared__ uint32_t s_hist[256];
   const int h = blockIdx.y, lb = blockIdx.z, b = lb % a.B;
   const int prob = lb * a.Hkv + h;
   const int M = a.G * a.T;
@@ -393,6 +398,7 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int key_base = blockIdx.x * (kKeyBlocks * 256);
   if (key_base >= nv) return;
   const int nkb = min(kKeyBlocks, (nv - key_base + 255) / 256);
+  for (int i = threadIdx.x; i < 256; i += kThreads) s_hist[i] = 0u;  // ordered by the set-up barrier
 
   // row statistics of this head as -(m_r + log2 l_r); padding rows get -inf (2^-inf = 0 on the
   // SFU, 2^-125 ~ 2e-38 on the FMA pipe: negligible)
@@ -551,12 +557,23 @@ colsum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const float total = colsum + x[kl];
         tc::mbar_arrive(&ctl->xempty[blk * 2 + slot]);
         const int n = key_base + kbi * 256 + blk * BM + kl;
-        if (n < nv) a.scores[(size_t)prob * a.nvis_max + n] = total * invM;
+        const bool valid = n < nv && STD_DCHECK(n < a.nvis_max, a.err);
+        const float score = total * invM;
+        if (valid) a.scores[(size_t)prob * a.nvis_max + n] = score;
+        if (a.hist) {  // lanes with the same digit add once, as a group
+          const uint32_t digit = valid ? score_order_key(score) >> 24 : 256u;
+          const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+          if (valid && lane == __ffs(peers) - 1) atomicAdd(&s_hist[digit], (uint32_t)__popc(peers));
+        }
       }
     }
   }
   tc::fence_before_sync();
   __syncthreads();
+  if (a.hist) {
+    for (int i = threadIdx.x; i < 256; i += kThreads)
+      if (s_hist[i]) atomicAdd(&a.hist[(size_t)prob * 256 + i], s_hist[i]);
+  }
   if (warp == 1) {
     __syncwarp();
     tc::fence_after_sync();

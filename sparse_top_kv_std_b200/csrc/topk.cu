@@ -19,16 +19,13 @@ namespace {
 constexpr int TOPK_THREADS = 1024;
 constexpr int TOPK_WARPS = TOPK_THREADS / 32;
 
-// Larger float -> larger key; -0.0 maps like +0.0.
-__device__ __forceinline__ uint32_t order_key(float x) {
-  uint32_t u = __float_as_uint(x);
-  if (u == 0x80000000u) u = 0u;
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
+__device__ __forceinline__ uint32_t order_key(float x) { return score_order_key(x); }
 
+// hist0 (optional): [rows][256] counts of the top 8 key bits of every row's n entries, made
+// while the scores were written; the first radix pass then reads it instead of the scores.
 __global__ void __launch_bounds__(TOPK_THREADS)
 topk_kernel(const float* scores, int64_t stride, const int32_t* n_dev, int n_const, int n_div,
-            int n_mod, int K, int32_t* idx, int* err) {
+            int n_mod, int K, int32_t* idx, const uint32_t* hist0, int* err) {
   pdl_wait();  // memory of earlier kernels in the stream is visible from here on
   pdl_trigger();
   __shared__ uint32_t hist[256];
@@ -59,9 +56,13 @@ topk_kernel(const float* scores, int64_t stride, const int32_t* n_dev, int n_con
     for (int i = tid; i < 256; i += TOPK_THREADS) hist[i] = 0u;
     __syncthreads();
     const uint32_t prefix = s_prefix, mask = s_mask;
-    for (int i = tid; i < n; i += TOPK_THREADS) {
-      const uint32_t k = order_key(row[i]);
-      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+    if (shift == 24 && hist0) {
+      for (int i = tid; i < 256; i += TOPK_THREADS) hist[i] = hist0[(size_t)p * 256 + i];
+    } else {
+      for (int i = tid; i < n; i += TOPK_THREADS) {
+        const uint32_t k = order_key(row[i]);
+        if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+      }
     }
     __syncthreads();
     if (tid == 0) {
@@ -122,20 +123,23 @@ topk_kernel(const float* scores, int64_t stride, const int32_t* n_dev, int n_con
     const int eq_rank = eq_seen + __popc(eq_bits & lt_mask);
     const bool take = valid && (k > tau || (is_eq && eq_rank < need_eq));
     const uint32_t take_bits = __ballot_sync(0xffffffffu, take);
-    if (take) out[out_pos + __popc(take_bits & lt_mask)] = i;
+    if (take && STD_DCHECK(out_pos + __popc(take_bits & lt_mask) < K && i < n, err))
+      out[out_pos + __popc(take_bits & lt_mask)] = i;
     out_pos += __popc(take_bits);
     eq_seen += __popc(eq_bits);
   }
+  // every warp's output run ends where the next one starts, the last one at K
+  (void)STD_DCHECK(out_pos == (warp + 1 < TOPK_WARPS ? w_out_before[warp + 1] : K), err);
 }
 
 }  // namespace
 
 cudaError_t launch_topk(const float* scores, int64_t stride, int rows, const int32_t* n_dev,
-                        int n_const, int n_div, int n_mod, int K, int32_t* idx, int* err,
+                        int n_const, int n_div, int n_mod, int K, int32_t* idx, const uint32_t* hist0, int* err,
                         cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   return launch_pdl(topk_kernel, dim3(rows), dim3(TOPK_THREADS), 0, s, scores, stride, n_dev, n_const, n_div, n_mod, K,
-                    idx, err);
+                    idx, hist0, err);
 }
 
 }  // namespace stdb

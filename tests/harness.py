@@ -61,3 +61,43 @@ def session_for(wl, K=None, gamma=None, splits_draft=0, splits_verify=0):
     return DecodeSession(wl.L, wl.B, wl.Hq, wl.Hkv, wl.d, dtype_code(wl), wl.cap_full, wl.cap_sparse,
                          wl.T, wl.K if K is None else K, wl.gamma if gamma is None else gamma,
                          wl.nvis_max, splits_draft, splits_verify)
+
+
+# ----------------------------------------------------------------------------- canaries
+
+GUARD_BYTES = 256
+_GUARD_BYTE = 0xA5
+
+
+class Canaries:
+    """Device buffers with GUARD_BYTES of a fixed byte pattern before and after each one:
+    a kernel that writes past either end of an output or workspace changes the pattern,
+    which check() reports (a cheap stand-in for a memory checker)."""
+
+    def __init__(self):
+        self._bufs = []
+
+    def tensor(self, shape, dtype, fill=None):
+        import math
+        n = math.prod(shape) * torch.empty((), dtype=dtype).element_size()
+        raw = torch.full((GUARD_BYTES * 2 + n,), _GUARD_BYTE, dtype=torch.uint8, device="cuda")
+        inner = raw[GUARD_BYTES:GUARD_BYTES + n].view(dtype).view(shape)
+        if fill is not None:
+            inner.fill_(fill)
+        self._bufs.append((raw, n))
+        return inner
+
+    def like(self, t, fill=None):
+        c = self.tensor(tuple(t.shape), t.dtype)
+        c.copy_(t)
+        if fill is not None:
+            c.fill_(fill)
+        return c
+
+    def check(self):
+        torch.cuda.synchronize()
+        for i, (raw, n) in enumerate(self._bufs):
+            head = raw[:GUARD_BYTES]
+            tail = raw[GUARD_BYTES + n:]
+            assert bool((head == _GUARD_BYTE).all()), f"buffer {i}: bytes before it were overwritten"
+            assert bool((tail == _GUARD_BYTE).all()), f"buffer {i}: bytes after it were overwritten"

@@ -129,6 +129,8 @@ def test_binding_constants_match_the_header():
     the built-in scratch size of the no-alloc verify) have the header's values."""
     src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
     values = {n: int(v) for n, v in re.findall(r"\b(STD_[A-Z0-9_]+)\s*=\s*(-?\d+)", src)}
+    values.update({n: int(v) for n, v in re.findall(r"#define\s+(STD_[A-Z0-9_]+)\s+(-?\d+)\s*$", src, re.M)})
+    assert "STD_ATTN_EARLY_KV" in values and "STD_DEVERR_DEBUG" in values
     shift = re.search(r"#define\s+STD_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", src)
     assert shift, "STD_NOALLOC_SCRATCH_BYTES must stay of the form (a << b)"
     values["STD_NOALLOC_SCRATCH_BYTES"] = int(shift.group(1)) << int(shift.group(2))

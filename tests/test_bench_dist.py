@@ -147,8 +147,11 @@ def test_draft_launch_modes_issue_per_layer_slices(monkeypatch):
     fake = types.SimpleNamespace(
         dims=lambda *a: ("dims",) + a,
         std_get_device_error=lambda clear=True: 0,
+        STD_ATTN_EARLY_KV=1,
         std_sparse_decode_attn_append=lambda dims, q, k, v, ln, off, kn, vn, o, sp, ws: calls.append(
-            (dims, q, k, v, ln, off, kn, vn, o)))
+            (dims, q, k, v, ln, off, kn, vn, o, None)),
+        std_sparse_decode_attn_append_ex=lambda dims, q, k, v, ln, off, kn, vn, o, sp, fl, ws: calls.append(
+            (dims, q, k, v, ln, off, kn, vn, o, fl)))
     wl = types.SimpleNamespace(L=L, B=Bn, Hq=Hq, Hkv=Hkv, d=d, K=K, T=T, cap_full=20, cap_sparse=12)
     sess = types.SimpleNamespace(dims="batched-dims", k_sparse=torch.zeros(L, Bn, Hkv, 12, d),
                                  v_sparse=torch.ones(L, Bn, Hkv, 12, d), len_sparse=torch.zeros(Bn, dtype=torch.int32))
@@ -157,17 +160,21 @@ def test_draft_launch_modes_issue_per_layer_slices(monkeypatch):
     res = bench.draft_launch_modes(fake, sess, wl, 1, q, kn, vn, o, None, None, reps=2)
     assert "error" not in res, res
     assert sess.len_sparse.tolist() == [K + T]
-    # batched: 1 + 2 calls; per-layer eager: (1 + 2) x L; graph: capture L, then 1 + 2 replays of L
-    assert len(calls) == 3 + 3 * L + 3 * L
+    # batched: 1 + 2 calls; per-layer eager: (1 + 2) x L; each of the two graphs: capture L, then
+    # 1 + 2 replays of L (the second graph's launches fetch K/V early)
+    assert len(calls) == 3 + 3 * L + 3 * L + 3 * L
     assert res["launches_per_step"] == {"batched": 1, "per_layer": L}
     assert res["batched_us"] == res["per_layer_eager_us"] == res["per_layer_graph_us"] == 1e3
+    assert res["per_layer_graph_early_kv_us"] == 1e3
+    assert [c[9] for c in calls[3:3 + 6 * L]] == [0] * (6 * L)
+    assert [c[9] for c in calls[3 + 6 * L:]] == [1] * (3 * L)
     first = calls[0]
     assert first[0] == "batched-dims" and first[1] is q and first[5] == 1
     for l, c in enumerate(calls[3:3 + L]):
         assert c[0][:3] == ("dims", 1, Bn)                  # one layer per launch
         for got, full in zip((c[1], c[2], c[3], c[6], c[7], c[8]), (q, sess.k_sparse, sess.v_sparse, kn, vn, o)):
             assert got.data_ptr() == full[l].data_ptr() and got.shape == full.shape[1:]
-    replayed = calls[3 + 3 * L:]
+    replayed = calls[3 + 3 * L:3 + 6 * L]
     assert [c[1].data_ptr() for c in replayed] == [q[l].data_ptr() for l in range(L)] * 3
     # a failing library call is reported, not raised
     fake.std_sparse_decode_attn_append = lambda *a: (_ for _ in ()).throw(RuntimeError("boom"))

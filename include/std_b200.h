@@ -215,8 +215,9 @@ int std_gather_sparse(const std_dims* dims, const void* k_full, const void* v_fu
  * head) problems form one sequence that the CTAs split into equal slices;
  * `splits` = 0 launches one CTA per SM -- or one CTA per problem when there are
  * between half and all as many problems as SMs and `cap` is short (at most 2048
- * keys for up to 16 query rows, 8192 otherwise) -- and splits = s > 0 launches
- * s x L x B x Hkv CTAs.  fp32 operands (and bf16 with B > 64) use split-K
+ * keys for up to 16 query rows, 8192 otherwise), or, when all problems together
+ * have fewer than 4 tiles per SM (at `cap` keys), about one CTA per 4 tiles --
+ * and splits = s > 0 launches s x L x B x Hkv CTAs.  fp32 operands (and bf16 with B > 64) use split-K
  * kernels with `splits` key ranges per problem (0 = automatic).  Either way
  * the partial results go to the workspace.  The tensor-core kernel merges them
  * itself: the last CTA to finish a slice of a problem (an arrival counter per

@@ -162,10 +162,25 @@ int plan_attn(const std_dims* dims, int nq, int64_t cap, int splits, AttnPlan* p
       // heads, kernels timed alone): 7 query rows, 1024 keys 19.6 -> 14.7 us, 4352 keys
       // 48.6 -> 47.9 us but slower inside a decode step; 63 rows, 4352 keys 62.2 -> 50.4
       // us, 8192 keys 95.4 -> 85.9 us, 32768 keys 297 -> 328 us.  cap bounds the keys.
+      //
+      // With few tiles in all (a single layer's draft: 4 problems of ~35 tiles), one CTA per
+      // SM would cut every problem into dozens of one-tile segments whose partials the last
+      // CTA merges one batch after another; instead give each CTA about four tiles, so a
+      // problem has a handful of segments (28 launches of one layer's draft, 4 x 4352 keys,
+      // in a CUDA graph: 33 us each with 148 CTAs, 19 us with 32).
       int sms;
       STD_TRY(device_state(nullptr, &sms));
       const int64_t short_cap = a.rows <= 16 ? 2048 : 8192;
-      ctas = (probs <= sms && 2 * probs >= sms && cap <= short_cap) ? probs : sms;
+      const int64_t tiles_max = (int64_t)probs * ((cap + 127) / 128);
+      constexpr int64_t kMinTilesPerCta = 4;
+      if (probs <= sms && 2 * probs >= sms && cap <= short_cap) {
+        ctas = probs;
+      } else if (tiles_max < (int64_t)sms * kMinTilesPerCta) {
+        const int64_t c = (tiles_max + kMinTilesPerCta - 1) / kMinTilesPerCta;
+        ctas = (int)(c < probs ? probs : c);
+      } else {
+        ctas = sms;
+      }
     }
     a.splits = ctas;
     p->ws_bytes = stdb::attn_tc_ws_floats(probs, ctas, a.rows, a.d) * sizeof(float);

@@ -23,7 +23,7 @@
 // M = 64, which spreads the rows over all four TMEM lane quarters, so all four
 // SM sub-partitions share the softmax, two threads per row):
 //   TMA        K tile and V tile (128 keys x d, 128-byte swizzle) -> stage ring
-//   MMA        S = Q K^T  -> TMEM S buffer (double-buffered, 128 fp32 columns)
+//   MMA        S = Q K^T  -> TMEM S buffer (a ring of three, 128 fp32 columns each)
 //   softmax    row max, lazy rescale of O (only when the max grows by more than
 //              2^8), P = 2^(x - m) as bf16 written back over S in TMEM
 //   MMA        O += P V   (A = P from TMEM, B = V from shared memory, MN-major)
@@ -46,7 +46,9 @@ constexpr int kThreads = 192;
 constexpr int STAGES = 3;
 constexpr int kMaxB = 64;         // sequences per call handled by this kernel
 constexpr int kTmemCols = 512;
-constexpr uint32_t kColS = 128;   // TMEM column of S/P buffer 0 (buffer 1 at 256); O at column 0
+constexpr uint32_t kColS = 128;   // TMEM column of S/P buffer 0 (buffer b at 128 + 128 b); O at column 0
+constexpr int NSB = 3;            // S/P buffers: S of tile u + 1 is computed while tile u - 1's P V runs
+static_assert(kColS + NSB * 128 <= kTmemCols, "O and the S/P ring must fit the TMEM allocation");
 constexpr float kTau = 8.f;       // log2 growth of a row max that forces an O rescale
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kMergeSegs = 4;     // segments a merge loads per L2 round trip
@@ -54,7 +56,7 @@ constexpr int kMergeSegs = 4;     // segments a merge loads per L2 round trip
 struct Ctl {
   uint64_t kv_full[STAGES], kv_empty[STAGES];
   uint64_t q_full, q_empty, done;
-  uint64_t s_full[2], p_full[2], s_free[2];
+  uint64_t s_full[NSB], p_full[NSB], s_free[NSB];
   uint64_t o_ready, o_free;
   uint64_t pub, flag;  // partial published by all 128 row threads / merge decision made
   uint64_t nr_ready;   // fused append: the CTA's new cache rows are written (30 copy lanes)
@@ -336,7 +338,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc::mbar_init(&ctl->q_full, 1);
     tc::mbar_init(&ctl->q_empty, 1);
     tc::mbar_init(&ctl->done, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NSB; ++i) {
       tc::mbar_init(&ctl->s_full[i], 1);
       tc::mbar_init(&ctl->p_full[i], 128);
       tc::mbar_init(&ctl->s_free[i], 1);
@@ -502,8 +504,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       int pu = -1, ps = 0, pseg = 0;
       bool pfirst = false, any = false, ok = true;
       auto issue_pv = [&](int vu, int vs, bool vfirst, bool vlast, int vseg) -> bool {
-        const int vb = vu & 1;
-        if (!tc::mbar_wait(&ctl->p_full[vb], (vu >> 1) & 1, abort_flag, a.err)) return false;
+        const int vb = vu % NSB;
+        if (!tc::mbar_wait(&ctl->p_full[vb], (vu / NSB) & 1, abort_flag, a.err)) return false;
         if (vfirst && !tc::mbar_wait(&ctl->o_free, (vseg & 1) ^ 1, abort_flag, a.err)) return false;
         tc::fence_after_sync();
         const uint32_t p_tm = tmem + kColS + vb * 128;
@@ -526,8 +528,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int s = kv % STAGES;
         if (!tc::mbar_wait(&ctl->kv_full[s], (kv / STAGES) & 1, abort_flag, a.err)) { ok = false; break; }
         *(volatile int*)&ctl->consumed = kv + 1;
-        const int bu = u & 1;
-        if (!tc::mbar_wait(&ctl->s_free[bu], ((u >> 1) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
+        const int bu = u % NSB;
+        if (!tc::mbar_wait(&ctl->s_free[bu], ((u / NSB) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
         tc::fence_after_sync();
         const uint32_t s_tm = tmem + kColS + bu * 128;
         const uint32_t sk = sKV + s * C::ST_BYTES;
@@ -599,10 +601,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         lim = min(base + (row < a.rows ? row % a.nq : 0), a.row_end);
         lim_max = min(base + a.nq - 1, a.row_end);
       }
-      const int bu = u & 1;
+      const int bu = u % NSB;
       const int s = kv % STAGES;
       const int key0 = (it.t + ctl->tb) * TK;
-      if (!tc::mbar_wait_warp(&ctl->s_full[bu], (u >> 1) & 1, abort_flag, a.err)) break;
+      if (!tc::mbar_wait_warp(&ctl->s_full[bu], (u / NSB) & 1, abort_flag, a.err)) break;
       tc::fence_after_sync();
       if (key0 + TK > lim_max || key0 < a.row_begin) {
         // last tile of the problem (or first tile of a key range): zero the V rows past
@@ -683,7 +685,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const bool resc = (m != -INFINITY) && (mx - m) * sc > kTau;
         if (__any_sync(0xffffffffu, resc)) {
           // the previous tile's P V must have landed in O before O is rescaled
-          if (!tc::mbar_wait_warp(&ctl->s_free[(u - 1) & 1], ((u - 1) >> 1) & 1, abort_flag, a.err)) break;
+          // (u >= 1 here: a rescale needs an earlier tile of the same segment)
+          if (!tc::mbar_wait_warp(&ctl->s_free[(u - 1) % NSB], ((u - 1) / NSB) & 1, abort_flag, a.err)) break;
           tc::fence_after_sync();
           const float f = resc ? ex2((m - mx) * sc) : 1.f;
   #pragma unroll

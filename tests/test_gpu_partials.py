@@ -77,7 +77,7 @@ def test_verify_ranges_merge_to_full_verify(name, cuts):
     x = synth.host_inputs(wl, seed=7)
     kf, vf = _verify_inputs(wl, x)
     cap = wl.cap_full
-    cuts = tuple(cap if c is None else c for c in cuts)
+    cuts = tuple(cap if c is None else min(c, cap) for c in cuts)
     n_ctx = np.array(wl.nvis) + wl.T
     d = B.dims(wl.L, wl.B, wl.Hq, wl.Hkv, wl.d, B.STD_BF16, cap, wl.cap_sparse)
     q, kd, vd = H.to_dev(x["q_verify"][0]), H.to_dev(kf), H.to_dev(vf)

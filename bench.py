@@ -51,6 +51,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-draft-modes", action="store_true",
                     help="skip the draft launch-mode figures (batched / per layer / per-layer CUDA graph)")
     ap.add_argument("--threads", type=int, default=0, help="host threads for input generation")
+    ap.add_argument("--eager", action="store_true",
+                    help="issue every step's launches from the host instead of replaying a CUDA graph of one step")
     return ap.parse_args(argv)
 
 
@@ -487,20 +489,20 @@ def run_std(args, rank, world, local_rank):
         (selection and verify only, unless draft_ev: events between kernels cost overlap)."""
         sess.len_full.copy_(len0, non_blocking=True)
         if ev is not None:
-            ev["sel0"].record(stream)
+            ev["sel0"].record()
         sess.select(q_text, keep_scores=False)
         if ev is not None:
-            ev["sel1"].record(stream)
+            ev["sel1"].record()
         rounds(ev, draft_ev)
 
     def rounds(ev=None, draft_ev=False):
         for r in range(R):
             o = outs[r]
             if ev is not None and not draft_ev:
-                ev["dc0"][r].record(stream)
+                ev["dc0"][r].record()
             for j in range(wl.gamma):  # draft step j: append its input's row, attend (one launch)
                 if draft_ev:
-                    ev["d0"][r * wl.gamma + j].record(stream)
+                    ev["d0"][r * wl.gamma + j].record()
                 # steps after the first follow the previous step, which writes no length, no q and
                 # only the sparse row before this step's: they may start reading early (not after
                 # an event, which ends the overlap anyway)
@@ -509,26 +511,28 @@ def run_std(args, rank, world, local_rank):
                                                    sess.len_sparse, j + 1, view("k_draft", r)[j],
                                                    view("v_draft", r)[j], o["o_draft"][j], 0, flags, ws)
                 if draft_ev:
-                    ev["d1"][r * wl.gamma + j].record(stream)
+                    ev["d1"][r * wl.gamma + j].record()
             if ev is not None and not draft_ev:
-                ev["dc1"][r].record(stream)
+                ev["dc1"][r].record()
             B.std_kv_append(sess.dims, sess.k_full, sess.v_full, wl.cap_full, sess.len_full, 0,
                             view("k_verify", r), view("v_verify", r), wl.gamma + 1)
             if ev is not None:
-                ev["v0"][r].record(stream)
+                ev["v0"][r].record()
             B.std_dense_verify_attn(sess.dims, view("q_verify", r), wl.gamma, sess.k_full, sess.v_full,
                                     sess.len_full, o["o_verify"], 0, ws)
             if ev is not None:
-                ev["v1"][r].record(stream)
+                ev["v1"][r].record()
             B.std_accept_prefix(wl.B, wl.gamma, dv["draft_tokens"][r], dv["dense_tokens"][r], o["n_plus_1"],
                                 o["accepted"])
             B.std_kv_commit(sess.dims, sess.k_full, sess.v_full, sess.k_sparse, sess.v_sparse, sess.len_full,
                             sess.len_sparse, o["n_plus_1"], wl.gamma + 1)
         if ev is not None:
-            ev["end"].record(stream)
+            ev["end"].record()
 
-    def new_events():
-        E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    def new_events(external=False):
+        # external: recorded as event nodes when captured in a CUDA graph, so that every replay
+        # records them and their times can be read afterwards
+        E = lambda: torch.cuda.Event(enable_timing=True, external=external)  # noqa: E731
         return {"sel0": E(), "sel1": E(), "end": E(), "d0": [E() for _ in range(R * wl.gamma)],
                 "d1": [E() for _ in range(R * wl.gamma)], "v0": [E() for _ in range(R)],
                 "v1": [E() for _ in range(R)], "dc0": [E() for _ in range(R)], "dc1": [E() for _ in range(R)]}
@@ -547,8 +551,30 @@ def run_std(args, rank, world, local_rank):
     draft_b, verify_b, verify_round_b = attention_bytes(wl, R, accepted)
     step_attn = draft_b + verify_b
 
+    # ---- one step captured in a CUDA graph (as a serving loop runs its decode steps): the
+    # timed steps replay it, so the launches of a step are not issued one by one from Python.
+    # The library counts its launches while the graph is captured: that count per step is
+    # what every replay launches.
+    graph, graph_error, gev = None, None, None
+    if not args.eager:
+        try:
+            gev = new_events(external=True)
+            graph = torch.cuda.CUDAGraph()
+            n0 = B.std_launch_count()
+            with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+                step(gev)
+            per_step_launches = B.std_launch_count() - n0
+            graph.replay()  # one untimed replay
+            torch.cuda.synchronize()
+            flags = B.std_get_device_error(clear=True)
+            if flags:
+                raise RuntimeError(f"device error flags {flags:#x} in the graph replay")
+        except Exception as ex:  # the eager loop below still measures the step
+            graph, graph_error = None, f"{type(ex).__name__}: {ex}"
+            torch.cuda.synchronize()
+
     # ---- timed region
-    evs = [new_events() for _ in range(args.steps)]
+    evs = [gev] if graph is not None else [new_events() for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if pg:
         pg.barrier()
@@ -557,11 +583,14 @@ def run_std(args, rank, world, local_rank):
     launches0 = B.std_launch_count()  # the library's own count of the kernels it launches
     t0.record(stream)
     for i in range(args.steps):
-        step(evs[i])
+        if graph is not None:
+            graph.replay()  # the per-kernel events inside it keep the last replay's times
+        else:
+            step(evs[i])
     t1.record(stream)
     torch.cuda.synchronize()
     w1 = time.time()
-    launches = B.std_launch_count() - launches0
+    launches = per_step_launches * args.steps if graph is not None else B.std_launch_count() - launches0
     clocks = clk.stop(window=(w0, w1))
     if pg:
         pg.barrier()
@@ -687,6 +716,9 @@ def run_std(args, rank, world, local_rank):
                      "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                      "peak_source": f"{peak_src} HBM copy bandwidth"},
         "gpu_launches": launches,
+        "launch": ("one CUDA graph per step (captured once, replayed each step; the library's launch count is "
+                   "taken while capturing)" if graph is not None else "eager (host-issued launches)"
+                   + (f"; graph capture failed: {graph_error}" if graph_error else "")),
         "clocks": clocks,
         "e2e": e2e,
         "input_gen_s": t_gen,

@@ -906,19 +906,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           tc::mbar_arrive(&ctl->o_free);  // O may be reused: the rest reads global memory only
         }
         if (c0 != c1) {
-          // publish the partial, count the arrival; the last CTA merges every slot of the problem
-          __threadfence();
+          // publish the partial, count the arrival; the last CTA merges every slot of the problem.
+          // The CTA's partial writes reach thread 0 through the mbarrier (release / acquire in
+          // the CTA); thread 0's device-scope fence before the counter publishes them all, and
+          // its fence after the counter makes the other CTAs' partials visible to the merge,
+          // which the other threads order after through the second mbarrier.
           tc::mbar_arrive(&ctl->pub);
           if (tid == 0) {
             if (!tc::mbar_wait(&ctl->pub, npub & 1, abort_flag, a.err)) break;
             __threadfence();
             ctl->last_flag = arrive_last(ctr + prob, a.epoch, c1 - c0 + 1) ? 1 : 0;
+            if (ctl->last_flag) __threadfence();
             tc::mbar_arrive(&ctl->flag);
           }
           if (!tc::mbar_wait(&ctl->flag, npub & 1, abort_flag, a.err)) break;
           ++npub;
           if (ctl->last_flag && STD_DCHECK((size_t)prob + c1 < nslots && c0 <= c1, a.err)) {
-            __threadfence();
             // all 128 softmax threads share the merge
             merge_problem<D, HALF>(a.o, a.partial ? a.ml : nullptr, a.ws, wml, a.rows, (size_t)(prob + c0) * a.rows,
                                    c1 - c0 + 1, orow0, tid);

@@ -799,6 +799,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const float w = ex2(m * sc - ref);  // 0 for a quarter that saw no key
           // quarters 0 and 1 store w O into redA / redB, then quarters 2 and 3 add theirs: every
           // element is written by one thread at a time, in a fixed order
+          // (16-byte chunk k of a row is stored at chunk k ^ (row & 7): the eight rows a
+          // quarter-warp stores at once then fall in eight different bank groups)
           float* red = (qd & 1) ? redB : redA;
           if (qd < 2) {
 #pragma unroll
@@ -809,7 +811,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               tc::tmem_ld_wait(o);
               if (row < a.rows) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) red[row * D + hh * OC + c * 32 + j] = w * __uint_as_float(o[j]);
+                for (int j = 0; j < 8; ++j) {
+                  const int k = ((hh * OC + c * 32) / 4 + j) ^ (row & 7);
+                  *reinterpret_cast<float4*>(red + row * D + 4 * k) =
+                      make_float4(w * __uint_as_float(o[4 * j]), w * __uint_as_float(o[4 * j + 1]),
+                                  w * __uint_as_float(o[4 * j + 2]), w * __uint_as_float(o[4 * j + 3]));
+                }
               }
             }
           }
@@ -824,7 +831,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               tc::tmem_ld_wait(o);
               if (row < a.rows) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) red[row * D + hh * OC + c * 32 + j] += w * __uint_as_float(o[j]);
+                for (int j = 0; j < 8; ++j) {
+                  float4* dst = reinterpret_cast<float4*>(red + row * D + 4 * (((hh * OC + c * 32) / 4 + j) ^ (row & 7)));
+                  const float4 x = *dst;
+                  *dst = make_float4(x.x + w * __uint_as_float(o[4 * j]), x.y + w * __uint_as_float(o[4 * j + 1]),
+                                     x.z + w * __uint_as_float(o[4 * j + 2]), x.w + w * __uint_as_float(o[4 * j + 3]));
+                }
               }
             }
           }
@@ -835,8 +847,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           ++nx;
           for (int e = tid; e < a.rows * (D / 4); e += 128) {
             const int r = e / (D / 4), col = (e % (D / 4)) * 4;
-            const float4 xa = *reinterpret_cast<const float4*>(redA + r * D + col);
-            const float4 xb = *reinterpret_cast<const float4*>(redB + r * D + col);
+            const int sw = 4 * ((e % (D / 4)) ^ (r & 7));  // where the chunk of col sits
+            const float4 xa = *reinterpret_cast<const float4*>(redA + r * D + sw);
+            const float4 xb = *reinterpret_cast<const float4*>(redB + r * D + sw);
             const float4 x = make_float4(xa.x + xb.x, xa.y + xb.y, xa.z + xb.z, xa.w + xb.w);
             const float Mr = ctl->xrow[r][0], Lr = ctl->xrow[r][1];
             if (c0 == c1) {

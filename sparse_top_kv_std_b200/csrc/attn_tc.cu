@@ -972,6 +972,541 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   }
 }
 
+// ---------------------------------------------------------------------------
+// Keys-on-lanes layout (at most 16 query rows, d = 128: the draft step).  With a
+// handful of query rows the M = 64 MMAs above are mostly padding, so here every
+// MMA is transposed and the tile's 128 keys fill its M = 128 side:
+//   MMA      S^T = K Q^T     A = K tile, B = the 16-row query tile (both K-major)
+//                            -> TMEM S buffer: lane = key, column = query row
+//   softmax  thread t of the four softmax warps owns key t of the tile and reads
+//            its 16 logits; the warps combine their per-row maxima once per tile
+//            through shared memory (lazy rescale of O as above) and thread t writes
+//            P^T[row][t] as bf16 into a shared buffer [16 rows][128 keys]
+//   MMA      O^T += V^T P^T  A = V tile read MN-major, B = the P buffer (K-major)
+//                            -> TMEM O: lane = element of d, column = query row
+// One tile costs 16 MMAs of 128 x 16 x 16 instead of 16 of 64 x 128 x 16, each
+// softmax thread evaluates one exponential per real query row, and the segment end
+// needs no combine of lane quarters: thread t holds element t of every output row.
+struct CtlT : Ctl {
+  uint64_t xmax[2];      // per tile parity: the four warps' row maxima are in wmax
+  uint64_t xsum;         // segment end: the four warps' row sums are in wsum
+  alignas(16) float wmax[2][16][4];  // [tile parity][query row][softmax warp], read as float4
+  alignas(16) float wsum[16][4];
+};
+static_assert(alignof(CtlT) >= 16, "the float4 reads of wmax / wsum need 16-byte alignment");
+
+struct CfgT {
+  static constexpr int D = 128;
+  static constexpr int KB = D / 64;
+  static constexpr uint32_t Q_BYTES = KB * 16 * 128;   // 16 query rows
+  static constexpr uint32_t P_BYTES = 2 * 16 * 128;    // one P buffer: 16 rows x 128 keys, bf16
+  static constexpr uint32_t T_BYTES = KB * TK * 128;   // one K or V tile
+  static constexpr uint32_t ST_BYTES = 2 * T_BYTES;
+  static constexpr uint32_t KV_OFF = Q_BYTES + NSB * P_BYTES;
+  static constexpr uint32_t SMEM = 1024 + KV_OFF + STAGES * ST_BYTES + sizeof(CtlT);
+  static_assert(KV_OFF % 1024 == 0, "stages must start on a 1024-byte swizzle atom");
+  static_assert(SMEM <= 232448, "dynamic shared memory above the 227 KB a CTA may use");
+};
+constexpr int kTmemColsT = 64;     // O^T at columns 0..15, S^T buffer b at 16 + 16 b
+constexpr uint32_t kColST = 16;
+
+// Per-row sums of a warp's N values per lane (N = 8 or 16) over its 32 lanes.  Each
+// halving step keeps half of a lane's values (lane bit 4 picks the upper half, then bit
+// 3, ...) and adds its partner's; the lanes then sum the rest of the warp.  Afterwards
+// lane i * (32 / N) + j, j < 32 / N, holds the sum of value i.  Fixed order: the sums
+// are deterministic.
+template <int N>
+__device__ __forceinline__ float warp_row_sums(const float (&v)[N], int lane) {
+  float a[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) a[i] = v[i];
+  int bit = 16;
+#pragma unroll
+  for (int n = N; n > 1; n >>= 1, bit >>= 1) {
+    const bool hi = lane & bit;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i)
+      a[i] = (hi ? a[i + n / 2] : a[i]) + __shfl_xor_sync(0xffffffffu, hi ? a[i] : a[i + n / 2], bit);
+  }
+#pragma unroll
+  for (int b = (32 / N) / 2; b >= 1; b >>= 1) a[0] += __shfl_xor_sync(0xffffffffu, a[0], b);
+  return a[0];
+}
+
+// RT: query rows a softmax thread handles (8 or 16; rows up to RT of the 16-row tile)
+template <int RT>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k16,
+               const __grid_constant__ CUtensorMap tm_v16, const AttnArgs a) {
+  constexpr int D = 128;
+  using C = CfgT;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sQ = smem_u32(smem);
+  const uint32_t sP = sQ + C::Q_BYTES;
+  const uint32_t sKV = sQ + C::KV_OFF;
+  CtlT* ctl = reinterpret_cast<CtlT*>(smem + C::KV_OFF + STAGES * C::ST_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(&ctl->kv_full[s], 1);
+      tc::mbar_init(&ctl->kv_empty[s], 1);
+    }
+    tc::mbar_init(&ctl->q_full, 1);
+    tc::mbar_init(&ctl->q_empty, 1);
+    tc::mbar_init(&ctl->done, 1);
+    for (int i = 0; i < NSB; ++i) {
+      tc::mbar_init(&ctl->s_full[i], 1);
+      tc::mbar_init(&ctl->p_full[i], 128);
+      tc::mbar_init(&ctl->s_free[i], 1);
+    }
+    tc::mbar_init(&ctl->o_ready, 1);
+    tc::mbar_init(&ctl->o_free, 128);
+    tc::mbar_init(&ctl->pub, 128);
+    tc::mbar_init(&ctl->flag, 1);
+    tc::mbar_init(&ctl->nr_ready, 30);
+    tc::mbar_init(&ctl->xmax[0], 128);
+    tc::mbar_init(&ctl->xmax[1], 128);
+    tc::mbar_init(&ctl->xsum, 128);
+    ctl->abort_flag = 0;
+    ctl->consumed = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tc::tmem_alloc(&ctl->tmem, kTmemColsT);
+    tc::tmem_relinquish();
+  }
+  if (!a.early) {
+    pdl_wait();
+    pdl_trigger();
+  }
+  if (threadIdx.x == 0) {
+    int sum = 0;
+    for (int b = 0; b < a.B; ++b) {
+      ctl->tiles_b[b] = seq_tiles(a, b, blockIdx.x == 0);
+      ctl->len_b[b] = a.len[b];
+      ctl->pre_b[b] = a.Hkv * sum;
+      sum += ctl->tiles_b[b];
+    }
+    ctl->tl = a.Hkv * sum;
+    ctl->tb = a.row_begin / TK;
+    ctl->total = a.L * ctl->tl;
+    ctl->per = ctl->total > 0 ? (ctl->total + gridDim.x - 1) / gridDim.x : 1;
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = ctl->tmem;
+  volatile int* abort_flag = &ctl->abort_flag;
+  const int g0 = min(ctl->total, (int)blockIdx.x * ctl->per);
+  const int g1 = min(ctl->total, g0 + ctl->per);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producers
+    if (lane == 0 && g0 < g1) {
+      tc::prefetch_tmap(&tm_k);
+      tc::prefetch_tmap(&tm_v);
+      tc::prefetch_tmap(&tm_k16);
+      tc::prefetch_tmap(&tm_v16);
+      Iter it;
+      iter_seek(it, ctl, a, g0, g1);
+      int kv = 0;
+      bool rows_ready = a.k_new == nullptr;
+      bool waited = !a.early;
+      while (it.g < it.g_end) {
+        const int prob = (it.l * a.B + it.b) * a.Hkv + it.h;
+        const int s = kv % STAGES;
+        const int tabs = it.t + ctl->tb;
+        if (!waited && (tabs + 1) * TK > ctl->len_b[it.b] + a.new_off - 1) {
+          pdl_wait();
+          waited = true;
+        }
+        if (!rows_ready) {
+          const int p0 = ctl->len_b[it.b] + a.new_off;
+          if (tabs * TK < p0 + a.new_rows && p0 < (tabs + 1) * TK) {
+            if (!tc::mbar_wait(&ctl->nr_ready, 0, abort_flag, a.err)) break;
+            rows_ready = true;
+          }
+        }
+        if (!tc::mbar_wait(&ctl->kv_empty[s], ((kv / STAGES) & 1) ^ 1, abort_flag, a.err)) break;
+        if (!STD_DCHECK(tabs * TK < a.cap && prob < a.L * a.B * a.Hkv, a.err)) break;
+        const int row = prob * (int)a.cap + tabs * TK;
+        const uint32_t st = sKV + s * C::ST_BYTES;
+        const int nvalid = min(ctl->len_b[it.b] + a.len_off + a.nq - 1, a.row_end) - tabs * TK;
+        if (nvalid >= TK) {
+          tc::mbar_expect_tx(&ctl->kv_full[s], C::ST_BYTES);
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb) {
+            tc::tma_load_2d(st + kb * TK * 128, &tm_k, kb * 64, row, &ctl->kv_full[s]);
+            tc::tma_load_2d(st + C::T_BYTES + kb * TK * 128, &tm_v, kb * 64, row, &ctl->kv_full[s]);
+          }
+        } else {
+          const int nb = (nvalid + 15) >> 4;
+          tc::mbar_expect_tx(&ctl->kv_full[s], (uint32_t)nb * 16 * 128 * C::KB * 2);
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb) {
+            for (int i = 0; i < nb; ++i) {
+              tc::tma_load_2d(st + kb * TK * 128 + i * 16 * 128, &tm_k16, kb * 64, row + i * 16, &ctl->kv_full[s]);
+              tc::tma_load_2d(st + C::T_BYTES + kb * TK * 128 + i * 16 * 128, &tm_v16, kb * 64, row + i * 16,
+                              &ctl->kv_full[s]);
+            }
+          }
+        }
+        ++kv;
+        iter_next(it, ctl, a);
+      }
+      if (*abort_flag) {
+        for (int k = *(volatile int*)&ctl->consumed; k < kv; ++k) drain_wait(&ctl->kv_full[k % STAGES], (k / STAGES) & 1);
+      }
+    } else if (lane == 1 && g0 < g1) {
+      tc::prefetch_tmap(&tm_q);
+      Iter it;
+      iter_seek(it, ctl, a, g0, g1);
+      int seg = 0;
+      bool waited = !a.early;
+      while (it.g < it.g_end) {
+        if (it.first) {
+          if (!waited && !(a.early & STD_ATTN_EARLY_Q)) {
+            pdl_wait();
+            pdl_trigger();
+            waited = true;
+          }
+          if (!tc::mbar_wait(&ctl->q_empty, (seg & 1) ^ 1, abort_flag, a.err)) break;
+          tc::mbar_expect_tx(&ctl->q_full, C::Q_BYTES);
+          const int qrow = ((it.l * a.B + it.b) * a.Hq + it.h * a.G) * a.nq;
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb) tc::tma_load_2d(sQ + kb * 16 * 128, &tm_q, kb * 64, qrow, &ctl->q_full);
+          ++seg;
+          if (!waited) {
+            pdl_wait();
+            pdl_trigger();
+            waited = true;
+          }
+        }
+        iter_next(it, ctl, a);
+      }
+      if (*abort_flag && seg > 0) drain_wait(&ctl->q_full, (seg - 1) & 1);
+    } else if (lane >= 2 && g0 < g1 && a.k_new != nullptr) {
+      if (a.early) pdl_wait();
+      copy_new_rows<D>(a, ctl, g0, g1, lane - 2);
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      tc::mbar_arrive(&ctl->nr_ready);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && g0 < g1) {
+      constexpr uint32_t idS = tc::idesc_bf16(128, 16);               // S^T: M = keys, N = query rows
+      constexpr uint32_t idPV = tc::idesc_bf16(128, 16) | (1u << 15);  // O^T: A = V^T read MN-major
+      Iter it;
+      iter_seek(it, ctl, a, g0, g1);
+      int seg = -1, kv = 0, u = 0;
+      int pu = -1, ps = 0, pseg = 0;
+      bool pfirst = false, any = false, ok = true;
+      auto issue_pv = [&](int vu, int vs, bool vfirst, bool vlast, int vseg) -> bool {
+        const int vb = vu % NSB;
+        if (!tc::mbar_wait(&ctl->p_full[vb], (vu / NSB) & 1, abort_flag, a.err)) return false;
+        if (vfirst && !tc::mbar_wait(&ctl->o_free, (vseg & 1) ^ 1, abort_flag, a.err)) return false;
+        tc::fence_after_sync();
+        const uint32_t sp = sP + vb * C::P_BYTES;
+        const uint32_t sv = sKV + vs * C::ST_BYTES + C::T_BYTES;
+#pragma unroll
+        for (int k = 0; k < TK / 16; ++k)
+          tc::umma_bf16(tmem, tc::sdesc_sw128_mn(sv + k * 16 * 128, TK * 128),
+                        tc::sdesc_sw128(sp + (k >> 2) * 16 * 128 + (k & 3) * 32), idPV,
+                        (vfirst && k == 0) ? 0u : 1u);
+        tc::umma_commit(&ctl->kv_empty[vs]);
+        tc::umma_commit(&ctl->s_free[vb]);
+        if (vlast) tc::umma_commit(&ctl->o_ready);
+        return true;
+      };
+      while (it.g < it.g_end) {
+        const bool first = it.first, last = iter_last(it);
+        if (first) {
+          ++seg;
+          if (!tc::mbar_wait(&ctl->q_full, seg & 1, abort_flag, a.err)) { ok = false; break; }
+        }
+        const int s = kv % STAGES;
+        if (!tc::mbar_wait(&ctl->kv_full[s], (kv / STAGES) & 1, abort_flag, a.err)) { ok = false; break; }
+        *(volatile int*)&ctl->consumed = kv + 1;
+        const int bu = u % NSB;
+        if (!tc::mbar_wait(&ctl->s_free[bu], ((u / NSB) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
+        tc::fence_after_sync();
+        const uint32_t sk = sKV + s * C::ST_BYTES;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k & 3) * 32;
+          tc::umma_bf16(tmem + kColST + bu * 16, tc::sdesc_sw128(sk + (k >> 2) * TK * 128 + off),
+                        tc::sdesc_sw128(sQ + (k >> 2) * 16 * 128 + off), idS, k > 0 ? 1u : 0u);
+        }
+        any = true;
+        tc::umma_commit(&ctl->s_full[bu]);
+        if (last) tc::umma_commit(&ctl->q_empty);
+        if (pu >= 0) {
+          if (!issue_pv(pu, ps, pfirst, false, pseg)) { ok = false; break; }
+          pu = -1;
+        }
+        if (last) {
+          if (!issue_pv(u, s, first, true, seg)) { ok = false; break; }
+        } else {
+          pu = u;
+          ps = s;
+          pfirst = first;
+          pseg = seg;
+        }
+        ++u;
+        ++kv;
+        iter_next(it, ctl, a);
+      }
+      if (!ok && any) {
+        tc::umma_commit(&ctl->done);
+        drain_wait(&ctl->done, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax threads
+    const int w = warp & 3;               // TMEM lane quarter of this warp
+    const int tk = w * 32 + lane;         // this thread's key of every tile, and its element of d
+    const uint32_t lane_base = tmem + ((uint32_t)(w * 32) << 16);
+    const float sc = kLog2e * rsqrtf((float)D);
+    const int tid = threadIdx.x - 64;
+    // where this thread's P^T elements go: key tk of row r in the 128-byte-swizzled [16][64] block
+    const uint32_t p_off = (uint32_t)(tk >> 6) * 16 * 128 + (uint32_t)(tk & 7) * 2;
+    const int p_chunk = (tk & 63) >> 3;
+    // the P buffers start as zeros: rows RT..15 are never written and must contribute nothing
+    for (int i = tid; i < (int)(NSB * C::P_BYTES / 16); i += 128)
+      *reinterpret_cast<uint4*>(smem + C::Q_BYTES + i * 16) = make_uint4(0, 0, 0, 0);
+    tc::fence_proxy_async();
+    Iter it;
+    iter_seek(it, ctl, a, g0, g1);
+    int seg = -1, kv = 0, u = 0, npub = 0, nxs = 0;
+    float m[RT], l[RT];
+    int lim[RT];
+    int lim_max = 0;
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+      m[r] = -INFINITY;
+      l[r] = 0.f;
+      lim[r] = 0;
+    }
+    while (it.g < it.g_end) {
+      const bool first = it.first, last = iter_last(it);
+      const int lb = it.l * a.B + it.b;
+      const int prob = lb * a.Hkv + it.h;
+      if (first) {
+        ++seg;
+        const int base = a.len[it.b] + a.len_off;
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          m[r] = -INFINITY;
+          l[r] = 0.f;
+          lim[r] = r < a.rows ? min(base + r % a.nq, a.row_end) : 0;  // keys below lim[r] are attended
+        }
+        lim_max = min(base + a.nq - 1, a.row_end);
+      }
+      const int bu = u % NSB;
+      const int s = kv % STAGES;
+      const int key0 = (it.t + ctl->tb) * TK;
+      if (!tc::mbar_wait_warp(&ctl->s_full[bu], (u / NSB) & 1, abort_flag, a.err)) break;
+      tc::fence_after_sync();
+      if (key0 + TK > lim_max || key0 < a.row_begin) {
+        // zero the V rows past the last query's limit and before the range (0 * garbage
+        // could be NaN)
+        if (!tc::mbar_wait_warp(&ctl->kv_full[s], (kv / STAGES) & 1, abort_flag, a.err)) break;
+        const int z0 = max(0, lim_max - key0);
+        const int zb = a.row_begin - key0;
+        uint8_t* vb = smem + C::KV_OFF + s * C::ST_BYTES + C::T_BYTES;
+        for (int i = tid; i < C::KB * TK * 8; i += 128) {
+          const int r = (i >> 3) % TK;
+          if (r >= z0 || r < zb)
+            *reinterpret_cast<uint4*>(vb + (i / (TK * 8)) * TK * 128 + r * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+        }
+        tc::fence_proxy_async();
+      }
+      // this thread's key against the query rows
+      float v[RT];
+      {
+        uint32_t r16[16];
+        __syncwarp();
+        tc::tmem_ld_x16(lane_base + kColST + bu * 16, r16);
+        tc::tmem_ld_wait16(r16);
+        const int kc = key0 + tk;
+        const bool in_range = kc >= a.row_begin;
+#pragma unroll
+        for (int r = 0; r < RT; ++r) v[r] = (in_range && kc < lim[r]) ? __uint_as_float(r16[r]) : -INFINITY;
+      }
+      // row maxima of the tile: per warp (every lane gets them), then across the four warps
+      const int par = u & 1;
+      {
+        float mine = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          const float wm = warp_max_f32(v[r]);
+          mine = lane == r ? wm : mine;
+        }
+        if (lane < RT) ctl->wmax[par][lane][w] = mine;
+      }
+      tc::mbar_arrive(&ctl->xmax[par]);
+      if (!tc::mbar_wait_warp(&ctl->xmax[par], (u >> 1) & 1, abort_flag, a.err)) break;
+      bool need = false;
+      float f[RT];
+#pragma unroll
+      for (int r = 0; r < RT; ++r) {
+        const float4 q4 = *reinterpret_cast<const float4*>(ctl->wmax[par][r]);
+        const float mt = fmaxf(fmaxf(q4.x, q4.y), fmaxf(q4.z, q4.w));
+        // lazy rescale: only when the max grows by more than 2^kTau (the same decision in
+        // every thread: all see the same m and mt); branch-free
+        const float mr = m[r];
+        const bool fresh = mr == -INFINITY;
+        const bool resc = !fresh && (mt - mr) * sc > kTau;
+        f[r] = ex2(resc ? (mr - mt) * sc : 0.f);
+        need |= resc;
+        m[r] = (resc || fresh) ? mt : mr;
+      }
+      if (need) {
+        // the previous tile's P V must have landed in O before O is rescaled (u >= 1: a
+        // rescale needs an earlier tile of the same segment)
+        if (!tc::mbar_wait_warp(&ctl->s_free[(u - 1) % NSB], ((u - 1) / NSB) & 1, abort_flag, a.err)) break;
+        tc::fence_after_sync();
+        uint32_t o16[16];
+        __syncwarp();
+        tc::tmem_ld_x16(lane_base, o16);
+        tc::tmem_ld_wait16(o16);
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          o16[r] = __float_as_uint(__uint_as_float(o16[r]) * f[r]);
+          l[r] *= f[r];
+        }
+        __syncwarp();
+        tc::tmem_st_x16(lane_base, o16);
+        tc::tmem_st_wait();
+      }
+      // P^T[r][tk] = 2^(x - m) as bf16 into the tile's P buffer (a row that has seen no key
+      // yet has m = -inf and only -inf logits: its P is 2^-inf = 0)
+      {
+        uint8_t* pb = smem + C::Q_BYTES + bu * C::P_BYTES + p_off;
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          const float msc = (m[r] == -INFINITY ? 0.f : m[r]) * sc;
+          const float p = ex2(fmaf(v[r], sc, -msc));
+          l[r] += p;
+          *reinterpret_cast<__nv_bfloat16*>(pb + r * 128 + ((p_chunk ^ (r & 7)) << 4)) = __float2bfloat16_rn(p);
+        }
+      }
+      tc::fence_proxy_async();
+      tc::fence_before_sync();
+      tc::mbar_arrive(&ctl->p_full[bu]);
+      if (last) {
+        if (!tc::mbar_wait_warp(&ctl->o_ready, seg & 1, abort_flag, a.err)) break;
+        tc::fence_after_sync();
+        if (a.early) pdl_wait();  // outputs, partials and merge counters: after the previous kernel
+        // row sums over the 128 key threads
+        {
+          const float ws = warp_row_sums<RT>(l, lane);
+          if ((lane & (32 / RT - 1)) == 0) ctl->wsum[lane / (32 / RT)][w] = ws;
+        }
+        tc::mbar_arrive(&ctl->xsum);
+        if (!tc::mbar_wait_warp(&ctl->xsum, nxs & 1, abort_flag, a.err)) break;
+        ++nxs;
+        float L[RT];
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          const float4 q4 = *reinterpret_cast<const float4*>(ctl->wsum[r]);
+          L[r] = (q4.x + q4.y) + (q4.z + q4.w);
+        }
+        uint32_t o16[16];
+        __syncwarp();
+        tc::tmem_ld_x16(lane_base, o16);
+        tc::tmem_ld_wait16(o16);
+        tc::fence_before_sync();
+        tc::mbar_arrive(&ctl->o_free);  // O may be reused: the rest reads registers and global memory
+        // (m, L) of row tk, for the thread that writes them
+        float m_tk = 0.f, L_tk = 0.f;
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          m_tk = tk == r ? m[r] : m_tk;
+          L_tk = tk == r ? L[r] : L_tk;
+        }
+        const int start = it.l * ctl->tl + ctl->pre_b[it.b] + it.h * it.nt;
+        const int c0 = start / ctl->per, c1 = (start + it.nt - 1) / ctl->per;
+        const size_t orow0 = (size_t)(lb * a.Hq + it.h * a.G) * a.nq;
+        const size_t nslots = (size_t)a.L * a.B * a.Hkv + gridDim.x;
+        float* wml = a.ws + nslots * a.rows * D;
+        unsigned long long* ctr = reinterpret_cast<unsigned long long*>(wml + nslots * a.rows * 2);
+        const int slot = prob + blockIdx.x;
+        if (c0 == c1) {
+          // this CTA saw the whole problem: the output (partials: unnormalised, with (m, l))
+#pragma unroll
+          for (int r = 0; r < RT; ++r) {
+            if (r < a.rows) {
+              const float inv = a.partial ? 1.f : (L[r] > 0.f ? 1.f / L[r] : 0.f);
+              a.o[(orow0 + r) * D + tk] = __uint_as_float(o16[r]) * inv;
+            }
+          }
+          if (a.partial && tk < a.rows) {
+            a.ml[(orow0 + tk) * 2] = m_tk * rsqrtf((float)D);
+            a.ml[(orow0 + tk) * 2 + 1] = L_tk;
+          }
+        } else {
+          if (!STD_DCHECK((size_t)slot < nslots, a.err)) break;
+#pragma unroll
+          for (int r = 0; r < RT; ++r)
+            if (r < a.rows) a.ws[((size_t)slot * a.rows + r) * D + tk] = __uint_as_float(o16[r]);
+          if (tk < a.rows) {
+            wml[((size_t)slot * a.rows + tk) * 2] = m_tk * sc;
+            wml[((size_t)slot * a.rows + tk) * 2 + 1] = L_tk;
+          }
+          // publish the partial, count the arrival; the last CTA merges every slot of the
+          // problem (the same protocol as the kernel above)
+          tc::mbar_arrive(&ctl->pub);
+          if (tid == 0) {
+            if (!tc::mbar_wait(&ctl->pub, npub & 1, abort_flag, a.err)) break;
+            __threadfence();
+            ctl->last_flag = arrive_last(ctr + prob, a.epoch, c1 - c0 + 1) ? 1 : 0;
+            if (ctl->last_flag) __threadfence();
+            tc::mbar_arrive(&ctl->flag);
+          }
+          if (!tc::mbar_wait(&ctl->flag, npub & 1, abort_flag, a.err)) break;
+          ++npub;
+          if (ctl->last_flag && STD_DCHECK((size_t)prob + c1 < nslots && c0 <= c1, a.err)) {
+            merge_problem<D, true>(a.o, a.partial ? a.ml : nullptr, a.ws, wml, a.rows, (size_t)(prob + c0) * a.rows,
+                                   c1 - c0 + 1, orow0, tid);
+            if (tid == 0) atomicExch(ctr + prob, (unsigned long long)a.epoch << 32);  // ready for a replay
+          }
+        }
+      }
+      ++u;
+      ++kv;
+      iter_next(it, ctl, a);
+    }
+    if (a.partial && blockIdx.x == 0) {
+      // partials of a sequence with no key in the range: o = 0, m = -inf, l = 0
+      const int per_b = a.Hq * a.nq;
+      for (int b = 0; b < a.B; ++b) {
+        if (ctl->tiles_b[b] != 0) continue;
+        for (int i = tid; i < a.L * per_b * (D / 4); i += 128) {
+          const int l_ = i / (per_b * (D / 4)), rem = i % (per_b * (D / 4));
+          const size_t orow = (size_t)(l_ * a.B + b) * per_b + rem / (D / 4);
+          *reinterpret_cast<float4*>(a.o + orow * D + (rem % (D / 4)) * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (rem % (D / 4) == 0) {
+            a.ml[orow * 2] = -INFINITY;
+            a.ml[orow * 2 + 1] = 0.f;
+          }
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemColsT);
+  }
+}
+
 template <int D>
 cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   using C = Cfg<D>;
@@ -987,9 +1522,14 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
       !make_tmap_bf16_2d(&tk, a.k, D, krows, TK) || !make_tmap_bf16_2d(&tv, a.v, D, krows, TK) ||
       !make_tmap_bf16_2d(&tk16, a.k, D, krows, 16) || !make_tmap_bf16_2d(&tv16, a.v, D, krows, 16))
     return cudaErrorInvalidValue;
-  const int variant = split ? 2 : half ? 1 : 0;
-  auto kern = split ? attn_tc_kernel<D, true, true> : half ? attn_tc_kernel<D, true, false>
-                                                            : attn_tc_kernel<D, false, false>;
+  // d = 128 with at most 16 rows: the keys-on-lanes kernel; d = 64 keeps the quarter split
+  const bool keys_on_lanes = split && D == 128;
+  const int variant = keys_on_lanes ? (a.rows <= 8 ? 3 : 2) : split ? 2 : half ? 1 : 0;
+  auto kern = keys_on_lanes ? (a.rows <= 8 ? attn_tq_kernel<8> : attn_tq_kernel<16>)
+              : split       ? attn_tc_kernel<D, true, true>
+              : half        ? attn_tc_kernel<D, true, false>
+                            : attn_tc_kernel<D, false, false>;
+  const uint32_t smem_bytes = keys_on_lanes ? CfgT::SMEM : C::SMEM;
   // the shared-memory size is a per-device attribute of each kernel: set it once per device
   static std::atomic<uint64_t> attr_done{0};
   int dev = 0;
@@ -997,11 +1537,11 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const uint64_t bit = 1ull << ((dev & 15) * 4 + variant);
   if (!(attr_done.load(std::memory_order_acquire) & bit)) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(bit, std::memory_order_release);
   }
-  return launch_pdl(kern, dim3(a.splits), dim3(kThreads), C::SMEM, s, tq, tk, tv, tk16, tv16, a);
+  return launch_pdl(kern, dim3(a.splits), dim3(kThreads), smem_bytes, s, tq, tk, tv, tk16, tv16, a);
 }
 
 }  // namespace

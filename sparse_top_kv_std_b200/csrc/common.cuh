@@ -87,10 +87,17 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
 }
 
 // 2^x on the special-function unit (flushes subnormals; 2^-inf = 0).
+// (not volatile: no side effects, so the compiler may schedule, predicate or speculate it)
 __device__ __forceinline__ float ex2(float x) {
   float y;
-  asm volatile("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
+}
+// Maximum of v over the 32 lanes of the warp, in every lane (all lanes must be converged).
+__device__ __forceinline__ float warp_max_f32(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
 }
 
 // ---------------------------------------------------------------- packed fp32 pairs (sm_100)

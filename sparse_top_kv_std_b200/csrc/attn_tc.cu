@@ -1351,21 +1351,23 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc::mbar_arrive(&ctl->xmax[par]);
       if (!tc::mbar_wait_warp(&ctl->xmax[par], (u >> 1) & 1, abort_flag, a.err)) break;
       bool need = false;
-      float f[RT];
+      float mt[RT];
 #pragma unroll
       for (int r = 0; r < RT; ++r) {
         const float4 q4 = *reinterpret_cast<const float4*>(ctl->wmax[par][r]);
-        const float mt = fmaxf(fmaxf(q4.x, q4.y), fmaxf(q4.z, q4.w));
+        mt[r] = fmaxf(fmaxf(q4.x, q4.y), fmaxf(q4.z, q4.w));
         // lazy rescale: only when the max grows by more than 2^kTau (the same decision in
-        // every thread: all see the same m and mt); branch-free
-        const float mr = m[r];
-        const bool fresh = mr == -INFINITY;
-        const bool resc = !fresh && (mt - mr) * sc > kTau;
-        f[r] = ex2(resc ? (mr - mt) * sc : 0.f);
-        need |= resc;
-        m[r] = (resc || fresh) ? mt : mr;
+        // every thread: all see the same m and mt)
+        need |= m[r] != -INFINITY && (mt[r] - m[r]) * sc > kTau;
       }
       if (need) {
+        float f[RT];
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          const bool resc = m[r] != -INFINITY && (mt[r] - m[r]) * sc > kTau;
+          f[r] = resc ? ex2((m[r] - mt[r]) * sc) : 1.f;
+          m[r] = resc ? mt[r] : m[r];
+        }
         // the previous tile's P V must have landed in O before O is rescaled (u >= 1: a
         // rescale needs an earlier tile of the same segment)
         if (!tc::mbar_wait_warp(&ctl->s_free[(u - 1) % NSB], ((u - 1) / NSB) & 1, abort_flag, a.err)) break;
@@ -1383,6 +1385,8 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc::tmem_st_x16(lane_base, o16);
         tc::tmem_st_wait();
       }
+#pragma unroll
+      for (int r = 0; r < RT; ++r) m[r] = m[r] == -INFINITY ? mt[r] : m[r];  // first keys the row sees
       // P^T[r][tk] = 2^(x - m) as bf16 into the tile's P buffer (a row that has seen no key
       // yet has m = -inf and only -inf logits: its P is 2^-inf = 0)
       {

@@ -390,7 +390,17 @@ def workload_config(wl, R):
             "nvis": list(wl.nvis) if wl.B > 1 else wl.nvis[0], "T": wl.T, "K": wl.K, "gamma": wl.gamma,
             "rounds_per_step": R, "p_match": wl.p_match, "storage": wl.dtype,
             "step": f"prefill top-K selection + {R} draft/verify rounds (one StD decode)",
-            "l2": "inputs larger than L2 (no flush)" if kv_bytes(wl) > 126e6 else "L2-resident inputs"}
+            "l2": ("inputs larger than L2 (no flush)" if not needs_l2_flush(wl)
+                   else "L2 flushed before every timed step (256 MB written outside the step's events)")}
+
+
+# The KV cache must exceed the 126 MB L2 by a margin for back-to-back steps to start cold;
+# smaller workloads get the L2 overwritten between timed steps instead.
+L2_BYTES = 126e6
+
+
+def needs_l2_flush(wl):
+    return kv_bytes(wl) < 2 * L2_BYTES
 
 
 def kv_bytes(wl):
@@ -576,6 +586,10 @@ def run_std(args, rank, world, local_rank):
     # ---- timed region
     evs = [gev] if graph is not None else [new_events() for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # small workloads: overwrite L2 before every step, outside that step's own events
+    flush = torch.empty(int(2 * L2_BYTES), dtype=torch.uint8, device=dev) if needs_l2_flush(wl) else None
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)] if flush is not None else None
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
@@ -583,10 +597,15 @@ def run_std(args, rank, world, local_rank):
     launches0 = B.std_launch_count()  # the library's own count of the kernels it launches
     t0.record(stream)
     for i in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+            step_ev[i][0].record(stream)
         if graph is not None:
             graph.replay()  # the per-kernel events inside it keep the last replay's times
         else:
             step(evs[i])
+        if flush is not None:
+            step_ev[i][1].record(stream)
     t1.record(stream)
     torch.cuda.synchronize()
     w1 = time.time()
@@ -594,7 +613,7 @@ def run_std(args, rank, world, local_rank):
     clocks = clk.stop(window=(w0, w1))
     if pg:
         pg.barrier()
-    elapsed_ms = t0.elapsed_time(t1)
+    elapsed_ms = t0.elapsed_time(t1) if flush is None else sum(a.elapsed_time(b) for a, b in step_ev)
     flags = B.std_get_device_error(clear=True)
     if flags:
         raise RuntimeError(f"device error flags {flags:#x} in the timed region")
@@ -696,6 +715,8 @@ def run_std(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == B.STD_BF16 else "f32",
         "data": "synthetic", "config": workload_config(wl, R),
         "us_per_round": 1e3 * statistics.mean(rounds_ms) / R,
+        # the same draft + verify bytes over the rounds' own time (the step without its selection)
+        "rounds_GBps": step_attn / (statistics.mean(rounds_ms) / 1e3) / 1e9,
         "select_ms": sel_avg,
         "kernels": {
             "dense_verify_attn": {"ms_per_launch": v_avg_ms, "bytes_per_launch": v_bytes_avg,

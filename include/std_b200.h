@@ -179,6 +179,78 @@ int std_select_topk_ex(const std_dims* dims, const void* q_text, int T, const vo
 int std_topk_from_scores(const float* scores, int rows, int n, int K, int32_t* idx_out,
                          std_stream_t stream);
 
+/* ---------------------------------------------------------------- selection over a cache split by position
+ *
+ * When one sequence's prompt cache is split by position over several GPUs (one part
+ * each), the selection above runs in four steps with two exchanges between them, and
+ * gives the indices the single-GPU call gives (up to ties at the K-th score).  Per text
+ * row r of a problem the softmax over all visual keys is exp(x_rn - m_r) / l_r; split
+ * over parts, every part computes its own rows' (m, l) over its keys, the parts' values
+ * merge into the whole row's, every part scores its keys against the merged (m, l) --
+ * the same scores -- and keeps its own top-K, and the global top-K is the top-K of the
+ * parts' candidates (every one of its keys is among its own part's top-K):
+ *   1. std_select_rowstats on every part;          all-gather (row_m, row_l)
+ *   2. std_merge_rowstats on every part;
+ *      std_select_candidates on every part;        all-gather (cand_idx, cand_score)
+ *   3. std_merge_candidates on every part          (the global idx, ascending)
+ *   4. std_gather_sparse_part on every part;       all-reduce (sum) of the sparse caches
+ * The row statistics are in the exp2 domain: for the scaled logit x = q . k / sqrt(d),
+ * m = log2(e) * max_n x_n and l = sum_n 2^(log2(e) x_n - m).  Only the default score
+ * (flags 0: the softmax over the visual keys) splits this way.  A part's buffers hold
+ * the same per-(layer, sequence, KV head) layout as the full cache, restricted to the
+ * part's positions; every part must hold at least K visual keys of every sequence.
+ */
+
+/* Step 1: the row statistics of this part's visual keys: keys n < nvis[b] at rows
+ * n_prefix + n of k_full (this part's buffer; n_prefix here is the part's first visual
+ * row, nvis[b] its visual keys, 1 <= nvis[b] <= nvis_max, n_prefix + nvis_max <= cap_full).
+ * row_m, row_l  device float [L][B][Hkv][G * T], G = Hq / Hkv, row g * T + t. */
+int std_select_rowstats(const std_dims* dims, const void* q_text, int T, const void* k_full, const int32_t* nvis,
+                        int nvis_max, int n_prefix, float* row_m, float* row_l, std_stream_t stream);
+
+/* Step 2a: merge n_parts parts' row statistics, m_parts / l_parts device float
+ * [n_parts][n] (part-major, n = L * B * Hkv * G * T), into row_m / row_l [n]:
+ * m = max_i m_i, l = sum_i l_i 2^(m_i - m) (a part with l_i = 0 contributes nothing). */
+int std_merge_rowstats(int64_t n, int n_parts, const float* m_parts, const float* l_parts, float* row_m, float* row_l,
+                       std_stream_t stream);
+
+/* Device workspace bytes std_select_candidates needs (the part's scores). */
+size_t std_select_candidates_workspace_size(const std_dims* dims, int nvis_max);
+
+/* Step 2b: this part's scores against the merged row statistics (row_m, row_l from
+ * std_merge_rowstats) and its K highest: cand_idx device int32 [L][B][Hkv][K] (positions
+ * within the part's visual keys, ascending, ties to the lower position), cand_score device
+ * float [L][B][Hkv][K] their scores.  K <= nvis[b] is checked on the device
+ * (STD_DEVERR_K_RANGE).  scores_out: device float [L][B][Hkv][nvis_max] or NULL. */
+int std_select_candidates(const std_dims* dims, const void* q_text, int T, const void* k_full, const int32_t* nvis,
+                          int nvis_max, int n_prefix, const float* row_m, const float* row_l, int K,
+                          int32_t* cand_idx, float* cand_score, float* scores_out, void* ws, size_t ws_bytes,
+                          std_stream_t stream);
+
+/* Device workspace bytes std_merge_candidates needs. */
+size_t std_merge_candidates_workspace_size(const std_dims* dims, int n_parts, int K);
+
+/* Step 3: the global top-K from n_parts parts' candidates, cand_idx / cand_score device
+ * [n_parts][L][B][Hkv][K] (part-major; parts in increasing position order), and
+ * part_offset device int32 [n_parts][B]: the global visual index of each part's first
+ * visual key per sequence.  idx_out [L][B][Hkv][K] receives global visual indices of the
+ * K highest candidates, ties to the lower index, ascending -- what std_select_topk_ex
+ * gives on the whole cache (its ties to the lower position agree with the candidates'
+ * order because the parts come in position order). */
+int std_merge_candidates(const std_dims* dims, int n_parts, int K, const int32_t* cand_idx, const float* cand_score,
+                         const int32_t* part_offset, int32_t* idx_out, void* ws, size_t ws_bytes,
+                         std_stream_t stream);
+
+/* Step 4: std_gather_sparse on one part.  k_full / v_full hold the global cache positions
+ * [part_pos0, part_pos0 + part_rows) of the prompt [n_prefix rows | nvis[b] visual rows |
+ * T text rows] (dims->cap_full = the part buffer's capacity >= part_rows); idx and nvis
+ * are global (std_merge_candidates' output, the whole sequence's visual count).  Sparse
+ * rows whose source lies in this part are copied, the others written as zeros, so the
+ * parts' sparse caches sum (an all-reduce) to the one std_gather_sparse builds. */
+int std_gather_sparse_part(const std_dims* dims, const void* k_full, const void* v_full, const int32_t* nvis,
+                           const int32_t* idx, int K, int T, int n_prefix, int64_t part_pos0, int64_t part_rows,
+                           void* k_sparse, void* v_sparse, int32_t* len_sparse, std_stream_t stream);
+
 /* ---------------------------------------------------------------- streaming draft baseline
  *
  * Not the method's selection.  The gist.science summary ("Experimentelle

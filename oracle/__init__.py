@@ -13,12 +13,17 @@ from .std_oracle import (  # noqa: F401
     gather_sparse,
     kv_append,
     kv_commit,
+    merge_candidates,
     merge_partials,
+    merge_rowstats,
     select_topk,
     selection_scores,
+    selection_rowstats,
     selection_scores_causal,
+    selection_scores_given_rowstats,
     softmax,
     sparse_decode_attn,
     streaming_indices,
+    topk_candidates,
     topk_indices,
 )

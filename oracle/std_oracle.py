@@ -158,6 +158,61 @@ def select_topk(q_text: np.ndarray, k_full: np.ndarray, v_full: np.ndarray, nvis
     return idx, scores, k_sp, v_sp, lsp
 
 
+# --------------------------------------------------------------------------- selection over parts [P-M4]
+#
+# The selection score of [P-M4] for a cache split by position into parts (one per GPU).
+# Each text row's softmax over all visual keys is exp(x_n - m) / l with m the row's
+# maximum and l its sum of exp(x_n - m); a part can form its rows' (m, l) over its own
+# keys, the parts' pairs give the whole row's, and each part then scores its own keys
+# with the whole row's (m, l).  The global top-K keys are each among their own part's
+# top-K, so the top-K of the parts' candidates is the selection.
+
+def selection_rowstats(q_text: np.ndarray, k_vis: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Per text row of one (layer, KV head) over the given visual keys: m[r] = max_n
+    x_rn and l[r] = sum_n exp(x_rn - m[r]), x = q . k / sqrt(d).  q_text [G, T, d],
+    k_vis [n, d]; returns (m, l), each [G * T], fp64."""
+    q = np.asarray(q_text, np.float64).reshape(-1, q_text.shape[-1])
+    x = (q @ np.asarray(k_vis, np.float64).T) / math.sqrt(q.shape[-1])
+    m = x.max(axis=1)
+    return m, np.exp(x - m[:, None]).sum(axis=1)
+
+
+def merge_rowstats(ms, ls) -> Tuple[np.ndarray, np.ndarray]:
+    """(m, l) over the union of the parts' keys from each part's (m_i, l_i): m = max_i m_i,
+    l = sum_i l_i exp(m_i - m)."""
+    ms = np.asarray(ms, np.float64)
+    ls = np.asarray(ls, np.float64)
+    m = ms.max(axis=0)
+    return m, (ls * np.exp(ms - m)).sum(axis=0)
+
+
+def selection_scores_given_rowstats(q_text: np.ndarray, k_vis: np.ndarray, m: np.ndarray,
+                                    l: np.ndarray) -> np.ndarray:
+    """The selection score of the given keys when (m, l) are the whole rows' statistics:
+    score[n] = mean over rows r of exp(x_rn - m[r]) / l[r].  With (m, l) over exactly these
+    keys this is selection_scores."""
+    q = np.asarray(q_text, np.float64).reshape(-1, q_text.shape[-1])
+    x = (q @ np.asarray(k_vis, np.float64).T) / math.sqrt(q.shape[-1])
+    return (np.exp(x - m[:, None]) / l[:, None]).mean(axis=0)
+
+
+def topk_candidates(scores: np.ndarray, K: int) -> Tuple[np.ndarray, np.ndarray]:
+    """A part's candidates: its K highest scores' positions (ties to the lower position,
+    ascending) and those scores."""
+    idx = topk_indices(scores, K)
+    return idx, np.asarray(scores)[idx]
+
+
+def merge_candidates(parts, K: int) -> np.ndarray:
+    """The top-K of the parts' candidates.  parts: (offset, idx, score) per part, offset the
+    global index of the part's first key; returns the K highest candidates' global indices,
+    ties to the lower global index, ascending.  int32."""
+    gidx = np.concatenate([np.asarray(i, np.int64) + off for off, i, _ in parts])
+    sc = np.concatenate([np.asarray(v, np.float64) for _, _, v in parts])
+    order = np.lexsort((gidx, -sc))   # primary: score descending; then global index ascending
+    return np.sort(gidx[order[:K]]).astype(np.int32)
+
+
 # --------------------------------------------------------------------------- streaming draft baseline
 
 def streaming_indices(nv: int, K: int, n_sink: int) -> np.ndarray:

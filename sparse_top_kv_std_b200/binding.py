@@ -74,6 +74,13 @@ SIGNATURES = {
     "std_topk_from_scores": (_I, [_P, _I, _I, _I, _P, _P]),
     "std_streaming_indices": (_I, [_DP, _P, _I, _I, _P, _P]),
     "std_gather_sparse": (_I, [_DP, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P]),
+    "std_select_rowstats": (_I, [_DP, _P, _I, _P, _P, _I, _I, _P, _P, _P]),
+    "std_merge_rowstats": (_I, [_I64, _I, _P, _P, _P, _P, _P]),
+    "std_select_candidates_workspace_size": (_SZ, [_DP, _I]),
+    "std_select_candidates": (_I, [_DP, _P, _I, _P, _P, _I, _I, _P, _P, _I, _P, _P, _P, _P, _SZ, _P]),
+    "std_merge_candidates_workspace_size": (_SZ, [_DP, _I, _I]),
+    "std_merge_candidates": (_I, [_DP, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
+    "std_gather_sparse_part": (_I, [_DP, _P, _P, _P, _P, _I, _I, _I, _I64, _I64, _P, _P, _P, _P]),
     "std_attn_workspace_size": (_SZ, [_DP, _I, _I64, _I]),
     "std_attn_splits": (_I, [_DP, _I, _I64, _I]),
     "std_sparse_decode_attn": (_I, [_DP, _P, _P, _P, _P, _I, _P, _I, _P, _SZ, _P]),
@@ -215,6 +222,45 @@ def std_gather_sparse(d: StdDims, k_full, v_full, nvis, idx, K, T, k_sparse, v_s
                       n_prefix=0, stream=None) -> None:
     _check(lib().std_gather_sparse(ctypes.byref(d), _ptr(k_full), _ptr(v_full), _ptr(nvis), _ptr(idx), K, T,
                                    n_prefix, _ptr(k_sparse), _ptr(v_sparse), _ptr(len_sparse), _stream(stream)))
+
+
+# selection over a cache split by position (one part per GPU)
+
+def std_select_rowstats(d: StdDims, q_text, T, k_full, nvis, nvis_max, n_prefix, row_m, row_l, stream=None) -> None:
+    _check(lib().std_select_rowstats(ctypes.byref(d), _ptr(q_text), T, _ptr(k_full), _ptr(nvis), nvis_max, n_prefix,
+                                     _ptr(row_m), _ptr(row_l), _stream(stream)))
+
+
+def std_merge_rowstats(n, n_parts, m_parts, l_parts, row_m, row_l, stream=None) -> None:
+    _check(lib().std_merge_rowstats(n, n_parts, _ptr(m_parts), _ptr(l_parts), _ptr(row_m), _ptr(row_l),
+                                    _stream(stream)))
+
+
+def std_select_candidates_workspace_size(d: StdDims, nvis_max: int) -> int:
+    return lib().std_select_candidates_workspace_size(ctypes.byref(d), nvis_max)
+
+
+def std_select_candidates(d: StdDims, q_text, T, k_full, nvis, nvis_max, n_prefix, row_m, row_l, K, cand_idx,
+                          cand_score, scores_out, ws, stream=None) -> None:
+    _check(lib().std_select_candidates(ctypes.byref(d), _ptr(q_text), T, _ptr(k_full), _ptr(nvis), nvis_max, n_prefix,
+                                       _ptr(row_m), _ptr(row_l), K, _ptr(cand_idx), _ptr(cand_score),
+                                       _ptr(scores_out), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def std_merge_candidates_workspace_size(d: StdDims, n_parts: int, K: int) -> int:
+    return lib().std_merge_candidates_workspace_size(ctypes.byref(d), n_parts, K)
+
+
+def std_merge_candidates(d: StdDims, n_parts, K, cand_idx, cand_score, part_offset, idx_out, ws, stream=None) -> None:
+    _check(lib().std_merge_candidates(ctypes.byref(d), n_parts, K, _ptr(cand_idx), _ptr(cand_score), _ptr(part_offset),
+                                      _ptr(idx_out), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def std_gather_sparse_part(d: StdDims, k_full, v_full, nvis, idx, K, T, n_prefix, part_pos0, part_rows, k_sparse,
+                           v_sparse, len_sparse, stream=None) -> None:
+    _check(lib().std_gather_sparse_part(ctypes.byref(d), _ptr(k_full), _ptr(v_full), _ptr(nvis), _ptr(idx), K, T,
+                                        n_prefix, part_pos0, part_rows, _ptr(k_sparse), _ptr(v_sparse),
+                                        _ptr(len_sparse), _stream(stream)))
 
 
 def std_attn_workspace_size(d: StdDims, q_rows: int, cap: int, splits: int) -> int:

@@ -363,6 +363,167 @@ int std_select_topk_ex(const std_dims* dims, const void* q_text, int T, const vo
   return ok();
 }
 
+// ---------------------------------------------------------------- selection over parts
+
+namespace {
+
+// Checks shared by the two score steps of a part; fills the score arguments.
+int part_score_args(const std_dims* dims, const void* q_text, int T, const void* k_full, const int32_t* nvis,
+                    int nvis_max, int n_prefix, stdb::ScoreArgs* s) {
+  STD_TRY(check_dims(dims));
+  STD_TRY(check_ptr(q_text, 16, "q_text"));
+  STD_TRY(check_ptr(k_full, 16, "k_full"));
+  STD_TRY(check_ptr(nvis, 4, "nvis"));
+  if (T < 1) return fail(STD_ERR_INVALID_ARG, "T = %d must be >= 1", T);
+  if (nvis_max < 1) return fail(STD_ERR_INVALID_ARG, "nvis_max = %d must be >= 1", nvis_max);
+  if (n_prefix < 0) return fail(STD_ERR_INVALID_ARG, "n_prefix = %d must be >= 0", n_prefix);
+  if ((int64_t)n_prefix + nvis_max > dims->cap_full)
+    return fail(STD_ERR_CAPACITY, "n_prefix + nvis_max = %lld exceeds cap_full = %lld", (long long)n_prefix + nvis_max,
+                (long long)dims->cap_full);
+  int* err;
+  STD_TRY(device_state(&err, nullptr));
+  *s = stdb::ScoreArgs{};
+  s->q_text = q_text; s->k_full = k_full; s->nvis = nvis; s->nvis_max = nvis_max;
+  s->L = dims->L; s->B = dims->B; s->Hq = dims->Hq; s->Hkv = dims->Hkv; s->G = dims->Hq / dims->Hkv; s->T = T;
+  s->d = dims->d; s->dtype = dims->dtype; s->cap = dims->cap_full; s->err = err; s->prefix = n_prefix;
+  s->keys_only = 1;
+  return STD_OK;
+}
+
+}  // namespace
+
+int std_select_rowstats(const std_dims* dims, const void* q_text, int T, const void* k_full, const int32_t* nvis,
+                        int nvis_max, int n_prefix, float* row_m, float* row_l, std_stream_t stream) {
+  STD_NVTX_RANGE();
+  stdb::ScoreArgs s;
+  STD_TRY(part_score_args(dims, q_text, T, k_full, nvis, nvis_max, n_prefix, &s));
+  STD_TRY(check_ptr(row_m, 4, "row_m"));
+  STD_TRY(check_ptr(row_l, 4, "row_l"));
+  s.row_m = row_m; s.row_l = row_l; s.passes = 1;
+  bool hist_done = false;
+  cudaError_t e = stdb::launch_select_scores(s, stream, &hist_done);
+  if (e != cudaSuccess) return cuda_fail(e, "selection row-statistics launch");
+  return ok();
+}
+
+int std_merge_rowstats(int64_t n, int n_parts, const float* m_parts, const float* l_parts, float* row_m, float* row_l,
+                       std_stream_t stream) {
+  STD_NVTX_RANGE();
+  if (n < 1) return fail(STD_ERR_INVALID_ARG, "n = %lld must be >= 1", (long long)n);
+  if (n_parts < 1) return fail(STD_ERR_INVALID_ARG, "n_parts = %d must be >= 1", n_parts);
+  STD_TRY(check_ptr(m_parts, 4, "m_parts"));
+  STD_TRY(check_ptr(l_parts, 4, "l_parts"));
+  STD_TRY(check_ptr(row_m, 4, "row_m"));
+  STD_TRY(check_ptr(row_l, 4, "row_l"));
+  STD_TRY(device_state(nullptr, nullptr));
+  cudaError_t e = stdb::launch_merge_rowstats(m_parts, l_parts, n_parts, n, row_m, row_l, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "row-statistics merge launch");
+  return ok();
+}
+
+size_t std_select_candidates_workspace_size(const std_dims* dims, int nvis_max) {
+  if (check_dims(dims) || nvis_max < 1) return 0;
+  return (size_t)probs_of(dims) * nvis_max * sizeof(float) + 256;
+}
+
+int std_select_candidates(const std_dims* dims, const void* q_text, int T, const void* k_full, const int32_t* nvis,
+                          int nvis_max, int n_prefix, const float* row_m, const float* row_l, int K,
+                          int32_t* cand_idx, float* cand_score, float* scores_out, void* ws, size_t ws_bytes,
+                          std_stream_t stream) {
+  STD_NVTX_RANGE();
+  stdb::ScoreArgs s;
+  STD_TRY(part_score_args(dims, q_text, T, k_full, nvis, nvis_max, n_prefix, &s));
+  STD_TRY(check_ptr(row_m, 4, "row_m"));
+  STD_TRY(check_ptr(row_l, 4, "row_l"));
+  STD_TRY(check_ptr(cand_idx, 4, "cand_idx"));
+  STD_TRY(check_ptr(cand_score, 4, "cand_score"));
+  if (scores_out) STD_TRY(check_ptr(scores_out, 4, "scores_out"));
+  if (K < 1 || K > nvis_max) return fail(STD_ERR_INVALID_ARG, "K = %d must be in [1, nvis_max = %d]", K, nvis_max);
+  const size_t need = std_select_candidates_workspace_size(dims, nvis_max);
+  if (!scores_out && (!ws || ws_bytes < need))
+    return fail(STD_ERR_WORKSPACE, "candidate workspace: need %zu bytes, got %zu", need, ws ? ws_bytes : 0);
+  if (!scores_out) STD_TRY(check_ptr(ws, 16, "ws"));
+  float* scores = scores_out ? scores_out : static_cast<float*>(ws);
+  s.row_m = const_cast<float*>(row_m); s.row_l = const_cast<float*>(row_l); s.scores = scores; s.passes = 2;
+  bool hist_done = false;
+  cudaError_t e = stdb::launch_select_scores(s, stream, &hist_done);
+  if (e != cudaSuccess) return cuda_fail(e, "selection score launch");
+  const int probs = probs_of(dims);
+  e = stdb::launch_topk(scores, nvis_max, probs, nvis, 0, dims->Hkv, dims->B, K, cand_idx, nullptr, s.err, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "top-K launch");
+  e = stdb::launch_candidate_scores(scores, nvis_max, cand_idx, probs, K, cand_score, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "candidate score launch");
+  return ok();
+}
+
+size_t std_merge_candidates_workspace_size(const std_dims* dims, int n_parts, int K) {
+  if (check_dims(dims) || n_parts < 1 || K < 1) return 0;
+  // the candidates' scores per problem in part order, then the chosen positions
+  return (size_t)probs_of(dims) * ((size_t)n_parts * K * sizeof(float) + (size_t)K * sizeof(int32_t)) + 512;
+}
+
+int std_merge_candidates(const std_dims* dims, int n_parts, int K, const int32_t* cand_idx, const float* cand_score,
+                         const int32_t* part_offset, int32_t* idx_out, void* ws, size_t ws_bytes,
+                         std_stream_t stream) {
+  STD_NVTX_RANGE();
+  STD_TRY(check_dims(dims));
+  if (n_parts < 1) return fail(STD_ERR_INVALID_ARG, "n_parts = %d must be >= 1", n_parts);
+  if (K < 1) return fail(STD_ERR_INVALID_ARG, "K = %d must be >= 1", K);
+  if ((int64_t)n_parts * K > (1 << 30)) return fail(STD_ERR_INVALID_ARG, "n_parts * K too large");
+  STD_TRY(check_ptr(cand_idx, 4, "cand_idx"));
+  STD_TRY(check_ptr(cand_score, 4, "cand_score"));
+  STD_TRY(check_ptr(part_offset, 4, "part_offset"));
+  STD_TRY(check_ptr(idx_out, 4, "idx_out"));
+  const size_t need = std_merge_candidates_workspace_size(dims, n_parts, K);
+  if (!ws || ws_bytes < need)
+    return fail(STD_ERR_WORKSPACE, "candidate merge workspace: need %zu bytes, got %zu", need, ws ? ws_bytes : 0);
+  STD_TRY(check_ptr(ws, 16, "ws"));
+  int* err;
+  STD_TRY(device_state(&err, nullptr));
+  const int probs = probs_of(dims);
+  float* cat = static_cast<float*>(ws);
+  int32_t* pos = reinterpret_cast<int32_t*>(cat + (size_t)probs * n_parts * K);
+  cudaError_t e = stdb::launch_concat_candidates(cand_score, n_parts, probs, K, cat, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "candidate layout launch");
+  e = stdb::launch_topk(cat, (int64_t)n_parts * K, probs, nullptr, n_parts * K, 1, 1, K, pos, nullptr, err, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "top-K launch");
+  e = stdb::launch_map_candidates(pos, cand_idx, part_offset, n_parts, probs, K, dims->B, dims->Hkv, idx_out, err,
+                                  stream);
+  if (e != cudaSuccess) return cuda_fail(e, "candidate index launch");
+  return ok();
+}
+
+int std_gather_sparse_part(const std_dims* dims, const void* k_full, const void* v_full, const int32_t* nvis,
+                           const int32_t* idx, int K, int T, int n_prefix, int64_t part_pos0, int64_t part_rows,
+                           void* k_sparse, void* v_sparse, int32_t* len_sparse, std_stream_t stream) {
+  STD_NVTX_RANGE();
+  STD_TRY(check_dims(dims));
+  STD_TRY(check_ptr(k_full, 16, "k_full"));
+  STD_TRY(check_ptr(v_full, 16, "v_full"));
+  STD_TRY(check_ptr(nvis, 4, "nvis"));
+  STD_TRY(check_ptr(idx, 4, "idx"));
+  STD_TRY(check_ptr(k_sparse, 16, "k_sparse"));
+  STD_TRY(check_ptr(v_sparse, 16, "v_sparse"));
+  STD_TRY(check_ptr(len_sparse, 4, "len_sparse"));
+  if (K < 1 || T < 0 || n_prefix < 0) return fail(STD_ERR_INVALID_ARG, "need K >= 1, T >= 0, n_prefix >= 0");
+  if (part_pos0 < 0 || part_rows < 1 || part_rows > dims->cap_full)
+    return fail(STD_ERR_INVALID_ARG, "part [%lld, +%lld) must be non-empty and fit cap_full = %lld",
+                (long long)part_pos0, (long long)part_rows, (long long)dims->cap_full);
+  if ((int64_t)n_prefix + K + T > dims->cap_sparse)
+    return fail(STD_ERR_CAPACITY, "n_prefix + K + T = %lld exceeds cap_sparse = %lld", (long long)n_prefix + K + T,
+                (long long)dims->cap_sparse);
+  int* err;
+  STD_TRY(device_state(&err, nullptr));
+  stdb::GatherArgs g{};
+  g.k_full = k_full; g.v_full = v_full; g.k_sp = k_sparse; g.v_sp = v_sparse; g.idx = idx; g.nvis = nvis;
+  g.len_sparse = len_sparse; g.L = dims->L; g.B = dims->B; g.Hkv = dims->Hkv; g.T = T; g.K = K;
+  g.row_bytes = dims->d * elem_bytes(dims->dtype); g.cap_full = dims->cap_full; g.cap_sparse = dims->cap_sparse;
+  g.prefix = n_prefix; g.err = err; g.part_pos0 = part_pos0; g.part_rows = part_rows;
+  cudaError_t e = stdb::launch_gather(g, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+  return ok();
+}
+
 int std_streaming_indices(const std_dims* dims, const int32_t* nvis, int K, int n_sink, int32_t* idx_out,
                           std_stream_t stream) {
   STD_NVTX_RANGE();

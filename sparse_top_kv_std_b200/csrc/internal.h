@@ -105,6 +105,12 @@ struct ScoreArgs {
   // [prob][256]: counts of the top 8 bits of score_order_key over each problem's scores,
   // made by the tensor-core score pass as it writes the scores (the top-K's first radix pass)
   uint32_t* hist;
+  // which passes run: bit 0 the row statistics (into row_m / row_l), bit 1 the scores from
+  // the row statistics already there; 0 means both
+  int passes;
+  // nonzero: the buffer holds no text rows after the visual keys (one part of a cache split
+  // by position): the extent check is prefix + nvis <= cap (the default score reads no text key)
+  int keys_only;
 };
 // *hist_done: whether the path that ran filled a.hist (the tensor-core path does).
 cudaError_t launch_select_scores(const ScoreArgs& a, cudaStream_t s, bool* hist_done);
@@ -132,8 +138,25 @@ struct GatherArgs {
   int prefix;  // prompt rows before the visual block, copied first
   int64_t cap_full, cap_sparse;
   int* err;
+  // part_rows > 0: k_full / v_full hold only global cache positions [part_pos0, part_pos0 +
+  // part_rows) (cap_full is then that buffer's capacity); sparse rows whose source lies
+  // elsewhere are written as zeros, so that the parts' sparse caches sum to the whole one
+  int64_t part_pos0, part_rows;
 };
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s);
+// Selection split by position: merge of the parts' row statistics ([n_parts][n] each, exp2
+// domain: M = max m_i, L = sum l_i 2^(m_i - M)); each part's top-K candidates' scores
+// (cand_score[p][j] = scores[p * stride + idx[p][j]]); the parts' candidate scores laid out
+// per problem in part order (cat[p][i * K + j] = part_score[i][p][j]); and the merged
+// selection's positions in that layout mapped back to global visual indices.
+cudaError_t launch_merge_rowstats(const float* m_parts, const float* l_parts, int n_parts, int64_t n, float* m_out,
+                                  float* l_out, cudaStream_t s);
+cudaError_t launch_candidate_scores(const float* scores, int64_t stride, const int32_t* idx, int probs, int K,
+                                    float* cand_score, cudaStream_t s);
+cudaError_t launch_concat_candidates(const float* part_score, int n_parts, int probs, int K, float* cat,
+                                     cudaStream_t s);
+cudaError_t launch_map_candidates(const int32_t* pos, const int32_t* part_idx, const int32_t* part_offset, int n_parts,
+                                  int probs, int K, int B, int Hkv, int32_t* idx_out, int* err, cudaStream_t s);
 // Sink + recent-window index set: idx[prob][j] = j (j < n_sink), else nvis[b] - K + j.
 cudaError_t launch_streaming_indices(const int32_t* nvis, int L, int B, int Hkv, int K, int n_sink, int32_t* idx,
                                      int* err, cudaStream_t s);

@@ -16,6 +16,10 @@ __device__ __forceinline__ void copy_row(uint8_t* dst, const uint8_t* src, int b
     *reinterpret_cast<uint4*>(dst + off) = *reinterpret_cast<const uint4*>(src + off);
 }
 
+__device__ __forceinline__ void zero_row(uint8_t* dst, int bytes, int lane) {
+  for (int off = lane * 16; off < bytes; off += 32 * 16) *reinterpret_cast<uint4*>(dst + off) = make_uint4(0, 0, 0, 0);
+}
+
 // Sparse cache rows [0, K) <- full rows idx[0..K); rows [K, K + T) <- text rows.
 __global__ void __launch_bounds__(ROWS_PER_CTA * 32) gather_kernel(const GatherArgs a) {
   pdl_wait();  // memory of earlier kernels in the stream is visible from here on
@@ -25,7 +29,8 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) gather_kernel(const GatherA
   const int j = blockIdx.x * ROWS_PER_CTA + warp;
   const int prob = lb * a.Hkv + h;
   const int nv = a.nvis[b];
-  if (a.K > nv || (int64_t)a.prefix + nv + a.T > a.cap_full) {
+  // (a part holds only [part_pos0, part_pos0 + part_rows) of the cache: no extent check here)
+  if (a.K > nv || (a.part_rows == 0 && (int64_t)a.prefix + nv + a.T > a.cap_full)) {
     if (j == 0 && h == 0 && lane == 0) flag_error(a.err, STD_DEVERR_K_RANGE);
     return;
   }
@@ -43,9 +48,18 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) gather_kernel(const GatherA
   } else {
     src = a.prefix + nv + (j - a.prefix - a.K);
   }
+  const size_t dof = ((size_t)prob * a.cap_sparse + j) * a.row_bytes;
+  if (a.part_rows > 0) {
+    if (src < a.part_pos0 || src >= a.part_pos0 + a.part_rows) {  // another part's row: zeros here
+      zero_row(static_cast<uint8_t*>(a.k_sp) + dof, a.row_bytes, lane);
+      zero_row(static_cast<uint8_t*>(a.v_sp) + dof, a.row_bytes, lane);
+      if (blockIdx.x == 0 && h == 0 && blockIdx.z / a.B == 0 && threadIdx.x == 0) a.len_sparse[b] = a.prefix + a.K + a.T;
+      return;
+    }
+    src -= (int)a.part_pos0;
+  }
   if (!STD_DCHECK(src >= 0 && src < a.cap_full && j < a.cap_sparse, a.err)) return;
   const size_t so = ((size_t)prob * a.cap_full + src) * a.row_bytes;
-  const size_t dof = ((size_t)prob * a.cap_sparse + j) * a.row_bytes;
   copy_row(static_cast<uint8_t*>(a.k_sp) + dof, static_cast<const uint8_t*>(a.k_full) + so, a.row_bytes, lane);
   copy_row(static_cast<uint8_t*>(a.v_sp) + dof, static_cast<const uint8_t*>(a.v_full) + so, a.row_bytes, lane);
   if (blockIdx.x == 0 && h == 0 && blockIdx.z / a.B == 0 && threadIdx.x == 0) a.len_sparse[b] = a.prefix + a.K + a.T;

@@ -28,7 +28,7 @@ constexpr int P1_STAGES = 3;
 __device__ __forceinline__ bool visual_ok(const ScoreArgs& a, int b, int* nv_out) {
   const int nv = a.nvis[b];
   *nv_out = nv;
-  return nv >= 1 && nv <= a.nvis_max && (int64_t)a.prefix + nv + a.T <= a.cap;
+  return nv >= 1 && nv <= a.nvis_max && (int64_t)a.prefix + nv + (a.keys_only ? 0 : a.T) <= a.cap;
 }
 
 // Q fragments (m16n8k16 A operand) of 16 text rows starting at r_base.
@@ -300,8 +300,12 @@ cudaError_t launch_bf16_scores(const ScoreArgs& a, cudaStream_t s) {
   constexpr int smem1 = P1_STAGES * TKS * D * 2;
   cudaError_t e = cudaFuncSetAttribute(rowstats_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
   if (e != cudaSuccess) return e;
-  if ((e = launch_pdl(rowstats_bf16_kernel<D>, dim3((M + 63) / 64, a.Hkv, a.L * a.B), dim3(128), smem1, s, a)) != cudaSuccess) return e;
-  if (a.causal_text && (e = launch_text_rowstats(a, s)) != cudaSuccess) return e;
+  const int passes = a.passes ? a.passes : 3;
+  if ((passes & 1) &&
+      (e = launch_pdl(rowstats_bf16_kernel<D>, dim3((M + 63) / 64, a.Hkv, a.L * a.B), dim3(128), smem1, s, a)) != cudaSuccess)
+    return e;
+  if ((passes & 1) && a.causal_text && (e = launch_text_rowstats(a, s)) != cudaSuccess) return e;
+  if (!(passes & 2)) return cudaSuccess;
   constexpr int smem2 = TKS * D * 2;
   return launch_pdl(colsum_bf16_kernel<D>, dim3((a.nvis_max + TKS - 1) / TKS, a.Hkv, a.L * a.B), dim3(128), smem2, s, a);
 }
@@ -309,9 +313,13 @@ cudaError_t launch_bf16_scores(const ScoreArgs& a, cudaStream_t s) {
 template <int D>
 cudaError_t launch_f32_scores(const ScoreArgs& a, cudaStream_t s) {
   const int M = a.G * a.T;
-  cudaError_t e = launch_pdl(rowstats_f32_kernel<D>, dim3((M + 127) / 128, a.Hkv, a.L * a.B), dim3(128), 0, s, a);
-  if (e != cudaSuccess) return e;
-  if (a.causal_text && (e = launch_text_rowstats(a, s)) != cudaSuccess) return e;
+  const int passes = a.passes ? a.passes : 3;
+  cudaError_t e = cudaSuccess;
+  if ((passes & 1) &&
+      (e = launch_pdl(rowstats_f32_kernel<D>, dim3((M + 127) / 128, a.Hkv, a.L * a.B), dim3(128), 0, s, a)) != cudaSuccess)
+    return e;
+  if ((passes & 1) && a.causal_text && (e = launch_text_rowstats(a, s)) != cudaSuccess) return e;
+  if (!(passes & 2)) return cudaSuccess;
   return launch_pdl(colsum_f32_kernel<D>, dim3((a.nvis_max + 127) / 128, a.Hkv, a.L * a.B), dim3(128), 0, s, a);
 }
 

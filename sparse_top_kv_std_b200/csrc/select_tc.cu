@@ -65,7 +65,7 @@ struct Ctl {
 __device__ __forceinline__ bool visual_ok(const ScoreArgs& a, int b, int* nv_out) {
   const int nv = a.nvis[b];
   *nv_out = nv;
-  return nv >= 1 && nv <= a.nvis_max && (int64_t)a.prefix + nv + a.T <= a.cap;
+  return nv >= 1 && nv <= a.nvis_max && (int64_t)a.prefix + nv + (a.keys_only ? 0 : a.T) <= a.cap;
 }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -625,10 +625,14 @@ static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s) {
   e = cudaFuncSetAttribute(colsum_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, P2<D>::SMEM);
   if (e != cudaSuccess) return e;
   const int M = a.G * a.T;
-  e = launch_pdl(rowstats_tc_kernel<D>, dim3((M + BM - 1) / BM, a.Hkv, a.L * a.B), dim3(kP1Threads), P1<D>::SMEM, s,
-                 tq128, tk, a);
-  if (e != cudaSuccess) return e;
-  if (a.causal_text && (e = launch_text_rowstats(a, s)) != cudaSuccess) return e;
+  const int passes = a.passes ? a.passes : 3;
+  if (passes & 1) {
+    e = launch_pdl(rowstats_tc_kernel<D>, dim3((M + BM - 1) / BM, a.Hkv, a.L * a.B), dim3(kP1Threads), P1<D>::SMEM, s,
+                   tq128, tk, a);
+    if (e != cudaSuccess) return e;
+    if (a.causal_text && (e = launch_text_rowstats(a, s)) != cudaSuccess) return e;
+  }
+  if (!(passes & 2)) return cudaSuccess;
   return launch_pdl(colsum_tc_kernel<D>, dim3((a.nvis_max + kKeyBlocks * 256 - 1) / (kKeyBlocks * 256), a.Hkv,
                                               a.L * a.B),
                     dim3(kThreads), P2<D>::SMEM, s, tq128, tk, a);

@@ -507,6 +507,49 @@ def check_range_partials_vs_torch(orc, seed: int = 15) -> None:
     np.testing.assert_allclose(l1, l2, atol=1e-14)
 
 
+# ----------------------------------------------------------------------------- selection over parts
+
+def check_split_selection(orc, seed: int = 16) -> None:
+    """The selection over a cache split by position: each part's (m, l) against torch
+    (max, exp(logsumexp - max)); the parts' merged (m, l), the parts' scores against them
+    and the top-K of the parts' candidates against the whole-cache selection; the
+    candidates' tie rule on a hand-made case."""
+    import torch
+    rng = np.random.default_rng(seed)
+    G, T, d, nv = 3, 4, 8, 90
+    q = rng.standard_normal((G, T, d)) * 1.5
+    k = rng.standard_normal((nv, d)) * 1.5
+    k[17] += 3 * q[0, 0]                              # a salient key
+    whole = orc.selection_scores(q, k)
+    for cuts in ((0, 90), (0, 1, 90), (0, 30, 31, 64, 90), (0, 45, 89, 90), (0, 20, 55, 90), (0, 12, 90)):
+        ranges = list(zip(cuts[:-1], cuts[1:]))
+        stats = [orc.selection_rowstats(q, k[a:b]) for a, b in ranges]
+        for (a, b), (m, l) in zip(ranges, stats):
+            x = torch.from_numpy(q.reshape(-1, d)) @ torch.from_numpy(k[a:b]).T / math.sqrt(d)
+            mx = x.max(dim=1).values
+            np.testing.assert_allclose(m, mx.numpy(), atol=1e-12, rtol=0)
+            np.testing.assert_allclose(l, torch.exp(torch.logsumexp(x, 1) - mx).numpy(), rtol=1e-12)
+        m, l = orc.merge_rowstats([s[0] for s in stats], [s[1] for s in stats])
+        m0, l0 = orc.selection_rowstats(q, k)
+        np.testing.assert_allclose(m, m0, atol=1e-12, rtol=0)
+        np.testing.assert_allclose(l, l0, rtol=1e-12)
+        part_scores = [orc.selection_scores_given_rowstats(q, k[a:b], m, l) for a, b in ranges]
+        np.testing.assert_allclose(np.concatenate(part_scores), whole, rtol=1e-11)
+        smallest = min(b - a for a, b in ranges)   # every part holds at least K keys
+        for K in sorted({1, min(5, smallest), smallest}):
+            parts = []
+            for (a, b), sc in zip(ranges, part_scores):
+                idx, val = orc.topk_candidates(sc, K)
+                np.testing.assert_array_equal(idx, orc.topk_indices(sc, K))
+                np.testing.assert_array_equal(val, sc[idx])
+                parts.append((a, idx, val))
+            np.testing.assert_array_equal(orc.merge_candidates(parts, K), orc.topk_indices(whole, K))
+    # ties across parts go to the lower global index
+    parts = [(0, np.array([1, 2]), np.array([0.5, 0.3])), (10, np.array([0, 4]), np.array([0.5, 0.5]))]
+    np.testing.assert_array_equal(orc.merge_candidates(parts, 2), [1, 10])
+    np.testing.assert_array_equal(orc.merge_candidates(parts, 3), [1, 10, 14])
+
+
 ALL_CHECKS = [
     check_golden_attention, check_golden_verify, check_golden_draft_round, check_append_offsets,
     check_attention_vs_sdpa,
@@ -515,5 +558,5 @@ ALL_CHECKS = [
     check_selection_prefix, check_streaming_and_gather,
     check_topk_bruteforce, check_topk_special, check_full_k_sparse_equals_dense,
     check_golden_accept, check_accept_bruteforce, check_commit, check_round_lossless_extremes,
-    check_golden_partials, check_range_partials_vs_torch,
+    check_golden_partials, check_range_partials_vs_torch, check_split_selection,
 ]

@@ -182,6 +182,25 @@ def _range_ignores_pos0(q, k, v, limit, pos0, row_begin, row_end):
     return so.attn_range_partial(q, k, v, limit, 0, row_begin, row_end)
 
 
+def _merge_rowstats_no_rescale(ms, ls):
+    return np.max(ms, axis=0), np.sum(ls, axis=0)
+
+
+def _part_scores_own_stats(q_text, k_vis, m, l):
+    return so.selection_scores(q_text, k_vis)
+
+
+def _merge_candidates_ties_high(parts, K):
+    gidx = np.concatenate([np.asarray(i, np.int64) + off for off, i, _ in parts])
+    sc = np.concatenate([np.asarray(v, np.float64) for _, _, v in parts])
+    order = np.lexsort((-gidx, -sc))
+    return np.sort(gidx[order[:K]]).astype(np.int32)
+
+
+def _merge_candidates_local_idx(parts, K):
+    return so.merge_candidates([(0, i, v) for _, i, v in parts], K)
+
+
 MUTANTS = {
     "merge without the exp(m_k - M) rescale": _mutant(merge_partials=_merge_without_rescale),
     "partial returns the normalised output": _mutant(attend_partial=_partial_normalised),
@@ -207,6 +226,10 @@ MUTANTS = {
     "accept counts all matches": _mutant(accept_prefix=_accept_count_all),
     "bonus token from the draft": _mutant(accept_prefix=_accept_bonus_from_draft),
     "commit window shifted": _mutant(kv_commit=_commit_shifted),
+    "row statistics merged without the exp(m_i - m) rescale": _mutant(merge_rowstats=_merge_rowstats_no_rescale),
+    "part scores use the part's own row statistics": _mutant(selection_scores_given_rowstats=_part_scores_own_stats),
+    "candidate merge ties to the higher index": _mutant(merge_candidates=_merge_candidates_ties_high),
+    "candidate merge ignores the part offsets": _mutant(merge_candidates=_merge_candidates_local_idx),
 }
 
 

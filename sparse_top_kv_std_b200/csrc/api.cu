@@ -380,14 +380,12 @@ int part_score_args(const std_dims* dims, const void* q_text, int T, const void*
   if ((int64_t)n_prefix + nvis_max > dims->cap_full)
     return fail(STD_ERR_CAPACITY, "n_prefix + nvis_max = %lld exceeds cap_full = %lld", (long long)n_prefix + nvis_max,
                 (long long)dims->cap_full);
-  int* err;
-  STD_TRY(device_state(&err, nullptr));
   *s = stdb::ScoreArgs{};
   s->q_text = q_text; s->k_full = k_full; s->nvis = nvis; s->nvis_max = nvis_max;
   s->L = dims->L; s->B = dims->B; s->Hq = dims->Hq; s->Hkv = dims->Hkv; s->G = dims->Hq / dims->Hkv; s->T = T;
-  s->d = dims->d; s->dtype = dims->dtype; s->cap = dims->cap_full; s->err = err; s->prefix = n_prefix;
+  s->d = dims->d; s->dtype = dims->dtype; s->cap = dims->cap_full; s->prefix = n_prefix;
   s->keys_only = 1;
-  return STD_OK;
+  return STD_OK;  // s->err is set by the caller once every host check has passed
 }
 
 }  // namespace
@@ -399,6 +397,7 @@ int std_select_rowstats(const std_dims* dims, const void* q_text, int T, const v
   STD_TRY(part_score_args(dims, q_text, T, k_full, nvis, nvis_max, n_prefix, &s));
   STD_TRY(check_ptr(row_m, 4, "row_m"));
   STD_TRY(check_ptr(row_l, 4, "row_l"));
+  STD_TRY(device_state(&s.err, nullptr));
   s.row_m = row_m; s.row_l = row_l; s.passes = 1;
   bool hist_done = false;
   cudaError_t e = stdb::launch_select_scores(s, stream, &hist_done);
@@ -443,6 +442,7 @@ int std_select_candidates(const std_dims* dims, const void* q_text, int T, const
   if (!scores_out && (!ws || ws_bytes < need))
     return fail(STD_ERR_WORKSPACE, "candidate workspace: need %zu bytes, got %zu", need, ws ? ws_bytes : 0);
   if (!scores_out) STD_TRY(check_ptr(ws, 16, "ws"));
+  STD_TRY(device_state(&s.err, nullptr));
   float* scores = scores_out ? scores_out : static_cast<float*>(ws);
   s.row_m = const_cast<float*>(row_m); s.row_l = const_cast<float*>(row_l); s.scores = scores; s.passes = 2;
   bool hist_done = false;

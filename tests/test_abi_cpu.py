@@ -104,6 +104,28 @@ FAKE = 1 << 40  # a 16-byte aligned non-null "pointer": never dereferenced, chec
     (lambda: lib_().std_kv_append(ctypes.byref(_dims()), FAKE, FAKE, 100, FAKE, -1, FAKE, FAKE, 2, None), B.STD_ERR_INVALID_ARG),
     (lambda: lib_().std_kv_commit(ctypes.byref(_dims()), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 33, None), B.STD_ERR_INVALID_ARG),
     (lambda: lib_().std_decode_round(ctypes.byref(_dims()), 4, None, None, 0, 0, None, 0, None), B.STD_ERR_INVALID_ARG),
+    # the selection over a cache split by position
+    (lambda: lib_().std_select_rowstats(None, FAKE, 64, FAKE, FAKE, 512, 0, FAKE, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_select_rowstats(ctypes.byref(_dims()), FAKE, 0, FAKE, FAKE, 512, 0, FAKE, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_select_rowstats(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, 0, 0, FAKE, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_select_rowstats(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, 512, -1, FAKE, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_select_rowstats(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, 900, 101, FAKE, FAKE, None), B.STD_ERR_CAPACITY),
+    (lambda: lib_().std_select_rowstats(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, 512, 0, None, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_merge_rowstats(0, 2, FAKE, FAKE, FAKE, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_merge_rowstats(100, 0, FAKE, FAKE, FAKE, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_merge_rowstats(100, 2, None, FAKE, FAKE, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_select_candidates(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, 512, 0, FAKE, FAKE, 0, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_select_candidates(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, 512, 0, FAKE, FAKE, 513, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_select_candidates(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, 512, 0, FAKE, FAKE, 16, FAKE, FAKE, None, FAKE, 16, None), B.STD_ERR_WORKSPACE),
+    (lambda: lib_().std_select_candidates(ctypes.byref(_dims()), FAKE, 64, FAKE, FAKE, 512, 0, None, FAKE, 16, FAKE, FAKE, None, FAKE, 1 << 30, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_merge_candidates(ctypes.byref(_dims()), 0, 16, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_merge_candidates(ctypes.byref(_dims()), 2, 0, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_merge_candidates(ctypes.byref(_dims()), 2, 16, FAKE, FAKE, FAKE, FAKE, FAKE, 16, None), B.STD_ERR_WORKSPACE),
+    (lambda: lib_().std_merge_candidates(ctypes.byref(_dims()), 2, 16, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_gather_sparse_part(ctypes.byref(_dims()), FAKE, FAKE, FAKE, FAKE, 16, 64, 0, 0, 0, FAKE, FAKE, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_gather_sparse_part(ctypes.byref(_dims()), FAKE, FAKE, FAKE, FAKE, 16, 64, 0, 0, 1001, FAKE, FAKE, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_gather_sparse_part(ctypes.byref(_dims()), FAKE, FAKE, FAKE, FAKE, 16, 64, 0, -5, 100, FAKE, FAKE, FAKE, None), B.STD_ERR_INVALID_ARG),
+    (lambda: lib_().std_gather_sparse_part(ctypes.byref(_dims()), FAKE, FAKE, FAKE, FAKE, 240, 64, 0, 0, 100, FAKE, FAKE, FAKE, None), B.STD_ERR_CAPACITY),
     (lambda: lib_().std_probe_wait_timeout(None, None), B.STD_ERR_INVALID_ARG),
     (lambda: lib_().std_probe_wait_timeout(FAKE + 2, None), B.STD_ERR_INVALID_ARG),
 ])

@@ -988,8 +988,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 // softmax thread evaluates one exponential per real query row, and the segment end
 // needs no combine of lane quarters: thread t holds element t of every output row.
 struct CtlT : Ctl {
-  uint64_t xmax[2];      // per tile parity: the four warps' row maxima are in wmax
-  uint64_t xsum;         // segment end: the four warps' row sums are in wsum
+  uint64_t xmax[2][2];   // [row group][tile parity]: the group's four warps' row maxima are in wmax
+  uint64_t xsum[2];      // [row group] segment end: the group's four warps' row sums are in wsum
   alignas(16) float wmax[2][16][4];  // [tile parity][query row][softmax warp], read as float4
   alignas(16) float wsum[16][4];
 };
@@ -1033,13 +1033,17 @@ __device__ __forceinline__ float warp_row_sums(const float (&v)[N], int lane) {
   return a[0];
 }
 
-// RT: query rows a softmax thread handles (8 or 16; rows up to RT of the 16-row tile)
-template <int RT>
-__global__ void __launch_bounds__(kThreads, 1)
+// RT: query rows handled (8 or 16; rows up to RT of the 16-row tile).  NG: softmax row
+// groups -- 1: four softmax warps, each thread all RT rows of its key; 2: eight warps, two
+// per TMEM lane quarter, group g taking rows g RT/2 .. (g + 1) RT/2 - 1 of the same keys.
+template <int RT, int NG>
+__global__ void __launch_bounds__(64 + 128 * NG, 1)
 attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k16,
                const __grid_constant__ CUtensorMap tm_v16, const AttnArgs a) {
   constexpr int D = 128;
+  constexpr int RTT = RT / NG;        // query rows per softmax thread
+  constexpr int NSM = 128 * NG;       // softmax threads
   using C = CfgT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1059,17 +1063,19 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc::mbar_init(&ctl->done, 1);
     for (int i = 0; i < NSB; ++i) {
       tc::mbar_init(&ctl->s_full[i], 1);
-      tc::mbar_init(&ctl->p_full[i], 128);
+      tc::mbar_init(&ctl->p_full[i], NSM);
       tc::mbar_init(&ctl->s_free[i], 1);
     }
     tc::mbar_init(&ctl->o_ready, 1);
-    tc::mbar_init(&ctl->o_free, 128);
-    tc::mbar_init(&ctl->pub, 128);
+    tc::mbar_init(&ctl->o_free, NSM);
+    tc::mbar_init(&ctl->pub, NSM);
     tc::mbar_init(&ctl->flag, 1);
     tc::mbar_init(&ctl->nr_ready, 30);
-    tc::mbar_init(&ctl->xmax[0], 128);
-    tc::mbar_init(&ctl->xmax[1], 128);
-    tc::mbar_init(&ctl->xsum, 128);
+    for (int g = 0; g < NG; ++g) {
+      tc::mbar_init(&ctl->xmax[g][0], 128);
+      tc::mbar_init(&ctl->xmax[g][1], 128);
+      tc::mbar_init(&ctl->xsum[g], 128);
+    }
     ctl->abort_flag = 0;
     ctl->consumed = 0;
     tc::fence_mbar_init();
@@ -1268,6 +1274,10 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   } else {
     // ------------------------------------------------------------ softmax threads
     const int w = warp & 3;               // TMEM lane quarter of this warp
+    const int grp = NG == 1 ? 0 : (warp - 2) >> 2;  // row group
+    const int r0 = grp * RTT;                       // the group's first query row
+    // value r0 + r of a 16-column load, with compile-time register indices only
+    auto pick = [&](const uint32_t(&x)[16], int r) -> uint32_t { return (NG == 2 && grp) ? x[RTT + r] : x[r]; };
     const int tk = w * 32 + lane;         // this thread's key of every tile, and its element of d
     const uint32_t lane_base = tmem + ((uint32_t)(w * 32) << 16);
     const float sc = kLog2e * rsqrtf((float)D);
@@ -1276,17 +1286,17 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t p_off = (uint32_t)(tk >> 6) * 16 * 128 + (uint32_t)(tk & 7) * 2;
     const int p_chunk = (tk & 63) >> 3;
     // the P buffers start as zeros: rows RT..15 are never written and must contribute nothing
-    for (int i = tid; i < (int)(NSB * C::P_BYTES / 16); i += 128)
+    for (int i = tid; i < (int)(NSB * C::P_BYTES / 16); i += NSM)
       *reinterpret_cast<uint4*>(smem + C::Q_BYTES + i * 16) = make_uint4(0, 0, 0, 0);
     tc::fence_proxy_async();
     Iter it;
     iter_seek(it, ctl, a, g0, g1);
     int seg = -1, kv = 0, u = 0, npub = 0, nxs = 0;
-    float m[RT], l[RT];
-    int lim[RT];
+    float m[RTT], l[RTT];  // this thread's rows r0 + i
+    int lim[RTT];
     int lim_max = 0;
 #pragma unroll
-    for (int r = 0; r < RT; ++r) {
+    for (int r = 0; r < RTT; ++r) {
       m[r] = -INFINITY;
       l[r] = 0.f;
       lim[r] = 0;
@@ -1299,10 +1309,10 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ++seg;
         const int base = a.len[it.b] + a.len_off;
 #pragma unroll
-        for (int r = 0; r < RT; ++r) {
+        for (int r = 0; r < RTT; ++r) {
           m[r] = -INFINITY;
           l[r] = 0.f;
-          lim[r] = r < a.rows ? min(base + r % a.nq, a.row_end) : 0;  // keys below lim[r] are attended
+          lim[r] = r0 + r < a.rows ? min(base + (r0 + r) % a.nq, a.row_end) : 0;  // keys below lim[r] are attended
         }
         lim_max = min(base + a.nq - 1, a.row_end);
       }
@@ -1318,7 +1328,7 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int z0 = max(0, lim_max - key0);
         const int zb = a.row_begin - key0;
         uint8_t* vb = smem + C::KV_OFF + s * C::ST_BYTES + C::T_BYTES;
-        for (int i = tid; i < C::KB * TK * 8; i += 128) {
+        for (int i = tid; i < C::KB * TK * 8; i += NSM) {
           const int r = (i >> 3) % TK;
           if (r >= z0 || r < zb)
             *reinterpret_cast<uint4*>(vb + (i / (TK * 8)) * TK * 128 + r * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
@@ -1326,7 +1336,7 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc::fence_proxy_async();
       }
       // this thread's key against the query rows
-      float v[RT];
+      float v[RTT];
       {
         uint32_t r16[16];
         __syncwarp();
@@ -1335,35 +1345,35 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int kc = key0 + tk;
         const bool in_range = kc >= a.row_begin;
 #pragma unroll
-        for (int r = 0; r < RT; ++r) v[r] = (in_range && kc < lim[r]) ? __uint_as_float(r16[r]) : -INFINITY;
+        for (int r = 0; r < RTT; ++r) v[r] = (in_range && kc < lim[r]) ? __uint_as_float(pick(r16, r)) : -INFINITY;
       }
       // row maxima of the tile: per warp (every lane gets them), then across the four warps
       const int par = u & 1;
       {
         float mine = -INFINITY;
 #pragma unroll
-        for (int r = 0; r < RT; ++r) {
+        for (int r = 0; r < RTT; ++r) {
           const float wm = warp_max_f32(v[r]);
           mine = lane == r ? wm : mine;
         }
-        if (lane < RT) ctl->wmax[par][lane][w] = mine;
+        if (lane < RTT) ctl->wmax[par][r0 + lane][w] = mine;
       }
-      tc::mbar_arrive(&ctl->xmax[par]);
-      if (!tc::mbar_wait_warp(&ctl->xmax[par], (u >> 1) & 1, abort_flag, a.err)) break;
+      tc::mbar_arrive(&ctl->xmax[grp][par]);
+      if (!tc::mbar_wait_warp(&ctl->xmax[grp][par], (u >> 1) & 1, abort_flag, a.err)) break;
       bool need = false;
-      float mt[RT];
+      float mt[RTT];
 #pragma unroll
-      for (int r = 0; r < RT; ++r) {
-        const float4 q4 = *reinterpret_cast<const float4*>(ctl->wmax[par][r]);
+      for (int r = 0; r < RTT; ++r) {
+        const float4 q4 = *reinterpret_cast<const float4*>(ctl->wmax[par][r0 + r]);
         mt[r] = fmaxf(fmaxf(q4.x, q4.y), fmaxf(q4.z, q4.w));
         // lazy rescale: only when the max grows by more than 2^kTau (the same decision in
         // every thread: all see the same m and mt)
         need |= m[r] != -INFINITY && (mt[r] - m[r]) * sc > kTau;
       }
       if (need) {
-        float f[RT];
+        float f[RTT];
 #pragma unroll
-        for (int r = 0; r < RT; ++r) {
+        for (int r = 0; r < RTT; ++r) {
           const bool resc = m[r] != -INFINITY && (mt[r] - m[r]) * sc > kTau;
           f[r] = resc ? ex2((m[r] - mt[r]) * sc) : 1.f;
           m[r] = resc ? mt[r] : m[r];
@@ -1372,31 +1382,43 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // rescale needs an earlier tile of the same segment)
         if (!tc::mbar_wait_warp(&ctl->s_free[(u - 1) % NSB], ((u - 1) / NSB) & 1, abort_flag, a.err)) break;
         tc::fence_after_sync();
-        uint32_t o16[16];
-        __syncwarp();
-        tc::tmem_ld_x16(lane_base, o16);
-        tc::tmem_ld_wait16(o16);
+        if constexpr (NG == 1) {
+          uint32_t o16[16];
+          __syncwarp();
+          tc::tmem_ld_x16(lane_base, o16);
+          tc::tmem_ld_wait16(o16);
 #pragma unroll
-        for (int r = 0; r < RT; ++r) {
-          o16[r] = __float_as_uint(__uint_as_float(o16[r]) * f[r]);
-          l[r] *= f[r];
+          for (int r = 0; r < RTT; ++r) o16[r] = __float_as_uint(__uint_as_float(o16[r]) * f[r]);
+          __syncwarp();
+          tc::tmem_st_x16(lane_base, o16);
+        } else {  // only this group's columns: the other group rescales its own
+          static_assert(RTT == 4, "two row groups of four rows");
+          uint32_t o4[4];
+          __syncwarp();
+          tc::tmem_ld_x4(lane_base + r0, o4);
+          tc::tmem_ld_wait4(o4);
+#pragma unroll
+          for (int r = 0; r < 4; ++r) o4[r] = __float_as_uint(__uint_as_float(o4[r]) * f[r]);
+          __syncwarp();
+          tc::tmem_st_x4(lane_base + r0, o4);
         }
-        __syncwarp();
-        tc::tmem_st_x16(lane_base, o16);
         tc::tmem_st_wait();
+#pragma unroll
+        for (int r = 0; r < RTT; ++r) l[r] *= f[r];
       }
 #pragma unroll
-      for (int r = 0; r < RT; ++r) m[r] = m[r] == -INFINITY ? mt[r] : m[r];  // first keys the row sees
+      for (int r = 0; r < RTT; ++r) m[r] = m[r] == -INFINITY ? mt[r] : m[r];  // first keys the row sees
       // P^T[r][tk] = 2^(x - m) as bf16 into the tile's P buffer (a row that has seen no key
       // yet has m = -inf and only -inf logits: its P is 2^-inf = 0)
       {
         uint8_t* pb = smem + C::Q_BYTES + bu * C::P_BYTES + p_off;
 #pragma unroll
-        for (int r = 0; r < RT; ++r) {
+        for (int r = 0; r < RTT; ++r) {
           const float msc = (m[r] == -INFINITY ? 0.f : m[r]) * sc;
           const float p = ex2(fmaf(v[r], sc, -msc));
           l[r] += p;
-          *reinterpret_cast<__nv_bfloat16*>(pb + r * 128 + ((p_chunk ^ (r & 7)) << 4)) = __float2bfloat16_rn(p);
+          const int row = r0 + r;
+          *reinterpret_cast<__nv_bfloat16*>(pb + row * 128 + ((p_chunk ^ (row & 7)) << 4)) = __float2bfloat16_rn(p);
         }
       }
       tc::fence_proxy_async();
@@ -1408,16 +1430,16 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (a.early) pdl_wait();  // outputs, partials and merge counters: after the previous kernel
         // row sums over the 128 key threads
         {
-          const float ws = warp_row_sums<RT>(l, lane);
-          if ((lane & (32 / RT - 1)) == 0) ctl->wsum[lane / (32 / RT)][w] = ws;
+          const float ws = warp_row_sums<RTT>(l, lane);
+          if ((lane & (32 / RTT - 1)) == 0) ctl->wsum[r0 + lane / (32 / RTT)][w] = ws;
         }
-        tc::mbar_arrive(&ctl->xsum);
-        if (!tc::mbar_wait_warp(&ctl->xsum, nxs & 1, abort_flag, a.err)) break;
+        tc::mbar_arrive(&ctl->xsum[grp]);
+        if (!tc::mbar_wait_warp(&ctl->xsum[grp], nxs & 1, abort_flag, a.err)) break;
         ++nxs;
-        float L[RT];
+        float L[RTT];
 #pragma unroll
-        for (int r = 0; r < RT; ++r) {
-          const float4 q4 = *reinterpret_cast<const float4*>(ctl->wsum[r]);
+        for (int r = 0; r < RTT; ++r) {
+          const float4 q4 = *reinterpret_cast<const float4*>(ctl->wsum[r0 + r]);
           L[r] = (q4.x + q4.y) + (q4.z + q4.w);
         }
         uint32_t o16[16];
@@ -1428,10 +1450,11 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc::mbar_arrive(&ctl->o_free);  // O may be reused: the rest reads registers and global memory
         // (m, L) of row tk, for the thread that writes them
         float m_tk = 0.f, L_tk = 0.f;
+        const bool own_tk = tk >= r0 && tk < r0 + RTT;  // row tk is one of this group's rows
 #pragma unroll
-        for (int r = 0; r < RT; ++r) {
-          m_tk = tk == r ? m[r] : m_tk;
-          L_tk = tk == r ? L[r] : L_tk;
+        for (int r = 0; r < RTT; ++r) {
+          m_tk = tk == r0 + r ? m[r] : m_tk;
+          L_tk = tk == r0 + r ? L[r] : L_tk;
         }
         const int start = it.l * ctl->tl + ctl->pre_b[it.b] + it.h * it.nt;
         const int c0 = start / ctl->per, c1 = (start + it.nt - 1) / ctl->per;
@@ -1443,22 +1466,22 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (c0 == c1) {
           // this CTA saw the whole problem: the output (partials: unnormalised, with (m, l))
 #pragma unroll
-          for (int r = 0; r < RT; ++r) {
-            if (r < a.rows) {
+          for (int r = 0; r < RTT; ++r) {
+            if (r0 + r < a.rows) {
               const float inv = a.partial ? 1.f : (L[r] > 0.f ? 1.f / L[r] : 0.f);
-              a.o[(orow0 + r) * D + tk] = __uint_as_float(o16[r]) * inv;
+              a.o[(orow0 + r0 + r) * D + tk] = __uint_as_float(pick(o16, r)) * inv;
             }
           }
-          if (a.partial && tk < a.rows) {
+          if (a.partial && own_tk && tk < a.rows) {
             a.ml[(orow0 + tk) * 2] = m_tk * rsqrtf((float)D);
             a.ml[(orow0 + tk) * 2 + 1] = L_tk;
           }
         } else {
           if (!STD_DCHECK((size_t)slot < nslots, a.err)) break;
 #pragma unroll
-          for (int r = 0; r < RT; ++r)
-            if (r < a.rows) a.ws[((size_t)slot * a.rows + r) * D + tk] = __uint_as_float(o16[r]);
-          if (tk < a.rows) {
+          for (int r = 0; r < RTT; ++r)
+            if (r0 + r < a.rows) a.ws[((size_t)slot * a.rows + r0 + r) * D + tk] = __uint_as_float(pick(o16, r));
+          if (own_tk && tk < a.rows) {
             wml[((size_t)slot * a.rows + tk) * 2] = m_tk * sc;
             wml[((size_t)slot * a.rows + tk) * 2 + 1] = L_tk;
           }
@@ -1474,7 +1497,7 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
           if (!tc::mbar_wait(&ctl->flag, npub & 1, abort_flag, a.err)) break;
           ++npub;
-          if (ctl->last_flag && STD_DCHECK((size_t)prob + c1 < nslots && c0 <= c1, a.err)) {
+          if (ctl->last_flag && tid < 128 && STD_DCHECK((size_t)prob + c1 < nslots && c0 <= c1, a.err)) {
             merge_problem<D, true>(a.o, a.partial ? a.ml : nullptr, a.ws, wml, a.rows, (size_t)(prob + c0) * a.rows,
                                    c1 - c0 + 1, orow0, tid);
             if (tid == 0) atomicExch(ctr + prob, (unsigned long long)a.epoch << 32);  // ready for a replay
@@ -1485,7 +1508,7 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       ++kv;
       iter_next(it, ctl, a);
     }
-    if (a.partial && blockIdx.x == 0) {
+    if (a.partial && blockIdx.x == 0 && tid < 128) {
       // partials of a sequence with no key in the range: o = 0, m = -inf, l = 0
       const int per_b = a.Hq * a.nq;
       for (int b = 0; b < a.B; ++b) {
@@ -1529,7 +1552,7 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   // d = 128 with at most 16 rows: the keys-on-lanes kernel; d = 64 keeps the quarter split
   const bool keys_on_lanes = split && D == 128;
   const int variant = keys_on_lanes ? (a.rows <= 8 ? 3 : 2) : split ? 2 : half ? 1 : 0;
-  auto kern = keys_on_lanes ? (a.rows <= 8 ? attn_tq_kernel<8> : attn_tq_kernel<16>)
+  auto kern = keys_on_lanes ? (a.rows <= 8 ? attn_tq_kernel<8, 2> : attn_tq_kernel<16, 1>)
               : split       ? attn_tc_kernel<D, true, true>
               : half        ? attn_tc_kernel<D, true, false>
                             : attn_tc_kernel<D, false, false>;
@@ -1545,7 +1568,8 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(bit, std::memory_order_release);
   }
-  return launch_pdl(kern, dim3(a.splits), dim3(kThreads), smem_bytes, s, tq, tk, tv, tk16, tv16, a);
+  const int threads = keys_on_lanes && a.rows <= 8 ? 64 + 128 * 2 : kThreads;
+  return launch_pdl(kern, dim3(a.splits), dim3(threads), smem_bytes, s, tq, tk, tv, tk16, tv16, a);
 }
 
 }  // namespace

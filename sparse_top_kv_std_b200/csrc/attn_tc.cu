@@ -161,7 +161,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Merge of a problem's segment partials (m, l, o) into its output, by the 128 softmax
+// Merge of a problem's segment partials (m, l, o) into its output, by the NTHREADS softmax
 // threads of the last CTA to finish the problem.  One item = 4 columns of one query row.
 // BATCHED: the segments are taken kMergeSegs at a time, every load of a batch issued
 // before any is used (one L2 round trip per batch instead of one per segment), and the
@@ -170,7 +170,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 // kernel, already near the register limit, keeps the two-pass form (max over all
 // segments, then the weighted sums).  Partial k of row r sits at slot0 + k * rows + r;
 // output row r at orow0 + r.
-template <int D, bool BATCHED>
+template <int D, bool BATCHED, int NTHREADS = 128>
 __device__ __forceinline__ void merge_problem(float* out, float* ml_out, const float* ws, const float* ml, int rows,
                                            size_t slot0, int nseg, size_t orow0, int tid) {
   const int nitems = rows * (D / 4);
@@ -205,7 +205,7 @@ __device__ __forceinline__ void merge_problem(float* out, float* ml_out, const f
     }
     write(r, col, M, L, acc);
   };
-  for (int item = tid; item < nitems; item += 128) {
+  for (int item = tid; item < nitems; item += NTHREADS) {
     if (!BATCHED) {
       two_pass(item);
       continue;
@@ -1497,9 +1497,10 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
           if (!tc::mbar_wait(&ctl->flag, npub & 1, abort_flag, a.err)) break;
           ++npub;
-          if (ctl->last_flag && tid < 128 && STD_DCHECK((size_t)prob + c1 < nslots && c0 <= c1, a.err)) {
-            merge_problem<D, true>(a.o, a.partial ? a.ml : nullptr, a.ws, wml, a.rows, (size_t)(prob + c0) * a.rows,
-                                   c1 - c0 + 1, orow0, tid);
+          if (ctl->last_flag && STD_DCHECK((size_t)prob + c1 < nslots && c0 <= c1, a.err)) {
+            // all NSM softmax threads share the merge
+            merge_problem<D, true, NSM>(a.o, a.partial ? a.ml : nullptr, a.ws, wml, a.rows,
+                                        (size_t)(prob + c0) * a.rows, c1 - c0 + 1, orow0, tid);
             if (tid == 0) atomicExch(ctr + prob, (unsigned long long)a.epoch << 32);  // ready for a replay
           }
         }

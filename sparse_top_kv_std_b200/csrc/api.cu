@@ -165,14 +165,15 @@ int plan_attn(const std_dims* dims, int nq, int64_t cap, int splits, AttnPlan* p
       //
       // With few tiles in all (a single layer's draft: 4 problems of ~35 tiles), one CTA per
       // SM would cut every problem into dozens of one-tile segments whose partials the last
-      // CTA merges one batch after another; instead give each CTA about four tiles, so a
+      // CTA merges one batch after another; instead give each CTA about five tiles, so a
       // problem has a handful of segments (28 launches of one layer's draft, 4 x 4352 keys,
-      // in a CUDA graph: 33 us each with 148 CTAs, 19 us with 32).
+      // in a CUDA graph, us per launch: 25.8 with 148 CTAs, 17.9 with 48, 15.1 with 32,
+      // 18.0 with 24).
       int sms;
       STD_TRY(device_state(nullptr, &sms));
       const int64_t short_cap = a.rows <= 16 ? 2048 : 8192;
       const int64_t tiles_max = (int64_t)probs * ((cap + 127) / 128);
-      constexpr int64_t kMinTilesPerCta = 4;
+      constexpr int64_t kMinTilesPerCta = 5;
       if (probs <= sms && 2 * probs >= sms && cap <= short_cap) {
         ctas = probs;
       } else if (tiles_max < (int64_t)sms * kMinTilesPerCta) {

@@ -78,17 +78,28 @@ struct Ctl {
 
 // Arrival on the merge counter of one problem: the counter holds (epoch << 32) |
 // arrivals; a stale epoch (an earlier call, or uninitialised memory) restarts the
-// count.  Returns true for the arrival that completes `need`.  Lock-free: a CAS
-// retry loop, never a wait on another CTA.
+// count.  Returns true for the arrival that completes `need`.  The merging CTA leaves
+// the counter at ((epoch + 1) << 32) | 0, and the host numbers calls in issue order, so
+// in a run of calls on one workspace the next call finds its own epoch and each arrival
+// is one atomic add, however many CTAs arrive together.  An add that lands on a stale
+// epoch is wiped when the count restarts, so that arrival counts itself again with a
+// CAS loop.  Lock-free: never a wait on another CTA.
 __device__ __forceinline__ bool arrive_last(unsigned long long* ctr, uint32_t epoch, int need) {
-  unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(ctr);
+  const unsigned long long old = atomicAdd(ctr, 1ull);
+  if ((uint32_t)(old >> 32) == epoch) return (int)(old & 0xffffffffull) + 1 == need;
+  unsigned long long cur = old + 1ull;
   for (;;) {
     const unsigned long long want =
-        (uint32_t)(old >> 32) == epoch ? old + 1 : (((unsigned long long)epoch << 32) | 1ull);
-    const unsigned long long prev = atomicCAS(ctr, old, want);
-    if (prev == old) return (int)(want & 0xffffffffull) == need;
-    old = prev;
+        (uint32_t)(cur >> 32) == epoch ? cur + 1 : (((unsigned long long)epoch << 32) | 1ull);
+    const unsigned long long prev = atomicCAS(ctr, cur, want);
+    if (prev == cur) return (int)(want & 0xffffffffull) == need;
+    cur = prev;
   }
+}
+
+// The counter value the merging CTA leaves for the next call on the workspace.
+__device__ __forceinline__ unsigned long long next_call_counter(uint32_t epoch) {
+  return (unsigned long long)(uint32_t)(epoch + 1u) << 32;
 }
 
 
@@ -938,7 +949,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // all 128 softmax threads share the merge
             merge_problem<D, HALF>(a.o, a.partial ? a.ml : nullptr, a.ws, wml, a.rows, (size_t)(prob + c0) * a.rows,
                                    c1 - c0 + 1, orow0, tid);
-            if (tid == 0) atomicExch(ctr + prob, (unsigned long long)a.epoch << 32);  // ready for a replay
+            if (tid == 0) atomicExch(ctr + prob, next_call_counter(a.epoch));
           }
         }
       }
@@ -1501,7 +1512,7 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // all NSM softmax threads share the merge
             merge_problem<D, true, NSM>(a.o, a.partial ? a.ml : nullptr, a.ws, wml, a.rows,
                                         (size_t)(prob + c0) * a.rows, c1 - c0 + 1, orow0, tid);
-            if (tid == 0) atomicExch(ctr + prob, (unsigned long long)a.epoch << 32);  // ready for a replay
+            if (tid == 0) atomicExch(ctr + prob, next_call_counter(a.epoch));
           }
         }
       }

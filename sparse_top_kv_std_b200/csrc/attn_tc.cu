@@ -342,6 +342,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
+    // the tensor maps are kernel parameters: fetch them while the barriers are set up
+    // (and, launched early, while the previous kernel finishes)
+    tc::prefetch_tmap(&tm_q);
+    tc::prefetch_tmap(&tm_k);
+    tc::prefetch_tmap(&tm_v);
+    tc::prefetch_tmap(&tm_k16);
+    tc::prefetch_tmap(&tm_v16);
     for (int s = 0; s < STAGES; ++s) {
       tc::mbar_init(&ctl->kv_full[s], 1);
       tc::mbar_init(&ctl->kv_empty[s], 1);
@@ -402,10 +409,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producers
     if (lane == 0 && g0 < g1) {
-      tc::prefetch_tmap(&tm_k);
-      tc::prefetch_tmap(&tm_v);
-      tc::prefetch_tmap(&tm_k16);
-      tc::prefetch_tmap(&tm_v16);
       Iter it;
       iter_seek(it, ctl, a, g0, g1);
       int kv = 0;
@@ -460,7 +463,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int k = *(volatile int*)&ctl->consumed; k < kv; ++k) drain_wait(&ctl->kv_full[k % STAGES], (k / STAGES) & 1);
       }
     } else if (lane == 1 && g0 < g1) {
-      tc::prefetch_tmap(&tm_q);
       Iter it;
       iter_seek(it, ctl, a, g0, g1);
       int seg = 0;
@@ -1065,6 +1067,13 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
+    // the tensor maps are kernel parameters: fetch them while the barriers are set up
+    // (and, launched early, while the previous kernel finishes)
+    tc::prefetch_tmap(&tm_q);
+    tc::prefetch_tmap(&tm_k);
+    tc::prefetch_tmap(&tm_v);
+    tc::prefetch_tmap(&tm_k16);
+    tc::prefetch_tmap(&tm_v16);
     for (int s = 0; s < STAGES; ++s) {
       tc::mbar_init(&ctl->kv_full[s], 1);
       tc::mbar_init(&ctl->kv_empty[s], 1);
@@ -1124,10 +1133,6 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producers
     if (lane == 0 && g0 < g1) {
-      tc::prefetch_tmap(&tm_k);
-      tc::prefetch_tmap(&tm_v);
-      tc::prefetch_tmap(&tm_k16);
-      tc::prefetch_tmap(&tm_v16);
       Iter it;
       iter_seek(it, ctl, a, g0, g1);
       int kv = 0;
@@ -1179,7 +1184,6 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int k = *(volatile int*)&ctl->consumed; k < kv; ++k) drain_wait(&ctl->kv_full[k % STAGES], (k / STAGES) & 1);
       }
     } else if (lane == 1 && g0 < g1) {
-      tc::prefetch_tmap(&tm_q);
       Iter it;
       iter_seek(it, ctl, a, g0, g1);
       int seg = 0;

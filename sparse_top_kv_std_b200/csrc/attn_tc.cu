@@ -1001,6 +1001,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 // softmax thread evaluates one exponential per real query row, and the segment end
 // needs no combine of lane quarters: thread t holds element t of every output row.
 struct CtlT : Ctl {
+  uint64_t prev_done;    // early start: the previous kernel has completed (its writes are visible)
   uint64_t xmax[2][2];   // [row group][tile parity]: the group's four warps' row maxima are in wmax
   uint64_t xsum[2];      // [row group] segment end: the group's four warps' row sums are in wsum
   alignas(16) float wmax[2][16][4];  // [tile parity][query row][softmax warp], read as float4
@@ -1022,6 +1023,9 @@ struct CfgT {
 };
 constexpr int kTmemColsT = 64;     // O^T at columns 0..15, S^T buffer b at 16 + 16 b
 constexpr uint32_t kColST = 16;
+// Early start: the roles wait for prev_done, which the waiting warp signals once its
+// griddepcontrol.wait returns; the previous kernel may run for long, hence a long bound.
+constexpr uint64_t kPrevWaitNs = 20ull * 1000 * 1000 * 1000;
 
 // Per-row sums of a warp's N values per lane (N = 8 or 16) over its 32 lanes.  Each
 // halving step keeps half of a lane's values (lane bit 4 picks the upper half, then bit
@@ -1049,8 +1053,13 @@ __device__ __forceinline__ float warp_row_sums(const float (&v)[N], int lane) {
 // RT: query rows handled (8 or 16; rows up to RT of the 16-row tile).  NG: softmax row
 // groups -- 1: four softmax warps, each thread all RT rows of its key; 2: eight warps, two
 // per TMEM lane quarter, group g taking rows g RT/2 .. (g + 1) RT/2 - 1 of the same keys.
+// Warps: 0 the K/V producer (lane 0) and the Q loader (lane 1), 1 the MMA issuer, 2 ..
+// 1 + 4 NG the softmax, 2 + 4 NG the waiting warp.  griddepcontrol.wait stalls every lane
+// of the warp that runs it, so with an early start only the waiting warp runs it (then
+// copies the appended rows); the other roles wait for its prev_done signal, each only
+// where it needs the previous kernel's writes, and keep streaming K/V until then.
 template <int RT, int NG>
-__global__ void __launch_bounds__(64 + 128 * NG, 1)
+__global__ void __launch_bounds__(96 + 128 * NG, 1)
 attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k16,
                const __grid_constant__ CUtensorMap tm_v16, const AttnArgs a) {
@@ -1091,6 +1100,7 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc::mbar_init(&ctl->pub, NSM);
     tc::mbar_init(&ctl->flag, 1);
     tc::mbar_init(&ctl->nr_ready, 30);
+    tc::mbar_init(&ctl->prev_done, 1);
     for (int g = 0; g < NG; ++g) {
       tc::mbar_init(&ctl->xmax[g][0], 128);
       tc::mbar_init(&ctl->xmax[g][1], 128);
@@ -1143,7 +1153,8 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int s = kv % STAGES;
         const int tabs = it.t + ctl->tb;
         if (!waited && (tabs + 1) * TK > ctl->len_b[it.b] + a.new_off - 1) {
-          pdl_wait();
+          // this tile holds rows the previous kernel may write
+          if (!tc::mbar_wait(&ctl->prev_done, 0, abort_flag, a.err, kPrevWaitNs)) break;
           waited = true;
         }
         if (!rows_ready) {
@@ -1184,15 +1195,16 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int k = *(volatile int*)&ctl->consumed; k < kv; ++k) drain_wait(&ctl->kv_full[k % STAGES], (k / STAGES) & 1);
       }
     } else if (lane == 1 && g0 < g1) {
+      // ---------------------------------------------------------- Q loader (one 16-row box
+      // per segment; with an early start but no early Q, after the previous kernel)
       Iter it;
       iter_seek(it, ctl, a, g0, g1);
       int seg = 0;
-      bool waited = !a.early;
+      bool waited = !a.early || (a.early & STD_ATTN_EARLY_Q);
       while (it.g < it.g_end) {
         if (it.first) {
-          if (!waited && !(a.early & STD_ATTN_EARLY_Q)) {
-            pdl_wait();
-            pdl_trigger();
+          if (!waited) {
+            if (!tc::mbar_wait(&ctl->prev_done, 0, abort_flag, a.err, kPrevWaitNs)) break;
             waited = true;
           }
           if (!tc::mbar_wait(&ctl->q_empty, (seg & 1) ^ 1, abort_flag, a.err)) break;
@@ -1201,20 +1213,10 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
           for (int kb = 0; kb < C::KB; ++kb) tc::tma_load_2d(sQ + kb * 16 * 128, &tm_q, kb * 64, qrow, &ctl->q_full);
           ++seg;
-          if (!waited) {
-            pdl_wait();
-            pdl_trigger();
-            waited = true;
-          }
         }
         iter_next(it, ctl, a);
       }
       if (*abort_flag && seg > 0) drain_wait(&ctl->q_full, (seg - 1) & 1);
-    } else if (lane >= 2 && g0 < g1 && a.k_new != nullptr) {
-      if (a.early) pdl_wait();
-      copy_new_rows<D>(a, ctl, g0, g1, lane - 2);
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-      tc::mbar_arrive(&ctl->nr_ready);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -1285,6 +1287,19 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc::umma_commit(&ctl->done);
         drain_wait(&ctl->done, 0);
       }
+    }
+  } else if (warp == 2 + 4 * NG) {
+    // ------------------------------------------------------------ waiting warp
+    if (a.early) {
+      pdl_wait();
+      pdl_trigger();  // only after this CTA's wait: the next kernel may start early itself
+      if (lane == 0) tc::mbar_arrive(&ctl->prev_done);
+    }
+    if (lane >= 2 && g0 < g1 && a.k_new != nullptr) {
+      // the previous kernel may still read the tile these rows land in: after the wait
+      copy_new_rows<D>(a, ctl, g0, g1, lane - 2);
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      tc::mbar_arrive(&ctl->nr_ready);
     }
   } else {
     // ------------------------------------------------------------ softmax threads
@@ -1442,7 +1457,8 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (last) {
         if (!tc::mbar_wait_warp(&ctl->o_ready, seg & 1, abort_flag, a.err)) break;
         tc::fence_after_sync();
-        if (a.early) pdl_wait();  // outputs, partials and merge counters: after the previous kernel
+        // outputs, partials and merge counters: after the previous kernel
+        if (a.early && !tc::mbar_wait_warp(&ctl->prev_done, 0, abort_flag, a.err, kPrevWaitNs)) break;
         // row sums over the 128 key threads
         {
           const float ws = warp_row_sums<RTT>(l, lane);
@@ -1524,7 +1540,8 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       ++kv;
       iter_next(it, ctl, a);
     }
-    if (a.partial && blockIdx.x == 0 && tid < 128) {
+    if (a.partial && blockIdx.x == 0 && tid < 128 &&
+        (!a.early || tc::mbar_wait(&ctl->prev_done, 0, abort_flag, a.err, kPrevWaitNs))) {
       // partials of a sequence with no key in the range: o = 0, m = -inf, l = 0
       const int per_b = a.Hq * a.nq;
       for (int b = 0; b < a.B; ++b) {
@@ -1584,7 +1601,7 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(bit, std::memory_order_release);
   }
-  const int threads = keys_on_lanes && a.rows <= 8 ? 64 + 128 * 2 : kThreads;
+  const int threads = keys_on_lanes ? 96 + 128 * (a.rows <= 8 ? 2 : 1) : kThreads;
   return launch_pdl(kern, dim3(a.splits), dim3(threads), smem_bytes, s, tq, tk, tv, tk16, tv16, a);
 }
 

@@ -46,9 +46,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Returns false if the
-// CTA-wide abort flag is raised or the wait exceeds kWaitTimeoutNs (then it
-// raises the abort flag itself and records the timeout in the error word).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err) {
+// CTA-wide abort flag is raised or the wait exceeds limit_ns (then it raises the
+// abort flag itself and records the timeout in the error word).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err,
+                                          uint64_t limit_ns = kWaitTimeoutNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer();
@@ -56,7 +57,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(a, parity)) return true;
     if ((i & 63) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitTimeoutNs) {
+      if (globaltimer() - t0 > limit_ns) {
         *abort_flag = 1;
         flag_error(err, kDevErrTimeout);
         return false;
@@ -67,8 +68,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 
 // Same, but every lane of the warp gets the same answer (needed before the
 // warp-collective .sync.aligned tcgen05 instructions).
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err) {
-  const bool ok = mbar_wait(bar, parity, abort_flag, err);
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err,
+                                               uint64_t limit_ns = kWaitTimeoutNs) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, err, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 

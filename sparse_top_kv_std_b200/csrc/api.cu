@@ -138,7 +138,7 @@ struct AttnPlan {
   size_t ws_bytes;
 };
 
-int plan_attn(const std_dims* dims, int nq, int64_t cap, int splits, AttnPlan* p) {
+int plan_attn(const std_dims* dims, int nq, int64_t cap, int splits, AttnPlan* p, int early = 0) {
   if (splits < 0 || splits > 1024) return fail(STD_ERR_INVALID_ARG, "splits %d out of range [0, 1024]", splits);
   const int G = dims->Hq / dims->Hkv;
   stdb::AttnArgs& a = p->a;
@@ -151,10 +151,14 @@ int plan_attn(const std_dims* dims, int nq, int64_t cap, int splits, AttnPlan* p
   const int probs = probs_of(dims);
   p->tc = stdb::attn_tc_supported(a);
   if (p->tc) {
-    int ctas = splits;
+    // keys-on-lanes kernel: CTAs cut problems into equal parts instead of stream-K ranges
+    // wherever there are at most about as many CTAs as SMs (parts = 0: stream-K)
+    const bool aligned = stdb::attn_tc_keys_on_lanes(a);
+    int ctas = splits, parts = 0;
     if (splits > 0) {
       const int64_t want = (int64_t)splits * probs;
       ctas = (int)(want > 65535 ? 65535 : want);
+      if (aligned && want <= 65535) parts = splits;
     } else {
       // One persistent CTA per SM (stream-K), unless the problems are short and nearly
       // fill the SMs: then one CTA per problem saves the segment partials and their merge,
@@ -162,27 +166,51 @@ int plan_attn(const std_dims* dims, int nq, int64_t cap, int splits, AttnPlan* p
       // heads, kernels timed alone): 7 query rows, 1024 keys 19.6 -> 14.7 us, 4352 keys
       // 48.6 -> 47.9 us but slower inside a decode step; 63 rows, 4352 keys 62.2 -> 50.4
       // us, 8192 keys 95.4 -> 85.9 us, 32768 keys 297 -> 328 us.  cap bounds the keys.
+      // With an early start the SMs left idle are where the next kernel's CTAs start
+      // early, so short-query calls take one CTA per problem up to 8192 keys too (the
+      // long-video draft, 112 problems of 4353 keys: a chain of early-started steps 46.2 ->
+      // 43.9 us per launch, 55.4 -> 53.7 us inside the decode step).  The workspace query,
+      // which knows no flags, sizes for the larger grid.
       //
       // With few tiles in all (a single layer's draft: 4 problems of ~35 tiles), one CTA per
       // SM would cut every problem into dozens of one-tile segments whose partials the last
-      // CTA merges one batch after another; instead give each CTA about five tiles, so a
-      // problem has a handful of segments (28 launches of one layer's draft, 4 x 4352 keys,
-      // in a CUDA graph, us per launch: 25.8 with 148 CTAs, 17.9 with 48, 15.1 with 32,
-      // 18.0 with 24).
+      // CTA merges; instead each problem gets a few CTAs.  The keys-on-lanes kernel cuts a
+      // problem into equal parts of about kTilesPerPart tiles (a part fits the three K/V
+      // stages, so with an early start all of it is fetched before the previous kernel
+      // ends; 28 launches of one layer's draft, 4 x 4352 keys, in a CUDA graph with early
+      // K/V, us per step: 361 with 35 parts, 269 with 18, 279 with 14, 279 with 12, 308
+      // with 10, 330 with 7; without early start 337 with 18 parts); the other kernel
+      // takes stream-K ranges of about kMinTilesPerCta tiles (the same launches, us per
+      // launch: 25.8 with 148 CTAs, 17.9 with 48, 15.1 with 32, 18.0 with 24).
       int sms;
       STD_TRY(device_state(nullptr, &sms));
-      const int64_t short_cap = a.rows <= 16 ? 2048 : 8192;
-      const int64_t tiles_max = (int64_t)probs * ((cap + 127) / 128);
+      const int64_t short_cap = a.rows <= 16 && !early ? 2048 : 8192;
+      const int64_t nt_cap = (cap + 127) / 128;
+      const int64_t tiles_max = (int64_t)probs * nt_cap;
       constexpr int64_t kMinTilesPerCta = 5;
+      constexpr int64_t kTilesPerPart = 2;
       if (probs <= sms && 2 * probs >= sms && cap <= short_cap) {
         ctas = probs;
+        parts = aligned ? 1 : 0;
       } else if (tiles_max < (int64_t)sms * kMinTilesPerCta) {
-        const int64_t c = (tiles_max + kMinTilesPerCta - 1) / kMinTilesPerCta;
-        ctas = (int)(c < probs ? probs : c);
+        if (aligned) {
+          // at most half the SMs: the next launch's CTAs fit beside this one's and can
+          // start early (the same launches with 19 parts, 76 CTAs: 322 us per step)
+          int64_t k = (nt_cap + kTilesPerPart - 1) / kTilesPerPart;
+          const int64_t k_fit = sms / (2 * (int64_t)probs);
+          if (k > k_fit) k = k_fit;
+          if (k < 1) k = 1;
+          parts = (int)k;
+          ctas = (int)(k * probs);
+        } else {
+          const int64_t c = (tiles_max + kMinTilesPerCta - 1) / kMinTilesPerCta;
+          ctas = (int)(c < probs ? probs : c);
+        }
       } else {
         ctas = sms;
       }
     }
+    a.parts = parts;
     a.splits = ctas;
     p->ws_bytes = stdb::attn_tc_ws_floats(probs, ctas, a.rows, a.d) * sizeof(float);
   } else {
@@ -211,7 +239,7 @@ int run_attn(const std_dims* dims, const void* q, const void* k, const void* v, 
              cudaStream_t stream, const void* k_new = nullptr, const void* v_new = nullptr, int new_rows = 0,
              int new_off = 0, int early = 0, const RangeOpt* range = nullptr) {
   AttnPlan p;
-  STD_TRY(plan_attn(dims, nq, cap, splits, &p));
+  STD_TRY(plan_attn(dims, nq, cap, splits, &p, early));
   if (range && !p.tc)
     return fail(STD_ERR_UNSUPPORTED, "key-range partials need the bf16 tensor-core kernel (d 64 or 128, "
                 "G * query rows <= 128, at most 64 sequences)");

@@ -1137,8 +1137,20 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   tc::fence_after_sync();
   const uint32_t tmem = ctl->tmem;
   volatile int* abort_flag = &ctl->abort_flag;
-  const int g0 = min(ctl->total, (int)blockIdx.x * ctl->per);
-  const int g1 = min(ctl->total, g0 + ctl->per);
+  // this CTA's slice [g0, g1) of the flat (problem, tile) sequence
+  int g0, g1;
+  if (a.parts > 0) {  // part r of problem p: tiles [r nt / k, (r + 1) nt / k), k = min(parts, nt)
+    const int p = blockIdx.x / a.parts, r = blockIdx.x % a.parts;
+    const int h = p % a.Hkv, b = (p / a.Hkv) % a.B, l = p / (a.Hkv * a.B);
+    const int nt = l < a.L ? ctl->tiles_b[b] : 0;
+    const int k = min(a.parts, nt);
+    const int start = l < a.L ? l * ctl->tl + ctl->pre_b[b] + h * nt : ctl->total;
+    g0 = start + (r < k ? r * nt / k : nt);
+    g1 = start + (r < k ? (r + 1) * nt / k : nt);
+  } else {
+    g0 = min(ctl->total, (int)blockIdx.x * ctl->per);
+    g1 = min(ctl->total, g0 + ctl->per);
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producers
@@ -1487,8 +1499,10 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           m_tk = tk == r0 + r ? m[r] : m_tk;
           L_tk = tk == r0 + r ? L[r] : L_tk;
         }
+        // the CTAs c0 .. c1 that hold a segment of this problem
         const int start = it.l * ctl->tl + ctl->pre_b[it.b] + it.h * it.nt;
-        const int c0 = start / ctl->per, c1 = (start + it.nt - 1) / ctl->per;
+        const int c0 = a.parts > 0 ? prob * a.parts : start / ctl->per;
+        const int c1 = a.parts > 0 ? c0 + min(a.parts, it.nt) - 1 : (start + it.nt - 1) / ctl->per;
         const size_t orow0 = (size_t)(lb * a.Hq + it.h * a.G) * a.nq;
         const size_t nslots = (size_t)a.L * a.B * a.Hkv + gridDim.x;
         float* wml = a.ws + nslots * a.rows * D;
@@ -1583,7 +1597,7 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
       !make_tmap_bf16_2d(&tk16, a.k, D, krows, 16) || !make_tmap_bf16_2d(&tv16, a.v, D, krows, 16))
     return cudaErrorInvalidValue;
   // d = 128 with at most 16 rows: the keys-on-lanes kernel; d = 64 keeps the quarter split
-  const bool keys_on_lanes = split && D == 128;
+  const bool keys_on_lanes = attn_tc_keys_on_lanes(a);
   const int variant = keys_on_lanes ? (a.rows <= 8 ? 3 : 2) : split ? 2 : half ? 1 : 0;
   auto kern = keys_on_lanes ? (a.rows <= 8 ? attn_tq_kernel<8, 2> : attn_tq_kernel<16, 1>)
               : split       ? attn_tc_kernel<D, true, true>
@@ -1606,6 +1620,8 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+bool attn_tc_keys_on_lanes(const AttnArgs& a) { return a.d == 128 && a.rows <= 16; }
 
 bool attn_tc_supported(const AttnArgs& a) {
   return a.dtype == STD_BF16 && (a.d == 64 || a.d == 128) && a.rows <= 128 && a.B <= kMaxB &&

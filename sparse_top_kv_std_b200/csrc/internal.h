@@ -46,6 +46,10 @@ struct AttnArgs {
   int L, B, Hq, Hkv, G, nq, rows, d, dtype;
   int64_t cap;
   int splits;
+  // Problem-aligned split (keys-on-lanes kernel; 0: stream-K over the flat tile sequence):
+  // CTA c takes part c % parts of problem c / parts, an equal share of that problem's
+  // tiles, so no CTA's range straddles two problems; splits = problems x parts.
+  int parts;
   float* ws;  // partials: [prob][split][rows_pad][d] then [prob][split][rows_pad][2]
   int* err;
   uint32_t epoch;  // per-call tag of the merge counters (tensor-core kernel)
@@ -83,6 +87,9 @@ cudaError_t launch_decode_attn(const AttnArgs& a, cudaStream_t s);
 // stream-K over 128-key tiles, a.splits = number of CTAs; workspace holds
 // (problems + CTAs) partial slots.
 bool attn_tc_supported(const AttnArgs& a);
+// The tensor-core call runs the keys-on-lanes kernel (d = 128, at most 16 query rows per
+// problem), the one that honours AttnArgs::parts.
+bool attn_tc_keys_on_lanes(const AttnArgs& a);
 size_t attn_tc_ws_floats(int probs, int ctas, int rows, int d);
 cudaError_t launch_decode_attn_tc(const AttnArgs& a, cudaStream_t s);
 

@@ -489,7 +489,11 @@ def run_std(args, rank, world, local_rank):
     nvis_dev = torch.tensor(list(wl.nvis), dtype=torch.int32, device=dev)
     sess.nvis.copy_(nvis_dev)
     outs = [sess.round_outputs() for _ in range(R)]
-    sp_d = B.std_attn_splits(sess.dims, 1, wl.cap_sparse, 0) if wl.gamma > 0 else 1
+    # draft CTAs: step 0 of a round, and the early-started steps after it
+    sp_d = ({"step_0": B.std_attn_splits(sess.dims, 1, wl.cap_sparse, 0),
+             "steps_1_on": B.std_attn_splits_ex(sess.dims, 1, wl.cap_sparse, 0,
+                                                B.STD_ATTN_EARLY_KV | B.STD_ATTN_EARLY_Q)}
+            if wl.gamma > 0 else 1)
     sp_v = B.std_attn_splits(sess.dims, wl.gamma + 1, wl.cap_full, 0)
     ws = sess.ws_round
     q_text = view("q_text")

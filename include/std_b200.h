@@ -316,6 +316,12 @@ size_t std_attn_workspace_size(const std_dims* dims, int q_rows, int64_t cap, in
  * STD_ERR_* code. */
 int std_attn_splits(const std_dims* dims, int q_rows, int64_t cap, int splits);
 
+/* The same for a call with early-start flags (bits of STD_ATTN_EARLY_*, defined
+ * below; unknown bits, or STD_ATTN_EARLY_Q without STD_ATTN_EARLY_KV, are
+ * STD_ERR_INVALID_ARG): an early-started call may use fewer CTAs, never more
+ * workspace. */
+int std_attn_splits_ex(const std_dims* dims, int q_rows, int64_t cap, int splits, int flags);
+
 /*
  * Sparse draft attention ("Methodik" item 2: the draft model M_s uses top-K
  * attention over the selected KV).  For every query head:

@@ -83,6 +83,7 @@ SIGNATURES = {
     "std_gather_sparse_part": (_I, [_DP, _P, _P, _P, _P, _I, _I, _I, _I64, _I64, _P, _P, _P, _P]),
     "std_attn_workspace_size": (_SZ, [_DP, _I, _I64, _I]),
     "std_attn_splits": (_I, [_DP, _I, _I64, _I]),
+    "std_attn_splits_ex": (_I, [_DP, _I, _I64, _I, _I]),
     "std_sparse_decode_attn": (_I, [_DP, _P, _P, _P, _P, _I, _P, _I, _P, _SZ, _P]),
     "std_dense_verify_attn": (_I, [_DP, _P, _I, _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "std_dense_verify_attn_noalloc": (_I, [_DP, _P, _I, _P, _P, _P, _P, _I, _P]),
@@ -269,6 +270,13 @@ def std_attn_workspace_size(d: StdDims, q_rows: int, cap: int, splits: int) -> i
 
 def std_attn_splits(d: StdDims, q_rows: int, cap: int, splits: int = 0) -> int:
     rc = lib().std_attn_splits(ctypes.byref(d), q_rows, cap, splits)
+    if rc < 0:
+        _check(rc)
+    return rc
+
+
+def std_attn_splits_ex(d: StdDims, q_rows: int, cap: int, splits: int = 0, flags: int = 0) -> int:
+    rc = lib().std_attn_splits_ex(ctypes.byref(d), q_rows, cap, splits, flags)
     if rc < 0:
         _check(rc)
     return rc

@@ -616,13 +616,21 @@ size_t std_attn_workspace_size(const std_dims* dims, int q_rows, int64_t cap, in
   return p.ws_bytes;
 }
 
-int std_attn_splits(const std_dims* dims, int q_rows, int64_t cap, int splits) {
+int std_attn_splits_ex(const std_dims* dims, int q_rows, int64_t cap, int splits, int flags) {
   STD_TRY(check_dims(dims));
   if (cap < 1 || q_rows < 1) return fail(STD_ERR_INVALID_ARG, "cap = %lld, q_rows = %d", (long long)cap, q_rows);
+  if (flags & ~(STD_ATTN_EARLY_KV | STD_ATTN_EARLY_Q))
+    return fail(STD_ERR_INVALID_ARG, "unknown attention flags %#x", flags);
+  if ((flags & STD_ATTN_EARLY_Q) && !(flags & STD_ATTN_EARLY_KV))
+    return fail(STD_ERR_INVALID_ARG, "STD_ATTN_EARLY_Q needs STD_ATTN_EARLY_KV");
   AttnPlan p;
-  STD_TRY(plan_attn(dims, q_rows, cap, splits, &p));
+  STD_TRY(plan_attn(dims, q_rows, cap, splits, &p, flags));
   ok();
   return p.a.splits;
+}
+
+int std_attn_splits(const std_dims* dims, int q_rows, int64_t cap, int splits) {
+  return std_attn_splits_ex(dims, q_rows, cap, splits, 0);
 }
 
 int std_sparse_decode_attn(const std_dims* dims, const void* q, const void* k_sparse, const void* v_sparse,

@@ -60,9 +60,28 @@ def test_workspace_queries_host_only(lib):
     assert B.std_attn_workspace_size(f, 9, 1000, 4) == probs * 4 * 63 * (64 + 2) * 4
     assert B.std_select_workspace_size(_dims(dtype=7), 64, 512) == 0
     assert B.std_attn_workspace_size(_dims(Hq=5), 1, 1000, 4) == 0
+    # explicit splits: the CTA count needs no device, with or without early-start flags
+    assert B.std_attn_splits(d, 1, 300, 4) == 4 * probs
+    assert B.std_attn_splits_ex(d, 1, 300, 4, B.STD_ATTN_EARLY_KV | B.STD_ATTN_EARLY_Q) == 4 * probs
+    assert lib.std_attn_splits_ex(ctypes.byref(d), 1, 300, 4, 4) == B.STD_ERR_INVALID_ARG
+    assert lib.std_attn_splits_ex(ctypes.byref(d), 1, 300, 4, B.STD_ATTN_EARLY_Q) == B.STD_ERR_INVALID_ARG
 
 
 FAKE = 1 << 40  # a 16-byte aligned non-null "pointer": never dereferenced, checks fail first
+
+
+def _gpu_visible():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+# The calls below hand made-up device addresses to the library and rely on its host checks
+# rejecting them first.  They belong to the CPU suite: where a GPU is visible they are
+# skipped, so that a check that stopped firing can never become a launch on invalid memory.
+no_gpu_only = pytest.mark.skipif(_gpu_visible(), reason="made-up device addresses: host-only test")
 
 
 @pytest.mark.parametrize("call,code", [
@@ -129,6 +148,7 @@ FAKE = 1 << 40  # a 16-byte aligned non-null "pointer": never dereferenced, chec
     (lambda: lib_().std_probe_wait_timeout(None, None), B.STD_ERR_INVALID_ARG),
     (lambda: lib_().std_probe_wait_timeout(FAKE + 2, None), B.STD_ERR_INVALID_ARG),
 ])
+@no_gpu_only
 def test_host_side_rejections(lib, call, code):
     assert call() == code
     assert B.std_last_error() != ""
@@ -138,6 +158,7 @@ def lib_():
     return B.lib()
 
 
+@no_gpu_only
 def test_launch_count_ignores_rejected_calls(lib):
     n0 = B.std_launch_count()
     assert n0 >= 0

@@ -596,3 +596,51 @@ def test_launch_count_matches_the_calls():
     assert B.std_get_device_error() == 0
     assert (n1 - n0, n2 - n1) == (4, wl.gamma + 5)
 
+
+
+@pytest.mark.parametrize("early", [False, True])
+@pytest.mark.parametrize("splits", [1, 2, 7, 40, 0])
+def test_sparse_decode_ragged_lengths_problem_aligned_parts(splits, early):
+    """The keys-on-lanes draft kernel over sequences of different lengths -- one shorter
+    than a 128-key tile, one with fewer tiles than a 7- or 40-part split, one over nine
+    tiles -- with the step's row appended in the same launch: explicit splits (equal parts
+    of every problem), the automatic plan, and the early start behind another attention
+    call on the same stream and workspace.  Against the oracle's sparse draft attention
+    over rows j < len[b] + 1 after the append [S-M2, S-M3]; the appended rows bit-exact."""
+    L, Bn, Hq, Hkv, d, cap = 2, 3, 28, 4, 128, 1200
+    lens = np.array([90, 300, 1100], np.int32)
+    rng = np.random.default_rng(11)
+
+    def draw(shape, scale=1.0):
+        return synth.storage(rng.standard_normal(shape).astype(np.float32) * scale, "bf16")
+
+    k, v = draw((L, Bn, Hkv, cap, d), 0.5), draw((L, Bn, Hkv, cap, d))
+    q = draw((L, Bn, Hq, 1, d))
+    kn, vn = draw((L, Bn, Hkv, 1, d), 0.5), draw((L, Bn, Hkv, 1, d))
+    dims = B.dims(L, Bn, Hq, Hkv, d, B.STD_BF16, cap, cap)
+    ws = torch.empty(max(B.std_attn_workspace_size(dims, 1, cap, splits), 16), dtype=torch.uint8, device="cuda")
+    kd, vd, qd = H.to_dev(k), H.to_dev(v), H.to_dev(q)
+    lens_d = torch.from_numpy(lens).cuda()
+    o = torch.full((L, Bn, Hq, 1, d), float("nan"), device="cuda")
+    flags = 0
+    if early:
+        # the predecessor writes only its own output and the workspace: the rows below the
+        # appended one, the lengths and q may be read before it finishes
+        o0 = torch.empty_like(o)
+        B.std_sparse_decode_attn(dims, qd, kd, vd, lens_d, 0, o0, splits, ws)
+        flags = B.STD_ATTN_EARLY_KV | B.STD_ATTN_EARLY_Q
+    B.std_sparse_decode_attn_append_ex(dims, qd, kd, vd, lens_d, 1, H.to_dev(kn), H.to_dev(vn), o, splits, flags, ws)
+    torch.cuda.synchronize()
+    assert B.std_get_device_error() == 0
+    k_ref, v_ref = k.copy(), v.copy()
+    for b in range(Bn):
+        k_ref[:, b, :, lens[b]] = kn[:, b, :, 0]
+        v_ref[:, b, :, lens[b]] = vn[:, b, :, 0]
+    assert np.array_equal(H.to_host_bits(kd), k_ref) and np.array_equal(H.to_host_bits(vd), v_ref)
+    wl = type("W", (), {"dtype": "bf16"})()
+    want = oracle.sparse_decode_attn(H.f64(q, wl), H.f64(k_ref, wl), H.f64(v_ref, wl), lens + 1)
+    err = np.abs(o.cpu().numpy() - want).max()
+    assert err <= H.attn_tol(wl), err
+    if early:
+        want0 = oracle.sparse_decode_attn(H.f64(q, wl), H.f64(k, wl), H.f64(v, wl), lens)
+        assert np.abs(o0.cpu().numpy() - want0).max() <= H.attn_tol(wl)

@@ -290,10 +290,12 @@ int std_gather_sparse(const std_dims* dims, const void* k_full, const void* v_fu
  * keys for up to 16 query rows, 8192 otherwise), or, when all problems together
  * have fewer than 5 tiles per SM (at `cap` keys), a few CTAs per problem: for head
  * dim 128 and at most 16 query rows per problem (the draft) each problem is cut
- * into equal parts of about 2 tiles, one CTA each (at most half as many CTAs
- * as SMs in all), otherwise about one CTA per 5 tiles of the whole sequence -- and
+ * into equal parts of about 3 tiles, one CTA each (at most 16 parts, and at
+ * most half as many CTAs as SMs in all), otherwise about one CTA per 5 tiles of the whole sequence -- and
  * splits = s > 0 launches s x L x B x Hkv CTAs (for the draft's kernel: s equal
- * parts of every problem).  With an early start (STD_ATTN_EARLY_*) and at most 16
+ * parts of every problem; with 2 to 16 parts, the parts of a problem form one
+ * thread-block cluster and merge in distributed shared memory where such a
+ * cluster fits the device).  With an early start (STD_ATTN_EARLY_*) and at most 16
  * query rows, one CTA per problem applies up to 8192 keys; such a call never
  * needs more workspace than the same call without the flags.  fp32 operands (and
  * bf16 with B > 64) use split-K kernels with `splits` key ranges per problem (0 =

@@ -177,9 +177,11 @@ int plan_attn(const std_dims* dims, int nq, int64_t cap, int splits, AttnPlan* p
       // CTA merges; instead each problem gets a few CTAs.  The keys-on-lanes kernel cuts a
       // problem into equal parts of about kTilesPerPart tiles (a part fits the three K/V
       // stages, so with an early start all of it is fetched before the previous kernel
-      // ends; 28 launches of one layer's draft, 4 x 4352 keys, in a CUDA graph with early
-      // K/V, us per step: 361 with 35 parts, 269 with 18, 279 with 14, 279 with 12, 308
-      // with 10, 330 with 7; without early start 337 with 18 parts); the other kernel
+      // ends) and, up to 16 parts, merged inside a thread-block cluster.  28 launches of
+      // one layer's draft, 4 x 4352 keys, in a CUDA graph, us per step without (with) an
+      // early K/V start: 313 (277) with 12 parts in clusters, 330 (286) with 16 in
+      // clusters, 377 (313) with 8 in clusters; merged through global memory: 341 (276)
+      // with 18 parts, 362 (287) with 16, 361 with 35 early; the other kernel
       // takes stream-K ranges of about kMinTilesPerCta tiles (the same launches, us per
       // launch: 25.8 with 148 CTAs, 17.9 with 48, 15.1 with 32, 18.0 with 24).
       int sms;
@@ -188,17 +190,20 @@ int plan_attn(const std_dims* dims, int nq, int64_t cap, int splits, AttnPlan* p
       const int64_t nt_cap = (cap + 127) / 128;
       const int64_t tiles_max = (int64_t)probs * nt_cap;
       constexpr int64_t kMinTilesPerCta = 5;
-      constexpr int64_t kTilesPerPart = 2;
+      constexpr int64_t kTilesPerPart = 3;
+      constexpr int64_t kMaxParts = 16;
       if (probs <= sms && 2 * probs >= sms && cap <= short_cap) {
         ctas = probs;
         parts = aligned ? 1 : 0;
       } else if (tiles_max < (int64_t)sms * kMinTilesPerCta) {
         if (aligned) {
           // at most half the SMs: the next launch's CTAs fit beside this one's and can
-          // start early (the same launches with 19 parts, 76 CTAs: 322 us per step)
+          // start early (the same launches with 19 parts, 76 CTAs: 322 us per step); at
+          // most 16, so that a problem's parts form one thread-block cluster
           int64_t k = (nt_cap + kTilesPerPart - 1) / kTilesPerPart;
           const int64_t k_fit = sms / (2 * (int64_t)probs);
           if (k > k_fit) k = k_fit;
+          if (k > kMaxParts) k = kMaxParts;
           if (k < 1) k = 1;
           parts = (int)k;
           ctas = (int)(k * probs);

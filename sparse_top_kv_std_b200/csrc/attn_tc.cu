@@ -1023,6 +1023,8 @@ struct CfgT {
 };
 constexpr int kTmemColsT = 64;     // O^T at columns 0..15, S^T buffer b at 16 + 16 b
 constexpr uint32_t kColST = 16;
+// Largest thread-block cluster the keys-on-lanes kernel merges a problem's parts in.
+constexpr int kMaxClusterT = 16;
 // Early start: the roles wait for prev_done, which the waiting warp signals once its
 // griddepcontrol.wait returns; the previous kernel may run for long, hence a long bound.
 constexpr uint64_t kPrevWaitNs = 20ull * 1000 * 1000 * 1000;
@@ -1508,7 +1510,18 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         float* wml = a.ws + nslots * a.rows * D;
         unsigned long long* ctr = reinterpret_cast<unsigned long long*>(wml + nslots * a.rows * 2);
         const int slot = prob + blockIdx.x;
-        if (c0 == c1) {
+        if (a.cluster > 1) {
+          // the problem's parts form a cluster: this part's partial stays in shared memory
+          // (K/V stage 0, idle once the segment's last P V has run) for the cluster merge
+          float* po = reinterpret_cast<float*>(smem + C::KV_OFF);
+#pragma unroll
+          for (int r = 0; r < RTT; ++r)
+            if (r0 + r < a.rows) po[(r0 + r) * D + tk] = __uint_as_float(pick(o16, r));
+          if (own_tk && tk < a.rows) {
+            po[RT * D + tk] = m_tk * sc;
+            po[RT * D + RT + tk] = L_tk;
+          }
+        } else if (c0 == c1) {
           // this CTA saw the whole problem: the output (partials: unnormalised, with (m, l))
 #pragma unroll
           for (int r = 0; r < RTT; ++r) {
@@ -1554,6 +1567,11 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       ++kv;
       iter_next(it, ctl, a);
     }
+    if (a.cluster > 1 && seg < 0 && tid < RT) {  // no part of the problem here: an empty partial
+      float* po = reinterpret_cast<float*>(smem + C::KV_OFF);
+      po[RT * D + tid] = -INFINITY;
+      po[RT * D + RT + tid] = 0.f;
+    }
     if (a.partial && blockIdx.x == 0 && tid < 128 &&
         (!a.early || tc::mbar_wait(&ctl->prev_done, 0, abort_flag, a.err, kPrevWaitNs))) {
       // partials of a sequence with no key in the range: o = 0, m = -inf, l = 0
@@ -1571,6 +1589,49 @@ attn_tq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
       }
     }
+  }
+  if (a.cluster > 1) {
+    // Cluster merge: every CTA of the cluster holds one part of problem blockIdx.x / parts
+    // (or an empty partial); rank k's softmax threads combine items [k, k + 1) x rows x D /
+    // cluster of the outputs from all parts' shared memory, in rank order (deterministic).
+    tc::cluster_sync();
+    if (warp >= 2 && warp < 2 + 4 * NG) {
+      const int tid = threadIdx.x - 64;
+      const int cs = a.cluster;
+      const int rank = (int)tc::cluster_ctarank();
+      const int p = blockIdx.x / a.parts;
+      const size_t orow0 = (size_t)((p / a.Hkv) * a.Hq + (p % a.Hkv) * a.G) * a.nq;
+      const uint32_t pb = smem_u32(smem + C::KV_OFF);
+      const int items = a.rows * D;
+      const int i1 = (rank + 1) * items / cs;
+      // outputs after the previous kernel (an early start)
+      const bool go = !a.early || tc::mbar_wait(&ctl->prev_done, 0, abort_flag, a.err, kPrevWaitNs);
+      for (int i = rank * items / cs + tid; go && i < i1; i += NSM) {
+        const int r = i / D, c = i % D;
+        float mk[kMaxClusterT];
+        float M = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < kMaxClusterT; ++k) {
+          mk[k] = k < cs ? tc::ld_dsmem_f32(tc::dsmem_addr(pb + (RT * D + r) * 4, k)) : -INFINITY;
+          M = fmaxf(M, mk[k]);
+        }
+        float L = 0.f, acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMaxClusterT; ++k) {
+          if (mk[k] != -INFINITY) {  // an empty part contributes nothing (its o is not read)
+            const float w = ex2(mk[k] - M);
+            L += w * tc::ld_dsmem_f32(tc::dsmem_addr(pb + (RT * D + RT + r) * 4, k));
+            acc += w * tc::ld_dsmem_f32(tc::dsmem_addr(pb + (r * D + c) * 4, k));
+          }
+        }
+        a.o[(orow0 + r) * D + c] = a.partial ? acc : (L > 0.f ? acc / L : 0.f);
+        if (a.partial && c == 0) {
+          a.ml[(orow0 + r) * 2] = M * kLn2;
+          a.ml[(orow0 + r) * 2 + 1] = L;
+        }
+      }
+    }
+    tc::cluster_sync();  // no CTA leaves while another may still read its shared memory
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -1616,7 +1677,49 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
     attr_done.fetch_or(bit, std::memory_order_release);
   }
   const int threads = keys_on_lanes ? 96 + 128 * (a.rows <= 8 ? 2 : 1) : kThreads;
-  return launch_pdl(kern, dim3(a.splits), dim3(threads), smem_bytes, s, tq, tk, tv, tk16, tv16, a);
+  // keys-on-lanes kernel with 2 .. 16 parts per problem: each problem's parts form one
+  // thread-block cluster (merged in distributed shared memory) if a cluster that large can
+  // be resident on this device (asked once per device and kernel)
+  int cl = 0;
+  if (keys_on_lanes && a.parts >= 2 && a.parts <= kMaxClusterT) {
+    static std::atomic<int> cl_max[16][2];  // largest resident cluster + 1; 0: not asked yet
+    std::atomic<int>& slot = cl_max[dev & 15][a.rows <= 8 ? 1 : 0];
+    int m = slot.load(std::memory_order_acquire);
+    if (m == 0) {
+      m = 1;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+        for (int c = kMaxClusterT; c >= 2 && m == 1; c /= 2) {
+          cudaLaunchConfig_t cfg = {};
+          cfg.gridDim = dim3(c);
+          cfg.blockDim = dim3(threads);
+          cfg.dynamicSmemBytes = smem_bytes;
+          cudaLaunchAttribute at[1];
+          at[0].id = cudaLaunchAttributeClusterDimension;
+          at[0].val.clusterDim.x = c;
+          at[0].val.clusterDim.y = 1;
+          at[0].val.clusterDim.z = 1;
+          cfg.attrs = at;
+          cfg.numAttrs = 1;
+          int n = 0;
+          if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+            (void)cudaGetLastError();  // a refused query leaves no error behind
+          } else if (n > 0) {
+            m = c + 1;
+          }
+        }
+      } else {
+        (void)cudaGetLastError();
+      }
+      slot.store(m, std::memory_order_release);
+    }
+    if (a.parts <= m - 1) cl = a.parts;
+  }
+  AttnArgs b = a;
+  b.cluster = cl;
+  if (cl > 1)
+    return launch_pdl_cluster(kern, dim3(a.splits), dim3(threads), smem_bytes, s, (unsigned)cl, tq, tk, tv, tk16, tv16,
+                              b);
+  return launch_pdl(kern, dim3(a.splits), dim3(threads), smem_bytes, s, tq, tk, tv, tk16, tv16, b);
 }
 
 }  // namespace

@@ -33,6 +33,30 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return e;
 }
 
+// The same with the CTAs grouped into thread-block clusters of `cluster` consecutive CTAs
+// (gridDim.x a multiple of it).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                               unsigned cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  if (e == cudaSuccess) g_launch_count.fetch_add(1, std::memory_order_relaxed);
+  return e;
+}
+
 // One decode-attention launch: query row r of a KV head (r = g * nq + i, g the
 // query head in the group, i the query position) attends to keys
 // j < len[b] + len_off + i.
@@ -50,6 +74,10 @@ struct AttnArgs {
   // CTA c takes part c % parts of problem c / parts, an equal share of that problem's
   // tiles, so no CTA's range straddles two problems; splits = problems x parts.
   int parts;
+  // With parts: the parts of a problem form one thread-block cluster of `cluster` CTAs
+  // and merge their partials through distributed shared memory (set by the launch;
+  // 0: the global partials and the arrival counter).
+  int cluster;
   float* ws;  // partials: [prob][split][rows_pad][d] then [prob][split][rows_pad][2]
   int* err;
   uint32_t epoch;  // per-call tag of the merge counters (tensor-core kernel)

@@ -179,8 +179,8 @@ int plan_attn(const std_dims* dims, int nq, int64_t cap, int splits, AttnPlan* p
       // stages, so with an early start all of it is fetched before the previous kernel
       // ends) and, up to 16 parts, merged inside a thread-block cluster.  28 launches of
       // one layer's draft, 4 x 4352 keys, in a CUDA graph, us per step without (with) an
-      // early K/V start: 313 (277) with 12 parts in clusters, 330 (286) with 16 in
-      // clusters, 377 (313) with 8 in clusters; merged through global memory: 341 (276)
+      // early K/V start: 312 (276) with 12 parts in clusters, 328 (286) with 13, 324
+      // (283) with 14, 330 (286) with 16, 377 (313) with 8; merged through global memory: 341 (276)
       // with 18 parts, 362 (287) with 16, 361 with 35 early; the other kernel
       // takes stream-K ranges of about kMinTilesPerCta tiles (the same launches, us per
       // launch: 25.8 with 148 CTAs, 17.9 with 48, 15.1 with 32, 18.0 with 24).
@@ -200,7 +200,7 @@ int plan_attn(const std_dims* dims, int nq, int64_t cap, int splits, AttnPlan* p
           // at most half the SMs: the next launch's CTAs fit beside this one's and can
           // start early (the same launches with 19 parts, 76 CTAs: 322 us per step); at
           // most 16, so that a problem's parts form one thread-block cluster
-          int64_t k = (nt_cap + kTilesPerPart - 1) / kTilesPerPart;
+          int64_t k = nt_cap / kTilesPerPart;  // parts of at least kTilesPerPart tiles at cap
           const int64_t k_fit = sms / (2 * (int64_t)probs);
           if (k > k_fit) k = k_fit;
           if (k > kMaxParts) k = kMaxParts;

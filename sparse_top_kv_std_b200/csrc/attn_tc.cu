@@ -14,7 +14,9 @@
 // otherwise it writes one partial (m, l, o) per run of tiles of the same
 // problem ("segment") into slot problem + cta, and the last CTA to finish a
 // problem (an epoch-tagged arrival counter per problem, no waiting) merges the
-// partials of that problem.
+// partials of that problem.  The keys-on-lanes kernel for the draft (further down)
+// can instead cut each problem into equal parts, one CTA each, whose CTAs form one
+// thread-block cluster and merge through distributed shared memory.
 //
 // Per tile, inside a CTA (warp 0: TMA producers, lane 0 for K/V and lane 1 for
 // Q; warp 1: TMEM owner and MMA issuer; warps 2-5: softmax -- one thread per

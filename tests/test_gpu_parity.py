@@ -644,3 +644,25 @@ def test_sparse_decode_ragged_lengths_problem_aligned_parts(splits, early):
     if early:
         want0 = oracle.sparse_decode_attn(H.f64(q, wl), H.f64(k, wl), H.f64(v, wl), lens)
         assert np.abs(o0.cpu().numpy() - want0).max() <= H.attn_tol(wl)
+
+
+def test_automatic_draft_grids():
+    """The planner's automatic grid for the draft kernel on this device: a single layer's
+    draft (4 problems of up to 4640 keys) is cut into equal parts of at least three tiles
+    at cap, at most 16 and at most half as many CTAs as SMs; the 28-layer draft takes one
+    CTA per SM, or one CTA per problem when it starts early; an early plan never needs
+    more workspace than the plain one."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    cap = 4640
+    d1 = B.dims(1, 1, 28, 4, 128, B.STD_BF16, 200000, cap)
+    parts = max(1, min((cap + 127) // 128 // 3, 16, sms // (2 * 4)))
+    assert B.std_attn_splits(d1, 1, cap, 0) == 4 * parts
+    d28 = B.dims(28, 1, 28, 4, 128, B.STD_BF16, 200000, cap)
+    assert B.std_attn_splits(d28, 1, cap, 0) == sms
+    early = B.STD_ATTN_EARLY_KV | B.STD_ATTN_EARLY_Q
+    if 112 <= sms <= 224:
+        assert B.std_attn_splits_ex(d28, 1, cap, 0, early) == 112
+    # explicit splits are parts of every problem, with or without the flags
+    assert B.std_attn_splits_ex(d1, 1, cap, 7, early) == 28
+    # the early plan's grid (one CTA per problem) is that of splits = 1
+    assert B.std_attn_workspace_size(d28, 1, cap, 0) >= B.std_attn_workspace_size(d28, 1, cap, 1)

@@ -45,7 +45,7 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="video_140k")
     ap.add_argument("--rounds", type=int, default=None, help="draft+verify rounds per step (default: workload's)")
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-draft-modes", action="store_true",
@@ -498,6 +498,19 @@ def run_std(args, rank, world, local_rank):
     ws = sess.ws_round
     q_text = view("q_text")
 
+    class BufSet:
+        """One decode's device state: a session (caches, lengths, workspaces), the round
+        inputs on the device and the round outputs."""
+
+        def __init__(self, s, d, o):
+            self.sess, self.dv, self.outs, self.ws = s, d, o, s.ws_round
+
+        def view(self, n, r=None):
+            t = self.dv[n] if r is None else self.dv[n][r]
+            return t.view(sd) if t.dtype == torch.int16 else t
+
+    bs0 = BufSet(sess, dv, outs)
+
     def step(ev=None, draft_ev=False):
         """One StD decode: reset lengths, select, R rounds.  ev: dict of event lists to record
         (selection and verify only, unless draft_ev: events between kernels cost overlap)."""
@@ -509,7 +522,9 @@ def run_std(args, rank, world, local_rank):
             ev["sel1"].record()
         rounds(ev, draft_ev)
 
-    def rounds(ev=None, draft_ev=False):
+    def rounds(ev=None, draft_ev=False, bs=None):
+        bs = bs or bs0
+        sess, outs, ws, view, dv = bs.sess, bs.outs, bs.ws, bs.view, bs.dv
         for r in range(R):
             o = outs[r]
             if ev is not None and not draft_ev:
@@ -642,55 +657,73 @@ def run_std(args, rank, world, local_rank):
         acc_dev = torch.zeros((R, wl.B, wl.gamma + 1), dtype=torch.int32, device=dev)
 
         copy_stream = torch.cuda.Stream(device=dev)
-        layer_ev = [torch.cuda.Event() for _ in range(wl.L)]
-        rest_ev = torch.cuda.Event()
         d1 = B.dims(1, wl.B, wl.Hq, wl.Hkv, wl.d, dt, wl.cap_full, wl.cap_sparse)
-        kf_h, vf_h = sess.k_full.view(host_t), sess.v_full.view(host_t)
+        # two buffer sets, taken in turn: the next prompt's cache uploads while this one decodes
+        sets = [bs0]
+        if args.e2e_steps >= 2:
+            s2 = DecodeSession(wl.L, wl.B, wl.Hq, wl.Hkv, wl.d, dt, wl.cap_full, wl.cap_sparse, wl.T, wl.K,
+                               wl.gamma, wl.nvis_max, device=dev)
+            s2.nvis.copy_(nvis_dev)
+            sets.append(BufSet(s2, {n: to_dev(pin[n]) for n in pin}, [s2.round_outputs() for _ in range(R)]))
+        layer_ev = [[torch.cuda.Event() for _ in range(wl.L)] for _ in sets]
+        rest_ev = [torch.cuda.Event() for _ in sets]
+        done_ev = [torch.cuda.Event() for _ in sets]
 
-        def e2e_step():
+        def e2e_step(k):
             # the prompt cache and the text queries arrive layer by layer on a copy stream, and
             # each layer's selection starts as soon as its rows have landed; the rounds need
             # every layer, so they wait for the whole copy
-            copy_stream.wait_stream(stream)  # the previous step is done with these buffers
+            bs = sets[k]
+            s = bs.sess
+            copy_stream.wait_event(done_ev[k])  # the step before on this set is done with it
             with torch.cuda.stream(copy_stream):
+                kf_h, vf_h = s.k_full.view(host_t), s.v_full.view(host_t)
                 for l in range(wl.L):
                     kf_h[l].copy_(pin_k[l], non_blocking=True)
                     vf_h[l].copy_(pin_v[l], non_blocking=True)
-                    dv["q_text"][l].copy_(pin["q_text"][l], non_blocking=True)
-                    layer_ev[l].record(copy_stream)
+                    bs.dv["q_text"][l].copy_(pin["q_text"][l], non_blocking=True)
+                    layer_ev[k][l].record(copy_stream)
                 for n in pin:
                     if n != "q_text":
-                        dv[n].copy_(pin[n], non_blocking=True)
-                rest_ev.record(copy_stream)
-            sess.len_full.copy_(len0, non_blocking=True)
+                        bs.dv[n].copy_(pin[n], non_blocking=True)
+                rest_ev[k].record(copy_stream)
+            s.len_full.copy_(len0, non_blocking=True)
+            qt = bs.view("q_text")
             for l in range(wl.L):
-                stream.wait_event(layer_ev[l])
-                B.std_select_topk(d1, q_text[l], wl.T, sess.k_full[l], sess.v_full[l], sess.nvis, wl.nvis_max, wl.K,
-                                  sess.idx[l], sess.k_sparse[l], sess.v_sparse[l], sess.len_sparse, None,
-                                  sess.ws_select)
-            stream.wait_event(rest_ev)
-            rounds()
+                stream.wait_event(layer_ev[k][l])
+                B.std_select_topk(d1, qt[l], wl.T, s.k_full[l], s.v_full[l], s.nvis, wl.nvis_max, wl.K, s.idx[l],
+                                  s.k_sparse[l], s.v_sparse[l], s.len_sparse, None, s.ws_select)
+            stream.wait_event(rest_ev[k])
+            rounds(bs=bs)
             for r in range(R):
-                acc_dev[r].copy_(outs[r]["accepted"], non_blocking=True)
+                acc_dev[r].copy_(bs.outs[r]["accepted"], non_blocking=True)
             acc_host.copy_(acc_dev, non_blocking=True)
+            done_ev[k].record(stream)
 
-        e2e_step()
+        for k in range(len(sets)):
+            e2e_step(k)
         torch.cuda.synchronize()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if pg:
             pg.barrier()
         torch.cuda.synchronize()
         a0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        for i in range(args.e2e_steps):
+            e2e_step(i % len(sets))
         a1.record(stream)
         torch.cuda.synchronize()
         e_ms = dist_max(a0.elapsed_time(a1), pg, dev)
+        # the same prompt in either buffer set: the accepted tokens read back must equal the
+        # timed region's
+        if not torch.equal(acc_host, torch.stack([o["accepted"] for o in outs]).cpu()):
+            raise RuntimeError("end-to-end steps accepted other tokens than the timed steps")
         h2d = pin_k.numel() * pin_k.element_size() * 2 + sum(t.numel() * t.element_size() for t in pin.values())
         d2h = acc_host.numel() * 4
         e2e = {"value": weak_scaling_value(step_attn, args.e2e_steps, world, e_ms), "unit": "GB/s",
                "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps,
-               "pipeline": "prompt cache copied layer by layer on a second stream, each layer selected as it lands",
+               "pipeline": "two buffer sets taken in turn: each prompt's cache is copied layer by layer on a "
+                           "second stream while the previous prompt decodes, and each layer is selected as it "
+                           "lands",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     if rank != 0:

@@ -599,13 +599,14 @@ def test_launch_count_matches_the_calls():
 
 
 @pytest.mark.parametrize("early", [False, True])
-@pytest.mark.parametrize("splits", [1, 2, 7, 40, 0])
+@pytest.mark.parametrize("splits", [1, 2, 7, 16, 40, 0])
 def test_sparse_decode_ragged_lengths_problem_aligned_parts(splits, early):
     """The keys-on-lanes draft kernel over sequences of different lengths -- one shorter
     than a 128-key tile, one with fewer tiles than a 7- or 40-part split, one over nine
     tiles -- with the step's row appended in the same launch: explicit splits (equal parts
-    of every problem), the automatic plan, and the early start behind another attention
-    call on the same stream and workspace.  Against the oracle's sparse draft attention
+    of every problem; 2 to 16 of them merge inside a thread-block cluster, 16 being the
+    largest, non-portable size), the automatic plan, and the early start behind another
+    attention call on the same stream and workspace.  Against the oracle's sparse draft attention
     over rows j < len[b] + 1 after the append [S-M2, S-M3]; the appended rows bit-exact."""
     L, Bn, Hq, Hkv, d, cap = 2, 3, 28, 4, 128, 1200
     lens = np.array([90, 300, 1100], np.int32)
